@@ -1,0 +1,333 @@
+#!/usr/bin/env python3
+"""Benchmark of the bidirectional SSD mixer on B200.
+
+One step = one ssd_bidir_fwd call over a whole batch of the 130M-shape mixer
+workload (batch 32, L 1024, 24 heads x 64, d_state 128, per-head B/C, bf16
+I/O): both scans, the D terms and the output write. Inputs are synthetic
+(seeded, ssd_inputs) and already resident in HBM when timing starts; they
+total ~1 GB per GPU, well above the 126 MB L2, so no flush is needed between
+steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--path auto|simt|chunked|fused]
+
+Under torchrun every rank runs the same per-GPU workload (independent
+batches: weak scaling, no collective on the data path); rank 0 prints one
+JSON line with the whole-job throughput, timed on the device as the max over
+ranks. `--impl reference` times the fp64 CPU oracle on the host cores
+instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "bidir SSD tokens/s at 130M shape L=1024 (1×B200) + % roofline"
+DEFAULT_WORKLOAD = "mixer130m_b32_L1024"
+PATH_IDS = {"auto": 0, "simt": 1, "chunked": 2, "fused": 3}
+# kernels each path launches per ssd_bidir_fwd call (bf16)
+LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1}
+# source file holding the kernel each path spends its time in
+KERNEL_SOURCE = {"simt": "ssd_simt.cu", "chunked": "ssd_tc.cu", "fused": "ssd_tc.cu"}
+
+
+def algorithmic_bytes(w) -> int:
+    """Unavoidable HBM bytes of one bidirectional call: x read once, dt/B/C of
+    both directions read once, out written once, A and D (fp32)."""
+    io = 4 if w.dtype == "f32" else 2
+    tok = w.batch * w.seqlen
+    elems = tok * w.nheads * w.headdim * 2 + 2 * tok * w.nheads + 4 * tok * w.ngroups * w.dstate
+    return io * elems + 4 * 4 * w.nheads
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def traffic_record(path: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    if it was taken on the current kernel source (else None)."""
+    rec = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(rec):
+        return None
+    with open(rec) as f:
+        d = json.load(f)
+    e = d.get(f"{workload}:{path}")
+    if not e:
+        return None
+    src = os.path.join(ROOT, "bidirectional_mamba_ssd_b200", "csrc", KERNEL_SOURCE[path])
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if e.get("source_sha") != sha:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(w, budget_s: float = 12.0):
+    """The fp64 oracle, as it stands, on the host cores over a bounded sample of
+    the workload: whole batch elements (all heads, both directions), several
+    per call so every core has a (batch, head) unit, until ~budget_s of work
+    or the workload's batch is used up."""
+    import math
+    import torch
+    import oracle
+    import ssd_inputs as si
+    cores = oracle.threads(0)
+    per_call = max(1, min(w.batch, math.ceil(cores / w.nheads)))
+    used = min(cores, per_call * w.nheads)
+    done, t_used, calls = 0, 0.0, 0
+    while t_used < budget_s and done < w.batch:
+        k = min(per_call, w.batch - done)
+        inp = si.bidir_inputs(k, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.dtype,
+                              seed=100 + calls, device="cpu")
+        arrs = [inp[n].to(torch.float64).numpy() for n in ("x", "dt", "A", "B", "C", "D")]
+        t0 = time.perf_counter()
+        oracle.bidir(*arrs)
+        t_used += time.perf_counter() - t0
+        done += k
+        calls += 1
+    tokens = done * w.seqlen
+    return {"value": tokens / t_used, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{done} of {w.batch} batch elements x {w.seqlen} tokens x {w.nheads} heads, "
+                      f"both directions, fp64 sequential recurrence, {t_used:.1f} s on {used} threads"}
+
+
+def run_reference(args, w):
+    """Reference arm: the fp64 CPU oracle timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    vals = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        info = cpu_baseline(w, budget_s=4.0)
+        if i >= args.warmup:
+            vals.append(info["value"])
+    v = statistics.median(vals)
+    info["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * w.tokens / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, **{k: getattr(w, k) for k in
+                       ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "chunk")},
+                       "io_dtype": w.dtype},
+            "cpu_baseline": info,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--path", default="auto", choices=list(PATH_IDS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    import ssd_inputs as si
+    w = si.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import bidirectional_mamba_ssd_b200 as ssd
+    path = PATH_IDS[args.path]
+    if path == 0:
+        path = ssd.lib.ssd_select_path(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                                       w.chunk, 1 if w.dtype == "bf16" else 0)
+    path_name = {v: k for k, v in PATH_IDS.items()}[path]
+
+    inp = si.workload_inputs(w, seed=1000 + rank, device=dev)
+    names = ("x", "dt", "A", "B", "C", "D")
+    out = torch.empty_like(inp["x"])
+    ws = ssd.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssd.ssd_bidir_fwd(*(inp[n] for n in names), out=out, chunk=w.chunk, path=path, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc = ws.status()
+    if rc != 0:
+        raise SystemExit(f"device status {rc} after warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    ms_step = ms / args.steps
+    tokens_job = w.tokens * world
+    value = tokens_job * args.steps / (ms / 1e3)
+
+    # end to end through the public API: pinned host inputs -> device -> mixer -> host output
+    e2e = None
+    if not args.no_e2e:
+        host = {n: inp[n].cpu().pin_memory() for n in names}
+        dev_in = {n: torch.empty_like(inp[n]) for n in names}
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for n in names:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            ssd.ssd_bidir_fwd(*(dev_in[n] for n in names), out=out, chunk=w.chunk, path=path, workspace=ws)
+            host_out.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        k = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": tokens_job * k / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = measured_peaks()
+    abytes = algorithmic_bytes(w)
+    launches = LAUNCHES_PER_CALL[path_name]
+    achieved = abytes / (ms_step / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_record(path_name, w.name),
+            "peak_source": f"{peaks['source']} STREAM-copy HBM GB/s",
+            "algorithmic_bytes_per_launch": abytes,
+            "kernel": {"simt": "scan_simt_kernel", "chunked": "tc_state/tc_pass/tc_out kernels (whole step)",
+                       "fused": "tc_fused_kernel"}[path_name]}
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, **{k: getattr(w, k) for k in
+                       ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "chunk")},
+                       "io_dtype": w.dtype, "state_dtype": "f32", "path": path_name,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": roof,
+            "e2e": e2e,
+            "gpu_launches": launches * args.steps,
+            "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

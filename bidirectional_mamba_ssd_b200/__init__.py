@@ -1,0 +1,230 @@
+"""Bidirectional Mamba-2 SSD mixer for B200 (sm_100a): Python binding.
+
+A thin layer over the C ABI of libssd_bidir.so (include/ssd_bidir.h): it
+checks that the torch tensors it is handed are contiguous CUDA tensors of
+the expected dtype, passes their device pointers, sizes and the current CUDA
+stream to the library, and allocates outputs and the workspace with torch.
+Every step of the computation runs in the library's kernels.
+
+Functions carry the C names:
+  ssd_bidir_fwd(x, dt, A, B, C, D, chunk=256)          -> out
+  ssd_prefix_state(x, dt, A, B, init=None, chunk=256)  -> state (batch, H, P, N) fp32
+  ssd_block_step(x, dt, A, B, C, D, prefix_state)      -> out
+Shapes (row-major, natural token order; [0] forward, [1] reverse):
+  x (batch, L, H, P); dt (2, batch, L, H); A, D (2, H) fp32;
+  B, C (2, batch, L, G, N); out like x.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib as _c
+from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED,  # noqa: F401
+                   SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA,
+                   SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT, SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE,
+                   SSD_OP_BLOCK_STEP)
+
+__all__ = ["ssd_bidir_fwd", "ssd_prefix_state", "ssd_block_step", "ssd_workspace_bytes",
+           "ssd_get_device_status", "SSDError", "Workspace", "lib"]
+
+lib = _c.load()
+
+_DT = {torch.float32: _c.SSD_F32, torch.bfloat16: _c.SSD_BF16}
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.ssd_error_string(status).decode()} (status {status})")
+
+
+def _check(rc: int, what: str):
+    if rc != _c.SSD_OK:
+        raise SSDError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t, name, dtype=None, device=None, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims (got {tuple(t.shape)})")
+
+
+def ssd_workspace_bytes(op, batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype) -> int:
+    code = _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return int(lib.ssd_workspace_bytes(op, batch, seqlen, nheads, headdim, dstate, ngroups,
+                                       chunk, code))
+
+
+class Workspace:
+    """A device buffer for the library's workspace, grown on demand.
+
+    The first 256 bytes are the status header; the buffer is zero-filled on
+    (re)allocation, which initialises it. One Workspace must not be shared by
+    calls that overlap on the device (different streams)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+    def status(self) -> int:
+        """Synchronise the current stream and read (and clear) the status header."""
+        if self.buf is None:
+            return _c.SSD_OK
+        return int(lib.ssd_get_device_status(_ptr(self.buf), ctypes.c_void_p(_stream(self.device))))
+
+
+_default_ws: dict = {}
+
+
+def _workspace(device, stream, ws):
+    if ws is not None:
+        return ws
+    key = (device.index, stream)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def ssd_get_device_status(ws: Workspace | None = None) -> int:
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = _workspace(dev, _stream(dev), ws)
+    return w.status()
+
+
+def _dims(x, B):
+    batch, L, H, P = x.shape
+    G, N = B.shape[-2], B.shape[-1]
+    return batch, L, H, P, G, N
+
+
+def ssd_bidir_fwd(x, dt, A, B, C, D, out=None, *, chunk: int = 256, path: int = SSD_PATH_AUTO,
+                  workspace: Workspace | None = None):
+    """Bidirectional SSD mixer over whole sequences (include/ssd_bidir.h: ssd_bidir_fwd)."""
+    _need(x, "x", ndim=4)
+    dev, io = x.device, x.dtype
+    if io not in _DT:
+        raise ValueError(f"x dtype {io} not supported (float32 or bfloat16)")
+    _need(dt, "dt", io, dev, 4)
+    _need(B, "B", io, dev, 5)
+    _need(C, "C", io, dev, 5)
+    _need(A, "A", torch.float32, dev, 2)
+    _need(D, "D", torch.float32, dev, 2)
+    batch, L, H, P, G, N = _dims(x, B)
+    if tuple(dt.shape) != (2, batch, L, H) or tuple(B.shape) != (2, batch, L, G, N) \
+            or tuple(C.shape) != tuple(B.shape) or tuple(A.shape) != (2, H) or tuple(D.shape) != (2, H):
+        raise ValueError("shape mismatch: want x (b,L,H,P), dt (2,b,L,H), B/C (2,b,L,G,N), A/D (2,H)")
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _need(out, "out", io, dev, 4)
+        if out.shape != x.shape:
+            raise ValueError("out must have x's shape")
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    nbytes = ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, L, H, P, N, G, chunk, io)
+    if nbytes == 0:
+        _check(_c.SSD_ERR_UNSUPPORTED, "ssd_bidir_fwd")
+    buf = ws.get(nbytes)
+    rc = lib.ssd_bidir_fwd_path(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(out),
+                                batch, L, H, P, N, G, chunk, _DT[io], int(path),
+                                _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_bidir_fwd")
+    return out
+
+
+def ssd_prefix_state(x, dt, A, B, init=None, out=None, *, chunk: int = 256,
+                     workspace: Workspace | None = None):
+    """Forward-only state after the last token (include/ssd_bidir.h: ssd_prefix_state).
+    dt (batch, L, H), A (H), B (batch, L, G, N): the forward direction's."""
+    _need(x, "x", ndim=4)
+    dev, io = x.device, x.dtype
+    if io not in _DT:
+        raise ValueError(f"x dtype {io} not supported (float32 or bfloat16)")
+    _need(dt, "dt", io, dev, 3)
+    _need(B, "B", io, dev, 4)
+    _need(A, "A", torch.float32, dev, 1)
+    batch, L, H, P = x.shape
+    G, N = B.shape[-2], B.shape[-1]
+    if tuple(dt.shape) != (batch, L, H) or tuple(B.shape) != (batch, L, G, N) or tuple(A.shape) != (H,):
+        raise ValueError("shape mismatch: want x (b,L,H,P), dt (b,L,H), B (b,L,G,N), A (H)")
+    if init is not None:
+        _need(init, "init", torch.float32, dev, 4)
+        if tuple(init.shape) != (batch, H, P, N):
+            raise ValueError("init must be (batch, H, P, N)")
+    if out is None:
+        out = torch.empty(batch, H, P, N, dtype=torch.float32, device=dev)
+    else:
+        _need(out, "out", torch.float32, dev, 4)
+        if tuple(out.shape) != (batch, H, P, N):
+            raise ValueError("out must be (batch, H, P, N)")
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    nbytes = ssd_workspace_bytes(SSD_OP_PREFIX_STATE, batch, L, H, P, N, G, chunk, io)
+    if nbytes == 0:
+        _check(_c.SSD_ERR_UNSUPPORTED, "ssd_prefix_state")
+    buf = ws.get(nbytes)
+    rc = lib.ssd_prefix_state(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init), _ptr(out),
+                              batch, L, H, P, N, G, chunk, _DT[io],
+                              _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_prefix_state")
+    return out
+
+
+def ssd_block_step(x, dt, A, B, C, D, prefix_state, out=None, *, workspace: Workspace | None = None):
+    """One block-diffusion step on the active block (include/ssd_bidir.h: ssd_block_step)."""
+    _need(x, "x", ndim=4)
+    dev, io = x.device, x.dtype
+    if io not in _DT:
+        raise ValueError(f"x dtype {io} not supported (float32 or bfloat16)")
+    _need(dt, "dt", io, dev, 4)
+    _need(B, "B", io, dev, 5)
+    _need(C, "C", io, dev, 5)
+    _need(A, "A", torch.float32, dev, 2)
+    _need(D, "D", torch.float32, dev, 2)
+    batch, T, H, P, G, N = _dims(x, B)
+    if tuple(dt.shape) != (2, batch, T, H) or tuple(B.shape) != (2, batch, T, G, N) \
+            or tuple(C.shape) != tuple(B.shape) or tuple(A.shape) != (2, H) or tuple(D.shape) != (2, H):
+        raise ValueError("shape mismatch: want x (b,T,H,P), dt (2,b,T,H), B/C (2,b,T,G,N), A/D (2,H)")
+    if prefix_state is not None:
+        _need(prefix_state, "prefix_state", torch.float32, dev, 4)
+        if tuple(prefix_state.shape) != (batch, H, P, N):
+            raise ValueError("prefix_state must be (batch, H, P, N)")
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _need(out, "out", io, dev, 4)
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    nbytes = ssd_workspace_bytes(SSD_OP_BLOCK_STEP, batch, T, H, P, N, G, 64, io)
+    if nbytes == 0:
+        _check(_c.SSD_ERR_UNSUPPORTED, "ssd_block_step")
+    buf = ws.get(nbytes)
+    rc = lib.ssd_block_step(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                            _ptr(prefix_state), _ptr(out), batch, T, H, P, N, G, _DT[io],
+                            _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_block_step")
+    return out

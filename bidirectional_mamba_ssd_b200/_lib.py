@@ -1,0 +1,54 @@
+"""ctypes declarations of libssd_bidir.so (see include/ssd_bidir.h).
+
+Loading fails loudly: there is no Python or CPU implementation behind these
+names, so a missing or stale library is an ImportError, not a fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd_bidir.so")
+
+# Values of include/ssd_bidir.h.
+SSD_F32, SSD_BF16 = 0, 1
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED = 0, -1, -2
+SSD_ERR_CUDA, SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT = -3, -4, -5
+SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE, SSD_OP_BLOCK_STEP = 0, 1, 2
+SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED = 0, 1, 2, 3
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+# name -> (restype, argtypes); the C-ABI surface the header declares.
+SIGNATURES = {
+    "ssd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "ssd_select_path": (_i, [_i] * 8),
+    "ssd_workspace_init": (_i, [_vp, _sz, _vp]),
+    "ssd_bidir_fwd": (_i, [_vp] * 7 + [_i] * 8 + [_vp, _sz, _vp]),
+    "ssd_bidir_fwd_path": (_i, [_vp] * 7 + [_i] * 9 + [_vp, _sz, _vp]),
+    "ssd_prefix_state": (_i, [_vp] * 6 + [_i] * 8 + [_vp, _sz, _vp]),
+    "ssd_block_step": (_i, [_vp] * 8 + [_i] * 7 + [_vp, _sz, _vp]),
+    "ssd_get_device_status": (_i, [_vp, _vp]),
+    "ssd_error_string": (ctypes.c_char_p, [_i]),
+    "ssd_version": (_i, []),
+}
+
+_lib = None
+
+
+def load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is not built; run `python -c 'import __graft_entry__ as g; g.build()'` "
+                "(nvcc, sm_100a). There is no fallback implementation.")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+    return _lib

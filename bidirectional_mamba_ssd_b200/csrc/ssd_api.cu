@@ -1,0 +1,244 @@
+// C ABI of the bidirectional SSD mixer: argument checks, workspace sizing and
+// dispatch to the kernels. Declarations and documentation: include/ssd_bidir.h.
+#include <stdint.h>
+#include <string.h>
+
+#include "ssd_bidir.h"
+#include "ssd_kernels.h"
+
+using ssd::SimtArgs;
+using ssd::TcArgs;
+
+namespace {
+
+constexpr int kHeaddim = 64;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Shape checks shared by every entry point. Returns SSD_OK or an error code.
+int check_shape(int batch, int seqlen, int nheads, int headdim, int dstate, int ngroups,
+                int chunk, int dtype, bool check_chunk) {
+    if (batch < 0 || seqlen < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (nheads % ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    if (headdim != kHeaddim) return SSD_ERR_UNSUPPORTED;
+    if (dstate != 64 && dstate != 128) return SSD_ERR_UNSUPPORTED;
+    if (check_chunk && chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_UNSUPPORTED;
+    // Index arithmetic uses 64-bit offsets, but token counts stay in int.
+    if ((long long)batch * seqlen > (1ll << 31) - 1) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+int to_status(cudaError_t e) {
+    if (e == cudaSuccess) return SSD_OK;
+    if (e == cudaErrorNotSupported) return SSD_ERR_UNSUPPORTED;
+    return SSD_ERR_CUDA;
+}
+
+size_t simt_scratch(int op, int batch, int seqlen, int nheads) {
+    if (op == SSD_OP_PREFIX_STATE) return 0;
+    return sizeof(float) * (size_t)batch * seqlen * nheads * kHeaddim;
+}
+
+size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+float *scratch_ptr(void *ws) { return reinterpret_cast<float *>(static_cast<char *>(ws) + ssd::kStatusBytes); }
+
+// Kernel choice of SSD_PATH_AUTO: bf16 runs on the tensor cores, in one
+// kernel per (batch, head) when there are enough of those to fill the GPU,
+// else in the tile-parallel chunked kernels; fp32 runs the sequential scan.
+int auto_path(int batch, int seqlen, int nheads, int ngroups, int dstate, int dtype) {
+    if (dtype != SSD_BF16) return SSD_PATH_SIMT;
+    if (ssd::tc_fused_supported(batch, seqlen, nheads, ngroups, dstate)) return SSD_PATH_FUSED;
+    return SSD_PATH_CHUNKED;
+}
+
+int bidir_impl(const void *x, const void *dt, const float *A, const void *B, const void *C,
+               const float *D, void *out, int batch, int seqlen, int nheads, int headdim,
+               int dstate, int ngroups, int chunk, int dtype, int path, void *workspace,
+               size_t ws_bytes, void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
+    if (rc != SSD_OK) return rc;
+    if (path < SSD_PATH_AUTO || path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, seqlen, nheads, headdim, dstate,
+                                       ngroups, chunk, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    if (!x || !dt || !A || !B || !C || !D || !out) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned16(C) || !aligned16(out) ||
+        !aligned4(A) || !aligned4(D))
+        return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (path == SSD_PATH_AUTO) path = auto_path(batch, seqlen, nheads, ngroups, dstate, dtype);
+
+    if (path == SSD_PATH_SIMT) {
+        SimtArgs a{};
+        a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
+        a.out = out; a.yacc = scratch_ptr(workspace);
+        a.dt_dir_stride = (long long)batch * seqlen * nheads;
+        a.bc_dir_stride = (long long)batch * seqlen * ngroups * dstate;
+        a.A_dir_stride = nheads;
+        a.batch = batch; a.L = seqlen; a.H = nheads; a.G = ngroups;
+        a.ndir = 2; a.has_output = 1;
+        return to_status(ssd::launch_scan_simt(a, dtype == SSD_BF16, dstate, s));
+    }
+    if (dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    TcArgs t{};
+    t.x = x; t.dt = dt; t.A = A; t.B = B; t.C = C; t.D = D; t.out = out;
+    t.workspace = workspace; t.ws_bytes = ws_bytes;
+    t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+    if (path == SSD_PATH_FUSED) return to_status(ssd::launch_tc_fused(t, s));
+    return to_status(ssd::launch_tc_chunked(t, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdim, int dstate,
+                           int ngroups, int chunk, int dtype) {
+    const bool use_chunk = op != SSD_OP_BLOCK_STEP;
+    if (check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, use_chunk) != SSD_OK)
+        return 0;
+    size_t scratch = simt_scratch(op, batch, seqlen, nheads);
+    if (dtype == SSD_BF16) {
+        if (op == SSD_OP_BIDIR_FWD) {
+            size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 2);
+            size_t f = ssd::tc_fused_scratch_bytes(batch, seqlen, nheads, dstate);
+            scratch = scratch > c ? scratch : c;
+            scratch = scratch > f ? scratch : f;
+        } else if (op == SSD_OP_PREFIX_STATE) {
+            size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 1);
+            scratch = scratch > c ? scratch : c;
+        }
+    }
+    return ssd::kStatusBytes + round256(scratch);
+}
+
+int ssd_select_path(int batch, int seqlen, int nheads, int headdim, int dstate, int ngroups,
+                    int chunk, int dtype) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
+    if (rc != SSD_OK) return rc;
+    return auto_path(batch, seqlen, nheads, ngroups, dstate, dtype);
+}
+
+int ssd_workspace_init(void *workspace, size_t ws_bytes, void *stream) {
+    if (!workspace || ws_bytes < ssd::kStatusBytes) return SSD_ERR_WORKSPACE;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, ssd::kStatusBytes, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+int ssd_bidir_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                  const float *D, void *out, int batch, int seqlen, int nheads, int headdim,
+                  int dstate, int ngroups, int chunk, int dtype, void *workspace, size_t ws_bytes,
+                  void *stream) {
+    return bidir_impl(x, dt, A, B, C, D, out, batch, seqlen, nheads, headdim, dstate, ngroups,
+                      chunk, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
+}
+
+int ssd_bidir_fwd_path(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                       const float *D, void *out, int batch, int seqlen, int nheads, int headdim,
+                       int dstate, int ngroups, int chunk, int dtype, int path, void *workspace,
+                       size_t ws_bytes, void *stream) {
+    return bidir_impl(x, dt, A, B, C, D, out, batch, seqlen, nheads, headdim, dstate, ngroups,
+                      chunk, dtype, path, workspace, ws_bytes, stream);
+}
+
+int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *B,
+                     const float *init_state, float *state_out, int batch, int seqlen, int nheads,
+                     int headdim, int dstate, int ngroups, int chunk, int dtype, void *workspace,
+                     size_t ws_bytes, void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
+    if (rc != SSD_OK) return rc;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_PREFIX_STATE, batch, seqlen, nheads, headdim, dstate,
+                                       ngroups, chunk, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0) return SSD_OK;
+    if (!state_out || !aligned16(state_out)) return SSD_ERR_INVALID_ARG;
+    if (init_state && !aligned16(init_state)) return SSD_ERR_INVALID_ARG;
+    if (seqlen > 0) {
+        if (!x || !dt || !A || !B) return SSD_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned4(A)) return SSD_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == SSD_BF16 && seqlen > 0) {
+        TcArgs t{};
+        t.x = x; t.dt = dt; t.A = A; t.B = B; t.init = init_state; t.state_out = state_out;
+        t.workspace = workspace; t.ws_bytes = ws_bytes;
+        t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 1;
+        cudaError_t e = ssd::launch_tc_chunked(t, s);
+        if (e != cudaErrorNotSupported) return to_status(e);
+        (void)cudaGetLastError();
+    }
+    SimtArgs a{};
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = nullptr; a.D = nullptr;
+    a.init = init_state; a.state_out = state_out;
+    a.dt_dir_stride = 0; a.bc_dir_stride = 0; a.A_dir_stride = 0;
+    a.batch = batch; a.L = seqlen; a.H = nheads; a.G = ngroups;
+    a.ndir = 1; a.has_output = 0;
+    return to_status(ssd::launch_scan_simt(a, dtype == SSD_BF16, dstate, s));
+}
+
+int ssd_block_step(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                   const float *D, const float *prefix_state, void *out, int batch, int blk_len,
+                   int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
+                   size_t ws_bytes, void *stream) {
+    int rc = check_shape(batch, blk_len, nheads, headdim, dstate, ngroups, 64, dtype, false);
+    if (rc != SSD_OK) return rc;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_BLOCK_STEP, batch, blk_len, nheads, headdim, dstate,
+                                       ngroups, 64, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0 || blk_len == 0) return SSD_OK;
+    if (!x || !dt || !A || !B || !C || !D || !out) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned16(C) || !aligned16(out) ||
+        !aligned4(A) || !aligned4(D))
+        return SSD_ERR_INVALID_ARG;
+    if (prefix_state && !aligned16(prefix_state)) return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SimtArgs a{};
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.init = prefix_state; a.state_out = nullptr;
+    a.out = out; a.yacc = scratch_ptr(workspace);
+    a.dt_dir_stride = (long long)batch * blk_len * nheads;
+    a.bc_dir_stride = (long long)batch * blk_len * ngroups * dstate;
+    a.A_dir_stride = nheads;
+    a.batch = batch; a.L = blk_len; a.H = nheads; a.G = ngroups;
+    a.ndir = 2; a.has_output = 1;
+    return to_status(ssd::launch_scan_simt(a, dtype == SSD_BF16, dstate, s));
+}
+
+int ssd_get_device_status(const void *workspace, void *stream) {
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ssd::DeviceStatus st;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SSD_ERR_CUDA;
+    if (cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+    if (st.flags == 0) return SSD_OK;
+    if (cudaMemset(const_cast<void *>(workspace), 0, sizeof(st)) != cudaSuccess) return SSD_ERR_CUDA;
+    return (st.flags & ssd::kFlagTimeout) ? SSD_ERR_TIMEOUT : SSD_ERR_CUDA;
+}
+
+const char *ssd_error_string(int status) {
+    switch (status) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size, ngroups does not divide nheads)";
+        case SSD_ERR_UNSUPPORTED: return "unsupported shape, chunk, dtype or path";
+        case SSD_ERR_CUDA: return "CUDA launch or runtime error";
+        case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSD_ERR_TIMEOUT: return "a bounded device-side wait expired";
+        default: return "unknown status";
+    }
+}
+
+int ssd_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// Internal launch interface between the C ABI (ssd_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "ssd_common.cuh"
+
+namespace ssd {
+
+// Arguments of the sequential CUDA-core scan (ssd_simt.cu).
+struct SimtArgs {
+    const void *x;            // (batch, L, H, 64) io
+    const void *dt;           // direction 0 base; + dir * dt_dir_stride elements
+    const float *A;           // A[dir * A_dir_stride + h]
+    const void *B;            // direction 0 base; + dir * bc_dir_stride elements
+    const void *C;            // as B; nullptr when no output is read
+    const float *D;           // (2, H) when has_output
+    const float *init;        // (batch, H, 64, N) start of the forward scan, or nullptr
+    float *state_out;         // (batch, H, 64, N) final forward state, or nullptr
+    void *out;                // (batch, L, H, 64) io when has_output
+    float *yacc;              // (batch, L, H, 64) fp32 scratch for the forward partial
+    long long dt_dir_stride, bc_dir_stride;
+    int A_dir_stride;
+    int batch, L, H, G;
+    int ndir;                 // 1: forward only, 2: forward + reverse
+    int has_output;
+};
+
+cudaError_t launch_scan_simt(const SimtArgs &a, bool bf16, int N, cudaStream_t stream);
+
+// Arguments of the tensor-core kernels (ssd_tc.cu). bf16 I/O only.
+struct TcArgs {
+    const void *x;            // (batch, L, H, 64) bf16
+    const void *dt;           // (2, batch, L, H) bf16 (forward only: (batch, L, H))
+    const float *A;           // (2, H) (forward only: (H))
+    const void *B;            // (2, batch, L, G, N) bf16
+    const void *C;            // (2, batch, L, G, N) bf16 or nullptr
+    const float *D;           // (2, H)
+    const float *init;        // (batch, H, 64, N) forward start state or nullptr
+    float *state_out;         // (batch, H, 64, N) or nullptr
+    void *out;                // (batch, L, H, 64) bf16
+    void *workspace;          // status header + scratch
+    size_t ws_bytes;
+    int batch, L, H, G, N;
+    int ndir;                 // 1 (prefix state) or 2
+};
+
+// Scratch bytes (after the status header) the tensor-core paths need.
+size_t tc_chunked_scratch_bytes(int batch, int L, int H, int N, int ndir);
+size_t tc_fused_scratch_bytes(int batch, int L, int H, int N);
+bool tc_fused_supported(int batch, int L, int H, int G, int N);
+
+cudaError_t launch_tc_chunked(const TcArgs &a, cudaStream_t stream);
+cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream);
+
+}  // namespace ssd

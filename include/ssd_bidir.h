@@ -1,0 +1,183 @@
+/*
+ * ssd_bidir.h - C ABI of the bidirectional Mamba-2 SSD mixer for B200 (sm_100a).
+ *
+ * What the mixer computes, per batch element b, head h and direction
+ * d in {forward, reverse} (head h reads B/C group g = h / (nheads/ngroups)):
+ *
+ *   forward,  t = 0 .. L-1:  h_t  = exp(dt_t A_h) h_{t-1}  + dt_t B_t x_t^T,  yf_t = C_t^T h_t
+ *   reverse,  t = L-1 .. 0:  h'_t = exp(dt'_t A'_h) h'_{t+1} + dt'_t B'_t x_t^T, yb_t = C'_t^T h'_t
+ *   out_t = yf_t + yb_t + (D_h + D'_h) x_t
+ *
+ * with an N x P state (N = dstate, P = headdim) starting at zero.
+ *  - "DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone",
+ *    Technical Summary, 2. Methodology, Core Architecture: a forward and a
+ *    backward Mamba-2 layer over the sequence, added.
+ *  - "DiffMamba - Checkpoints" model card, Model details: the backward
+ *    layer is Mamba-2 on the flipped sequence. The reverse scan here reads
+ *    its inputs in natural token order from the right end, which is the
+ *    same thing without materialising a flipped copy.
+ *  - The pages name Mamba-2 without printing its recurrence; the scalar-
+ *    decay selective SSM above is the standard Mamba-2 (SSD) definition.
+ *  - "Training Hybrid Block Diffusion Language Models with Partial
+ *    Bidirectionality", Abstract and Methodology: for block diffusion the
+ *    reverse scan is confined to the active block, so the forward state of
+ *    the prefix is a cache that is reused exactly (ssd_prefix_state,
+ *    ssd_block_step).
+ *
+ * Conventions for every entry point
+ *  - All tensor arguments are DEVICE pointers to dense row-major arrays in
+ *    natural token order, 16-byte aligned. The caller allocates and owns
+ *    every buffer, the workspace included; the library allocates nothing,
+ *    keeps no global state and never synchronises (except
+ *    ssd_get_device_status).
+ *  - "io" = the I/O dtype chosen by `dtype` (SSD_F32 or SSD_BF16): x, dt,
+ *    B, C and out use it. A, D and states are always fp32.
+ *  - Direction-stacked tensors have a leading dimension of 2:
+ *    [0] = forward, [1] = reverse.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
+ *    enqueued on it; results are ready when the stream reaches that point.
+ *  - Arguments are checked on the host before anything is launched; a bad
+ *    argument returns an error code and launches nothing. Launch failures
+ *    return SSD_ERR_CUDA. A device-side wait that ran out of its iteration
+ *    bound sets a flag in the workspace header that ssd_get_device_status
+ *    reports; the kernel then returns without finishing its output.
+ *  - Supported in this version: headdim == 64, dstate in {64, 128},
+ *    nheads % ngroups == 0, chunk in {64, 128, 256}, seqlen >= 0 (no
+ *    multiple-of-chunk requirement). Other shapes return
+ *    SSD_ERR_UNSUPPORTED.
+ *  - chunk is the chunk length of the chunked evaluation. The result does
+ *    not depend on it beyond floating-point rounding. The fp32 path runs a
+ *    sequential scan and ignores it; the bf16 tensor-core path evaluates
+ *    128-token tiles (see each function).
+ *  - Calls that share a workspace must not overlap on the device.
+ */
+#ifndef SSD_BIDIR_H
+#define SSD_BIDIR_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* I/O element type. */
+enum {
+    SSD_F32 = 0,  /* IEEE fp32 */
+    SSD_BF16 = 1  /* bfloat16; outputs rounded to nearest-even once, at the final store */
+};
+
+/* Status codes. */
+enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = -1,   /* null/misaligned pointer, negative size, ngroups not dividing nheads */
+    SSD_ERR_UNSUPPORTED = -2,   /* valid but not implemented: headdim, dstate, chunk, dtype */
+    SSD_ERR_CUDA = -3,          /* a CUDA launch or driver call failed (cudaGetLastError) */
+    SSD_ERR_WORKSPACE = -4,     /* workspace NULL or smaller than ssd_workspace_bytes() */
+    SSD_ERR_TIMEOUT = -5        /* a bounded device-side wait expired (from ssd_get_device_status) */
+};
+
+/* Operation ids for ssd_workspace_bytes. */
+enum { SSD_OP_BIDIR_FWD = 0, SSD_OP_PREFIX_STATE = 1, SSD_OP_BLOCK_STEP = 2 };
+
+/* Kernel selection for ssd_bidir_fwd_path (tests and benchmarks). */
+enum {
+    SSD_PATH_AUTO = 0,     /* what ssd_bidir_fwd uses */
+    SSD_PATH_SIMT = 1,     /* sequential fp32 scan on CUDA cores, any dtype */
+    SSD_PATH_CHUNKED = 2,  /* tensor-core chunked path in three kernels (states through the workspace) */
+    SSD_PATH_FUSED = 3     /* tensor-core path, one kernel per (batch, head) */
+};
+
+/* The SSD_PATH_* that ssd_bidir_fwd (SSD_PATH_AUTO) runs for these sizes, or
+ * a negative status for arguments it rejects. Host only; launches nothing. */
+int ssd_select_path(int batch, int seqlen, int nheads, int headdim, int dstate,
+                    int ngroups, int chunk, int dtype);
+
+/* Bytes of device workspace the operation needs for these sizes (always at
+ * least the 256-byte status header). `seqlen` is the block length for
+ * SSD_OP_BLOCK_STEP. Returns 0 for arguments the operation rejects. */
+size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdim,
+                           int dstate, int ngroups, int chunk, int dtype);
+
+/* Zero the workspace's status header (256 bytes) on `stream`. A workspace
+ * must be initialised once before first use (zero-filled memory counts). */
+int ssd_workspace_init(void *workspace, size_t ws_bytes, void *stream);
+
+/* Full-sequence bidirectional mixer (both scans over the whole sequence).
+ *   x    (batch, seqlen, nheads, headdim)           io
+ *   dt   (2, batch, seqlen, nheads)                 io, > 0 (already softplus'ed; used as given)
+ *   A    (2, nheads)                                fp32, <= 0
+ *   B, C (2, batch, seqlen, ngroups, dstate)        io
+ *   D    (2, nheads)                                fp32
+ *   out  (batch, seqlen, nheads, headdim)           io, overwritten; must not alias an input
+ * bf16 I/O runs the tensor-core path: state and accumulation fp32, the
+ * decay-masked C.B^T tile and the chunk states rounded to bf16 as MMA
+ * operands. fp32 I/O runs the sequential fp32 scan.
+ * Source: "DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone",
+ * Technical Summary, 2. Methodology, Core Architecture. */
+int ssd_bidir_fwd(const void *x, const void *dt, const float *A, const void *B,
+                  const void *C, const float *D, void *out,
+                  int batch, int seqlen, int nheads, int headdim, int dstate,
+                  int ngroups, int chunk, int dtype,
+                  void *workspace, size_t ws_bytes, void *stream);
+
+/* ssd_bidir_fwd with an explicit kernel choice (SSD_PATH_*). A path that
+ * cannot run these arguments returns SSD_ERR_UNSUPPORTED. The workspace
+ * must be at least ssd_workspace_bytes(SSD_OP_BIDIR_FWD, ...). */
+int ssd_bidir_fwd_path(const void *x, const void *dt, const float *A, const void *B,
+                       const void *C, const float *D, void *out,
+                       int batch, int seqlen, int nheads, int headdim, int dstate,
+                       int ngroups, int chunk, int dtype, int path,
+                       void *workspace, size_t ws_bytes, void *stream);
+
+/* Forward-only state after the last token of each sequence: the cache that
+ * block diffusion reuses ("Training Hybrid Block Diffusion Language Models
+ * with Partial Bidirectionality", Abstract: prefix-only states reused
+ * exactly; Technical Contribution: timestep-free prefix cache).
+ *   x          (batch, seqlen, nheads, headdim)     io
+ *   dt         (batch, seqlen, nheads)              io, forward direction only
+ *   A          (nheads)                             fp32
+ *   B          (batch, seqlen, ngroups, dstate)     io
+ *   init_state (batch, nheads, headdim, dstate)     fp32, NULL = zero start
+ *   state_out  (batch, nheads, headdim, dstate)     fp32; may equal init_state (in-place update,
+ *                                                   e.g. committing a finished block)
+ * The state is stored as headdim rows of dstate values: state[b][h][p][n] = h[n][p]. */
+int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *B,
+                     const float *init_state, float *state_out,
+                     int batch, int seqlen, int nheads, int headdim, int dstate,
+                     int ngroups, int chunk, int dtype,
+                     void *workspace, size_t ws_bytes, void *stream);
+
+/* One denoising step on the active block of blk_len tokens: the forward scan
+ * starts from the cached prefix state, the reverse scan starts from zero at
+ * the block's right end and sees only the block ("Training Hybrid Block
+ * Diffusion Language Models with Partial Bidirectionality", Methodology and
+ * Key Results: the reverse scan is restricted to the active block so states
+ * stay prefix-only). prefix_state is only read.
+ *   x            (batch, blk_len, nheads, headdim)        io
+ *   dt           (2, batch, blk_len, nheads)              io
+ *   A, D         (2, nheads)                              fp32
+ *   B, C         (2, batch, blk_len, ngroups, dstate)     io
+ *   prefix_state (batch, nheads, headdim, dstate)         fp32, NULL = zero prefix
+ *   out          (batch, blk_len, nheads, headdim)        io, overwritten */
+int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
+                   const void *C, const float *D, const float *prefix_state, void *out,
+                   int batch, int blk_len, int nheads, int headdim, int dstate,
+                   int ngroups, int dtype,
+                   void *workspace, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, read and clear the workspace's status header.
+ * Returns SSD_OK, SSD_ERR_TIMEOUT (a bounded device wait expired in a call
+ * since the last check) or SSD_ERR_CUDA (the stream reported an error). */
+int ssd_get_device_status(const void *workspace, void *stream);
+
+/* Static description of a status code. */
+const char *ssd_error_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_BIDIR_H */

@@ -1,0 +1,99 @@
+"""Error metrics and oracle sampling shared by the GPU parity tests.
+
+Tolerances (written here once, used by every parity test):
+  fp32 I/O:  max_i |y_i - o_i| / max(|o_i|, rms(o)) <= 1e-4
+             (elementwise relative error, floored at the output RMS so that
+             outputs near zero do not dominate);
+  bf16 I/O:  max_i e_i <= 2e-2 * rms(o), with
+             e_i = max(0, |y_i - o_i| - ulp_bf16(max(|y_i|, |o_i|)) / 2)
+             for outputs stored as bf16 (the error the computation adds on
+             top of the one mandatory round-to-nearest of the result), and
+             e_i = |y_i - o_i| for fp32 results such as states.
+o is the unrounded fp64 oracle output on the very same (rounded) inputs.
+Why the half ulp is excluded for bf16 outputs: these outputs are heavy
+tailed (max|o| / rms(o) is about 9 at the 130M shape), so rounding the exact
+result to bf16 already moves the largest ones by up to 2^-9 * 9 * rms ~ 0.018
+rms; a bare max-abs bound of 0.02 rms would reject correctly rounded answers.
+The RMS of the error is reported too (rms_err).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from ssd_inputs import to_f64
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+def rms(o):
+    return float(np.sqrt(np.mean(np.square(o)))) if o.size else 0.0
+
+
+def half_ulp_bf16(a):
+    """Half the bf16 spacing at |a| (8 significant bits)."""
+    a = np.abs(np.asarray(a, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 0.5 * np.exp2(e - 7)
+
+
+def err_f32(y, o):
+    y = np.asarray(y, dtype=np.float64)
+    floor = max(rms(o), 1e-30)
+    return float(np.max(np.abs(y - o) / np.maximum(np.abs(o), floor))) if o.size else 0.0
+
+
+def err_bf16(y, o, rounded_output=True):
+    y = np.asarray(y, dtype=np.float64)
+    if not o.size:
+        return 0.0
+    d = np.abs(y - o)
+    if rounded_output:
+        d = np.maximum(d - half_ulp_bf16(np.maximum(np.abs(y), np.abs(o))), 0.0)
+    return float(np.max(d) / max(rms(o), 1e-30))
+
+
+def rms_err(y, o):
+    return float(np.sqrt(np.mean((np.asarray(y, np.float64) - o) ** 2)) / max(rms(o), 1e-30)) if o.size else 0.0
+
+
+def check(y, o, io_dtype, what="", state=False):
+    """Assert the parity bar for the I/O dtype; return the error.
+    state=True: y is an fp32 result (a state), not a bf16-rounded output."""
+    assert np.isfinite(np.asarray(y, dtype=np.float64)).all(), f"{what}: non-finite output"
+    if io_dtype == torch.float32:
+        e = err_f32(y, o)
+        assert e <= TOL_F32, f"{what}: fp32 max rel err {e:.3e} > {TOL_F32}"
+    else:
+        e = err_bf16(y, o, rounded_output=not state)
+        assert e <= TOL_BF16, f"{what}: bf16 err / rms {e:.3e} > {TOL_BF16} (rms err {rms_err(y, o):.2e})"
+    return e
+
+
+def unit_problem(inp, b, h):
+    """The (1, L, 1, P) sub-problem of unit (b, h), as float64 numpy, G = 1."""
+    H = inp["x"].shape[2]
+    G = inp["B"].shape[3]
+    g = h // (H // G)
+    return (to_f64(inp["x"][b:b + 1, :, h:h + 1]), to_f64(inp["dt"][:, b:b + 1, :, h:h + 1]),
+            to_f64(inp["A"][:, h:h + 1]), to_f64(inp["B"][:, b:b + 1, :, g:g + 1]),
+            to_f64(inp["C"][:, b:b + 1, :, g:g + 1]), to_f64(inp["D"][:, h:h + 1]))
+
+
+def oracle_units(inp, units, nthreads=0):
+    """Oracle outputs (L, P) for each sampled unit (b, h)."""
+    res = {}
+    for b, h in units:
+        res[(b, h)] = oracle.bidir(*unit_problem(inp, b, h), nthreads=nthreads)[0, :, 0]
+    return res
+
+
+def sample_units(batch, H, k, seed=0):
+    rng = np.random.default_rng(seed)
+    allu = [(b, h) for b in range(batch) for h in range(H)]
+    pick = set([allu[0], allu[-1]])
+    while len(pick) < min(k, len(allu)):
+        pick.add(allu[int(rng.integers(len(allu)))])
+    return sorted(pick)

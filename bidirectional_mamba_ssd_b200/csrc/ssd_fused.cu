@@ -1,0 +1,686 @@
+// Fused bidirectional SSD kernel for sm_100a: one persistent CTA per SM walks
+// (batch, head) units; for each unit it computes both scans and writes the
+// summed output once.
+//
+// Per unit, in two phases over 128-token tiles (the tile algebra is the one
+// described in ssd_tc.cu):
+//   phase 1, tiles right to left: the reverse scan's tile states
+//            S' = B'^T diag(w') X on the tensor cores, chained in fp32
+//            registers into the reverse state entering each tile from the
+//            right; those states (bf16, the MMA operand of phase 2) go to
+//            the workspace and stay L2-resident until phase 2 reads them;
+//   phase 2, tiles left to right: C.B^T of both directions, the decay mask,
+//            (M_f + M_b) X, C_f.H_f and C_b.H_b, the forward state chained
+//            in fp32 registers, y = Yd + e_f Yo_f + e_b Yo_b + (D_f + D_b) x,
+//            one bf16 TMA store per tile.
+// Forward and reverse scans, added: "DiffuMamba: High-Throughput Diffusion
+// LMs with Mamba Backbone", Technical Summary, 2. Methodology, Core
+// Architecture; reverse = forward on the flipped sequence: "DiffMamba -
+// Checkpoints" model card, Model details.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: x tiles (2 slots), B/C tiles (3-slot ring),
+//               reverse states (1 slot)
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2..5  epilogue: thread r owns tile row r = 32 * (warp % 4) + lane
+//               (its TMEM lane): decay sums, diag(w) X, the masked matrix,
+//               state chains, outputs.
+// Phase-1 inputs (x, B') are loaded with an L2 evict-last hint and re-read in
+// phase 2 with evict-first, so the re-read mostly hits L2.
+//
+// Every wait is an mbarrier wait bounded in time (sm100.cuh); a lost arrival
+// sets the workspace's timeout flag and the CTA runs to its end.
+#include <cuda.h>
+#include <stdint.h>
+
+#include "sm100.cuh"
+#include "ssd_kernels.h"
+#include "ssd_tmap.h"
+
+namespace ssd {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTile = 128;
+constexpr int kP = 64;
+constexpr uint32_t kSlab = 16384;       // 128 rows x 128 bytes
+constexpr int kRing = 3;                // B/C ring slots (32 KB each)
+constexpr int kThreads = 192;
+
+struct FusedParams {
+    const __nv_bfloat16 *dt;   // (2, batch, L, H)
+    const float *A;            // (2, H)
+    const float *D;            // (2, H)
+    __nv_bfloat16 *hb;         // (units, nt, N, 64) reverse states entering each tile
+    DeviceStatus *status;
+    int batch, L, H, G, nt, units;
+};
+
+// barrier indices
+enum {
+    B_RING_FULL = 0,                 // kRing
+    B_RING_EMPTY = B_RING_FULL + kRing,
+    B_X_FULL = B_RING_EMPTY + kRing, // 2
+    B_X_EMPTY = B_X_FULL + 2,        // 2
+    B_HB_FULL = B_X_EMPTY + 2,
+    B_HB_EMPTY,
+    B_HB_WRITTEN,                    // epilogue -> producer: phase-1 states are in global memory
+    B_G_READY,                       // MMA -> epilogue
+    B_S_READY,
+    B_Y_READY,
+    B_XW_READY,                      // epilogue -> MMA
+    B_M_READY,
+    B_S_FREE,
+    B_Y_FREE,
+    B_COUNT
+};
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0,
+                                                 int c1, int c2, int c3, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_5d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0,
+                                                 int c1, int c2, int c3, int c4, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+        "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0,
+                                                 int c1, int c2, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void st_global_v4_hint(void *p, uint4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// named barrier over the four epilogue warps
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ float bf2f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+// Inclusive scan over the 128 epilogue threads (row order), prefix or suffix.
+__device__ __forceinline__ float scan_rows(float v, bool suffix, int row, float *red) {
+    const int lane = row & 31, wq = row >> 5;
+    if (!suffix) {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            float n = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += n;
+        }
+        if (lane == 31) red[wq] = v;
+    } else {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            float n = __shfl_down_sync(0xffffffffu, v, o);
+            if (lane + o < 32) v += n;
+        }
+        if (lane == 0) red[wq] = v;
+    }
+    epi_sync();
+    float add = 0.f;
+    if (!suffix) {
+        for (int k = 0; k < wq; ++k) add += red[k];
+    } else {
+        for (int k = wq + 1; k < 4; ++k) add += red[k];
+    }
+    epi_sync();
+    return v + add;
+}
+
+template <int N>
+struct Smem {
+    static constexpr uint32_t kBC = N * 256;            // one B or C tile (N/64 slabs)
+    static constexpr uint32_t kH = N * 128;             // one bf16 (N, 64) state
+    static constexpr uint32_t x0 = 0;                   // 2 x slots
+    static constexpr uint32_t ring = x0 + 2 * kSlab;    // kRing slots of 32 KB
+    static constexpr uint32_t hb = ring + kRing * 2 * kSlab;
+    static constexpr uint32_t hf = hb + kH;
+    static constexpr uint32_t xw = hf + kH;             // diag(w) x
+    static constexpr uint32_t m = xw + kSlab;           // masked matrix, 2 slabs
+    static constexpr uint32_t small = m + 2 * kSlab;
+    static constexpr uint32_t bytes = small + 4096;     // barriers + per-tile vectors
+};
+
+template <int N>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
+                const __grid_constant__ CUtensorMap tm_out, const FusedParams p) {
+    using S = Smem<N>;
+    constexpr int NSLAB = N / 64;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *g = smem_raw + (base - smem_u32(smem_raw));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
+    float *red = reinterpret_cast<float *>(g + S::small + 256);   // 8 floats
+    float *af = red + 8;             // A_f * prefix sums of dt_f over the tile
+    float *ab = af + kTile;          // A_b * suffix sums of dt_b over the tile
+    float *colf = ab + kTile;        // per-column factors of the forward mask
+    float *colb = colf + kTile;      // per-column factors of the reverse mask
+    float *dtf = colb + kTile;
+    float *dtb = dtf + kTile;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+    if (tid == 0) {
+        *abort_flag = 0;
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(bar(B_RING_FULL + i), 1);
+            mbar_init(bar(B_RING_EMPTY + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(B_X_FULL + i), 1);
+            mbar_init(bar(B_X_EMPTY + i), 1);
+        }
+        for (int i = B_HB_FULL; i < B_COUNT; ++i) mbar_init(bar(i), 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tGf = tmem, tGb = tmem + 128, tYof = tmem + 256, tYob = tmem + 320,
+                   tYd = tmem + 384, tS = tmem + 448;
+    const int nt = p.nt;
+    const int hpg = p.H / p.G;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+            uint32_t kr = 0, kx = 0, kh = 0;  // loads issued into ring / x / hb
+            uint32_t units_done = 0;
+            auto ring_slot = [&](uint32_t k) -> uint32_t {
+                const uint32_t s = k % kRing;
+                if (k >= kRing) mbar_wait(bar(B_RING_EMPTY + s), ((k / kRing) - 1) & 1, abort_flag, p.status, 101);
+                return s;
+            };
+            auto x_slot = [&](uint32_t k) -> uint32_t {
+                const uint32_t s = k & 1;
+                if (k >= 2) mbar_wait(bar(B_X_EMPTY + s), ((k >> 1) - 1) & 1, abort_flag, p.status, 102);
+                return s;
+            };
+            for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++units_done) {
+                const int b = u / p.H, h = u % p.H, gg = h / hpg;
+                // phase 1: x and B' of every tile, right to left
+                for (int i = nt - 1; i >= 0; --i) {
+                    const uint32_t xs = x_slot(kx++);
+                    mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
+                    tma_load_4d_hint(base + S::x0 + xs * kSlab, &tm_x, bar(B_X_FULL + xs), 0, h, i * kTile, b, keep);
+                    const uint32_t rs = ring_slot(kr++);
+                    mbar_arrive_expect_tx(bar(B_RING_FULL + rs), S::kBC);
+                    for (int k = 0; k < NSLAB; ++k)
+                        tma_load_5d_hint(base + S::ring + rs * 2 * kSlab + k * kSlab, &tm_b, bar(B_RING_FULL + rs),
+                                         64 * k, gg, i * kTile, b, 1, keep);
+                }
+                // the reverse states of this unit must be in global memory
+                mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103);
+                // phase 2: x, C_f, B_f, C_b, B_b, H_b of every tile, left to right
+                for (int i = 0; i < nt; ++i) {
+                    const int t0 = i * kTile;
+                    const uint32_t xs = x_slot(kx++);
+                    mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
+                    tma_load_4d_hint(base + S::x0 + xs * kSlab, &tm_x, bar(B_X_FULL + xs), 0, h, t0, b, stream);
+                    const CUtensorMap *maps[4] = {&tm_c, &tm_b, &tm_c, &tm_b};
+                    const int dirs[4] = {0, 0, 1, 1};
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t rs = ring_slot(kr++);
+                        mbar_arrive_expect_tx(bar(B_RING_FULL + rs), S::kBC);
+                        for (int k = 0; k < NSLAB; ++k)
+                            tma_load_5d_hint(base + S::ring + rs * 2 * kSlab + k * kSlab, maps[j],
+                                             bar(B_RING_FULL + rs), 64 * k, gg, t0, b, dirs[j], stream);
+                    }
+                    if (kh >= 1) mbar_wait(bar(B_HB_EMPTY), (kh - 1) & 1, abort_flag, p.status, 104);
+                    ++kh;
+                    mbar_arrive_expect_tx(bar(B_HB_FULL), S::kH);
+                    tma_load_3d_hint(base + S::hb, &tm_h, bar(B_HB_FULL), 0, 0, u * nt + i, stream);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_state = idesc_bf16_f32(128, 64, true, true);   // B^T (MN) x X' (MN)
+            constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);    // C (K) x B (K)
+            constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);      // C (K) x H (MN); M (K) x X (MN)
+            uint32_t kr = 0, kx = 0, kh = 0;
+            uint32_t n_xw = 0, n_m = 0, n_sfree = 0, n_yfree = 0;
+            bool first_s = true, first_y = true;
+            auto wait_ring = [&](uint32_t k) -> uint32_t {
+                const uint32_t s = k % kRing;
+                mbar_wait(bar(B_RING_FULL + s), (k / kRing) & 1, abort_flag, p.status, 201);
+                return s;
+            };
+            for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+                // phase 1: S' = B'^T diag(w') X per tile
+                for (int i = nt - 1; i >= 0; --i) {
+                    const uint32_t xs_unused = kx++ & 1;
+                    (void)xs_unused;
+                    const uint32_t rs = wait_ring(kr++);
+                    mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 202);
+                    if (!first_s) mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 203);
+                    first_s = false;
+                    tc_fence_after();
+                    const uint32_t sB = base + S::ring + rs * 2 * kSlab;
+                    for (int k = 0; k < kTile / 16; ++k)
+                        mma_bf16_ss(tS, sdesc_sw128(sB + k * 2048, kSlab, 1024),
+                                    sdesc_sw128(base + S::xw + k * 2048, kSlab, 1024), id_state, k > 0);
+                    mma_commit(bar(B_S_READY));
+                    mma_commit(bar(B_RING_EMPTY + rs));
+                }
+                // phase 2. Issue order keeps the 3-slot ring moving: each slot is
+                // released by an MMA that needs no later load of the same tile
+                // (C_f after C_f.H_f, B_f after S_f, B_b after G_b, C_b after C_b.H_b).
+                for (int i = 0; i < nt; ++i) {
+                    const uint32_t xs = kx++ & 1;
+                    mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 204);
+                    const uint32_t rCf = wait_ring(kr++);
+                    const uint32_t rBf = wait_ring(kr++);
+                    const uint32_t sCf = base + S::ring + rCf * 2 * kSlab, sBf = base + S::ring + rBf * 2 * kSlab;
+                    tc_fence_after();
+                    // 1. G_f = C_f B_f^T
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
+                        mma_bf16_ss(tGf, sdesc_sw128(sCf + ko, 0, 1024), sdesc_sw128(sBf + ko, 0, 1024), id_g, k > 0);
+                    }
+                    // 2. Yo_f = C_f H_f: previous outputs read, H_f of this tile written
+                    if (!first_y) mbar_wait(bar(B_Y_FREE), n_yfree++ & 1, abort_flag, p.status, 205);
+                    first_y = false;
+                    mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 206);
+                    tc_fence_after();
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
+                        mma_bf16_ss(tYof, sdesc_sw128(sCf + ko, 0, 1024),
+                                    sdesc_sw128(base + S::hf + k * 2048, kSlab, 1024), id_o, k > 0);
+                    }
+                    mma_commit(bar(B_RING_EMPTY + rCf));
+                    // 3. S_f = B_f^T diag(w_f) X
+                    mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 208);
+                    tc_fence_after();
+                    for (int k = 0; k < kTile / 16; ++k)
+                        mma_bf16_ss(tS, sdesc_sw128(sBf + k * 2048, kSlab, 1024),
+                                    sdesc_sw128(base + S::xw + k * 2048, kSlab, 1024), id_state, k > 0);
+                    mma_commit(bar(B_S_READY));
+                    mma_commit(bar(B_RING_EMPTY + rBf));
+                    // 4. G_b = C_b B_b^T
+                    const uint32_t rCb = wait_ring(kr++);
+                    const uint32_t rBb = wait_ring(kr++);
+                    const uint32_t sCb = base + S::ring + rCb * 2 * kSlab, sBb = base + S::ring + rBb * 2 * kSlab;
+                    tc_fence_after();
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
+                        mma_bf16_ss(tGb, sdesc_sw128(sCb + ko, 0, 1024), sdesc_sw128(sBb + ko, 0, 1024), id_g, k > 0);
+                    }
+                    mma_commit(bar(B_G_READY));
+                    mma_commit(bar(B_RING_EMPTY + rBb));
+                    // 5. Yo_b = C_b H_b
+                    mbar_wait(bar(B_HB_FULL), kh++ & 1, abort_flag, p.status, 207);
+                    tc_fence_after();
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
+                        mma_bf16_ss(tYob, sdesc_sw128(sCb + ko, 0, 1024),
+                                    sdesc_sw128(base + S::hb + k * 2048, kSlab, 1024), id_o, k > 0);
+                    }
+                    mma_commit(bar(B_RING_EMPTY + rCb));
+                    mma_commit(bar(B_HB_EMPTY));
+                    // 6. Yd = M X
+                    mbar_wait(bar(B_M_READY), n_m++ & 1, abort_flag, p.status, 209);
+                    tc_fence_after();
+                    const uint32_t sX = base + S::x0 + xs * kSlab;
+                    for (int k = 0; k < kTile / 16; ++k)
+                        mma_bf16_ss(tYd, sdesc_sw128(base + S::m + (k >> 2) * kSlab + (k & 3) * 32, 0, 1024),
+                                    sdesc_sw128(sX + k * 2048, kSlab, 1024), id_o, k > 0);
+                    mma_commit(bar(B_Y_READY));
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int row = ((warp & 3) << 5) | lane;          // TMEM lane == tile row
+        const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+        const uint64_t keep = policy_evict_last();
+        uint32_t kx = 0, n_g = 0, n_s = 0, n_y = 0;
+        uint32_t units_done = 0;
+        uint8_t *xw_row = g + S::xw + row * 128;
+        float hreg[kP];
+
+        // H_f operand starts at zero for every unit; written before the first
+        // S_FREE arrival, so the first C_f.H_f of each unit reads zeros.
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++units_done) {
+            const int b = u / p.H, h = u % p.H;
+            const float Af = p.A[h], Ab = p.A[p.H + h];
+            const float dsum = p.D[h] + p.D[p.H + h];
+            const size_t dt_dir = (size_t)p.batch * p.L * p.H;
+
+            // ---------------- phase 1: reverse states, right to left
+#pragma unroll
+            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
+            for (int i = nt - 1; i >= 0; --i) {
+                const int t = i * kTile + row;
+                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
+                const float cs = scan_rows(vb, true, row, red);      // suffix sums
+                if (row == 0) red[4] = cs;                            // tile total
+                // state entering tile i from the right (before this tile's update)
+                if (row < N) {
+                    __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 v = make_uint4(pack_bf16x2(hreg[8 * c], hreg[8 * c + 1]),
+                                             pack_bf16x2(hreg[8 * c + 2], hreg[8 * c + 3]),
+                                             pack_bf16x2(hreg[8 * c + 4], hreg[8 * c + 5]),
+                                             pack_bf16x2(hreg[8 * c + 6], hreg[8 * c + 7]));
+                        st_global_v4_hint(dst + 8 * c, v, keep);
+                    }
+                }
+                epi_sync();
+                const float total = red[4];
+                const float w = __expf(Ab * (total - cs)) * vb;      // exp(A' sum_{r<s} dt') dt'_s
+                // diag(w') X into the X' buffer (row-local scaling)
+                const uint32_t xs = kx++ & 1;
+                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 301);
+                {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(g + S::x0 + xs * kSlab + row * 128);
+                    uint4 *dst = reinterpret_cast<uint4 *>(xw_row);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 v = src[c];
+                        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) q[j] = pack_bf16x2(bf2f(q[j] & 0xffffu) * w, bf2f(q[j] >> 16) * w);
+                        dst[c] = v;
+                    }
+                }
+                fence_proxy_async_smem();
+                epi_sync();
+                if (row == 0) {
+                    mbar_arrive(bar(B_XW_READY));
+                    mbar_arrive(bar(B_X_EMPTY + xs));
+                }
+                // S' ready: chain the reverse state
+                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 302);
+                tc_fence_after();
+                const float gdec = __expf(Ab * total);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t v[32];
+                    tmem_ld32(tS + lane_off + half * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
+                }
+                if (i == 0) {
+                    // start of phase 2 for this unit: H_f operand = 0
+                    uint4 *hf = reinterpret_cast<uint4 *>(g + S::hf + row * 128);
+                    if (row < N) {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) hf[c] = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                }
+                tc_fence_before();
+                epi_sync();
+                if (row == 0) mbar_arrive(bar(B_S_FREE));
+            }
+            // all reverse states of this unit are written: hand them to the TMA proxy
+            fence_proxy_async_global();
+            epi_sync();
+            if (row == 0) mbar_arrive(bar(B_HB_WRITTEN));
+
+            // ---------------- phase 2: outputs, left to right
+#pragma unroll
+            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;      // forward state
+            for (int i = 0; i < nt; ++i) {
+                const int t0 = i * kTile, t = t0 + row;
+                const float vf = t < p.L ? __bfloat162float(p.dt[((size_t)b * p.L + t) * p.H + h]) : 0.f;
+                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
+                const float csf = scan_rows(vf, false, row, red);
+                const float csb = scan_rows(vb, true, row, red);
+                const float my_af = Af * csf, my_ab = Ab * csb;
+                af[row] = my_af;
+                ab[row] = my_ab;
+                dtf[row] = vf;
+                dtb[row] = vb;
+                if (row == kTile - 1) red[5] = csf;   // forward tile total
+                epi_sync();
+                // per-column mask factors: forward relative to the end of the
+                // row's 32-block, reverse relative to its start
+                colf[row] = __expf(af[row | 31] - my_af) * vf;
+                colb[row] = __expf(ab[row & ~31] - my_ab) * vb;
+                const float totf = red[5];
+                const float wf = __expf(Af * (totf - csf)) * vf;     // exp(A sum_{r>s} dt) dt_s
+                // diag(w_f) X
+                const uint32_t xs = kx++ & 1;
+                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 311);
+                uint8_t *xrow = g + S::x0 + xs * kSlab + row * 128;
+                {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(xrow);
+                    uint4 *dst = reinterpret_cast<uint4 *>(xw_row);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 v = src[c];
+                        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) q[j] = pack_bf16x2(bf2f(q[j] & 0xffffu) * wf, bf2f(q[j] >> 16) * wf);
+                        dst[c] = v;
+                    }
+                }
+                fence_proxy_async_smem();
+                epi_sync();
+                if (row == 0) mbar_arrive(bar(B_XW_READY));
+
+                // masked matrix M = M_f + M_b (bf16, K-major) from G_f, G_b
+                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 312);
+                tc_fence_after();
+                uint8_t *mrow = g + S::m;
+#pragma unroll 1
+                for (int J = 0; J < 4; ++J) {
+                    uint32_t gf[32], gb[32];
+                    tmem_ld32(tGf + lane_off + J * 32, gf);
+                    tmem_ld32(tGb + lane_off + J * 32, gb);
+                    tmem_wait_ld();
+                    const int s0 = J * 32;
+                    const bool f_full = row >= s0 + 31, f_none = row < s0;
+                    const bool b_full = row <= s0, b_none = row > s0 + 31;
+                    const float rf = f_full ? __expf(my_af - af[s0 + 31]) : 0.f;
+                    const float rb = b_full ? __expf(my_ab - ab[s0]) : 0.f;
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int q = 0; q < 32; q += 2) {
+                        float mv[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int s = s0 + q + e;
+                            float mf, mb;
+                            if (f_full) mf = __uint_as_float(gf[q + e]) * rf * colf[s];
+                            else if (f_none || s > row) mf = 0.f;
+                            else mf = __uint_as_float(gf[q + e]) * __expf(my_af - af[s]) * dtf[s];
+                            if (b_full) mb = __uint_as_float(gb[q + e]) * rb * colb[s];
+                            else if (b_none || s < row) mb = 0.f;
+                            else mb = __uint_as_float(gb[q + e]) * __expf(my_ab - ab[s]) * dtb[s];
+                            mv[e] = mf + mb;
+                        }
+                        packed[q / 2] = pack_bf16x2(mv[0], mv[1]);
+                    }
+                    uint8_t *slab = mrow + (J >> 1) * kSlab;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4 *>(slab + sw128_offset(row, (J & 1) * 4 + c)) =
+                            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (row == 0) mbar_arrive(bar(B_M_READY));
+
+                // forward state chain: H_f <- exp(A sum dt) H_f + S_f; bf16 copy for C_f.H_f
+                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 313);
+                tc_fence_after();
+                const float gdec = __expf(Af * totf);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t v[32];
+                    tmem_ld32(tS + lane_off + half * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
+                }
+                if (row < N) {
+                    uint8_t *hrow = g + S::hf;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4 *>(hrow + sw128_offset(row, c)) =
+                            make_uint4(pack_bf16x2(hreg[8 * c], hreg[8 * c + 1]),
+                                       pack_bf16x2(hreg[8 * c + 2], hreg[8 * c + 3]),
+                                       pack_bf16x2(hreg[8 * c + 4], hreg[8 * c + 5]),
+                                       pack_bf16x2(hreg[8 * c + 6], hreg[8 * c + 7]));
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (row == 0) mbar_arrive(bar(B_S_FREE));
+
+                // output tile, written over the x slot, then one TMA store
+                mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 314);
+                tc_fence_after();
+                const float ef = __expf(my_af), eb = __expf(my_ab);
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t yd[32], yf[32], yb[32];
+                    tmem_ld32(tYd + lane_off + half * 32, yd);
+                    tmem_ld32(tYof + lane_off + half * 32, yf);
+                    tmem_ld32(tYob + lane_off + half * 32, yb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 *q = reinterpret_cast<uint4 *>(xrow - row * 128 + sw128_offset(row, half * 4 + c));
+                        uint4 xv = *q;
+                        uint32_t *xu = reinterpret_cast<uint32_t *>(&xv);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = c * 8 + 2 * e;
+                            const float y0 = __uint_as_float(yd[i0]) + ef * __uint_as_float(yf[i0]) +
+                                             eb * __uint_as_float(yb[i0]) + dsum * bf2f(xu[e] & 0xffffu);
+                            const float y1 = __uint_as_float(yd[i0 + 1]) + ef * __uint_as_float(yf[i0 + 1]) +
+                                             eb * __uint_as_float(yb[i0 + 1]) + dsum * bf2f(xu[e] >> 16);
+                            xu[e] = pack_bf16x2(y0, y1);
+                        }
+                        *q = xv;
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (row == 0) {
+                    mbar_arrive(bar(B_Y_FREE));
+                    if (!*abort_flag) {
+                        tma_store_4d(&tm_out, base + S::x0 + xs * kSlab, 0, h, t0, b);
+                        tma_store_commit();
+                    }
+                    // the store must have read the slot before the producer refills it
+                    tma_store_wait_read();
+                    mbar_arrive(bar(B_X_EMPTY + xs));
+                }
+            }
+        }
+        if (row == 0) tma_store_wait_all();
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+template <int N>
+cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
+    using S = Smem<N>;
+    const int nt = (a.L + kTile - 1) / kTile;
+    const int units = a.batch * a.H;
+    if (a.ws_bytes < kStatusBytes + tc_fused_scratch_bytes(a.batch, a.L, a.H, N)) return cudaErrorInvalidValue;
+    FusedParams p{};
+    p.dt = static_cast<const __nv_bfloat16 *>(a.dt);
+    p.A = a.A;
+    p.D = a.D;
+    p.hb = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(a.workspace) + kStatusBytes);
+    p.status = static_cast<DeviceStatus *>(a.workspace);
+    p.batch = a.batch; p.L = a.L; p.H = a.H; p.G = a.G; p.nt = nt; p.units = units;
+
+    CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_out;
+    if (!tmap::map_x(&tm_x, a.x, a.batch, a.L, a.H) || !tmap::map_bc(&tm_b, a.B, 2, a.batch, a.L, a.G, N) ||
+        !tmap::map_bc(&tm_c, a.C, 2, a.batch, a.L, a.G, N) ||
+        !tmap::map_h(&tm_h, p.hb, (long long)units * nt, N) || !tmap::map_x(&tm_out, a.out, a.batch, a.L, a.H))
+        return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    auto k = tc_fused_kernel<N>;
+    const size_t smem = S::bytes + 1024;
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+    const int grid = units < sms ? units : sms;
+    k<<<grid, kThreads, smem, stream>>>(tm_x, tm_b, tm_c, tm_h, tm_out, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t tc_fused_scratch_bytes(int batch, int L, int H, int N) {
+    const size_t nt = (size_t)(L + kTile - 1) / kTile;
+    return align256((size_t)batch * H * nt * N * kP * 2);
+}
+
+bool tc_fused_supported(int batch, int L, int H, int G, int N) {
+    (void)G;
+    if (L <= 0 || batch <= 0) return false;
+    if (N != 64 && N != 128) return false;
+    // one unit per CTA at a time: worthwhile when the units fill the GPU
+    if ((long long)batch * H < 148) return false;
+    const long long entries = (long long)batch * H * ((L + kTile - 1) / kTile);
+    return entries < (1ll << 31);
+}
+
+cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream) {
+    if (a.L <= 0 || a.batch <= 0) return cudaErrorNotSupported;
+    if (!tmap::encode_fn()) return cudaErrorNotSupported;
+    const long long entries = (long long)a.batch * a.H * ((a.L + kTile - 1) / kTile);
+    if (entries >= (1ll << 31)) return cudaErrorNotSupported;
+    return a.N == 64 ? run_fused<64>(a, stream) : run_fused<128>(a, stream);
+}
+
+}  // namespace ssd

@@ -30,6 +30,7 @@ SIGNATURES = {
     "ssd_bidir_fwd_path": (_i, [_vp] * 7 + [_i] * 9 + [_vp, _sz, _vp]),
     "ssd_prefix_state": (_i, [_vp] * 6 + [_i] * 8 + [_vp, _sz, _vp]),
     "ssd_block_step": (_i, [_vp] * 8 + [_i] * 7 + [_vp, _sz, _vp]),
+    "ssd_bidir_fwd_noalloc": (_i, [_vp] * 7 + [_i] * 8 + [_vp]),
     "ssd_get_device_status": (_i, [_vp, _vp]),
     "ssd_error_string": (ctypes.c_char_p, [_i]),
     "ssd_version": (_i, []),

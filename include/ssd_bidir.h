@@ -165,6 +165,31 @@ int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
                    int ngroups, int dtype,
                    void *workspace, size_t ws_bytes, void *stream);
 
+/* ssd_bidir_fwd for callers that cannot allocate device memory when they
+ * call the mixer: code running under CUDA graph capture in the global mode,
+ * where cudaMalloc is not allowed; plug-ins inside a runtime that has already
+ * reserved the GPU's memory for its own pool; loops where an allocation would
+ * synchronise the device. (The pages describe no such interface; it has no
+ * counterpart there.) Arguments as for ssd_bidir_fwd, without the workspace.
+ *  - bf16 I/O only (the fused tensor-core kernel); fp32 returns
+ *    SSD_ERR_UNSUPPORTED.
+ *  - Scratch is a fixed 32 MiB array (plus a 256-byte status header) inside
+ *    the library, held by every GPU that loads the library until the process
+ *    exits. Problems needing more, i.e. batch * nheads * ceil(seqlen / 128) *
+ *    dstate * 128 bytes > 32 MiB, return SSD_ERR_WORKSPACE and launch nothing.
+ *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *  - The first call on each device looks the array's device address up (with
+ *    that device current); make that first call before any stream capture.
+ *  - Every call shares the one array: calls that overlap on the GPU (other
+ *    streams, other host threads) race and give wrong results. Each call
+ *    clears the status header and overwrites the state area before reading it.
+ *  - Device-side wait timeouts are recorded in the array's header and are not
+ *    reported by this entry point. */
+int ssd_bidir_fwd_noalloc(const void *x, const void *dt, const float *A, const void *B,
+                          const void *C, const float *D, void *out,
+                          int batch, int seqlen, int nheads, int headdim, int dstate,
+                          int ngroups, int chunk, int dtype, void *stream);
+
 /* Synchronise `stream`, read and clear the workspace's status header.
  * Returns SSD_OK, SSD_ERR_TIMEOUT (a bounded device wait expired in a call
  * since the last check) or SSD_ERR_CUDA (the stream reported an error). */

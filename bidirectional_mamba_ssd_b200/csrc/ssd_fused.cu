@@ -18,13 +18,18 @@
 // Architecture; reverse = forward on the flipped sequence: "DiffMamba -
 // Checkpoints" model card, Model details.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: x tiles (2 slots), B/C tiles (3-slot ring),
+// Warp roles (320 threads):
+//   warp 0      TMA producer: x tiles (2 slots), B/C tiles (4-slot ring),
 //               reverse states (1 slot)
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 2..5  epilogue: thread r owns tile row r = 32 * (warp % 4) + lane
-//               (its TMEM lane): decay sums, diag(w) X, the masked matrix,
-//               state chains, outputs.
+//   warps 2..5  epilogue group A ("mask"): decay sums, diag(w) X, the masked
+//               matrix, written as bf16 into TMEM over the consumed C_f.B_f^T
+//               columns and used there as the A operand of (M_f + M_b) X
+//   warps 6..9  epilogue group B ("state/output"): the fp32 state chains, the
+//               reverse states' store, the output tile and its TMA store
+// In both groups thread r owns tile row r = 32 * (warp % 4) + lane (its TMEM
+// lane). Group A runs one tile ahead of group B; per-tile vectors pass from A
+// to B through two shared-memory buffers.
 // Phase-1 inputs (x, B') are loaded with an L2 evict-last hint and re-read in
 // phase 2 with evict-first, so the re-read mostly hits L2.
 //
@@ -45,8 +50,8 @@ using namespace sm100;
 constexpr int kTile = 128;
 constexpr int kP = 64;
 constexpr uint32_t kSlab = 16384;       // 128 rows x 128 bytes
-constexpr int kRing = 3;                // B/C ring slots (32 KB each)
-constexpr int kThreads = 192;
+constexpr int kRing = 4;                // B/C ring slots (32 KB each)
+constexpr int kThreads = 320;
 
 struct FusedParams {
     const __nv_bfloat16 *dt;   // (2, batch, L, H)
@@ -65,15 +70,25 @@ enum {
     B_X_EMPTY = B_X_FULL + 2,        // 2
     B_HB_FULL = B_X_EMPTY + 2,
     B_HB_EMPTY,
-    B_HB_WRITTEN,                    // epilogue -> producer: phase-1 states are in global memory
-    B_G_READY,                       // MMA -> epilogue
-    B_S_READY,
-    B_Y_READY,
-    B_XW_READY,                      // epilogue -> MMA
-    B_M_READY,
-    B_S_FREE,
-    B_Y_FREE,
-    B_COUNT
+    B_HB_WRITTEN,                    // group B -> producer: phase-1 states are in global memory
+    B_G_READY,                       // MMA -> group A
+    B_S_READY,                       // MMA -> groups A and B
+    B_Y_READY,                       // MMA -> group B
+    B_XW_READY,                      // group A -> MMA
+    B_M_READY,                       // group A -> MMA
+    B_S_FREE,                        // group B -> MMA
+    B_Y_FREE,                        // group B -> MMA
+    B_VEC_READY,                     // 2: group A -> group B, per vector buffer
+    B_VEC_FREE = B_VEC_READY + 2,    // 2: group B -> group A
+    B_COUNT = B_VEC_FREE + 2
+};
+
+// Per-tile vectors group A hands to group B (and reads itself).
+struct TileVec {
+    float af[kTile];    // A_f * prefix sums of dt_f
+    float ab[kTile];    // A_b * suffix sums of dt_b
+    float totf, totb;   // tile sums of dt_f, dt_b
+    float pad[2];
 };
 
 __device__ __forceinline__ uint64_t policy_evict_last() {
@@ -119,12 +134,13 @@ __device__ __forceinline__ void st_global_v4_hint(void *p, uint4 v, uint64_t pol
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
-// named barrier over the four epilogue warps
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// named barriers of the two epilogue groups (128 threads each)
+__device__ __forceinline__ void sync_a() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void sync_b() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 __device__ __forceinline__ float bf2f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
-// Inclusive scan over the 128 epilogue threads (row order), prefix or suffix.
+// Inclusive scan over the 128 rows of group A (row order), prefix or suffix.
 __device__ __forceinline__ float scan_rows(float v, bool suffix, int row, float *red) {
     const int lane = row & 31, wq = row >> 5;
     if (!suffix) {
@@ -142,15 +158,30 @@ __device__ __forceinline__ float scan_rows(float v, bool suffix, int row, float 
         }
         if (lane == 0) red[wq] = v;
     }
-    epi_sync();
+    sync_a();
     float add = 0.f;
     if (!suffix) {
         for (int k = 0; k < wq; ++k) add += red[k];
     } else {
         for (int k = wq + 1; k < 4; ++k) add += red[k];
     }
-    epi_sync();
+    sync_a();
     return v + add;
+}
+
+// Row `row` of the x tile at `xt` scaled by w into `dst` (row-local: the
+// swizzle permutes 16-byte chunks within a row only).
+__device__ __forceinline__ void scale_row(const uint8_t *xt, uint8_t *dst, int row, float w) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(xt + row * 128);
+    uint4 *d = reinterpret_cast<uint4 *>(dst + row * 128);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 v = src[c];
+        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) q[j] = pack_bf16x2(bf2f(q[j] & 0xffffu) * w, bf2f(q[j] >> 16) * w);
+        d[c] = v;
+    }
 }
 
 template <int N>
@@ -162,9 +193,8 @@ struct Smem {
     static constexpr uint32_t hb = ring + kRing * 2 * kSlab;
     static constexpr uint32_t hf = hb + kH;
     static constexpr uint32_t xw = hf + kH;             // diag(w) x
-    static constexpr uint32_t m = xw + kSlab;           // masked matrix, 2 slabs
-    static constexpr uint32_t small = m + 2 * kSlab;
-    static constexpr uint32_t bytes = small + 4096;     // barriers + per-tile vectors
+    static constexpr uint32_t small = xw + kSlab;
+    static constexpr uint32_t bytes = small + 6144;     // barriers + per-tile vectors (~4.4 KB)
 };
 
 template <int N>
@@ -180,11 +210,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
-    float *red = reinterpret_cast<float *>(g + S::small + 256);   // 8 floats
-    float *af = red + 8;             // A_f * prefix sums of dt_f over the tile
-    float *ab = af + kTile;          // A_b * suffix sums of dt_b over the tile
-    float *colf = ab + kTile;        // per-column factors of the forward mask
-    float *colb = colf + kTile;      // per-column factors of the reverse mask
+    float *red = reinterpret_cast<float *>(g + S::small + 256);   // 8 floats, group A scans
+    TileVec *vec = reinterpret_cast<TileVec *>(g + S::small + 288);  // 2 buffers
+    float *colf = reinterpret_cast<float *>(vec + 2);   // group A: per-column mask factors
+    float *colb = colf + kTile;
     float *dtf = colb + kTile;
     float *dtb = dtf + kTile;
 
@@ -193,15 +222,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < kRing; ++i) {
-            mbar_init(bar(B_RING_FULL + i), 1);
-            mbar_init(bar(B_RING_EMPTY + i), 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(bar(B_X_FULL + i), 1);
-            mbar_init(bar(B_X_EMPTY + i), 1);
-        }
-        for (int i = B_HB_FULL; i < B_COUNT; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -212,6 +233,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // TMEM columns: G_f [0,128) (the bf16 masked matrix M reuses [0,64)),
+    // G_b [128,256), Yo_f [256,320), Yo_b [320,384), Yd [384,448), S [448,512)
     const uint32_t tGf = tmem, tGb = tmem + 128, tYof = tmem + 256, tYob = tmem + 320,
                    tYd = tmem + 384, tS = tmem + 448;
     const int nt = p.nt;
@@ -221,7 +244,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
-            uint32_t kr = 0, kx = 0, kh = 0;  // loads issued into ring / x / hb
+            uint32_t kr = 0, kx = 0, kh = 0;
             uint32_t units_done = 0;
             auto ring_slot = [&](uint32_t k) -> uint32_t {
                 const uint32_t s = k % kRing;
@@ -235,8 +258,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             };
             for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++units_done) {
                 const int b = u / p.H, h = u % p.H, gg = h / hpg;
-                // phase 1: x and B' of every tile, right to left
-                for (int i = nt - 1; i >= 0; --i) {
+                for (int i = nt - 1; i >= 0; --i) {       // phase 1: x, B' right to left
                     const uint32_t xs = x_slot(kx++);
                     mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
                     tma_load_4d_hint(base + S::x0 + xs * kSlab, &tm_x, bar(B_X_FULL + xs), 0, h, i * kTile, b, keep);
@@ -246,10 +268,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         tma_load_5d_hint(base + S::ring + rs * 2 * kSlab + k * kSlab, &tm_b, bar(B_RING_FULL + rs),
                                          64 * k, gg, i * kTile, b, 1, keep);
                 }
-                // the reverse states of this unit must be in global memory
                 mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103);
-                // phase 2: x, C_f, B_f, C_b, B_b, H_b of every tile, left to right
-                for (int i = 0; i < nt; ++i) {
+                for (int i = 0; i < nt; ++i) {            // phase 2: x, C_f, B_f, C_b, B_b, H_b
                     const int t0 = i * kTile;
                     const uint32_t xs = x_slot(kx++);
                     mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
@@ -284,116 +304,211 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 mbar_wait(bar(B_RING_FULL + s), (k / kRing) & 1, abort_flag, p.status, 201);
                 return s;
             };
+            auto slot_addr = [&](uint32_t s) { return base + S::ring + s * 2 * kSlab; };
             for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-                // phase 1: S' = B'^T diag(w') X per tile
-                for (int i = nt - 1; i >= 0; --i) {
-                    const uint32_t xs_unused = kx++ & 1;
-                    (void)xs_unused;
+                for (int i = nt - 1; i >= 0; --i) {        // phase 1: S' = B'^T diag(w') X
+                    ++kx;
                     const uint32_t rs = wait_ring(kr++);
                     mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 202);
                     if (!first_s) mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 203);
                     first_s = false;
                     tc_fence_after();
-                    const uint32_t sB = base + S::ring + rs * 2 * kSlab;
+                    const uint32_t sB = slot_addr(rs);
                     for (int k = 0; k < kTile / 16; ++k)
                         mma_bf16_ss(tS, sdesc_sw128(sB + k * 2048, kSlab, 1024),
                                     sdesc_sw128(base + S::xw + k * 2048, kSlab, 1024), id_state, k > 0);
                     mma_commit(bar(B_S_READY));
                     mma_commit(bar(B_RING_EMPTY + rs));
                 }
-                // phase 2. Issue order keeps the 3-slot ring moving: each slot is
-                // released by an MMA that needs no later load of the same tile
-                // (C_f after C_f.H_f, B_f after S_f, B_b after G_b, C_b after C_b.H_b).
-                for (int i = 0; i < nt; ++i) {
+                for (int i = 0; i < nt; ++i) {             // phase 2
                     const uint32_t xs = kx++ & 1;
-                    mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 204);
-                    const uint32_t rCf = wait_ring(kr++);
-                    const uint32_t rBf = wait_ring(kr++);
-                    const uint32_t sCf = base + S::ring + rCf * 2 * kSlab, sBf = base + S::ring + rBf * 2 * kSlab;
+                    const uint32_t rCf = wait_ring(kr++), rBf = wait_ring(kr++);
+                    const uint32_t rCb = wait_ring(kr++), rBb = wait_ring(kr++);
+                    const uint32_t sCf = slot_addr(rCf), sBf = slot_addr(rBf);
+                    const uint32_t sCb = slot_addr(rCb), sBb = slot_addr(rBb);
                     tc_fence_after();
-                    // 1. G_f = C_f B_f^T
+                    // G_f = C_f B_f^T, G_b = C_b B_b^T (the previous tile's M, kept in
+                    // G_f's columns, was read by the Yd MMA issued before these)
                     for (int k = 0; k < N / 16; ++k) {
                         const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
                         mma_bf16_ss(tGf, sdesc_sw128(sCf + ko, 0, 1024), sdesc_sw128(sBf + ko, 0, 1024), id_g, k > 0);
                     }
-                    // 2. Yo_f = C_f H_f: previous outputs read, H_f of this tile written
-                    if (!first_y) mbar_wait(bar(B_Y_FREE), n_yfree++ & 1, abort_flag, p.status, 205);
-                    first_y = false;
-                    mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 206);
-                    tc_fence_after();
-                    for (int k = 0; k < N / 16; ++k) {
-                        const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
-                        mma_bf16_ss(tYof, sdesc_sw128(sCf + ko, 0, 1024),
-                                    sdesc_sw128(base + S::hf + k * 2048, kSlab, 1024), id_o, k > 0);
-                    }
-                    mma_commit(bar(B_RING_EMPTY + rCf));
-                    // 3. S_f = B_f^T diag(w_f) X
-                    mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 208);
-                    tc_fence_after();
-                    for (int k = 0; k < kTile / 16; ++k)
-                        mma_bf16_ss(tS, sdesc_sw128(sBf + k * 2048, kSlab, 1024),
-                                    sdesc_sw128(base + S::xw + k * 2048, kSlab, 1024), id_state, k > 0);
-                    mma_commit(bar(B_S_READY));
-                    mma_commit(bar(B_RING_EMPTY + rBf));
-                    // 4. G_b = C_b B_b^T
-                    const uint32_t rCb = wait_ring(kr++);
-                    const uint32_t rBb = wait_ring(kr++);
-                    const uint32_t sCb = base + S::ring + rCb * 2 * kSlab, sBb = base + S::ring + rBb * 2 * kSlab;
-                    tc_fence_after();
                     for (int k = 0; k < N / 16; ++k) {
                         const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
                         mma_bf16_ss(tGb, sdesc_sw128(sCb + ko, 0, 1024), sdesc_sw128(sBb + ko, 0, 1024), id_g, k > 0);
                     }
                     mma_commit(bar(B_G_READY));
                     mma_commit(bar(B_RING_EMPTY + rBb));
-                    // 5. Yo_b = C_b H_b
+                    // the previous tile's outputs and state are consumed; H_f is this tile's
+                    if (!first_y) mbar_wait(bar(B_Y_FREE), n_yfree++ & 1, abort_flag, p.status, 205);
+                    first_y = false;
+                    mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 206);
+                    tc_fence_after();
+                    for (int k = 0; k < N / 16; ++k) {      // Yo_f = C_f H_f
+                        const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
+                        mma_bf16_ss(tYof, sdesc_sw128(sCf + ko, 0, 1024),
+                                    sdesc_sw128(base + S::hf + k * 2048, kSlab, 1024), id_o, k > 0);
+                    }
+                    mma_commit(bar(B_RING_EMPTY + rCf));
                     mbar_wait(bar(B_HB_FULL), kh++ & 1, abort_flag, p.status, 207);
                     tc_fence_after();
-                    for (int k = 0; k < N / 16; ++k) {
+                    for (int k = 0; k < N / 16; ++k) {      // Yo_b = C_b H_b
                         const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
                         mma_bf16_ss(tYob, sdesc_sw128(sCb + ko, 0, 1024),
                                     sdesc_sw128(base + S::hb + k * 2048, kSlab, 1024), id_o, k > 0);
                     }
                     mma_commit(bar(B_RING_EMPTY + rCb));
                     mma_commit(bar(B_HB_EMPTY));
-                    // 6. Yd = M X
+                    mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 208);
+                    tc_fence_after();
+                    for (int k = 0; k < kTile / 16; ++k)    // S_f = B_f^T diag(w_f) X
+                        mma_bf16_ss(tS, sdesc_sw128(sBf + k * 2048, kSlab, 1024),
+                                    sdesc_sw128(base + S::xw + k * 2048, kSlab, 1024), id_state, k > 0);
+                    mma_commit(bar(B_S_READY));
+                    mma_commit(bar(B_RING_EMPTY + rBf));
                     mbar_wait(bar(B_M_READY), n_m++ & 1, abort_flag, p.status, 209);
+                    mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 204);
                     tc_fence_after();
                     const uint32_t sX = base + S::x0 + xs * kSlab;
-                    for (int k = 0; k < kTile / 16; ++k)
-                        mma_bf16_ss(tYd, sdesc_sw128(base + S::m + (k >> 2) * kSlab + (k & 3) * 32, 0, 1024),
-                                    sdesc_sw128(sX + k * 2048, kSlab, 1024), id_o, k > 0);
+                    for (int k = 0; k < kTile / 16; ++k)    // Yd = M X, M from TMEM
+                        mma_bf16_ts(tYd, tGf + k * 8, sdesc_sw128(sX + k * 2048, kSlab, 1024), id_o, k > 0);
                     mma_commit(bar(B_Y_READY));
                 }
             }
         }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ group A
+        const int row = ((warp & 3) << 5) | lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+        uint32_t kx = 0, n_g = 0, nvec = 0, n_s = 0;   // n_s: S MMAs issued before this step
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+            const int b = u / p.H, h = u % p.H;
+            const float Af = p.A[h], Ab = p.A[p.H + h];
+            const size_t dt_dir = (size_t)p.batch * p.L * p.H;
+            // phase 1: reverse tile sums and diag(w') X
+            for (int i = nt - 1; i >= 0; --i) {
+                const int t = i * kTile + row;
+                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
+                const float cs = scan_rows(vb, true, row, red);
+                const uint32_t vb_i = nvec & 1;
+                if (nvec >= 2) mbar_wait(bar(B_VEC_FREE + vb_i), ((nvec >> 1) - 1) & 1, abort_flag, p.status, 301);
+                TileVec &V = vec[vb_i];
+                if (row == 0) V.totb = cs;
+                sync_a();
+                const float total = V.totb;
+                if (row == 0) mbar_arrive(bar(B_VEC_READY + vb_i));
+                ++nvec;
+                const float w = __expf(Ab * (total - cs)) * vb;
+                if (n_s > 0) mbar_wait(bar(B_S_READY), (n_s - 1) & 1, abort_flag, p.status, 302);
+                const uint32_t xs = kx++ & 1;
+                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 303);
+                scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, w);
+                fence_proxy_async_smem();
+                sync_a();
+                if (row == 0) {
+                    mbar_arrive(bar(B_XW_READY));
+                    mbar_arrive(bar(B_X_EMPTY + xs));
+                }
+                ++n_s;
+            }
+            // phase 2: decay sums, diag(w_f) X, masked matrix
+            for (int i = 0; i < nt; ++i) {
+                const int t = i * kTile + row;
+                const float vf = t < p.L ? __bfloat162float(p.dt[((size_t)b * p.L + t) * p.H + h]) : 0.f;
+                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
+                const float csf = scan_rows(vf, false, row, red);
+                const float csb = scan_rows(vb, true, row, red);
+                const float my_af = Af * csf, my_ab = Ab * csb;
+                const uint32_t vb_i = nvec & 1;
+                if (nvec >= 2) mbar_wait(bar(B_VEC_FREE + vb_i), ((nvec >> 1) - 1) & 1, abort_flag, p.status, 311);
+                TileVec &V = vec[vb_i];
+                V.af[row] = my_af;
+                V.ab[row] = my_ab;
+                if (row == kTile - 1) V.totf = csf;
+                if (row == 0) V.totb = csb;
+                dtf[row] = vf;
+                dtb[row] = vb;
+                sync_a();
+                if (row == 0) mbar_arrive(bar(B_VEC_READY + vb_i));
+                ++nvec;
+                // per-column factors: forward relative to the end of the row's
+                // 32-block, reverse relative to its start
+                colf[row] = __expf(V.af[row | 31] - my_af) * vf;
+                colb[row] = __expf(V.ab[row & ~31] - my_ab) * vb;
+                const float wf = __expf(Af * (V.totf - csf)) * vf;
+                if (n_s > 0) mbar_wait(bar(B_S_READY), (n_s - 1) & 1, abort_flag, p.status, 312);
+                const uint32_t xs = kx++ & 1;
+                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 313);
+                scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, wf);
+                fence_proxy_async_smem();
+                sync_a();
+                if (row == 0) mbar_arrive(bar(B_XW_READY));
+                ++n_s;
+
+                // masked matrix M = M_f + M_b, bf16 pairs into TMEM columns [0, 64)
+                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 314);
+                tc_fence_after();
+#pragma unroll 1
+                for (int J = 0; J < 4; ++J) {
+                    uint32_t gf[32], gb[32];
+                    tmem_ld32(tGf + lane_off + J * 32, gf);
+                    tmem_ld32(tGb + lane_off + J * 32, gb);
+                    tmem_wait_ld();
+                    const int s0 = J * 32;
+                    const bool f_full = row >= s0 + 31, f_none = row < s0;
+                    const bool b_full = row <= s0, b_none = row > s0 + 31;
+                    const float rf = f_full ? __expf(my_af - V.af[s0 + 31]) : 0.f;
+                    const float rb = b_full ? __expf(my_ab - V.ab[s0]) : 0.f;
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int q = 0; q < 32; q += 2) {
+                        float mv[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int s = s0 + q + e;
+                            float mf, mb;
+                            if (f_full) mf = __uint_as_float(gf[q + e]) * rf * colf[s];
+                            else if (f_none || s > row) mf = 0.f;
+                            else mf = __uint_as_float(gf[q + e]) * __expf(my_af - V.af[s]) * dtf[s];
+                            if (b_full) mb = __uint_as_float(gb[q + e]) * rb * colb[s];
+                            else if (b_none || s < row) mb = 0.f;
+                            else mb = __uint_as_float(gb[q + e]) * __expf(my_ab - V.ab[s]) * dtb[s];
+                            mv[e] = mf + mb;
+                        }
+                        packed[q / 2] = pack_bf16x2(mv[0], mv[1]);
+                    }
+                    tmem_st16(tGf + lane_off + J * 16, packed);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                sync_a();
+                if (row == 0) mbar_arrive(bar(B_M_READY));
+            }
+        }
     } else {
-        // ------------------------------------------------------------ epilogue
-        const int row = ((warp & 3) << 5) | lane;          // TMEM lane == tile row
+        // ------------------------------------------------------------ group B
+        const int row = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
         const uint64_t keep = policy_evict_last();
-        uint32_t kx = 0, n_g = 0, n_s = 0, n_y = 0;
+        uint32_t kx = 0, n_s = 0, n_y = 0, nvec = 0;
         uint32_t units_done = 0;
-        uint8_t *xw_row = g + S::xw + row * 128;
         float hreg[kP];
-
-        // H_f operand starts at zero for every unit; written before the first
-        // S_FREE arrival, so the first C_f.H_f of each unit reads zeros.
         for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++units_done) {
             const int b = u / p.H, h = u % p.H;
             const float Af = p.A[h], Ab = p.A[p.H + h];
             const float dsum = p.D[h] + p.D[p.H + h];
-            const size_t dt_dir = (size_t)p.batch * p.L * p.H;
-
-            // ---------------- phase 1: reverse states, right to left
+            // phase 1: reverse state chain, right to left
 #pragma unroll
             for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
             for (int i = nt - 1; i >= 0; --i) {
-                const int t = i * kTile + row;
-                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
-                const float cs = scan_rows(vb, true, row, red);      // suffix sums
-                if (row == 0) red[4] = cs;                            // tile total
-                // state entering tile i from the right (before this tile's update)
+                const uint32_t vb_i = nvec & 1;
+                mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 401);
+                const float totb = vec[vb_i].totb;
+                sync_b();
+                if (row == 0) mbar_arrive(bar(B_VEC_FREE + vb_i));
+                ++nvec;
+                ++kx;
+                // state entering tile i from the right
                 if (row < N) {
                     __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
 #pragma unroll
@@ -405,157 +520,56 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         st_global_v4_hint(dst + 8 * c, v, keep);
                     }
                 }
-                epi_sync();
-                const float total = red[4];
-                const float w = __expf(Ab * (total - cs)) * vb;      // exp(A' sum_{r<s} dt') dt'_s
-                // diag(w') X into the X' buffer (row-local scaling)
-                const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 301);
-                {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(g + S::x0 + xs * kSlab + row * 128);
-                    uint4 *dst = reinterpret_cast<uint4 *>(xw_row);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 v = src[c];
-                        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) q[j] = pack_bf16x2(bf2f(q[j] & 0xffffu) * w, bf2f(q[j] >> 16) * w);
-                        dst[c] = v;
-                    }
-                }
-                fence_proxy_async_smem();
-                epi_sync();
-                if (row == 0) {
-                    mbar_arrive(bar(B_XW_READY));
-                    mbar_arrive(bar(B_X_EMPTY + xs));
-                }
-                // S' ready: chain the reverse state
-                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 302);
+                const float gdec = __expf(Ab * totb);
+                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 402);
                 tc_fence_after();
-                const float gdec = __expf(Ab * total);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t v[32];
                     tmem_ld32(tS + lane_off + half * 32, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
+                    for (int j = 0; j < 32; ++j)
+                        hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
                 }
-                if (i == 0) {
-                    // start of phase 2 for this unit: H_f operand = 0
+                if (i == 0 && row < N) {       // phase 2 starts from H_f = 0
                     uint4 *hf = reinterpret_cast<uint4 *>(g + S::hf + row * 128);
-                    if (row < N) {
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) hf[c] = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
+                    for (int c = 0; c < 8; ++c) hf[c] = make_uint4(0, 0, 0, 0);
                 }
+                fence_proxy_async_smem();
                 tc_fence_before();
-                epi_sync();
+                sync_b();
                 if (row == 0) mbar_arrive(bar(B_S_FREE));
             }
-            // all reverse states of this unit are written: hand them to the TMA proxy
             fence_proxy_async_global();
-            epi_sync();
+            sync_b();
             if (row == 0) mbar_arrive(bar(B_HB_WRITTEN));
 
-            // ---------------- phase 2: outputs, left to right
+            // phase 2: forward state chain and outputs, left to right
 #pragma unroll
-            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;      // forward state
+            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
             for (int i = 0; i < nt; ++i) {
-                const int t0 = i * kTile, t = t0 + row;
-                const float vf = t < p.L ? __bfloat162float(p.dt[((size_t)b * p.L + t) * p.H + h]) : 0.f;
-                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
-                const float csf = scan_rows(vf, false, row, red);
-                const float csb = scan_rows(vb, true, row, red);
-                const float my_af = Af * csf, my_ab = Ab * csb;
-                af[row] = my_af;
-                ab[row] = my_ab;
-                dtf[row] = vf;
-                dtb[row] = vb;
-                if (row == kTile - 1) red[5] = csf;   // forward tile total
-                epi_sync();
-                // per-column mask factors: forward relative to the end of the
-                // row's 32-block, reverse relative to its start
-                colf[row] = __expf(af[row | 31] - my_af) * vf;
-                colb[row] = __expf(ab[row & ~31] - my_ab) * vb;
-                const float totf = red[5];
-                const float wf = __expf(Af * (totf - csf)) * vf;     // exp(A sum_{r>s} dt) dt_s
-                // diag(w_f) X
-                const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 311);
-                uint8_t *xrow = g + S::x0 + xs * kSlab + row * 128;
-                {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(xrow);
-                    uint4 *dst = reinterpret_cast<uint4 *>(xw_row);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 v = src[c];
-                        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) q[j] = pack_bf16x2(bf2f(q[j] & 0xffffu) * wf, bf2f(q[j] >> 16) * wf);
-                        dst[c] = v;
-                    }
-                }
-                fence_proxy_async_smem();
-                epi_sync();
-                if (row == 0) mbar_arrive(bar(B_XW_READY));
-
-                // masked matrix M = M_f + M_b (bf16, K-major) from G_f, G_b
-                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 312);
-                tc_fence_after();
-                uint8_t *mrow = g + S::m;
-#pragma unroll 1
-                for (int J = 0; J < 4; ++J) {
-                    uint32_t gf[32], gb[32];
-                    tmem_ld32(tGf + lane_off + J * 32, gf);
-                    tmem_ld32(tGb + lane_off + J * 32, gb);
-                    tmem_wait_ld();
-                    const int s0 = J * 32;
-                    const bool f_full = row >= s0 + 31, f_none = row < s0;
-                    const bool b_full = row <= s0, b_none = row > s0 + 31;
-                    const float rf = f_full ? __expf(my_af - af[s0 + 31]) : 0.f;
-                    const float rb = b_full ? __expf(my_ab - ab[s0]) : 0.f;
-                    uint32_t packed[16];
-#pragma unroll
-                    for (int q = 0; q < 32; q += 2) {
-                        float mv[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int s = s0 + q + e;
-                            float mf, mb;
-                            if (f_full) mf = __uint_as_float(gf[q + e]) * rf * colf[s];
-                            else if (f_none || s > row) mf = 0.f;
-                            else mf = __uint_as_float(gf[q + e]) * __expf(my_af - af[s]) * dtf[s];
-                            if (b_full) mb = __uint_as_float(gb[q + e]) * rb * colb[s];
-                            else if (b_none || s < row) mb = 0.f;
-                            else mb = __uint_as_float(gb[q + e]) * __expf(my_ab - ab[s]) * dtb[s];
-                            mv[e] = mf + mb;
-                        }
-                        packed[q / 2] = pack_bf16x2(mv[0], mv[1]);
-                    }
-                    uint8_t *slab = mrow + (J >> 1) * kSlab;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4 *>(slab + sw128_offset(row, (J & 1) * 4 + c)) =
-                            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                epi_sync();
-                if (row == 0) mbar_arrive(bar(B_M_READY));
-
-                // forward state chain: H_f <- exp(A sum dt) H_f + S_f; bf16 copy for C_f.H_f
-                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 313);
-                tc_fence_after();
+                const int t0 = i * kTile;
+                const uint32_t vb_i = nvec & 1;
+                mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 411);
+                const float my_af = vec[vb_i].af[row], my_ab = vec[vb_i].ab[row];
+                const float totf = vec[vb_i].totf;
+                sync_b();
+                if (row == 0) mbar_arrive(bar(B_VEC_FREE + vb_i));
+                ++nvec;
+                // forward chain: H_f <- exp(A sum dt) H_f + S_f; bf16 copy for C_f.H_f
                 const float gdec = __expf(Af * totf);
+                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 412);
+                tc_fence_after();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t v[32];
                     tmem_ld32(tS + lane_off + half * 32, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
+                    for (int j = 0; j < 32; ++j)
+                        hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
                 }
                 if (row < N) {
                     uint8_t *hrow = g + S::hf;
@@ -569,13 +583,15 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                epi_sync();
+                sync_b();
                 if (row == 0) mbar_arrive(bar(B_S_FREE));
 
-                // output tile, written over the x slot, then one TMA store
-                mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 314);
+                // output tile over the x slot, then one TMA store
+                const uint32_t xs = kx++ & 1;
+                mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 413);
                 tc_fence_after();
                 const float ef = __expf(my_af), eb = __expf(my_ab);
+                uint8_t *xt = g + S::x0 + xs * kSlab;
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     uint32_t yd[32], yf[32], yb[32];
@@ -585,7 +601,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        uint4 *q = reinterpret_cast<uint4 *>(xrow - row * 128 + sw128_offset(row, half * 4 + c));
+                        uint4 *q = reinterpret_cast<uint4 *>(xt + sw128_offset(row, half * 4 + c));
                         uint4 xv = *q;
                         uint32_t *xu = reinterpret_cast<uint32_t *>(&xv);
 #pragma unroll
@@ -602,15 +618,14 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                epi_sync();
+                sync_b();
                 if (row == 0) {
                     mbar_arrive(bar(B_Y_FREE));
                     if (!*abort_flag) {
                         tma_store_4d(&tm_out, base + S::x0 + xs * kSlab, 0, h, t0, b);
                         tma_store_commit();
                     }
-                    // the store must have read the slot before the producer refills it
-                    tma_store_wait_read();
+                    tma_store_wait_read();      // the store has read the slot
                     mbar_arrive(bar(B_X_EMPTY + xs));
                 }
             }

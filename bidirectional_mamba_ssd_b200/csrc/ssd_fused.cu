@@ -40,6 +40,7 @@
 
 #include "sm100.cuh"
 #include "ssd_kernels.h"
+#include "ssd_mask.cuh"
 #include "ssd_tmap.h"
 
 namespace ssd {
@@ -167,21 +168,6 @@ __device__ __forceinline__ float scan_rows(float v, bool suffix, int row, float 
     }
     sync_a();
     return v + add;
-}
-
-// Row `row` of the x tile at `xt` scaled by w into `dst` (row-local: the
-// swizzle permutes 16-byte chunks within a row only).
-__device__ __forceinline__ void scale_row(const uint8_t *xt, uint8_t *dst, int row, float w) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(xt + row * 128);
-    uint4 *d = reinterpret_cast<uint4 *>(dst + row * 128);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint4 v = src[c];
-        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) q[j] = pack_bf16x2(bf2f(q[j] & 0xffffu) * w, bf2f(q[j] >> 16) * w);
-        d[c] = v;
-    }
 }
 
 template <int N>
@@ -431,10 +417,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 sync_a();
                 if (row == 0) mbar_arrive(bar(B_VEC_READY + vb_i));
                 ++nvec;
-                // per-column factors: forward relative to the end of the row's
-                // 32-block, reverse relative to its start
-                colf[row] = __expf(V.af[row | 31] - my_af) * vf;
-                colb[row] = __expf(V.ab[row & ~31] - my_ab) * vb;
+                mask_column_factors(row, my_af, my_ab, vf, vb, V.af, V.ab, colf, colb);
                 const float wf = __expf(Af * (V.totf - csf)) * vf;
                 if (n_s > 0) mbar_wait(bar(B_S_READY), (n_s - 1) & 1, abort_flag, p.status, 312);
                 const uint32_t xs = kx++ & 1;
@@ -448,35 +431,14 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 // masked matrix M = M_f + M_b, bf16 pairs into TMEM columns [0, 64)
                 mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 314);
                 tc_fence_after();
+                const MaskVectors mv{V.af, V.ab, dtf, dtb, colf, colb};
 #pragma unroll 1
                 for (int J = 0; J < 4; ++J) {
-                    uint32_t gf[32], gb[32];
+                    uint32_t gf[32], gb[32], packed[16];
                     tmem_ld32(tGf + lane_off + J * 32, gf);
                     tmem_ld32(tGb + lane_off + J * 32, gb);
                     tmem_wait_ld();
-                    const int s0 = J * 32;
-                    const bool f_full = row >= s0 + 31, f_none = row < s0;
-                    const bool b_full = row <= s0, b_none = row > s0 + 31;
-                    const float rf = f_full ? __expf(my_af - V.af[s0 + 31]) : 0.f;
-                    const float rb = b_full ? __expf(my_ab - V.ab[s0]) : 0.f;
-                    uint32_t packed[16];
-#pragma unroll
-                    for (int q = 0; q < 32; q += 2) {
-                        float mv[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int s = s0 + q + e;
-                            float mf, mb;
-                            if (f_full) mf = __uint_as_float(gf[q + e]) * rf * colf[s];
-                            else if (f_none || s > row) mf = 0.f;
-                            else mf = __uint_as_float(gf[q + e]) * __expf(my_af - V.af[s]) * dtf[s];
-                            if (b_full) mb = __uint_as_float(gb[q + e]) * rb * colb[s];
-                            else if (b_none || s < row) mb = 0.f;
-                            else mb = __uint_as_float(gb[q + e]) * __expf(my_ab - V.ab[s]) * dtb[s];
-                            mv[e] = mf + mb;
-                        }
-                        packed[q / 2] = pack_bf16x2(mv[0], mv[1]);
-                    }
+                    mask_block(J, row, my_af, my_ab, gf, gb, mv, packed);
                     tmem_st16(tGf + lane_off + J * 16, packed);
                 }
                 tmem_wait_st();

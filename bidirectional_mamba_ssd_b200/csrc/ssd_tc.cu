@@ -34,6 +34,7 @@
 
 #include "sm100.cuh"
 #include "ssd_kernels.h"
+#include "ssd_mask.cuh"
 #include "ssd_tmap.h"
 
 namespace ssd {
@@ -169,7 +170,8 @@ __global__ void __launch_bounds__(128) tc_state_kernel(const __grid_constant__ C
         uint4 *dst = reinterpret_cast<uint4 *>(gbase + (sW - base) + tid * 128);
         uint4 *dstl = reinterpret_cast<uint4 *>(gbase + (sWl - base) + tid * 128);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int k = 0; k < 8; ++k) {
+            const int c = (k + tid) & 7;   // rows start at different chunks: no bank conflicts
             uint4 v = src[c], lo;
             uint32_t *u = reinterpret_cast<uint32_t *>(&v);
             uint32_t *ul = reinterpret_cast<uint32_t *>(&lo);
@@ -297,6 +299,8 @@ __global__ void __launch_bounds__(128) tc_out_kernel(const __grid_constant__ CUt
     float *ab = af + kTile;         // A_b * suffix sum of dt_b
     float *dtf = ab + kTile;
     float *dtb = dtf + kTile;
+    float *colf = dtb + kTile;      // per-column mask factors
+    float *colb = colf + kTile;
 
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / (p.H / p.G);
@@ -363,6 +367,7 @@ __global__ void __launch_bounds__(128) tc_out_kernel(const __grid_constant__ CUt
     dtb[tid] = vb;
     __syncthreads();
     const float my_af = af[tid], my_ab = ab[tid];
+    mask_column_factors(tid, my_af, my_ab, vf, vb, af, ab, colf, colb);
 
     mbar_wait(bar_load, 0, abort_flag, p.status, 11);
     __syncthreads();
@@ -389,29 +394,18 @@ __global__ void __launch_bounds__(128) tc_out_kernel(const __grid_constant__ CUt
     mbar_wait(bar_mma1, 0, abort_flag, p.status, 12);
     tc_fence_after();
 
-    // masked matrix M[t][s] = fwd (s <= t) + rev (s >= t), bf16, K-major into sM
+    // masked matrix M = M_f + M_b, bf16, K-major into sM (column factors ready:
+    // the load wait above is preceded by a block barrier)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     uint8_t *mrow = gbase + (sM - base);
+    const MaskVectors mv{af, ab, dtf, dtb, colf, colb};
 #pragma unroll 1
     for (int j = 0; j < 4; ++j) {
-        uint32_t gf[32], gb[32];
+        uint32_t gf[32], gb[32], packed[16];
         tmem_ld32(tG_f + lane_base + j * 32, gf);
         tmem_ld32(tG_b + lane_base + j * 32, gb);
         tmem_wait_ld();
-        uint32_t packed[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-            float m2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int s = j * 32 + i + u;
-                float m = 0.f;
-                if (s <= tid) m += __uint_as_float(gf[i + u]) * __expf(my_af - af[s]) * dtf[s];
-                if (s >= tid) m += __uint_as_float(gb[i + u]) * __expf(my_ab - ab[s]) * dtb[s];
-                m2[u] = m;
-            }
-            packed[i / 2] = pack_bf16x2(m2[0], m2[1]);
-        }
+        mask_block(j, tid, my_af, my_ab, gf, gb, mv, packed);
         // columns j*32 .. j*32+31 = slab j/2, chunks (j%2)*4 .. +3
         uint8_t *slab = mrow + (j >> 1) * kSlab;
 #pragma unroll
@@ -500,7 +494,7 @@ ChunkedLayout chunked_layout(int batch, int L, int H, int N, int ndir) {
 
 constexpr size_t state_smem(int N) { return (N / 64 + 3) * kSlab + 1024 + 256; }
 constexpr size_t out_smem(int N) {
-    return kSlab + 4 * (N / 64) * kSlab + 2 * (size_t)N * 128 + 2 * kSlab + 1024 + 64 + 32 + 4 * kTile * 4 + 64;
+    return kSlab + 4 * (N / 64) * kSlab + 2 * (size_t)N * 128 + 2 * kSlab + 1024 + 64 + 32 + 6 * kTile * 4 + 64;
 }
 
 template <int N>

@@ -41,6 +41,28 @@ LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1}
 KERNEL_SOURCE = {"simt": "ssd_simt.cu", "chunked": "ssd_tc.cu", "fused": "ssd_tc.cu"}
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch: independent problems, no shared data."""
+    return 1000 + rank
+
+
+def job_time_ms(local_ms: float, world: int, device=None) -> float:
+    """Device time of the whole job: the max over ranks (all-reduce MAX of one
+    float; the only collective, outside the timed region)."""
+    if world <= 1:
+        return local_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, job_ms: float) -> float:
+    """Whole-job tokens/s: the units all ranks processed over the max-over-ranks time."""
+    return tokens_per_rank_step * world * steps / (job_ms / 1e3)
+
+
 def algorithmic_bytes(w) -> int:
     """Unavoidable HBM bytes of one bidirectional call: x read once, dt/B/C of
     both directions read once, out written once, A and D (fp32)."""
@@ -186,6 +208,88 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def bench_blockstep(args, w, dev):
+    """Block diffusion on one GPU: prefill of the cached forward state over the
+    prefix, then per block `steps` denoising steps (each a block step on fresh
+    block inputs, reading the cached state) and the commit of the block into
+    the state. One bench step = one block: all its denoising steps plus the
+    commit, replayed as one CUDA graph. value = block tokens x denoising steps
+    per second."""
+    import torch
+    import bidirectional_mamba_ssd_b200 as ssd
+    import ssd_inputs as si
+    data = si.blockstep_inputs(w.batch, w.seqlen, w.block, w.steps, w.nheads, w.headdim, w.dstate,
+                               w.ngroups, w.dtype, seed=0, device=dev)
+    ws_pre, ws_step, ws_commit = ssd.Workspace(dev), ssd.Workspace(dev), ssd.Workspace(dev)
+    state = torch.empty(w.batch, w.nheads, w.headdim, w.dstate, dtype=torch.float32, device=dev)
+    # prefill timing (outside the graph)
+    for _ in range(2):
+        ssd.ssd_prefix_state(data["x_pre"], data["dt_pre"], data["A"][0], data["B_pre"], out=state,
+                             chunk=w.chunk, workspace=ws_pre)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    ssd.ssd_prefix_state(data["x_pre"], data["dt_pre"], data["A"][0], data["B_pre"], out=state,
+                         chunk=w.chunk, workspace=ws_pre)
+    e1.record()
+    torch.cuda.synchronize()
+    prefill_ms = e0.elapsed_time(e1)
+    outs = [torch.empty_like(st["x"]) for st in data["steps"]]
+    commit_state = state.clone()
+
+    def block():
+        for k, st in enumerate(data["steps"]):
+            ssd.ssd_block_step(st["x"], st["dt"], data["A"], st["B"], st["C"], data["D"], state,
+                               out=outs[k], workspace=ws_step)
+        last = data["steps"][-1]
+        ssd.ssd_prefix_state(last["x"], last["dt"][0], data["A"][0], last["B"][0], init=state,
+                             out=commit_state, chunk=w.chunk, workspace=ws_commit)
+
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        block()   # sizes the workspaces outside the capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            block()
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        t0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        t1.record()
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    tok = w.batch * w.block * w.steps
+    io = 2
+    step_bytes = (io * (w.batch * w.block * w.nheads * w.headdim * 2 + 2 * w.batch * w.block * w.nheads
+                        + 4 * w.batch * w.block * w.ngroups * w.dstate)
+                  + 4 * w.batch * w.nheads * w.headdim * w.dstate)
+    prefill_bytes = (io * (w.batch * w.seqlen * (w.nheads * w.headdim + w.nheads + w.ngroups * w.dstate))
+                     + 4 * w.batch * w.nheads * w.headdim * w.dstate)
+    peaks = measured_peaks()
+    line = {"metric": "block-diffusion denoising tokens/s (block x steps), cached prefix state",
+            "value": round(tok / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "prefix": w.seqlen, "block": w.block,
+                       "denoising_steps": w.steps, "nheads": w.nheads, "headdim": w.headdim,
+                       "dstate": w.dstate, "ngroups": w.ngroups, "graph": "one CUDA graph per block"},
+            "per_denoising_step_us": round(1e3 * ms / (w.steps + 1), 3),
+            "algorithmic_bytes_per_denoising_step": step_bytes,
+            "prefill": {"ms": round(prefill_ms, 4), "tokens_per_s": round(w.batch * w.seqlen / (prefill_ms / 1e3), 1),
+                        "algorithmic_bytes": prefill_bytes,
+                        "hbm_frac": round(prefill_bytes / (prefill_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "gpu_launches": args.steps * (3 * w.steps + 2),
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -218,13 +322,16 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     import bidirectional_mamba_ssd_b200 as ssd
+    if w.block:
+        bench_blockstep(args, w, dev)
+        return
     path = PATH_IDS[args.path]
     if path == 0:
         path = ssd.lib.ssd_select_path(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
                                        w.chunk, 1 if w.dtype == "bf16" else 0)
     path_name = {v: k for k, v in PATH_IDS.items()}[path]
 
-    inp = si.workload_inputs(w, seed=1000 + rank, device=dev)
+    inp = si.workload_inputs(w, seed=rank_seed(rank), device=dev)
     names = ("x", "dt", "A", "B", "C", "D")
     out = torch.empty_like(inp["x"])
     ws = ssd.Workspace(dev)
@@ -250,15 +357,12 @@ def main():
             step()
         ev1.record(stream)
         torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
+    ms = job_time_ms(ev0.elapsed_time(ev1), world, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     ms_step = ms / args.steps
     tokens_job = w.tokens * world
-    value = tokens_job * args.steps / (ms / 1e3)
+    value = job_throughput(w.tokens, args.steps, world, ms)
 
     # end to end through the public API: pinned host inputs -> device -> mixer -> host output
     e2e = None
@@ -287,12 +391,8 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": tokens_job * k / (ems / 1e3), "unit": "tokens/s",
+        ems = job_time_ms(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_throughput(w.tokens, k, world, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if world > 1:

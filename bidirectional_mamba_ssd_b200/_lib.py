@@ -32,6 +32,7 @@ SIGNATURES = {
     "ssd_block_step": (_i, [_vp] * 8 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_bidir_fwd_noalloc": (_i, [_vp] * 7 + [_i] * 8 + [_vp]),
     "ssd_get_device_status": (_i, [_vp, _vp]),
+    "ssd_selftest_wait_timeout": (_i, [_vp, _sz, _i, _vp]),
     "ssd_error_string": (ctypes.c_char_p, [_i]),
     "ssd_version": (_i, []),
 }

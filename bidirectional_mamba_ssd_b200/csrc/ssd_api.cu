@@ -115,6 +115,9 @@ size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdi
         } else if (op == SSD_OP_PREFIX_STATE) {
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 1);
             scratch = scratch > c ? scratch : c;
+        } else if (op == SSD_OP_BLOCK_STEP) {
+            size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 2);
+            scratch = scratch > c ? scratch : c;
         }
     }
     return ssd::kStatusBytes + round256(scratch);
@@ -204,6 +207,18 @@ int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
         return SSD_ERR_INVALID_ARG;
     if (prefix_state && !aligned16(prefix_state)) return SSD_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == SSD_BF16) {
+        // the bidirectional chunked tensor-core path over the block, with the
+        // forward scan starting from the cached state and the reverse from zero
+        TcArgs t{};
+        t.x = x; t.dt = dt; t.A = A; t.B = B; t.C = C; t.D = D; t.out = out;
+        t.init = prefix_state;
+        t.workspace = workspace; t.ws_bytes = ws_bytes;
+        t.batch = batch; t.L = blk_len; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+        cudaError_t e = ssd::launch_tc_chunked(t, s);
+        if (e != cudaErrorNotSupported) return to_status(e);
+        (void)cudaGetLastError();
+    }
     SimtArgs a{};
     a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
     a.init = prefix_state; a.state_out = nullptr;

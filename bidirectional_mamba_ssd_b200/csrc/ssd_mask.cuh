@@ -29,18 +29,21 @@ struct MaskVectors {
     const float *colf, *colb;   // per-column factors (see above)
 };
 
-// Columns [32 J, 32 J + 32) of row `row`, packed as 16 bf16 pairs.
-__device__ __forceinline__ void mask_block(int J, int row, float my_af, float my_ab,
-                                           const uint32_t (&gf)[32], const uint32_t (&gb)[32],
-                                           const MaskVectors &v, uint32_t (&packed)[16]) {
+// Columns [32 J + c0, 32 J + c0 + W) of row `row` (W = 16 or 32, c0 = 0 or
+// 16 with W = 16), packed as W/2 bf16 pairs.
+template <int W>
+__device__ __forceinline__ void mask_cols(int J, int c0, int row, float my_af, float my_ab,
+                                          const uint32_t (&gf)[W], const uint32_t (&gb)[W],
+                                          const MaskVectors &v, uint32_t (&packed)[W / 2]) {
     const int wq = row >> 5;
     const int s0 = J * 32;
-    float m[32];
+    const int s1 = s0 + c0;
+    float m[W];
     if (J < wq) {
         const float rf = __expf(my_af - v.af[s0 + 31]);
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-            const float4 c = *reinterpret_cast<const float4 *>(v.colf + s0 + q);
+        for (int q = 0; q < W; q += 4) {
+            const float4 c = *reinterpret_cast<const float4 *>(v.colf + s1 + q);
             m[q + 0] = __uint_as_float(gf[q + 0]) * (rf * c.x);
             m[q + 1] = __uint_as_float(gf[q + 1]) * (rf * c.y);
             m[q + 2] = __uint_as_float(gf[q + 2]) * (rf * c.z);
@@ -49,21 +52,21 @@ __device__ __forceinline__ void mask_block(int J, int row, float my_af, float my
     } else if (J > wq) {
         const float rb = __expf(my_ab - v.ab[s0]);
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-            const float4 c = *reinterpret_cast<const float4 *>(v.colb + s0 + q);
+        for (int q = 0; q < W; q += 4) {
+            const float4 c = *reinterpret_cast<const float4 *>(v.colb + s1 + q);
             m[q + 0] = __uint_as_float(gb[q + 0]) * (rb * c.x);
             m[q + 1] = __uint_as_float(gb[q + 1]) * (rb * c.y);
             m[q + 2] = __uint_as_float(gb[q + 2]) * (rb * c.z);
             m[q + 3] = __uint_as_float(gb[q + 3]) * (rb * c.w);
         }
     } else {
-        const int rr = row - s0;   // this row's position inside the block
+        const int rr = row - s1;   // this row's position relative to the first column
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-            const float4 af4 = *reinterpret_cast<const float4 *>(v.af + s0 + q);
-            const float4 ab4 = *reinterpret_cast<const float4 *>(v.ab + s0 + q);
-            const float4 df4 = *reinterpret_cast<const float4 *>(v.dtf + s0 + q);
-            const float4 db4 = *reinterpret_cast<const float4 *>(v.dtb + s0 + q);
+        for (int q = 0; q < W; q += 4) {
+            const float4 af4 = *reinterpret_cast<const float4 *>(v.af + s1 + q);
+            const float4 ab4 = *reinterpret_cast<const float4 *>(v.ab + s1 + q);
+            const float4 df4 = *reinterpret_cast<const float4 *>(v.dtf + s1 + q);
+            const float4 db4 = *reinterpret_cast<const float4 *>(v.dtb + s1 + q);
             const float afs[4] = {af4.x, af4.y, af4.z, af4.w};
             const float abs_[4] = {ab4.x, ab4.y, ab4.z, ab4.w};
             const float dfs[4] = {df4.x, df4.y, df4.z, df4.w};
@@ -81,7 +84,14 @@ __device__ __forceinline__ void mask_block(int J, int row, float my_af, float my
         }
     }
 #pragma unroll
-    for (int q = 0; q < 16; ++q) packed[q] = sm100::pack_bf16x2(m[2 * q], m[2 * q + 1]);
+    for (int q = 0; q < W / 2; ++q) packed[q] = sm100::pack_bf16x2(m[2 * q], m[2 * q + 1]);
+}
+
+// Columns [32 J, 32 J + 32) of row `row`, packed as 16 bf16 pairs.
+__device__ __forceinline__ void mask_block(int J, int row, float my_af, float my_ab,
+                                           const uint32_t (&gf)[32], const uint32_t (&gb)[32],
+                                           const MaskVectors &v, uint32_t (&packed)[16]) {
+    mask_cols<32>(J, 0, row, my_af, my_ab, gf, gb, v, packed);
 }
 
 // Per-column factors of column s (call once per column, before mask_block).

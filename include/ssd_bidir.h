@@ -158,7 +158,9 @@ int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *
  *   A, D         (2, nheads)                              fp32
  *   B, C         (2, batch, blk_len, ngroups, dstate)     io
  *   prefix_state (batch, nheads, headdim, dstate)         fp32, NULL = zero prefix
- *   out          (batch, blk_len, nheads, headdim)        io, overwritten */
+ *   out          (batch, blk_len, nheads, headdim)        io, overwritten
+ * bf16 I/O runs the tensor-core chunked kernels (the prefix state enters the
+ * C.H product as a bf16 operand); fp32 I/O runs the sequential fp32 scan. */
 int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
                    const void *C, const float *D, const float *prefix_state, void *out,
                    int batch, int blk_len, int nheads, int headdim, int dstate,
@@ -194,6 +196,13 @@ int ssd_bidir_fwd_noalloc(const void *x, const void *dt, const float *A, const v
  * Returns SSD_OK, SSD_ERR_TIMEOUT (a bounded device wait expired in a call
  * since the last check) or SSD_ERR_CUDA (the stream reported an error). */
 int ssd_get_device_status(const void *workspace, void *stream);
+
+/* Self-test of the bounded device waits: launches one CTA that waits on an
+ * mbarrier nothing arrives on, for at most limit_us microseconds (1 ..
+ * 2,000,000). The wait gives up, the kernel records SSD_ERR_TIMEOUT in the
+ * workspace's status header and exits; nothing faults and the context stays
+ * usable. Read the result with ssd_get_device_status. */
+int ssd_selftest_wait_timeout(void *workspace, size_t ws_bytes, int limit_us, void *stream);
 
 /* Static description of a status code. */
 const char *ssd_error_string(int status);

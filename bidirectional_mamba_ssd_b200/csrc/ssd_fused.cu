@@ -22,14 +22,18 @@
 //   warp 0      TMA producer: x tiles (2 slots), B/C tiles (4-slot ring),
 //               reverse states (1 slot)
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 2..5  epilogue group A ("mask"): decay sums, diag(w) X, the masked
-//               matrix, written as bf16 into TMEM over the consumed C_f.B_f^T
-//               columns and used there as the A operand of (M_f + M_b) X
-//   warps 6..9  epilogue group B ("state/output"): the fp32 state chains, the
-//               reverse states' store, the output tile and its TMA store
+//   warps 2..5  epilogue group A: decay sums (both directions in one scan),
+//               diag(w) X, the per-tile vectors, the first 16 columns of each
+//               32-column block of the masked matrix
+//   warps 6..9  epilogue group B: the last 16 columns of each block, the fp32
+//               state chains, the reverse states' store, the output tile and
+//               its TMA store
 // In both groups thread r owns tile row r = 32 * (warp % 4) + lane (its TMEM
-// lane). Group A runs one tile ahead of group B; per-tile vectors pass from A
-// to B through two shared-memory buffers.
+// lane). The masked matrix is written as bf16 into TMEM over the consumed
+// C_f.B_f^T columns and read there as the A operand of (M_f + M_b) X. In
+// phase 1, diag(w') X overwrites its own x slot and the tile states alternate
+// between two TMEM buffers (the C.B^T columns are idle then), so the tiles of
+// phase 1 pipeline instead of waiting on each other.
 // Phase-1 inputs (x, B') are loaded with an L2 evict-last hint and re-read in
 // phase 2 with evict-first, so the re-read mostly hits L2.
 //
@@ -72,22 +76,26 @@ enum {
     B_HB_FULL = B_X_EMPTY + 2,
     B_HB_EMPTY,
     B_HB_WRITTEN,                    // group B -> producer: phase-1 states are in global memory
-    B_G_READY,                       // MMA -> group A
-    B_S_READY,                       // MMA -> groups A and B
+    B_G_READY,                       // MMA -> groups A and B (phase 2)
+    B_S_READY,                       // MMA -> groups A and B (phase 2)
     B_Y_READY,                       // MMA -> group B
-    B_XW_READY,                      // group A -> MMA
-    B_M_READY,                       // group A -> MMA
-    B_S_FREE,                        // group B -> MMA
+    B_P1S_READY,                     // 2: MMA -> group B, phase-1 tile state per TMEM buffer
+    B_P1S_FREE = B_P1S_READY + 2,    // 2: group B -> MMA
+    B_XW_READY = B_P1S_FREE + 2,     // group A -> MMA
+    B_M_READY,                       // groups A and B -> MMA (count 2)
+    B_S_FREE,                        // group B -> MMA (phase 2)
     B_Y_FREE,                        // group B -> MMA
     B_VEC_READY,                     // 2: group A -> group B, per vector buffer
     B_VEC_FREE = B_VEC_READY + 2,    // 2: group B -> group A
     B_COUNT = B_VEC_FREE + 2
 };
 
-// Per-tile vectors group A hands to group B (and reads itself).
+// Per-tile vectors group A writes and both groups read.
 struct TileVec {
     float af[kTile];    // A_f * prefix sums of dt_f
     float ab[kTile];    // A_b * suffix sums of dt_b
+    float dtf[kTile], dtb[kTile];
+    float colf[kTile], colb[kTile];   // per-column mask factors
     float totf, totb;   // tile sums of dt_f, dt_b
     float pad[2];
 };
@@ -141,33 +149,34 @@ __device__ __forceinline__ void sync_b() { asm volatile("bar.sync 2, 128;" ::: "
 
 __device__ __forceinline__ float bf2f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
-// Inclusive scan over the 128 rows of group A (row order), prefix or suffix.
-__device__ __forceinline__ float scan_rows(float v, bool suffix, int row, float *red) {
+// Inclusive prefix sums of two values over the 128 rows of group A (row
+// order), and both totals.
+__device__ __forceinline__ void scan2(float &a, float &b, float &ta, float &tb, int row, float *red) {
     const int lane = row & 31, wq = row >> 5;
-    if (!suffix) {
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            float n = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += n;
+    for (int o = 1; o < 32; o <<= 1) {
+        const float na = __shfl_up_sync(0xffffffffu, a, o);
+        const float nb = __shfl_up_sync(0xffffffffu, b, o);
+        if (lane >= o) {
+            a += na;
+            b += nb;
         }
-        if (lane == 31) red[wq] = v;
-    } else {
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            float n = __shfl_down_sync(0xffffffffu, v, o);
-            if (lane + o < 32) v += n;
-        }
-        if (lane == 0) red[wq] = v;
+    }
+    if (lane == 31) {
+        red[wq] = a;
+        red[4 + wq] = b;
     }
     sync_a();
-    float add = 0.f;
-    if (!suffix) {
-        for (int k = 0; k < wq; ++k) add += red[k];
-    } else {
-        for (int k = wq + 1; k < 4; ++k) add += red[k];
+    float pa = 0.f, pb = 0.f;
+    for (int k = 0; k < wq; ++k) {
+        pa += red[k];
+        pb += red[4 + k];
     }
+    ta = (red[0] + red[1]) + (red[2] + red[3]);
+    tb = (red[4] + red[5]) + (red[6] + red[7]);
     sync_a();
-    return v + add;
+    a += pa;
+    b += pb;
 }
 
 template <int N>
@@ -180,7 +189,7 @@ struct Smem {
     static constexpr uint32_t hf = hb + kH;
     static constexpr uint32_t xw = hf + kH;             // diag(w) x
     static constexpr uint32_t small = xw + kSlab;
-    static constexpr uint32_t bytes = small + 6144;     // barriers + per-tile vectors (~4.4 KB)
+    static constexpr uint32_t bytes = small + 7168;     // barriers, scan scratch, 2 tile-vector buffers
 };
 
 template <int N>
@@ -196,19 +205,15 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
-    float *red = reinterpret_cast<float *>(g + S::small + 256);   // 8 floats, group A scans
-    TileVec *vec = reinterpret_cast<TileVec *>(g + S::small + 288);  // 2 buffers
-    float *colf = reinterpret_cast<float *>(vec + 2);   // group A: per-column mask factors
-    float *colb = colf + kTile;
-    float *dtf = colb + kTile;
-    float *dtb = dtf + kTile;
+    float *red = reinterpret_cast<float *>(g + S::small + 384);    // 8 floats, group A scans
+    TileVec *vec = reinterpret_cast<TileVec *>(g + S::small + 512);  // 2 buffers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), i == B_M_READY ? 2 : 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -219,12 +224,17 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM columns: G_f [0,128) (the bf16 masked matrix M reuses [0,64)),
-    // G_b [128,256), Yo_f [256,320), Yo_b [320,384), Yd [384,448), S [448,512)
+    // TMEM columns: G_f [0,128), G_b [128,256), Yo_f [256,320), Yo_b [320,384),
+    // Yd [384,448), S [448,512). The masked matrix M (bf16 pairs) reuses G_f's
+    // columns: matrix columns [16k, 16k + 16) go to TMEM columns [16k, 16k + 8),
+    // written by the group that consumed G_f's columns [16k, 16k + 16) (group A
+    // for even k, group B for odd k); phase-1 tile states alternate between
+    // TMEM columns [0,64) and [64,128).
     const uint32_t tGf = tmem, tGb = tmem + 128, tYof = tmem + 256, tYob = tmem + 320,
                    tYd = tmem + 384, tS = tmem + 448;
     const int nt = p.nt;
     const int hpg = p.H / p.G;
+    const size_t dt_dir = (size_t)p.batch * p.L * p.H;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -282,9 +292,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             constexpr uint32_t id_state = idesc_bf16_f32(128, 64, true, true);   // B^T (MN) x X' (MN)
             constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);    // C (K) x B (K)
             constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);      // C (K) x H (MN); M (K) x X (MN)
-            uint32_t kr = 0, kx = 0, kh = 0;
+            uint32_t kr = 0, kx = 0, kh = 0, n1 = 0;
             uint32_t n_xw = 0, n_m = 0, n_sfree = 0, n_yfree = 0;
-            bool first_s = true, first_y = true;
+            bool first2 = true;
             auto wait_ring = [&](uint32_t k) -> uint32_t {
                 const uint32_t s = k % kRing;
                 mbar_wait(bar(B_RING_FULL + s), (k / kRing) & 1, abort_flag, p.status, 201);
@@ -292,19 +302,20 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             };
             auto slot_addr = [&](uint32_t s) { return base + S::ring + s * 2 * kSlab; };
             for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-                for (int i = nt - 1; i >= 0; --i) {        // phase 1: S' = B'^T diag(w') X
-                    ++kx;
+                for (int i = nt - 1; i >= 0; --i, ++n1) {  // phase 1: S' = B'^T (diag(w') X in the x slot)
+                    const uint32_t xs = kx++ & 1;
                     const uint32_t rs = wait_ring(kr++);
                     mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 202);
-                    if (!first_s) mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 203);
-                    first_s = false;
+                    const uint32_t pb = n1 & 1;
+                    if (n1 >= 2) mbar_wait(bar(B_P1S_FREE + pb), ((n1 >> 1) - 1) & 1, abort_flag, p.status, 203);
                     tc_fence_after();
-                    const uint32_t sB = slot_addr(rs);
+                    const uint32_t sB = slot_addr(rs), sX = base + S::x0 + xs * kSlab;
                     for (int k = 0; k < kTile / 16; ++k)
-                        mma_bf16_ss(tS, sdesc_sw128(sB + k * 2048, kSlab, 1024),
-                                    sdesc_sw128(base + S::xw + k * 2048, kSlab, 1024), id_state, k > 0);
-                    mma_commit(bar(B_S_READY));
+                        mma_bf16_ss(tGf + 64 * pb, sdesc_sw128(sB + k * 2048, kSlab, 1024),
+                                    sdesc_sw128(sX + k * 2048, kSlab, 1024), id_state, k > 0);
+                    mma_commit(bar(B_P1S_READY + pb));
                     mma_commit(bar(B_RING_EMPTY + rs));
+                    mma_commit(bar(B_X_EMPTY + xs));
                 }
                 for (int i = 0; i < nt; ++i) {             // phase 2
                     const uint32_t xs = kx++ & 1;
@@ -313,8 +324,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     const uint32_t sCf = slot_addr(rCf), sBf = slot_addr(rBf);
                     const uint32_t sCb = slot_addr(rCb), sBb = slot_addr(rBb);
                     tc_fence_after();
-                    // G_f = C_f B_f^T, G_b = C_b B_b^T (the previous tile's M, kept in
-                    // G_f's columns, was read by the Yd MMA issued before these)
+                    // G_f = C_f B_f^T, G_b = C_b B_b^T (earlier readers of these TMEM
+                    // columns are MMAs issued before, which complete in order)
                     for (int k = 0; k < N / 16; ++k) {
                         const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
                         mma_bf16_ss(tGf, sdesc_sw128(sCf + ko, 0, 1024), sdesc_sw128(sBf + ko, 0, 1024), id_g, k > 0);
@@ -326,9 +337,11 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     mma_commit(bar(B_G_READY));
                     mma_commit(bar(B_RING_EMPTY + rBb));
                     // the previous tile's outputs and state are consumed; H_f is this tile's
-                    if (!first_y) mbar_wait(bar(B_Y_FREE), n_yfree++ & 1, abort_flag, p.status, 205);
-                    first_y = false;
-                    mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 206);
+                    if (!first2) {
+                        mbar_wait(bar(B_Y_FREE), n_yfree++ & 1, abort_flag, p.status, 205);
+                        mbar_wait(bar(B_S_FREE), n_sfree++ & 1, abort_flag, p.status, 206);
+                    }
+                    first2 = false;
                     tc_fence_after();
                     for (int k = 0; k < N / 16; ++k) {      // Yo_f = C_f H_f
                         const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
@@ -353,11 +366,11 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     mma_commit(bar(B_S_READY));
                     mma_commit(bar(B_RING_EMPTY + rBf));
                     mbar_wait(bar(B_M_READY), n_m++ & 1, abort_flag, p.status, 209);
-                    mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 204);
+                    mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 204);
                     tc_fence_after();
                     const uint32_t sX = base + S::x0 + xs * kSlab;
                     for (int k = 0; k < kTile / 16; ++k)    // Yd = M X, M from TMEM
-                        mma_bf16_ts(tYd, tGf + k * 8, sdesc_sw128(sX + k * 2048, kSlab, 1024), id_o, k > 0);
+                        mma_bf16_ts(tYd, tGf + 16 * k, sdesc_sw128(sX + k * 2048, kSlab, 1024), id_o, k > 0);
                     mma_commit(bar(B_Y_READY));
                 }
             }
@@ -366,103 +379,115 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // ------------------------------------------------------------ group A
         const int row = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
-        uint32_t kx = 0, n_g = 0, nvec = 0, n_s = 0;   // n_s: S MMAs issued before this step
-        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-            const int b = u / p.H, h = u % p.H;
+        uint32_t kx = 0, n_g = 0, nvec = 0, n_s = 0;   // n_s: phase-2 S MMAs issued so far
+        // dt of the step after the current one is fetched a step ahead
+        auto load_dt = [&](int u, int ph, int i, float &vf, float &vb) {
+            vf = 0.f;
+            vb = 0.f;
+            if (u >= p.units) return;
+            const int b = u / p.H, h = u % p.H, t = i * kTile + row;
+            if (t < p.L) {
+                const size_t o = ((size_t)b * p.L + t) * p.H + h;
+                vb = __bfloat162float(p.dt[dt_dir + o]);
+                if (ph == 2) vf = __bfloat162float(p.dt[o]);
+            }
+        };
+        int cu = blockIdx.x, cph = 1, ci = nt - 1;
+        float nvf, nvb;
+        load_dt(cu, cph, ci, nvf, nvb);
+        while (cu < p.units) {
+            const float vf = nvf, vb = nvb;
+            int xu = cu, xph = cph, xi = ci;          // next step
+            if (xph == 1) {
+                if (xi > 0) --xi;
+                else { xph = 2; xi = 0; }
+            } else if (xi < nt - 1) {
+                ++xi;
+            } else {
+                xu += gridDim.x; xph = 1; xi = nt - 1;
+            }
+            load_dt(xu, xph, xi, nvf, nvb);
+            const int b = cu / p.H, h = cu % p.H;
             const float Af = p.A[h], Ab = p.A[p.H + h];
-            const size_t dt_dir = (size_t)p.batch * p.L * p.H;
-            // phase 1: reverse tile sums and diag(w') X
-            for (int i = nt - 1; i >= 0; --i) {
-                const int t = i * kTile + row;
-                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
-                const float cs = scan_rows(vb, true, row, red);
-                const uint32_t vb_i = nvec & 1;
-                if (nvec >= 2) mbar_wait(bar(B_VEC_FREE + vb_i), ((nvec >> 1) - 1) & 1, abort_flag, p.status, 301);
-                TileVec &V = vec[vb_i];
-                if (row == 0) V.totb = cs;
-                sync_a();
-                const float total = V.totb;
-                if (row == 0) mbar_arrive(bar(B_VEC_READY + vb_i));
-                ++nvec;
-                const float w = __expf(Ab * (total - cs)) * vb;
-                if (n_s > 0) mbar_wait(bar(B_S_READY), (n_s - 1) & 1, abort_flag, p.status, 302);
-                const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 303);
-                scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, w);
+            const uint32_t vb_i = nvec & 1;
+            TileVec &V = vec[vb_i];
+            float pf = vf, pb = vb, totf, totb;
+            scan2(pf, pb, totf, totb, row, red);
+            const float csb = totb - pb + vb;          // suffix sum of dt_b from this row
+            if (nvec >= 2) mbar_wait(bar(B_VEC_FREE + vb_i), ((nvec >> 1) - 1) & 1, abort_flag, p.status, 301);
+            const uint32_t xs = kx++ & 1;
+            if (cph == 1) {
+                if (row == 0) {
+                    V.totb = totb;
+                    mbar_arrive(bar(B_VEC_READY + vb_i));
+                }
+                // diag(w') X in place in the x slot, w'_s = exp(A' sum_{r<s} dt') dt'_s
+                const float w = __expf(Ab * (totb - csb)) * vb;
+                mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 302);
+                uint8_t *xt = g + S::x0 + xs * kSlab;
+                scale_row(xt, xt, row, w);
                 fence_proxy_async_smem();
                 sync_a();
-                if (row == 0) {
-                    mbar_arrive(bar(B_XW_READY));
-                    mbar_arrive(bar(B_X_EMPTY + xs));
-                }
-                ++n_s;
-            }
-            // phase 2: decay sums, diag(w_f) X, masked matrix
-            for (int i = 0; i < nt; ++i) {
-                const int t = i * kTile + row;
-                const float vf = t < p.L ? __bfloat162float(p.dt[((size_t)b * p.L + t) * p.H + h]) : 0.f;
-                const float vb = t < p.L ? __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]) : 0.f;
-                const float csf = scan_rows(vf, false, row, red);
-                const float csb = scan_rows(vb, true, row, red);
-                const float my_af = Af * csf, my_ab = Ab * csb;
-                const uint32_t vb_i = nvec & 1;
-                if (nvec >= 2) mbar_wait(bar(B_VEC_FREE + vb_i), ((nvec >> 1) - 1) & 1, abort_flag, p.status, 311);
-                TileVec &V = vec[vb_i];
+                if (row == 0) mbar_arrive(bar(B_XW_READY));
+            } else {
+                const float my_af = Af * pf, my_ab = Ab * csb;
                 V.af[row] = my_af;
                 V.ab[row] = my_ab;
-                if (row == kTile - 1) V.totf = csf;
-                if (row == 0) V.totb = csb;
-                dtf[row] = vf;
-                dtb[row] = vb;
+                V.dtf[row] = vf;
+                V.dtb[row] = vb;
+                if (row == 0) {
+                    V.totf = totf;
+                    V.totb = totb;
+                }
+                sync_a();
+                mask_column_factors(row, my_af, my_ab, vf, vb, V.af, V.ab, V.colf, V.colb);
                 sync_a();
                 if (row == 0) mbar_arrive(bar(B_VEC_READY + vb_i));
-                ++nvec;
-                mask_column_factors(row, my_af, my_ab, vf, vb, V.af, V.ab, colf, colb);
-                const float wf = __expf(Af * (V.totf - csf)) * vf;
-                if (n_s > 0) mbar_wait(bar(B_S_READY), (n_s - 1) & 1, abort_flag, p.status, 312);
-                const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_X_FULL + xs), ((kx - 1) >> 1) & 1, abort_flag, p.status, 313);
+                // diag(w_f) X into the X' buffer, w_s = exp(A sum_{r>s} dt) dt_s
+                const float wf = __expf(Af * (totf - pf)) * vf;
+                if (n_s > 0) mbar_wait(bar(B_S_READY), (n_s - 1) & 1, abort_flag, p.status, 311);
+                mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 312);
                 scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, wf);
                 fence_proxy_async_smem();
                 sync_a();
                 if (row == 0) mbar_arrive(bar(B_XW_READY));
                 ++n_s;
-
-                // masked matrix M = M_f + M_b, bf16 pairs into TMEM columns [0, 64)
-                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 314);
+                // masked matrix, the first 16 columns of every 32-column block
+                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 313);
                 tc_fence_after();
-                const MaskVectors mv{V.af, V.ab, dtf, dtb, colf, colb};
+                const MaskVectors mv{V.af, V.ab, V.dtf, V.dtb, V.colf, V.colb};
 #pragma unroll 1
                 for (int J = 0; J < 4; ++J) {
-                    uint32_t gf[32], gb[32], packed[16];
-                    tmem_ld32(tGf + lane_off + J * 32, gf);
-                    tmem_ld32(tGb + lane_off + J * 32, gb);
+                    uint32_t gf[16], gb[16], packed[8];
+                    tmem_ld16(tGf + lane_off + J * 32, gf);
+                    tmem_ld16(tGb + lane_off + J * 32, gb);
                     tmem_wait_ld();
-                    mask_block(J, row, my_af, my_ab, gf, gb, mv, packed);
-                    tmem_st16(tGf + lane_off + J * 16, packed);
+                    mask_cols<16>(J, 0, row, my_af, my_ab, gf, gb, mv, packed);
+                    tmem_st8(tGf + lane_off + J * 32, packed);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 sync_a();
                 if (row == 0) mbar_arrive(bar(B_M_READY));
             }
+            ++nvec;
+            cu = xu; cph = xph; ci = xi;
         }
     } else {
         // ------------------------------------------------------------ group B
         const int row = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
         const uint64_t keep = policy_evict_last();
-        uint32_t kx = 0, n_s = 0, n_y = 0, nvec = 0;
-        uint32_t units_done = 0;
+        uint32_t kx = 0, n_s = 0, n_y = 0, n_g = 0, nvec = 0, n1 = 0;
         float hreg[kP];
-        for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++units_done) {
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             const int b = u / p.H, h = u % p.H;
             const float Af = p.A[h], Ab = p.A[p.H + h];
             const float dsum = p.D[h] + p.D[p.H + h];
             // phase 1: reverse state chain, right to left
 #pragma unroll
             for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
-            for (int i = nt - 1; i >= 0; --i) {
+            for (int i = nt - 1; i >= 0; --i, ++n1) {
                 const uint32_t vb_i = nvec & 1;
                 mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 401);
                 const float totb = vec[vb_i].totb;
@@ -483,46 +508,68 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     }
                 }
                 const float gdec = __expf(Ab * totb);
-                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 402);
+                const uint32_t pbuf = n1 & 1;
+                mbar_wait(bar(B_P1S_READY + pbuf), (n1 >> 1) & 1, abort_flag, p.status, 402);
                 tc_fence_after();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t v[32];
-                    tmem_ld32(tS + lane_off + half * 32, v);
+                    tmem_ld32(tGf + 64 * pbuf + lane_off + half * 32, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
                 }
-                if (i == 0 && row < N) {       // phase 2 starts from H_f = 0
-                    uint4 *hf = reinterpret_cast<uint4 *>(g + S::hf + row * 128);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) hf[c] = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
                 tc_fence_before();
                 sync_b();
-                if (row == 0) mbar_arrive(bar(B_S_FREE));
+                if (row == 0) mbar_arrive(bar(B_P1S_FREE + pbuf));
             }
+            // phase 2 starts from H_f = 0; the reverse states go to the TMA proxy
+            if (row < N) {
+                uint4 *hf = reinterpret_cast<uint4 *>(g + S::hf + row * 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) hf[c] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
             fence_proxy_async_global();
             sync_b();
             if (row == 0) mbar_arrive(bar(B_HB_WRITTEN));
 
-            // phase 2: forward state chain and outputs, left to right
+            // phase 2: masked matrix (columns 64..127), forward state chain, outputs
 #pragma unroll
             for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
             for (int i = 0; i < nt; ++i) {
                 const int t0 = i * kTile;
                 const uint32_t vb_i = nvec & 1;
                 mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 411);
-                const float my_af = vec[vb_i].af[row], my_ab = vec[vb_i].ab[row];
-                const float totf = vec[vb_i].totf;
+                const TileVec &V = vec[vb_i];
+                const float my_af = V.af[row], my_ab = V.ab[row];
+                const float gdec = __expf(Af * V.totf);
+                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 412);
+                tc_fence_after();
+                {
+                    const MaskVectors mv{V.af, V.ab, V.dtf, V.dtb, V.colf, V.colb};
+                    // the last 16 columns of every 32-column block
+#pragma unroll 1
+                    for (int J = 0; J < 4; ++J) {
+                        uint32_t gf[16], gb[16], packed[8];
+                        tmem_ld16(tGf + lane_off + J * 32 + 16, gf);
+                        tmem_ld16(tGb + lane_off + J * 32 + 16, gb);
+                        tmem_wait_ld();
+                        mask_cols<16>(J, 16, row, my_af, my_ab, gf, gb, mv, packed);
+                        tmem_st8(tGf + lane_off + J * 32 + 16, packed);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
                 sync_b();
-                if (row == 0) mbar_arrive(bar(B_VEC_FREE + vb_i));
+                if (row == 0) {
+                    mbar_arrive(bar(B_M_READY));
+                    mbar_arrive(bar(B_VEC_FREE + vb_i));
+                }
                 ++nvec;
                 // forward chain: H_f <- exp(A sum dt) H_f + S_f; bf16 copy for C_f.H_f
-                const float gdec = __expf(Af * totf);
-                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 412);
+                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 413);
                 tc_fence_after();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -550,7 +597,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
                 // output tile over the x slot, then one TMA store
                 const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 413);
+                mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 414);
                 tc_fence_after();
                 const float ef = __expf(my_af), eb = __expf(my_ab);
                 uint8_t *xt = g + S::x0 + xs * kSlab;

@@ -60,6 +60,9 @@ __device__ __forceinline__ void mask_cols(int J, int c0, int row, float my_af, f
             m[q + 3] = __uint_as_float(gb[q + 3]) * (rb * c.w);
         }
     } else {
+        // diagonal block: column s is either left of the row (forward term
+        // only), right of it (reverse term only) or the row's own token (both,
+        // decay 1), so one exp per entry
         const int rr = row - s1;   // this row's position relative to the first column
 #pragma unroll
         for (int q = 0; q < W; q += 4) {
@@ -74,12 +77,13 @@ __device__ __forceinline__ void mask_cols(int J, int c0, int row, float my_af, f
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int c = q + e;
-                // exponents clamped at 0 so the unselected side never overflows
-                const float ef = __expf(fminf(my_af - afs[e], 0.f)) * dfs[e];
-                const float eb = __expf(fminf(my_ab - abs_[e], 0.f)) * dbs[e];
-                const float mf = c <= rr ? __uint_as_float(gf[c]) * ef : 0.f;
-                const float mb = c >= rr ? __uint_as_float(gb[c]) * eb : 0.f;
-                m[c] = mf + mb;
+                const bool fwd = c < rr, rev = c > rr;
+                const float gfv = __uint_as_float(gf[c]), gbv = __uint_as_float(gb[c]);
+                // the exponent of the selected side is <= 0; the other side is
+                // never used, so its possible overflow is harmless
+                const float x = __expf(fwd ? my_af - afs[e] : my_ab - abs_[e]);
+                const float wv = fwd ? gfv * dfs[e] : gbv * dbs[e];
+                m[c] = (fwd || rev) ? wv * x : gfv * dfs[e] + gbv * dbs[e];
             }
         }
     }
@@ -108,18 +112,20 @@ __device__ __forceinline__ void mask_column_factors(int s, float a_s, float ab_s
 __device__ __forceinline__ void scale_row(const uint8_t *src_tile, uint8_t *dst_tile, int row, float w) {
     const uint4 *src = reinterpret_cast<const uint4 *>(src_tile + row * 128);
     uint4 *d = reinterpret_cast<uint4 *>(dst_tile + row * 128);
+    uint4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = src[(k + row) & 7];   // all loads first (src may equal dst)
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        const int c = (k + row) & 7;
-        uint4 v = src[c];
-        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
+        uint32_t *q = reinterpret_cast<uint32_t *>(&v[k]);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float lo = __uint_as_float(q[j] << 16) * w, hi = __uint_as_float(q[j] & 0xffff0000u) * w;
             q[j] = sm100::pack_bf16x2(lo, hi);
         }
-        d[c] = v;
     }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) d[(k + row) & 7] = v[k];
 }
 
 }  // namespace ssd

@@ -18,22 +18,25 @@
 // Architecture; reverse = forward on the flipped sequence: "DiffMamba -
 // Checkpoints" model card, Model details.
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: x tiles (2 slots), B/C tiles (4-slot ring),
-//               reverse states (1 slot)
-//   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 2..5  epilogue group A: decay sums (both directions in one scan),
-//               diag(w) X, the per-tile vectors, the first 16 columns of each
-//               32-column block of the masked matrix
-//   warps 6..9  epilogue group B: the last 16 columns of each block, the fp32
-//               state chains, the reverse states' store, the output tile and
-//               its TMA store
-// In both groups thread r owns tile row r = 32 * (warp % 4) + lane (its TMEM
-// lane). The masked matrix is written as bf16 into TMEM over the consumed
-// C_f.B_f^T columns and read there as the A operand of (M_f + M_b) X. In
-// phase 1, diag(w') X overwrites its own x slot and the tile states alternate
-// between two TMEM buffers (the C.B^T columns are idle then), so the tiles of
-// phase 1 pipeline instead of waiting on each other.
+// Warp roles (448 threads):
+//   warp 0       TMA producer: x tiles (2 slots), B/C tiles (4-slot ring),
+//                reverse states (1 slot)
+//   warp 1       TMEM owner and MMA issuer (one thread)
+//   warps 2..5   epilogue group C: decay sums (both directions in one scan),
+//                diag(w) X, the per-tile vectors, the fp32 state chains of
+//                both directions and the reverse states' store
+//   warps 6..9   epilogue group A: the first 16 columns of each 32-column
+//                block of the masked matrix
+//   warps 10..13 epilogue group B: the last 16 columns of each block, the
+//                output tile and its TMA store
+// In every group thread r owns tile row r = 32 * (warp % 4) + lane (its TMEM
+// lane). Group C prepares tile i + 1 while groups A and B build the masked
+// matrix of tile i. The masked matrix is written as bf16 into TMEM over the
+// consumed C_f.B_f^T columns and read there as the A operand of
+// (M_f + M_b) X. In phase 1, diag(w') X overwrites its own x slot and the
+// tile states alternate between two TMEM buffers (the C.B^T columns are idle
+// then); group C chains each tile's state one step late, so its scans and
+// scaling of the next tile overlap the MMA.
 // Phase-1 inputs (x, B') are loaded with an L2 evict-last hint and re-read in
 // phase 2 with evict-first, so the re-read mostly hits L2.
 //
@@ -56,7 +59,7 @@ constexpr int kTile = 128;
 constexpr int kP = 64;
 constexpr uint32_t kSlab = 16384;       // 128 rows x 128 bytes
 constexpr int kRing = 4;                // B/C ring slots (32 KB each)
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 
 struct FusedParams {
     const __nv_bfloat16 *dt;   // (2, batch, L, H)
@@ -77,20 +80,20 @@ enum {
     B_HB_EMPTY,
     B_HB_WRITTEN,                    // group B -> producer: phase-1 states are in global memory
     B_G_READY,                       // MMA -> groups A and B (phase 2)
-    B_S_READY,                       // MMA -> groups A and B (phase 2)
+    B_S_READY,                       // MMA -> group C (phase 2)
     B_Y_READY,                       // MMA -> group B
-    B_P1S_READY,                     // 2: MMA -> group B, phase-1 tile state per TMEM buffer
-    B_P1S_FREE = B_P1S_READY + 2,    // 2: group B -> MMA
-    B_XW_READY = B_P1S_FREE + 2,     // group A -> MMA
+    B_P1S_READY,                     // 2: MMA -> group C, phase-1 tile state per TMEM buffer
+    B_P1S_FREE = B_P1S_READY + 2,    // 2: group C -> MMA
+    B_XW_READY = B_P1S_FREE + 2,     // group C -> MMA
     B_M_READY,                       // groups A and B -> MMA (count 2)
-    B_S_FREE,                        // group B -> MMA (phase 2)
+    B_S_FREE,                        // group C -> MMA (phase 2)
     B_Y_FREE,                        // group B -> MMA
-    B_VEC_READY,                     // 2: group A -> group B, per vector buffer
-    B_VEC_FREE = B_VEC_READY + 2,    // 2: group B -> group A
+    B_VEC_READY,                     // 2: group C -> groups A and B, per vector buffer
+    B_VEC_FREE = B_VEC_READY + 2,    // 2: groups A and B -> group C (count 2)
     B_COUNT = B_VEC_FREE + 2
 };
 
-// Per-tile vectors group A writes and both groups read.
+// Per-tile vectors group C writes and groups A and B read.
 struct TileVec {
     float af[kTile];    // A_f * prefix sums of dt_f
     float ab[kTile];    // A_b * suffix sums of dt_b
@@ -143,13 +146,14 @@ __device__ __forceinline__ void st_global_v4_hint(void *p, uint4 v, uint64_t pol
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
-// named barriers of the two epilogue groups (128 threads each)
-__device__ __forceinline__ void sync_a() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ void sync_b() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// named barriers of the three epilogue groups (128 threads each)
+__device__ __forceinline__ void sync_c() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void sync_a() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void sync_b() { asm volatile("bar.sync 3, 128;" ::: "memory"); }
 
 __device__ __forceinline__ float bf2f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
-// Inclusive prefix sums of two values over the 128 rows of group A (row
+// Inclusive prefix sums of two values over the 128 rows of group C (row
 // order), and both totals.
 __device__ __forceinline__ void scan2(float &a, float &b, float &ta, float &tb, int row, float *red) {
     const int lane = row & 31, wq = row >> 5;
@@ -166,7 +170,7 @@ __device__ __forceinline__ void scan2(float &a, float &b, float &ta, float &tb, 
         red[wq] = a;
         red[4 + wq] = b;
     }
-    sync_a();
+    sync_c();
     float pa = 0.f, pb = 0.f;
     for (int k = 0; k < wq; ++k) {
         pa += red[k];
@@ -174,7 +178,7 @@ __device__ __forceinline__ void scan2(float &a, float &b, float &ta, float &tb, 
     }
     ta = (red[0] + red[1]) + (red[2] + red[3]);
     tb = (red[4] + red[5]) + (red[6] + red[7]);
-    sync_a();
+    sync_c();
     a += pa;
     b += pb;
 }
@@ -205,7 +209,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
-    float *red = reinterpret_cast<float *>(g + S::small + 384);    // 8 floats, group A scans
+    float *red = reinterpret_cast<float *>(g + S::small + 384);    // 8 floats, group C scans
     TileVec *vec = reinterpret_cast<TileVec *>(g + S::small + 512);  // 2 buffers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -213,7 +217,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), i == B_M_READY ? 2 : 1);
+        for (int i = 0; i < B_COUNT; ++i)
+            mbar_init(bar(i), (i == B_M_READY || i == B_VEC_FREE || i == B_VEC_FREE + 1) ? 2 : 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -376,10 +381,12 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
         }
     } else if (warp < 6) {
-        // ------------------------------------------------------------ group A
+        // ------------------------------------------------------------ group C
         const int row = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
-        uint32_t kx = 0, n_g = 0, nvec = 0, n_s = 0;   // n_s: phase-2 S MMAs issued so far
+        const uint64_t keep = policy_evict_last();
+        uint32_t kx = 0, n_s = 0, nvec = 0, n1 = 0;
+        float hreg[kP];
         // dt of the step after the current one is fetched a step ahead
         auto load_dt = [&](int u, int ph, int i, float &vf, float &vb) {
             vf = 0.f;
@@ -392,138 +399,78 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 if (ph == 2) vf = __bfloat162float(p.dt[o]);
             }
         };
+        auto next_step = [&](int &u, int &ph, int &i) {
+            if (ph == 1) {
+                if (i > 0) --i;
+                else { ph = 2; i = 0; }
+            } else if (i < nt - 1) {
+                ++i;
+            } else {
+                u += gridDim.x; ph = 1; i = nt - 1;
+            }
+        };
+        // one phase-1 chain step: store the state entering tile i, then fold in its tile state
+        auto chain1 = [&](int u, int i, float gdec) {
+            if (row < N) {
+                __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v = make_uint4(pack_bf16x2(hreg[8 * c], hreg[8 * c + 1]),
+                                         pack_bf16x2(hreg[8 * c + 2], hreg[8 * c + 3]),
+                                         pack_bf16x2(hreg[8 * c + 4], hreg[8 * c + 5]),
+                                         pack_bf16x2(hreg[8 * c + 6], hreg[8 * c + 7]));
+                    st_global_v4_hint(dst + 8 * c, v, keep);
+                }
+            }
+            const uint32_t pbuf = n1 & 1;
+            mbar_wait(bar(B_P1S_READY + pbuf), (n1 >> 1) & 1, abort_flag, p.status, 301);
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t v[32];
+                tmem_ld32(tGf + 64 * pbuf + lane_off + half * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
+            }
+            tc_fence_before();
+            sync_c();
+            if (row == 0) mbar_arrive(bar(B_P1S_FREE + pbuf));
+            ++n1;
+        };
         int cu = blockIdx.x, cph = 1, ci = nt - 1;
         float nvf, nvb;
         load_dt(cu, cph, ci, nvf, nvb);
         while (cu < p.units) {
-            const float vf = nvf, vb = nvb;
-            int xu = cu, xph = cph, xi = ci;          // next step
-            if (xph == 1) {
-                if (xi > 0) --xi;
-                else { xph = 2; xi = 0; }
-            } else if (xi < nt - 1) {
-                ++xi;
-            } else {
-                xu += gridDim.x; xph = 1; xi = nt - 1;
-            }
-            load_dt(xu, xph, xi, nvf, nvb);
-            const int b = cu / p.H, h = cu % p.H;
+            const int u = cu;
+            const int h = u % p.H;
             const float Af = p.A[h], Ab = p.A[p.H + h];
-            const uint32_t vb_i = nvec & 1;
-            TileVec &V = vec[vb_i];
-            float pf = vf, pb = vb, totf, totb;
-            scan2(pf, pb, totf, totb, row, red);
-            const float csb = totb - pb + vb;          // suffix sum of dt_b from this row
-            if (nvec >= 2) mbar_wait(bar(B_VEC_FREE + vb_i), ((nvec >> 1) - 1) & 1, abort_flag, p.status, 301);
-            const uint32_t xs = kx++ & 1;
-            if (cph == 1) {
-                if (row == 0) {
-                    V.totb = totb;
-                    mbar_arrive(bar(B_VEC_READY + vb_i));
-                }
-                // diag(w') X in place in the x slot, w'_s = exp(A' sum_{r<s} dt') dt'_s
-                const float w = __expf(Ab * (totb - csb)) * vb;
+            // ---------------- phase 1: reverse tile sums, diag(w') X in place, reverse chain
+#pragma unroll
+            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
+            int pend = -1;
+            float pend_g = 0.f;
+            for (int i = nt - 1; i >= 0; --i) {
+                const float vb = nvb;
+                next_step(cu, cph, ci);
+                load_dt(cu, cph, ci, nvf, nvb);
+                float pf = 0.f, pb = vb, totf, totb;
+                scan2(pf, pb, totf, totb, row, red);
+                const float csb = totb - pb + vb;       // suffix sum of dt_b from this row
+                const float w = __expf(Ab * (totb - csb)) * vb;   // exp(A' sum_{r<s} dt') dt'_s
+                const uint32_t xs = kx++ & 1;
                 mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 302);
                 uint8_t *xt = g + S::x0 + xs * kSlab;
                 scale_row(xt, xt, row, w);
                 fence_proxy_async_smem();
-                sync_a();
+                sync_c();
                 if (row == 0) mbar_arrive(bar(B_XW_READY));
-            } else {
-                const float my_af = Af * pf, my_ab = Ab * csb;
-                V.af[row] = my_af;
-                V.ab[row] = my_ab;
-                V.dtf[row] = vf;
-                V.dtb[row] = vb;
-                if (row == 0) {
-                    V.totf = totf;
-                    V.totb = totb;
-                }
-                sync_a();
-                mask_column_factors(row, my_af, my_ab, vf, vb, V.af, V.ab, V.colf, V.colb);
-                sync_a();
-                if (row == 0) mbar_arrive(bar(B_VEC_READY + vb_i));
-                // diag(w_f) X into the X' buffer, w_s = exp(A sum_{r>s} dt) dt_s
-                const float wf = __expf(Af * (totf - pf)) * vf;
-                if (n_s > 0) mbar_wait(bar(B_S_READY), (n_s - 1) & 1, abort_flag, p.status, 311);
-                mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 312);
-                scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, wf);
-                fence_proxy_async_smem();
-                sync_a();
-                if (row == 0) mbar_arrive(bar(B_XW_READY));
-                ++n_s;
-                // masked matrix, the first 16 columns of every 32-column block
-                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 313);
-                tc_fence_after();
-                const MaskVectors mv{V.af, V.ab, V.dtf, V.dtb, V.colf, V.colb};
-#pragma unroll 1
-                for (int J = 0; J < 4; ++J) {
-                    uint32_t gf[16], gb[16], packed[8];
-                    tmem_ld16(tGf + lane_off + J * 32, gf);
-                    tmem_ld16(tGb + lane_off + J * 32, gb);
-                    tmem_wait_ld();
-                    mask_cols<16>(J, 0, row, my_af, my_ab, gf, gb, mv, packed);
-                    tmem_st8(tGf + lane_off + J * 32, packed);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                sync_a();
-                if (row == 0) mbar_arrive(bar(B_M_READY));
+                if (pend >= 0) chain1(u, pend, pend_g);
+                pend = i;
+                pend_g = __expf(Ab * totb);
             }
-            ++nvec;
-            cu = xu; cph = xph; ci = xi;
-        }
-    } else {
-        // ------------------------------------------------------------ group B
-        const int row = ((warp & 3) << 5) | lane;
-        const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
-        const uint64_t keep = policy_evict_last();
-        uint32_t kx = 0, n_s = 0, n_y = 0, n_g = 0, nvec = 0, n1 = 0;
-        float hreg[kP];
-        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-            const int b = u / p.H, h = u % p.H;
-            const float Af = p.A[h], Ab = p.A[p.H + h];
-            const float dsum = p.D[h] + p.D[p.H + h];
-            // phase 1: reverse state chain, right to left
-#pragma unroll
-            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
-            for (int i = nt - 1; i >= 0; --i, ++n1) {
-                const uint32_t vb_i = nvec & 1;
-                mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 401);
-                const float totb = vec[vb_i].totb;
-                sync_b();
-                if (row == 0) mbar_arrive(bar(B_VEC_FREE + vb_i));
-                ++nvec;
-                ++kx;
-                // state entering tile i from the right
-                if (row < N) {
-                    __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 v = make_uint4(pack_bf16x2(hreg[8 * c], hreg[8 * c + 1]),
-                                             pack_bf16x2(hreg[8 * c + 2], hreg[8 * c + 3]),
-                                             pack_bf16x2(hreg[8 * c + 4], hreg[8 * c + 5]),
-                                             pack_bf16x2(hreg[8 * c + 6], hreg[8 * c + 7]));
-                        st_global_v4_hint(dst + 8 * c, v, keep);
-                    }
-                }
-                const float gdec = __expf(Ab * totb);
-                const uint32_t pbuf = n1 & 1;
-                mbar_wait(bar(B_P1S_READY + pbuf), (n1 >> 1) & 1, abort_flag, p.status, 402);
-                tc_fence_after();
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t v[32];
-                    tmem_ld32(tGf + 64 * pbuf + lane_off + half * 32, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
-                }
-                tc_fence_before();
-                sync_b();
-                if (row == 0) mbar_arrive(bar(B_P1S_FREE + pbuf));
-            }
+            chain1(u, pend, pend_g);
             // phase 2 starts from H_f = 0; the reverse states go to the TMA proxy
             if (row < N) {
                 uint4 *hf = reinterpret_cast<uint4 *>(g + S::hf + row * 128);
@@ -532,44 +479,47 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
             fence_proxy_async_smem();
             fence_proxy_async_global();
-            sync_b();
+            sync_c();
             if (row == 0) mbar_arrive(bar(B_HB_WRITTEN));
-
-            // phase 2: masked matrix (columns 64..127), forward state chain, outputs
+            // ---------------- phase 2: decay sums, vectors, diag(w_f) X, forward chain
 #pragma unroll
             for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
             for (int i = 0; i < nt; ++i) {
-                const int t0 = i * kTile;
+                const float vf = nvf, vb = nvb;
+                next_step(cu, cph, ci);
+                load_dt(cu, cph, ci, nvf, nvb);
+                float pf = vf, pb = vb, totf, totb;
+                scan2(pf, pb, totf, totb, row, red);
+                const float csb = totb - pb + vb;
+                const float my_af = Af * pf, my_ab = Ab * csb;
                 const uint32_t vb_i = nvec & 1;
-                mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 411);
-                const TileVec &V = vec[vb_i];
-                const float my_af = V.af[row], my_ab = V.ab[row];
-                const float gdec = __expf(Af * V.totf);
-                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 412);
-                tc_fence_after();
-                {
-                    const MaskVectors mv{V.af, V.ab, V.dtf, V.dtb, V.colf, V.colb};
-                    // the last 16 columns of every 32-column block
-#pragma unroll 1
-                    for (int J = 0; J < 4; ++J) {
-                        uint32_t gf[16], gb[16], packed[8];
-                        tmem_ld16(tGf + lane_off + J * 32 + 16, gf);
-                        tmem_ld16(tGb + lane_off + J * 32 + 16, gb);
-                        tmem_wait_ld();
-                        mask_cols<16>(J, 16, row, my_af, my_ab, gf, gb, mv, packed);
-                        tmem_st8(tGf + lane_off + J * 32 + 16, packed);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                sync_b();
+                if (nvec >= 2) mbar_wait(bar(B_VEC_FREE + vb_i), ((nvec >> 1) - 1) & 1, abort_flag, p.status, 311);
+                TileVec &V = vec[vb_i];
+                V.af[row] = my_af;
+                V.ab[row] = my_ab;
+                V.dtf[row] = vf;
+                V.dtb[row] = vb;
                 if (row == 0) {
-                    mbar_arrive(bar(B_M_READY));
-                    mbar_arrive(bar(B_VEC_FREE + vb_i));
+                    V.totf = totf;
+                    V.totb = totb;
                 }
+                sync_c();
+                mask_column_factors(row, my_af, my_ab, vf, vb, V.af, V.ab, V.colf, V.colb);
+                sync_c();
+                if (row == 0) mbar_arrive(bar(B_VEC_READY + vb_i));
                 ++nvec;
+                // diag(w_f) X into the X' buffer (the previous state MMA, which read
+                // it, completed before this group's last state step)
+                const float wf = __expf(Af * (totf - pf)) * vf;   // exp(A sum_{r>s} dt) dt_s
+                const uint32_t xs = kx++ & 1;
+                mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 312);
+                scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, wf);
+                fence_proxy_async_smem();
+                sync_c();
+                if (row == 0) mbar_arrive(bar(B_XW_READY));
                 // forward chain: H_f <- exp(A sum dt) H_f + S_f; bf16 copy for C_f.H_f
-                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 413);
+                const float gdec = __expf(Af * totf);
+                mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 313);
                 tc_fence_after();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -592,26 +542,68 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                sync_b();
+                sync_c();
                 if (row == 0) mbar_arrive(bar(B_S_FREE));
-
-                // output tile over the x slot, then one TMA store
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ groups A and B
+        const bool is_b = warp >= 10;
+        const int row = ((warp & 3) << 5) | lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+        const int c0 = is_b ? 16 : 0;       // which half of each 32-column block
+        auto sync_g = [&]() { if (is_b) sync_b(); else sync_a(); };
+        uint32_t kx = 0, n_g = 0, n_y = 0, nvec = 0;
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+            const int b = u / p.H, h = u % p.H;
+            const float dsum = p.D[h] + p.D[p.H + h];
+            kx += nt;                        // phase 1 uses the x slots without these groups
+            for (int i = 0; i < nt; ++i) {
+                const int t0 = i * kTile;
+                const uint32_t vb_i = nvec & 1;
+                mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 401);
+                const TileVec &V = vec[vb_i];
+                const float my_af = V.af[row], my_ab = V.ab[row];
+                mbar_wait(bar(B_G_READY), n_g++ & 1, abort_flag, p.status, 402);
+                tc_fence_after();
+                {
+                    const MaskVectors mv{V.af, V.ab, V.dtf, V.dtb, V.colf, V.colb};
+#pragma unroll 1
+                    for (int J = 0; J < 4; ++J) {
+                        uint32_t gf[16], gb[16], packed[8];
+                        tmem_ld16(tGf + lane_off + J * 32 + c0, gf);
+                        tmem_ld16(tGb + lane_off + J * 32 + c0, gb);
+                        tmem_wait_ld();
+                        mask_cols<16>(J, c0, row, my_af, my_ab, gf, gb, mv, packed);
+                        tmem_st8(tGf + lane_off + J * 32 + c0, packed);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                sync_g();
+                if (row == 0) {
+                    mbar_arrive(bar(B_M_READY));
+                    mbar_arrive(bar(B_VEC_FREE + vb_i));
+                }
+                ++nvec;
                 const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 414);
+                if (!is_b) continue;
+                // group B: output tile over the x slot, then one TMA store
+                mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 403);
                 tc_fence_after();
                 const float ef = __expf(my_af), eb = __expf(my_ab);
                 uint8_t *xt = g + S::x0 + xs * kSlab;
 #pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t yd[32], yf[32], yb[32];
-                    tmem_ld32(tYd + lane_off + half * 32, yd);
-                    tmem_ld32(tYof + lane_off + half * 32, yf);
-                    tmem_ld32(tYob + lane_off + half * 32, yb);
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t yd[16], yf[16], yb[16];
+                    tmem_ld16(tYd + lane_off + q * 16, yd);
+                    tmem_ld16(tYof + lane_off + q * 16, yf);
+                    tmem_ld16(tYob + lane_off + q * 16, yb);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 *q = reinterpret_cast<uint4 *>(xt + sw128_offset(row, half * 4 + c));
-                        uint4 xv = *q;
+                    for (int c = 0; c < 2; ++c) {
+                        uint4 *qp = reinterpret_cast<uint4 *>(xt + sw128_offset(row, q * 2 + c));
+                        uint4 xv = *qp;
                         uint32_t *xu = reinterpret_cast<uint32_t *>(&xv);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -622,7 +614,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                              eb * __uint_as_float(yb[i0 + 1]) + dsum * bf2f(xu[e] >> 16);
                             xu[e] = pack_bf16x2(y0, y1);
                         }
-                        *q = xv;
+                        *qp = xv;
                     }
                 }
                 fence_proxy_async_smem();
@@ -639,7 +631,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
             }
         }
-        if (row == 0) tma_store_wait_all();
+        if (is_b && row == 0) tma_store_wait_all();
     }
 
     // ------------------------------------------------------------ teardown

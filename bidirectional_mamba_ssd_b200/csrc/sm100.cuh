@@ -58,8 +58,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Time spent waiting is the sum of the global timer's forward steps between
+// polls, each step clipped to 1 ms: a timer that is stepped back, a torn read
+// or a long preemption of the kernel can then neither fake an expiry nor make
+// one come early.
+struct WaitClock {
+    uint64_t prev, spent = 0;
+    __device__ __forceinline__ WaitClock() : prev(globaltimer_ns()) {}
+    __device__ __forceinline__ bool expired(uint64_t limit_ns) {
+        const uint64_t now = globaltimer_ns();
+        const int64_t d = (int64_t)(now - prev);
+        prev = now;
+        if (d > 0) spent += d < 1000000 ? (uint64_t)d : 1000000ull;
+        return spent > limit_ns;
+    }
+};
+
 // Wait for the phase with the given parity to complete, for at most
-// `limit_ns` of wall time. On expiry: record a timeout in the status header,
+// `limit_ns` of waiting. On expiry: record a timeout in the status header,
 // raise the CTA's abort flag and return false. Once the abort flag is up,
 // later waits return false at once, so a CTA that lost an arrival runs to
 // its end (producing garbage that the status flag disowns) instead of hanging.
@@ -67,16 +83,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           DeviceStatus *st, uint32_t where,
                                           uint64_t limit_ns = 1000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    WaitClock clock;
     while (true) {
         if (*abort_flag) return false;
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) {
+        if (clock.expired(limit_ns)) {
             *abort_flag = 1;
             report_timeout(st, where);
             return false;
         }
     }
+}
+
+// Bounded wait that ignores the abort flag: used at teardown so that a CTA's
+// own asynchronous copies and MMAs have finished before it exits.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns = 100000000ull) {
+    if (mbar_try_wait(bar, parity)) return;
+    WaitClock clock;
+    while (!mbar_try_wait(bar, parity))
+        if (clock.expired(limit_ns)) return;
 }
 
 // ------------------------------------------------------------------ TMA

@@ -20,12 +20,6 @@ struct DeviceStatus {
 static_assert(sizeof(DeviceStatus) == kStatusBytes, "status header size");
 enum : unsigned int { kFlagTimeout = 1u };
 
-// Upper bound on polls of one mbarrier / flag wait before a kernel gives up.
-// Each poll is a try_wait that itself blocks for a hardware time slice, so
-// this is seconds of wall time on a healthy GPU: far beyond any legitimate
-// wait in these kernels, short enough that a lost arrival never hangs a GPU.
-constexpr uint32_t kMaxPolls = 1u << 22;
-
 __device__ __forceinline__ void report_timeout(DeviceStatus *st, unsigned int where) {
     if (st) {
         unsigned int old = atomicOr(&st->flags, kFlagTimeout);

@@ -26,9 +26,9 @@
 //                diag(w) X, the per-tile vectors, the fp32 state chains of
 //                both directions and the reverse states' store
 //   warps 6..9   epilogue group A: the first 16 columns of each 32-column
-//                block of the masked matrix
+//                block of the masked matrix, the first 32 output columns
 //   warps 10..13 epilogue group B: the last 16 columns of each block, the
-//                output tile and its TMA store
+//                last 32 output columns and the tile's TMA store
 // In every group thread r owns tile row r = 32 * (warp % 4) + lane (its TMEM
 // lane). Group C prepares tile i + 1 while groups A and B build the masked
 // matrix of tile i. The masked matrix is written as bf16 into TMEM over the
@@ -78,19 +78,24 @@ enum {
     B_X_EMPTY = B_X_FULL + 2,        // 2
     B_HB_FULL = B_X_EMPTY + 2,
     B_HB_EMPTY,
-    B_HB_WRITTEN,                    // group B -> producer: phase-1 states are in global memory
+    B_HB_WRITTEN,                    // group C -> producer: phase-1 states are in global memory
     B_G_READY,                       // MMA -> groups A and B (phase 2)
     B_S_READY,                       // MMA -> group C (phase 2)
-    B_Y_READY,                       // MMA -> group B
+    B_Y_READY,                       // MMA -> groups A and B
     B_P1S_READY,                     // 2: MMA -> group C, phase-1 tile state per TMEM buffer
     B_P1S_FREE = B_P1S_READY + 2,    // 2: group C -> MMA
-    B_XW_READY = B_P1S_FREE + 2,     // group C -> MMA
-    B_M_READY,                       // groups A and B -> MMA (count 2)
+    // 2: group C -> MMA, alternating by tile. In phase 1 group C folds tile
+    // states in one tile behind, so it can release diag(w) X of two tiles
+    // before the MMA issuer has taken the first: one barrier would complete
+    // two phases and the issuer's parity wait would miss both.
+    B_XW_READY = B_P1S_FREE + 2,
+    B_M_READY = B_XW_READY + 2,      // groups A and B -> MMA (count 2)
     B_S_FREE,                        // group C -> MMA (phase 2)
     B_Y_FREE,                        // group B -> MMA
     B_VEC_READY,                     // 2: group C -> groups A and B, per vector buffer
     B_VEC_FREE = B_VEC_READY + 2,    // 2: groups A and B -> group C (count 2)
-    B_COUNT = B_VEC_FREE + 2
+    B_MMA_DONE = B_VEC_FREE + 2,     // MMA issuer, at teardown
+    B_COUNT
 };
 
 // Per-tile vectors group C writes and groups A and B read.
@@ -245,51 +250,68 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+            // kr, kx, kh count the loads issued; each is issued only once its
+            // slot is free, so at most one load per barrier is ever in flight
             uint32_t kr = 0, kx = 0, kh = 0;
             uint32_t units_done = 0;
-            auto ring_slot = [&](uint32_t k) -> uint32_t {
-                const uint32_t s = k % kRing;
-                if (k >= kRing) mbar_wait(bar(B_RING_EMPTY + s), ((k / kRing) - 1) & 1, abort_flag, p.status, 101);
-                return s;
+            auto ring_slot = [&](uint32_t &s) -> bool {
+                s = kr % kRing;
+                return kr < kRing ||
+                       mbar_wait(bar(B_RING_EMPTY + s), ((kr / kRing) - 1) & 1, abort_flag, p.status, 101);
             };
-            auto x_slot = [&](uint32_t k) -> uint32_t {
-                const uint32_t s = k & 1;
-                if (k >= 2) mbar_wait(bar(B_X_EMPTY + s), ((k >> 1) - 1) & 1, abort_flag, p.status, 102);
-                return s;
+            auto x_slot = [&](uint32_t &s) -> bool {
+                s = kx & 1;
+                return kx < 2 || mbar_wait(bar(B_X_EMPTY + s), ((kx >> 1) - 1) & 1, abort_flag, p.status, 102);
             };
-            for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++units_done) {
+            // after an expired wait anywhere in the CTA, no further loads are issued
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++units_done) {
                 const int b = u / p.H, h = u % p.H, gg = h / hpg;
-                for (int i = nt - 1; i >= 0; --i) {       // phase 1: x, B' right to left
-                    const uint32_t xs = x_slot(kx++);
+                for (int i = nt - 1; ok && i >= 0; --i) {   // phase 1: x, B' right to left
+                    uint32_t xs, rs;
+                    if (!(ok = x_slot(xs))) break;
+                    ++kx;
                     mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
                     tma_load_4d_hint(base + S::x0 + xs * kSlab, &tm_x, bar(B_X_FULL + xs), 0, h, i * kTile, b, keep);
-                    const uint32_t rs = ring_slot(kr++);
+                    if (!(ok = ring_slot(rs))) break;
+                    ++kr;
                     mbar_arrive_expect_tx(bar(B_RING_FULL + rs), S::kBC);
                     for (int k = 0; k < NSLAB; ++k)
                         tma_load_5d_hint(base + S::ring + rs * 2 * kSlab + k * kSlab, &tm_b, bar(B_RING_FULL + rs),
                                          64 * k, gg, i * kTile, b, 1, keep);
                 }
-                mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103);
-                for (int i = 0; i < nt; ++i) {            // phase 2: x, C_f, B_f, C_b, B_b, H_b
+                if (!ok || !(ok = mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103))) break;
+                for (int i = 0; ok && i < nt; ++i) {        // phase 2: x, C_f, B_f, C_b, B_b, H_b
                     const int t0 = i * kTile;
-                    const uint32_t xs = x_slot(kx++);
+                    uint32_t xs;
+                    if (!(ok = x_slot(xs))) break;
+                    ++kx;
                     mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
                     tma_load_4d_hint(base + S::x0 + xs * kSlab, &tm_x, bar(B_X_FULL + xs), 0, h, t0, b, stream);
                     const CUtensorMap *maps[4] = {&tm_c, &tm_b, &tm_c, &tm_b};
                     const int dirs[4] = {0, 0, 1, 1};
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t rs = ring_slot(kr++);
+                    for (int j = 0; ok && j < 4; ++j) {
+                        uint32_t rs;
+                        if (!(ok = ring_slot(rs))) break;
+                        ++kr;
                         mbar_arrive_expect_tx(bar(B_RING_FULL + rs), S::kBC);
                         for (int k = 0; k < NSLAB; ++k)
                             tma_load_5d_hint(base + S::ring + rs * 2 * kSlab + k * kSlab, maps[j],
                                              bar(B_RING_FULL + rs), 64 * k, gg, t0, b, dirs[j], stream);
                     }
-                    if (kh >= 1) mbar_wait(bar(B_HB_EMPTY), (kh - 1) & 1, abort_flag, p.status, 104);
+                    if (!ok) break;
+                    if (kh >= 1 && !(ok = mbar_wait(bar(B_HB_EMPTY), (kh - 1) & 1, abort_flag, p.status, 104))) break;
                     ++kh;
                     mbar_arrive_expect_tx(bar(B_HB_FULL), S::kH);
                     tma_load_3d_hint(base + S::hb, &tm_h, bar(B_HB_FULL), 0, 0, u * nt + i, stream);
                 }
             }
+            // every load issued has landed before the CTA may exit (waited on only
+            // after an expired wait, when consumers may have stopped waiting)
+            for (uint32_t k = kr > kRing ? kr - kRing : 0; k < kr; ++k)
+                mbar_drain(bar(B_RING_FULL + k % kRing), (k / kRing) & 1);
+            for (uint32_t k = kx > 2 ? kx - 2 : 0; k < kx; ++k) mbar_drain(bar(B_X_FULL + (k & 1)), (k >> 1) & 1);
+            if (kh >= 1) mbar_drain(bar(B_HB_FULL), (kh - 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -306,11 +328,13 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 return s;
             };
             auto slot_addr = [&](uint32_t s) { return base + S::ring + s * 2 * kSlab; };
-            for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-                for (int i = nt - 1; i >= 0; --i, ++n1) {  // phase 1: S' = B'^T (diag(w') X in the x slot)
+            // after an expired wait anywhere in the CTA, no further tiles are issued
+            for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
+                for (int i = nt - 1; i >= 0 && !*abort_flag; --i, ++n1) {  // phase 1: S' = B'^T (diag(w') X in the x slot)
                     const uint32_t xs = kx++ & 1;
                     const uint32_t rs = wait_ring(kr++);
-                    mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 202);
+                    mbar_wait(bar(B_XW_READY + (n_xw & 1)), (n_xw >> 1) & 1, abort_flag, p.status, 202);
+                    ++n_xw;
                     const uint32_t pb = n1 & 1;
                     if (n1 >= 2) mbar_wait(bar(B_P1S_FREE + pb), ((n1 >> 1) - 1) & 1, abort_flag, p.status, 203);
                     tc_fence_after();
@@ -322,7 +346,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     mma_commit(bar(B_RING_EMPTY + rs));
                     mma_commit(bar(B_X_EMPTY + xs));
                 }
-                for (int i = 0; i < nt; ++i) {             // phase 2
+                for (int i = 0; i < nt && !*abort_flag; ++i) {   // phase 2
                     const uint32_t xs = kx++ & 1;
                     const uint32_t rCf = wait_ring(kr++), rBf = wait_ring(kr++);
                     const uint32_t rCb = wait_ring(kr++), rBb = wait_ring(kr++);
@@ -363,7 +387,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     }
                     mma_commit(bar(B_RING_EMPTY + rCb));
                     mma_commit(bar(B_HB_EMPTY));
-                    mbar_wait(bar(B_XW_READY), n_xw++ & 1, abort_flag, p.status, 208);
+                    mbar_wait(bar(B_XW_READY + (n_xw & 1)), (n_xw >> 1) & 1, abort_flag, p.status, 208);
+                    ++n_xw;
                     tc_fence_after();
                     for (int k = 0; k < kTile / 16; ++k)    // S_f = B_f^T diag(w_f) X
                         mma_bf16_ss(tS, sdesc_sw128(sBf + k * 2048, kSlab, 1024),
@@ -379,25 +404,34 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     mma_commit(bar(B_Y_READY));
                 }
             }
+            // all MMAs complete before TMEM is released
+            mma_commit(bar(B_MMA_DONE));
+            mbar_drain(bar(B_MMA_DONE), 0);
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ group C
         const int row = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
         const uint64_t keep = policy_evict_last();
-        uint32_t kx = 0, n_s = 0, nvec = 0, n1 = 0;
+        uint32_t kx = 0, n_s = 0, nvec = 0, n1 = 0, n_xw = 0;
         float hreg[kP];
         // dt of the step after the current one is fetched a step ahead
-        auto load_dt = [&](int u, int ph, int i, float &vf, float &vb) {
-            vf = 0.f;
-            vb = 0.f;
+        // (issued as volatile loads so the compiler keeps them a step early)
+        uint32_t rawf = 0, rawb = 0;
+        auto load_dt = [&](int u, int ph, int i) {
+            rawf = 0;
+            rawb = 0;
             if (u >= p.units) return;
             const int b = u / p.H, h = u % p.H, t = i * kTile + row;
             if (t < p.L) {
                 const size_t o = ((size_t)b * p.L + t) * p.H + h;
-                vb = __bfloat162float(p.dt[dt_dir + o]);
-                if (ph == 2) vf = __bfloat162float(p.dt[o]);
+                asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawb) : "l"(p.dt + dt_dir + o));
+                if (ph == 2) asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawf) : "l"(p.dt + o));
             }
+        };
+        auto take_dt = [&](float &vf, float &vb) {
+            vf = __uint_as_float(rawf << 16);
+            vb = __uint_as_float(rawb << 16);
         };
         auto next_step = [&](int &u, int &ph, int &i) {
             if (ph == 1) {
@@ -440,8 +474,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             ++n1;
         };
         int cu = blockIdx.x, cph = 1, ci = nt - 1;
-        float nvf, nvb;
-        load_dt(cu, cph, ci, nvf, nvb);
+        load_dt(cu, cph, ci);
         while (cu < p.units) {
             const int u = cu;
             const int h = u % p.H;
@@ -452,9 +485,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             int pend = -1;
             float pend_g = 0.f;
             for (int i = nt - 1; i >= 0; --i) {
-                const float vb = nvb;
+                float vf_unused, vb;
+                take_dt(vf_unused, vb);
                 next_step(cu, cph, ci);
-                load_dt(cu, cph, ci, nvf, nvb);
+                load_dt(cu, cph, ci);
                 float pf = 0.f, pb = vb, totf, totb;
                 scan2(pf, pb, totf, totb, row, red);
                 const float csb = totb - pb + vb;       // suffix sum of dt_b from this row
@@ -465,7 +499,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 scale_row(xt, xt, row, w);
                 fence_proxy_async_smem();
                 sync_c();
-                if (row == 0) mbar_arrive(bar(B_XW_READY));
+                if (row == 0) mbar_arrive(bar(B_XW_READY + (n_xw & 1)));
+                ++n_xw;
                 if (pend >= 0) chain1(u, pend, pend_g);
                 pend = i;
                 pend_g = __expf(Ab * totb);
@@ -485,9 +520,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
             for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
             for (int i = 0; i < nt; ++i) {
-                const float vf = nvf, vb = nvb;
+                float vf, vb;
+                take_dt(vf, vb);
                 next_step(cu, cph, ci);
-                load_dt(cu, cph, ci, nvf, nvb);
+                load_dt(cu, cph, ci);
                 float pf = vf, pb = vb, totf, totb;
                 scan2(pf, pb, totf, totb, row, red);
                 const float csb = totb - pb + vb;
@@ -516,7 +552,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, wf);
                 fence_proxy_async_smem();
                 sync_c();
-                if (row == 0) mbar_arrive(bar(B_XW_READY));
+                if (row == 0) mbar_arrive(bar(B_XW_READY + (n_xw & 1)));
+                ++n_xw;
                 // forward chain: H_f <- exp(A sum dt) H_f + S_f; bf16 copy for C_f.H_f
                 const float gdec = __expf(Af * totf);
                 mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 313);
@@ -551,8 +588,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const bool is_b = warp >= 10;
         const int row = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
-        const int c0 = is_b ? 16 : 0;       // which half of each 32-column block
+        const int c0 = is_b ? 16 : 0;       // which half of each 32-column block, and of the output
         auto sync_g = [&]() { if (is_b) sync_b(); else sync_a(); };
+        auto sync_ab = [&]() { asm volatile("bar.sync 4, 256;" ::: "memory"); };
         uint32_t kx = 0, n_g = 0, n_y = 0, nvec = 0;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             const int b = u / p.H, h = u % p.H;
@@ -587,14 +625,15 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 ++nvec;
                 const uint32_t xs = kx++ & 1;
-                if (!is_b) continue;
-                // group B: output tile over the x slot, then one TMA store
+                // output columns [2 c0, 2 c0 + 32) of the tile over the x slot
+                // (group A the first half, group B the second), then one TMA store
                 mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 403);
                 tc_fence_after();
                 const float ef = __expf(my_af), eb = __expf(my_ab);
                 uint8_t *xt = g + S::x0 + xs * kSlab;
+                const int q0 = c0 >> 3;              // 0 or 2: first 16-column quarter
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
+                for (int q = q0; q < q0 + 2; ++q) {
                     uint32_t yd[16], yf[16], yb[16];
                     tmem_ld16(tYd + lane_off + q * 16, yd);
                     tmem_ld16(tYof + lane_off + q * 16, yf);
@@ -619,8 +658,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                sync_b();
-                if (row == 0) {
+                sync_ab();
+                if (is_b && row == 0) {
                     mbar_arrive(bar(B_Y_FREE));
                     if (!*abort_flag) {
                         tma_store_4d(&tm_out, base + S::x0 + xs * kSlab, 0, h, t0, b);

@@ -189,7 +189,9 @@ __global__ void __launch_bounds__(128) tc_state_kernel(const __grid_constant__ C
     fence_proxy_async_smem();
     __syncthreads();
 
+    bool issued = false;   // thread 0: whether the MMAs were issued
     if (tid == 0 && !*abort_flag) {
+        issued = true;
         tc_fence_after();
         constexpr uint32_t idesc = idesc_bf16_f32(128, 64, true, true);
 #pragma unroll
@@ -223,7 +225,12 @@ __global__ void __launch_bounds__(128) tc_state_kernel(const __grid_constant__ C
                                      __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }
     }
-    if (tid == 0) p.g[entry] = __expf(A * total);
+    if (tid == 0) {
+        p.g[entry] = __expf(A * total);
+        // after an expired wait: the copies and MMAs this CTA started finish first
+        mbar_drain(bar_load, 0);
+        if (issued) mbar_drain(bar_mma, 0);
+    }
     tc_fence_before();
     __syncthreads();
     if (tid < 32) tmem_dealloc(tmem, 64);
@@ -371,7 +378,9 @@ __global__ void __launch_bounds__(128) tc_out_kernel(const __grid_constant__ CUt
 
     mbar_wait(bar_load, 0, abort_flag, p.status, 11);
     __syncthreads();
+    bool issued1 = false, issued2 = false;   // thread 0: which MMA groups were issued
     if (tid == 0 && !*abort_flag) {
+        issued1 = true;
         tc_fence_after();
         constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);
@@ -419,6 +428,7 @@ __global__ void __launch_bounds__(128) tc_out_kernel(const __grid_constant__ CUt
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && !*abort_flag) {
+        issued2 = true;
         tc_fence_after();
         constexpr uint32_t id_y = idesc_bf16_f32(128, 64, false, true);
 #pragma unroll
@@ -470,6 +480,10 @@ __global__ void __launch_bounds__(128) tc_out_kernel(const __grid_constant__ CUt
             tma_store_commit();
         }
         tma_store_wait_all();
+        // after an expired wait: the copies and MMAs this CTA started finish first
+        mbar_drain(bar_load, 0);
+        if (issued1) mbar_drain(bar_mma1, 0);
+        if (issued2) mbar_drain(bar_mma2, 0);
     }
     __syncthreads();
     if (tid < 32) tmem_dealloc(tmem, 512);

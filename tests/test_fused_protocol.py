@@ -1,0 +1,407 @@
+"""Barrier protocol of the fused tensor-core kernel (ssd_fused.cu), checked
+on the CPU.
+
+A discrete-event model of one CTA: the TMA producer, the MMA issuer, the
+prep/state group (C) and the two mask/output groups (A, B), each taking the
+same mbarrier waits and arrivals, named-barrier syncs, TMA loads, MMA commits
+and TMA stores, in the same order, as the kernel. Asynchronous completions
+(TMA loads, MMAs in issue order, the output store's read) land after random,
+heavy-tailed delays, and runnable roles are stepped in random order.
+
+Each schedule is checked for
+  * phase overrun: a barrier completing two phases past the one a role waits
+    for (the hardware parity wait would then miss both),
+  * deadlock: every role blocked with nothing in flight,
+  * data races: every buffer (x slots, the B/C ring, H_b, H_f, diag(w) X, the
+    TMEM accumulators by 16-column block, the per-tile vectors) carries the
+    version its last writer left, and each read names the version it needs.
+
+The model must be kept in step with the kernel when its protocol changes.
+A planted variant with a single diag(w) X barrier (the kernel's earlier
+design, which did overrun on the GPU) must be caught.
+"""
+import heapq
+import itertools
+import random
+
+
+class Bug(Exception):
+    pass
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.c = name, count, count, 0
+    def arrive(self):
+        self.pending -= 1
+        if self.pending < 0:
+            raise Bug(f"{self.name}: too many arrivals")
+        if self.pending == 0:
+            self.c += 1
+            self.pending = self.count
+
+class Sim:
+    def __init__(self, nt, units, seed, kRing=4, xw2=True, heavy=0.1):
+        self.r = random.Random(seed)
+        self.nt, self.units, self.kRing, self.xw2, self.heavy = nt, units, kRing, xw2, heavy
+        self.bars = {}
+        self.res = {}
+        self.t = 0.0
+        self.ev = []          # (time, seq, fn)
+        self.seq = itertools.count()
+        self.mma_done_t = 0.0
+    def bar(self, name, count=1):
+        if name not in self.bars:
+            self.bars[name] = Bar(name, count)
+        return self.bars[name]
+    def delay(self):
+        d = self.r.expovariate(1.0)
+        if self.r.random() < self.heavy:
+            d *= self.r.choice([10, 50, 200])
+        return d
+    def at(self, t, fn):
+        heapq.heappush(self.ev, (t, next(self.seq), fn))
+    def write(self, k, v):
+        self.res[k] = v
+    def read(self, k, v, who):
+        got = self.res.get(k)
+        if got != v:
+            raise Bug(f"{who}: read {k} expected {v} got {got} at t={self.t:.2f}")
+
+# ---------------------------------------------------------------- roles
+# A role is a generator yielding commands:
+#   ('wait', bar, k)      wait for completion of phase k (parity k & 1)
+#   ('arrive', bar)
+#   ('tma', bar, [(res, val)])          async load: writes then arrives
+#   ('mma', [(res,val)] reads, [(res,val)] writes)   in-order async
+#   ('commit', bar)                     arrives when all prior MMAs are done
+#   ('read', res, val) / ('write', res, val)
+#   ('sync', name, n)                   named barrier over n roles
+#   ('store', [(res,val)]) then ('store_wait',)
+
+def producer(S, units_list):
+    nt, R = S.nt, S.kRing
+    kr = kx = kh = 0
+    units_done = 0
+    for u in units_list:
+        for i in range(nt - 1, -1, -1):
+            xs = kx % 2
+            if kx >= 2:
+                yield ('wait', 'X_EMPTY%d' % xs, (kx >> 1) - 1)
+            kx += 1
+            yield ('tma', 'X_FULL%d' % xs, [(('x', xs, 0), ('x', u, 1, i)), (('x', xs, 1), ('x', u, 1, i))])
+            rs = kr % R
+            if kr >= R:
+                yield ('wait', 'RING_EMPTY%d' % rs, kr // R - 1)
+            kr += 1
+            yield ('tma', 'RING_FULL%d' % rs, [(('ring', rs), ('Bb1', u, i))])
+        yield ('wait', 'HB_WRITTEN', units_done)
+        for i in range(nt):
+            xs = kx % 2
+            if kx >= 2:
+                yield ('wait', 'X_EMPTY%d' % xs, (kx >> 1) - 1)
+            kx += 1
+            yield ('tma', 'X_FULL%d' % xs, [(('x', xs, 0), ('x', u, 2, i)), (('x', xs, 1), ('x', u, 2, i))])
+            for name in ('Cf', 'Bf', 'Cb', 'Bb'):
+                rs = kr % R
+                if kr >= R:
+                    yield ('wait', 'RING_EMPTY%d' % rs, kr // R - 1)
+                kr += 1
+                yield ('tma', 'RING_FULL%d' % rs, [(('ring', rs), (name, u, i))])
+            if kh >= 1:
+                yield ('wait', 'HB_EMPTY', kh - 1)
+            kh += 1
+            yield ('tma_hb', 'HB_FULL', u, i)
+        units_done += 1
+
+def mma(S, units_list):
+    nt, R = S.nt, S.kRing
+    kr = kx = kh = n1 = 0
+    n_xw = n_m = n_sfree = n_yfree = 0
+    first2 = True
+    def xw_bar(n):
+        return ('XW_READY%d' % (n & 1)) if S.xw2 else 'XW_READY'
+    def xw_phase(n):
+        return (n >> 1) if S.xw2 else n
+    for u in units_list:
+        for i in range(nt - 1, -1, -1):
+            xs = kx % 2; kx += 1
+            rs = kr % R
+            yield ('wait', 'RING_FULL%d' % rs, kr // R); kr += 1
+            yield ('wait', xw_bar(n_xw), xw_phase(n_xw)); n_xw += 1
+            pb = n1 % 2
+            if n1 >= 2:
+                yield ('wait', 'P1S_FREE%d' % pb, (n1 >> 1) - 1)
+            yield ('mma', [(('ring', rs), ('Bb1', u, i)), (('x', xs, 0), ('xw1', u, i)), (('x', xs, 1), ('xw1', u, i))],
+                   [(('tGf', b), ('S1', u, i)) for b in range(4 * pb, 4 * pb + 4)])
+            yield ('commit', 'P1S_READY%d' % pb)
+            yield ('commit', 'RING_EMPTY%d' % rs)
+            yield ('commit', 'X_EMPTY%d' % xs)
+            n1 += 1
+        for i in range(nt):
+            xs = kx % 2; kx += 1
+            slots = []
+            for name in ('Cf', 'Bf', 'Cb', 'Bb'):
+                rs = kr % R
+                yield ('wait', 'RING_FULL%d' % rs, kr // R); kr += 1
+                slots.append(rs)
+            rCf, rBf, rCb, rBb = slots
+            yield ('mma', [(('ring', rCf), ('Cf', u, i)), (('ring', rBf), ('Bf', u, i))],
+                   [(('tGf', b), ('Gf', u, i)) for b in range(8)])
+            yield ('mma', [(('ring', rCb), ('Cb', u, i)), (('ring', rBb), ('Bb', u, i))],
+                   [(('tGb', b), ('Gb', u, i)) for b in range(8)])
+            yield ('commit', 'G_READY')
+            yield ('commit', 'RING_EMPTY%d' % rBb)
+            if not first2:
+                yield ('wait', 'Y_FREE', n_yfree); n_yfree += 1
+                yield ('wait', 'S_FREE', n_sfree); n_sfree += 1
+            first2 = False
+            yield ('mma', [(('ring', rCf), ('Cf', u, i)), ('hf', ('hf', u, i))], [(('Yof', 0), ('Yof', u, i)), (('Yof', 1), ('Yof', u, i))])
+            yield ('commit', 'RING_EMPTY%d' % rCf)
+            yield ('wait', 'HB_FULL', kh); kh += 1
+            yield ('mma', [(('ring', rCb), ('Cb', u, i)), ('hb', ('hb', u, i))], [(('Yob', 0), ('Yob', u, i)), (('Yob', 1), ('Yob', u, i))])
+            yield ('commit', 'RING_EMPTY%d' % rCb)
+            yield ('commit', 'HB_EMPTY')
+            yield ('wait', xw_bar(n_xw), xw_phase(n_xw)); n_xw += 1
+            yield ('mma', [(('ring', rBf), ('Bf', u, i)), ('xw', ('xw', u, i))], [('S', ('S', u, i))])
+            yield ('commit', 'S_READY')
+            yield ('commit', 'RING_EMPTY%d' % rBf)
+            yield ('wait', 'M_READY', n_m); n_m += 1
+            yield ('wait', 'X_FULL%d' % xs, (kx - 1) >> 1)
+            yield ('mma', [(('tGf', b), ('M', u, i)) for b in range(8)] + [(('x', xs, 0), ('x', u, 2, i)), (('x', xs, 1), ('x', u, 2, i))],
+                   [(('Yd', 0), ('Yd', u, i)), (('Yd', 1), ('Yd', u, i))])
+            yield ('commit', 'Y_READY')
+
+def group_c(S, units_list):
+    nt = S.nt
+    kx = n_s = nvec = n1 = n_xw = 0
+    def xw_bar(n):
+        return ('XW_READY%d' % (n & 1)) if S.xw2 else 'XW_READY'
+    def chain1(u, i):
+        nonlocal n1
+        yield ('write', ('hbg', u, i), ('hbg', u, i))
+        pb = n1 % 2
+        yield ('wait', 'P1S_READY%d' % pb, n1 >> 1)
+        for b in range(4 * pb, 4 * pb + 4):
+            yield ('read', ('tGf', b), ('S1', u, i))
+        yield ('sync', 'c', 1)
+        yield ('arrive', 'P1S_FREE%d' % pb)
+        n1 += 1
+    for u in units_list:
+        pend = None
+        for i in range(nt - 1, -1, -1):
+            xs = kx % 2; kx += 1
+            yield ('wait', 'X_FULL%d' % xs, (kx - 1) >> 1)
+            for hh in (0, 1):
+                yield ('read', ('x', xs, hh), ('x', u, 1, i))
+            for hh in (0, 1):
+                yield ('write', ('x', xs, hh), ('xw1', u, i))
+            yield ('arrive', xw_bar(n_xw)); n_xw += 1
+            if pend is not None:
+                yield from chain1(u, pend)
+            pend = i
+        yield from chain1(u, pend)
+        yield ('write', 'hf', ('hf', u, 0))
+        yield ('arrive', 'HB_WRITTEN')
+        for i in range(nt):
+            vb = nvec % 2
+            if nvec >= 2:
+                yield ('wait', 'VEC_FREE%d' % vb, (nvec >> 1) - 1)
+            yield ('write', ('vec', vb), ('V', u, i))
+            yield ('arrive', 'VEC_READY%d' % vb)
+            nvec += 1
+            xs = kx % 2; kx += 1
+            yield ('wait', 'X_FULL%d' % xs, (kx - 1) >> 1)
+            for hh in (0, 1):
+                yield ('read', ('x', xs, hh), ('x', u, 2, i))
+            yield ('write', 'xw', ('xw', u, i))
+            yield ('arrive', xw_bar(n_xw)); n_xw += 1
+            yield ('wait', 'S_READY', n_s); n_s += 1
+            yield ('read', 'S', ('S', u, i))
+            yield ('write', 'hf', ('hf', u, i + 1))
+            yield ('read', 'S', ('S', u, i))
+            yield ('arrive', 'S_FREE')
+
+def group_ab(S, units_list, is_b):
+    nt = S.nt
+    kx = n_g = n_y = nvec = 0
+    half = 1 if is_b else 0
+    blocks = range(half, 8, 2)
+    for u in units_list:
+        kx += nt
+        for i in range(nt):
+            vb = nvec % 2
+            yield ('wait', 'VEC_READY%d' % vb, nvec >> 1)
+            yield ('read', ('vec', vb), ('V', u, i))
+            yield ('wait', 'G_READY', n_g); n_g += 1
+            for b in blocks:
+                yield ('read', ('tGf', b), ('Gf', u, i))
+                yield ('read', ('tGb', b), ('Gb', u, i))
+            for b in blocks:
+                yield ('write', ('tGf', b), ('M', u, i))
+            yield ('read', ('vec', vb), ('V', u, i))
+            yield ('sync', 'b' if is_b else 'a', 1)
+            yield ('arrive', 'M_READY')
+            yield ('arrive', 'VEC_FREE%d' % vb)
+            nvec += 1
+            xs = kx % 2; kx += 1
+            yield ('wait', 'Y_READY', n_y); n_y += 1
+            for nm in ('Yd', 'Yof', 'Yob'):
+                yield ('read', (nm, half), (nm, u, i))
+            yield ('read', ('x', xs, half), ('x', u, 2, i))
+            yield ('write', ('x', xs, half), ('y', u, i))
+            for nm in ('Yd', 'Yof', 'Yob'):
+                yield ('read', (nm, half), (nm, u, i))
+            yield ('sync', 'ab', 2)
+            if is_b:
+                yield ('arrive', 'Y_FREE')
+                yield ('store', [(('x', xs, 0), ('y', u, i)), (('x', xs, 1), ('y', u, i))])
+                yield ('store_wait',)
+                yield ('arrive', 'X_EMPTY%d' % xs)
+
+def run(S, units_list):
+    counts = {'M_READY': 2, 'VEC_FREE0': 2, 'VEC_FREE1': 2}
+    roles = {
+        'prod': producer(S, units_list), 'mma': mma(S, units_list), 'C': group_c(S, units_list),
+        'A': group_ab(S, units_list, False), 'B': group_ab(S, units_list, True),
+    }
+    cur = {k: None for k in roles}        # pending command per role
+    ready = {k: 0.0 for k in roles}
+    done = set()
+    syncs = {}                            # name -> set of roles arrived
+    store_pending = {}
+    def bar(n):
+        return S.bar(n, counts.get(n, 1))
+    def step_role(name):
+        """Try to make progress on role `name`; return True if it advanced."""
+        if cur[name] is None:
+            try:
+                cur[name] = next(roles[name])
+            except StopIteration:
+                done.add(name)
+                return True
+        c = cur[name]
+        op = c[0]
+        if op == 'wait':
+            b = bar(c[1]); k = c[2]
+            if b.c >= k + 2:
+                raise Bug(f"{name}: overrun on {c[1]}: waiting for phase {k}, completed {b.c}")
+            if (b.c & 1) != (k & 1):     # the phase with parity k&1 completed (c == k+1)
+                cur[name] = None
+                return True
+            return False
+        if op == 'arrive':
+            bar(c[1]).arrive()
+        elif op == 'tma':
+            bn, writes = c[1], c[2]
+            def land(writes=writes, bn=bn):
+                for k, v in writes:
+                    S.write(k, v)
+                bar(bn).arrive()
+            S.at(S.t + S.delay(), land)
+        elif op == 'tma_hb':
+            bn, u, i = c[1], c[2], c[3]
+            S.read(('hbg', u, i), ('hbg', u, i), name + ' hb load issue')
+            def land(bn=bn, u=u, i=i):
+                S.write('hb', ('hb', u, i))
+                bar(bn).arrive()
+            S.at(S.t + S.delay(), land)
+        elif op == 'mma':
+            reads, writes = c[1], c[2]
+            tdone = max(S.mma_done_t, S.t) + S.delay()
+            S.mma_done_t = tdone
+            def ex(reads=reads, writes=writes):
+                for k, v in reads:
+                    S.read(k, v, 'mma exec')
+                for k, v in writes:
+                    S.write(k, v)
+            S.at(tdone, ex)
+        elif op == 'commit':
+            bn = c[1]
+            S.at(max(S.mma_done_t, S.t) + 1e-6, lambda bn=bn: bar(bn).arrive())
+        elif op == 'read':
+            S.read(c[1], c[2], name)
+        elif op == 'write':
+            S.write(c[1], c[2])
+        elif op == 'sync':
+            nm, n = c[1], c[2]
+            if n == 1:
+                pass
+            else:
+                s = syncs.setdefault(nm, set())
+                s.add(name)
+                if len(s) < n:
+                    return False
+                # all arrived: release the others lazily
+                for other in list(s):
+                    if other != name and cur[other] == c:
+                        cur[other] = None
+                syncs[nm] = set()
+        elif op == 'store':
+            for k, v in c[1]:
+                S.read(k, v, 'store issue')
+            tr = S.t + S.delay()
+            store_pending[name] = (tr, c[1])
+            def rd(items=c[1]):
+                for k, v in items:
+                    S.read(k, v, 'store read')
+            S.at(tr, rd)
+        elif op == 'store_wait':
+            tr, _ = store_pending[name]
+            if S.t < tr:
+                return False
+        cur[name] = None
+        return True
+    while len(done) < len(roles):
+        progressed = True
+        while progressed:
+            progressed = False
+            order = [r for r in roles if r not in done]
+            S.r.shuffle(order)
+            for r in order:
+                if r in done or ready[r] > S.t:
+                    continue
+                # a sync waiter whose partner already released it
+                if step_role(r):
+                    ready[r] = S.t + (S.r.expovariate(4.0) if S.r.random() < 0.5 else 0.0)
+                    progressed = True
+        if len(done) == len(roles):
+            break
+        nxt = [ready[r] for r in roles if r not in done and ready[r] > S.t]
+        tnext = min(nxt) if nxt else None
+        if S.ev and (tnext is None or S.ev[0][0] <= tnext):
+            t, _, fn = heapq.heappop(S.ev)
+            S.t = max(S.t, t)
+            fn()
+        elif tnext is not None:
+            S.t = tnext
+        else:
+            state = {r: cur[r] for r in roles if r not in done}
+            raise Bug(f"deadlock at t={S.t:.2f}: {state}")
+    while S.ev:
+        t, _, fn = heapq.heappop(S.ev)
+        S.t = t
+        fn()
+
+
+def _schedules(n, xw2, seed0=0):
+    fails = []
+    for seed in range(seed0, seed0 + n):
+        r = random.Random(seed)
+        nt = r.choice([1, 2, 3, 4, 5])
+        nunits = r.choice([1, 2, 3])
+        S = Sim(nt, nunits, seed, xw2=xw2, heavy=r.choice([0.0, 0.05, 0.2, 0.5]))
+        try:
+            run(S, list(range(nunits)))
+        except Bug as e:
+            fails.append(f"seed {seed} nt {nt} units {nunits}: {e}")
+    return fails
+
+
+def test_fused_protocol_has_no_overrun_deadlock_or_race():
+    fails = _schedules(1200, xw2=True)
+    assert not fails, "\n".join(fails[:5])
+
+
+def test_model_catches_single_diag_w_x_barrier():
+    fails = _schedules(100, xw2=False)
+    assert fails and any("overrun on XW_READY" in f for f in fails)

@@ -37,8 +37,16 @@ DEFAULT_WORKLOAD = "mixer130m_b32_L1024"
 PATH_IDS = {"auto": 0, "simt": 1, "chunked": 2, "fused": 3}
 # kernels each path launches per ssd_bidir_fwd call (bf16)
 LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1}
-# source file holding the kernel each path spends its time in
-KERNEL_SOURCE = {"simt": "ssd_simt.cu", "chunked": "ssd_tc.cu", "fused": "ssd_tc.cu"}
+# sources each path's kernels compile from (a traffic record is valid only
+# while their hash is unchanged)
+KERNEL_SOURCE = {
+    "simt": ("ssd_simt.cu", "ssd_common.cuh"),
+    "chunked": ("ssd_tc.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
+    "fused": ("ssd_fused.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
+}
+# name of the kernel each path spends its time in (found in ncu's "Kernel Name")
+KERNEL_NAME = {"simt": "scan_simt_kernel", "chunked": "tc_out_kernel", "fused": "tc_fused_kernel"}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def rank_seed(rank: int) -> int:
@@ -81,22 +89,54 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
+def kernel_source_sha(path: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCE[path]:
+        with open(os.path.join(ROOT, "bidirectional_mamba_ssd_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_record(path: str, workload: str):
     """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
     if it was taken on the current kernel source (else None)."""
-    rec = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(rec):
+    if not os.path.exists(TRAFFIC_FILE):
         return None
-    with open(rec) as f:
+    with open(TRAFFIC_FILE) as f:
         d = json.load(f)
     e = d.get(f"{workload}:{path}")
-    if not e:
-        return None
-    src = os.path.join(ROOT, "bidirectional_mamba_ssd_b200", "csrc", KERNEL_SOURCE[path])
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if e.get("source_sha") != sha:
+    if not e or e.get("source_sha") != kernel_source_sha(path):
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def record_traffic(csv_path: str, path: str, workload: str, command: str):
+    """Store dram__bytes_read.sum + dram__bytes_write.sum per launch of the
+    path's dominant kernel, from `ncu -i <report> --page raw --csv` output."""
+    import csv
+    with open(csv_path, newline="") as f:
+        rows = list(csv.reader(f))
+    head, units = rows[0], rows[1]
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    col = {m: head.index(m) for m in ("Kernel Name", "dram__bytes_read.sum", "dram__bytes_write.sum")}
+    per = []
+    for r in rows[2:]:
+        if KERNEL_NAME[path] + "<" in r[col["Kernel Name"]] or KERNEL_NAME[path] + "(" in r[col["Kernel Name"]]:
+            per.append(sum(float(r[col[m]].replace(",", "")) * scale[units[col[m]]]
+                           for m in ("dram__bytes_read.sum", "dram__bytes_write.sum")))
+    if not per:
+        raise SystemExit(f"no {KERNEL_NAME[path]} launch in {csv_path}")
+    d = {}
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    d[f"{workload}:{path}"] = {"dram_bytes_per_launch": round(sum(per) / len(per)),
+                               "launches": len(per), "kernel": KERNEL_NAME[path],
+                               "source_sha": kernel_source_sha(path), "command": command}
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(d, f, indent=1, sort_keys=True)
+        f.write("\n")
+    print(json.dumps(d[f"{workload}:{path}"]))
 
 
 class ClockSampler:
@@ -300,7 +340,16 @@ def main():
     ap.add_argument("--path", default="auto", choices=list(PATH_IDS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--record-traffic", metavar="CSV",
+                    help="store the dominant kernel's DRAM bytes per launch from an ncu raw CSV "
+                         "(with --path and --workload; --capture-command names the capture) and exit")
+    ap.add_argument("--capture-command", default="")
     args = ap.parse_args()
+    if args.record_traffic:
+        if args.path == "auto":
+            ap.error("--record-traffic needs an explicit --path")
+        record_traffic(args.record_traffic, args.path, args.workload, args.capture_command)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

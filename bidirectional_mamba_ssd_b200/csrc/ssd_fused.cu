@@ -94,7 +94,8 @@ enum {
     B_Y_FREE,                        // group B -> MMA
     B_VEC_READY,                     // 2: group C -> groups A and B, per vector buffer
     B_VEC_FREE = B_VEC_READY + 2,    // 2: groups A and B -> group C (count 2)
-    B_MMA_DONE = B_VEC_FREE + 2,     // MMA issuer, at teardown
+    B_G1_READY = B_VEC_FREE + 2,     // 4: groups A/B -> group C, reverse-pass tile decay per buffer
+    B_MMA_DONE = B_G1_READY + 4,     // MMA issuer, at teardown
     B_COUNT
 };
 
@@ -188,6 +189,26 @@ __device__ __forceinline__ void scan2(float &a, float &b, float &ta, float &tb, 
     b += pb;
 }
 
+// Inclusive prefix sum of `a` over the 128 rows of an epilogue group and the
+// group's total, with `sync` the group's named barrier and `red` 4 floats of
+// the group's own scratch.
+template <typename Sync>
+__device__ __forceinline__ void scan1(float &a, float &ta, int row, float *red, Sync sync) {
+    const int lane = row & 31, wq = row >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float na = __shfl_up_sync(0xffffffffu, a, o);
+        if (lane >= o) a += na;
+    }
+    if (lane == 31) red[wq] = a;
+    sync();
+    float pa = 0.f;
+    for (int k = 0; k < wq; ++k) pa += red[k];
+    ta = (red[0] + red[1]) + (red[2] + red[3]);
+    sync();
+    a += pa;
+}
+
 template <int N>
 struct Smem {
     static constexpr uint32_t kBC = N * 256;            // one B or C tile (N/64 slabs)
@@ -214,6 +235,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
+    static_assert(8 * B_COUNT + 8 <= 320, "barrier area");
+    float *gdec1 = reinterpret_cast<float *>(g + S::small + 320);  // 4 reverse-pass tile decays
+    float *red_ab = reinterpret_cast<float *>(g + S::small + 352); // 2 x 4 floats, groups A and B scans
     float *red = reinterpret_cast<float *>(g + S::small + 384);    // 8 floats, group C scans
     TileVec *vec = reinterpret_cast<TileVec *>(g + S::small + 512);  // 2 buffers
 
@@ -415,10 +439,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const uint64_t keep = policy_evict_last();
         uint32_t kx = 0, n_s = 0, nvec = 0, n1 = 0, n_xw = 0;
         float hreg[kP];
-        // dt of the step after the current one is fetched a step ahead
-        // (issued as volatile loads so the compiler keeps them a step early)
+        // dt of the next output-pass tile is fetched a tile ahead (volatile
+        // loads, so the compiler keeps them a tile early)
         uint32_t rawf = 0, rawb = 0;
-        auto load_dt = [&](int u, int ph, int i) {
+        auto load_dt = [&](int u, int i) {
             rawf = 0;
             rawb = 0;
             if (u >= p.units) return;
@@ -426,86 +450,56 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if (t < p.L) {
                 const size_t o = ((size_t)b * p.L + t) * p.H + h;
                 asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawb) : "l"(p.dt + dt_dir + o));
-                if (ph == 2) asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawf) : "l"(p.dt + o));
+                asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawf) : "l"(p.dt + o));
             }
         };
         auto take_dt = [&](float &vf, float &vb) {
             vf = __uint_as_float(rawf << 16);
             vb = __uint_as_float(rawb << 16);
         };
-        auto next_step = [&](int &u, int &ph, int &i) {
-            if (ph == 1) {
-                if (i > 0) --i;
-                else { ph = 2; i = 0; }
-            } else if (i < nt - 1) {
-                ++i;
-            } else {
-                u += gridDim.x; ph = 1; i = nt - 1;
-            }
-        };
-        // one phase-1 chain step: store the state entering tile i, then fold in its tile state
-        auto chain1 = [&](int u, int i, float gdec) {
-            if (row < N) {
-                __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 v = make_uint4(pack_bf16x2(hreg[8 * c], hreg[8 * c + 1]),
-                                         pack_bf16x2(hreg[8 * c + 2], hreg[8 * c + 3]),
-                                         pack_bf16x2(hreg[8 * c + 4], hreg[8 * c + 5]),
-                                         pack_bf16x2(hreg[8 * c + 6], hreg[8 * c + 7]));
-                    st_global_v4_hint(dst + 8 * c, v, keep);
-                }
-            }
-            const uint32_t pbuf = n1 & 1;
-            mbar_wait(bar(B_P1S_READY + pbuf), (n1 >> 1) & 1, abort_flag, p.status, 301);
-            tc_fence_after();
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t v[32];
-                tmem_ld32(tGf + 64 * pbuf + lane_off + half * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
-            }
-            tc_fence_before();
-            sync_c();
-            if (row == 0) mbar_arrive(bar(B_P1S_FREE + pbuf));
-            ++n1;
-        };
-        int cu = blockIdx.x, cph = 1, ci = nt - 1;
-        load_dt(cu, cph, ci);
+        int cu = blockIdx.x, ci = 0;   // the output-pass tile whose dt is in flight
+        load_dt(cu, ci);
         while (cu < p.units) {
             const int u = cu;
             const int h = u % p.H;
             const float Af = p.A[h], Ab = p.A[p.H + h];
-            // ---------------- phase 1: reverse tile sums, diag(w') X in place, reverse chain
+            // ---------------- phase 1: the reverse chain, right to left. Groups A
+            // and B prepare the tiles (diag(w') X, tile decay); this group stores
+            // the state entering each tile and folds the tile's state in.
 #pragma unroll
             for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
-            int pend = -1;
-            float pend_g = 0.f;
-            for (int i = nt - 1; i >= 0; --i) {
-                float vf_unused, vb;
-                take_dt(vf_unused, vb);
-                next_step(cu, cph, ci);
-                load_dt(cu, cph, ci);
-                float pf = 0.f, pb = vb, totf, totb;
-                scan2(pf, pb, totf, totb, row, red);
-                const float csb = totb - pb + vb;       // suffix sum of dt_b from this row
-                const float w = __expf(Ab * (totb - csb)) * vb;   // exp(A' sum_{r<s} dt') dt'_s
-                const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 302);
-                uint8_t *xt = g + S::x0 + xs * kSlab;
-                scale_row(xt, xt, row, w);
-                fence_proxy_async_smem();
+            for (int i = nt - 1; i >= 0; --i, ++n1) {
+                if (row < N) {
+                    __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 v = make_uint4(pack_bf16x2(hreg[8 * c], hreg[8 * c + 1]),
+                                             pack_bf16x2(hreg[8 * c + 2], hreg[8 * c + 3]),
+                                             pack_bf16x2(hreg[8 * c + 4], hreg[8 * c + 5]),
+                                             pack_bf16x2(hreg[8 * c + 6], hreg[8 * c + 7]));
+                        st_global_v4_hint(dst + 8 * c, v, keep);
+                    }
+                }
+                const uint32_t pbuf = n1 & 1;
+                mbar_wait(bar(B_G1_READY + (n1 & 3)), (n1 >> 2) & 1, abort_flag, p.status, 303);
+                const float gdec = gdec1[n1 & 3];
+                mbar_wait(bar(B_P1S_READY + pbuf), (n1 >> 1) & 1, abort_flag, p.status, 301);
+                tc_fence_after();
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t v[32];
+                    tmem_ld32(tGf + 64 * pbuf + lane_off + half * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        hreg[half * 32 + j] = fmaf(gdec, hreg[half * 32 + j], __uint_as_float(v[j]));
+                }
+                tc_fence_before();
                 sync_c();
-                if (row == 0) mbar_arrive(bar(B_XW_READY + (n_xw & 1)));
-                ++n_xw;
-                if (pend >= 0) chain1(u, pend, pend_g);
-                pend = i;
-                pend_g = __expf(Ab * totb);
+                if (row == 0) mbar_arrive(bar(B_P1S_FREE + pbuf));
             }
-            chain1(u, pend, pend_g);
+            kx += nt;        // the reverse pass's x loads and diag(w') X releases
+            n_xw += nt;      // belong to groups A and B
             // phase 2 starts from H_f = 0; the reverse states go to the TMA proxy
             if (row < N) {
                 uint4 *hf = reinterpret_cast<uint4 *>(g + S::hf + row * 128);
@@ -522,8 +516,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             for (int i = 0; i < nt; ++i) {
                 float vf, vb;
                 take_dt(vf, vb);
-                next_step(cu, cph, ci);
-                load_dt(cu, cph, ci);
+                if (++ci == nt) { ci = 0; cu += gridDim.x; }
+                load_dt(cu, ci);
                 float pf = vf, pb = vb, totf, totb;
                 scan2(pf, pb, totf, totb, row, red);
                 const float csb = totb - pb + vb;
@@ -591,11 +585,52 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const int c0 = is_b ? 16 : 0;       // which half of each 32-column block, and of the output
         auto sync_g = [&]() { if (is_b) sync_b(); else sync_a(); };
         auto sync_ab = [&]() { asm volatile("bar.sync 4, 256;" ::: "memory"); };
-        uint32_t kx = 0, n_g = 0, n_y = 0, nvec = 0;
+        uint32_t kx = 0, n_g = 0, n_y = 0, nvec = 0, m1 = 0;
+        float *red_g = red_ab + (is_b ? 4 : 0);
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             const int b = u / p.H, h = u % p.H;
             const float dsum = p.D[h] + p.D[p.H + h];
-            kx += nt;                        // phase 1 uses the x slots without these groups
+            const float Ab = p.A[p.H + h];
+            // ---------------- phase 1: every other reverse-pass tile (by the CTA's
+            // running tile count m1: group A the even ones, group B the odd ones):
+            // w'_s = exp(A' sum_{r<s} dt'_r) dt'_s, diag(w') X in place in the x
+            // slot, and the tile decay exp(A' sum dt') for group C's chain.
+            uint32_t rawn = 0;               // dt' of this group's next tile, fetched a tile ahead
+            bool have = false;
+            for (int i = nt - 1; i >= 0; --i, ++m1, ++kx) {
+                if ((m1 & 1) != (uint32_t)is_b) continue;
+                float vb = 0.f;
+                if (have) {
+                    vb = bf2f(rawn);
+                } else {
+                    const int t = i * kTile + row;
+                    if (t < p.L) vb = __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]);
+                }
+                have = i >= 2;
+                rawn = 0;
+                if (have) {
+                    const int t = (i - 2) * kTile + row;
+                    if (t < p.L) {
+                        const size_t o = dt_dir + ((size_t)b * p.L + t) * p.H + h;
+                        asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawn) : "l"(p.dt + o));
+                    }
+                }
+                float pb = vb, totb;
+                scan1(pb, totb, row, red_g, sync_g);
+                const float w = __expf(Ab * (pb - vb)) * vb;
+                const uint32_t xs = kx & 1;
+                mbar_wait(bar(B_X_FULL + xs), (kx >> 1) & 1, abort_flag, p.status, 404);
+                uint8_t *xt = g + S::x0 + xs * kSlab;
+                scale_row(xt, xt, row, w);
+                fence_proxy_async_smem();
+                if (row == 0) gdec1[m1 & 3] = __expf(Ab * totb);
+                sync_g();
+                if (row == 0) {
+                    mbar_arrive(bar(B_XW_READY + (kx & 1)));
+                    mbar_arrive(bar(B_G1_READY + (m1 & 3)));
+                }
+            }
+            // ---------------- phase 2: masked matrix halves and output halves
             for (int i = 0; i < nt; ++i) {
                 const int t0 = i * kTile;
                 const uint32_t vb_i = nvec & 1;
@@ -606,13 +641,22 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 tc_fence_after();
                 {
                     const MaskVectors mv{V.af, V.ab, V.dtf, V.dtb, V.colf, V.colb};
+                    const int wq = warp & 3;        // this warp's row block
 #pragma unroll 1
                     for (int J = 0; J < 4; ++J) {
-                        uint32_t gf[16], gb[16], packed[8];
-                        tmem_ld16(tGf + lane_off + J * 32 + c0, gf);
-                        tmem_ld16(tGb + lane_off + J * 32 + c0, gb);
-                        tmem_wait_ld();
-                        mask_cols<16>(J, c0, row, my_af, my_ab, gf, gb, mv, packed);
+                        uint32_t packed[8];
+                        if (J != wq) {              // one direction: only its G is read
+                            uint32_t g[16];
+                            tmem_ld16((J < wq ? tGf : tGb) + lane_off + J * 32 + c0, g);
+                            tmem_wait_ld();
+                            mask_offdiag<16>(J, c0, row, my_af, my_ab, g, mv, packed);
+                        } else {
+                            uint32_t gf[16], gb[16];
+                            tmem_ld16(tGf + lane_off + J * 32 + c0, gf);
+                            tmem_ld16(tGb + lane_off + J * 32 + c0, gb);
+                            tmem_wait_ld();
+                            mask_diag<16>(J, c0, row, my_af, my_ab, gf, gb, mv, packed);
+                        }
                         tmem_st8(tGf + lane_off + J * 32 + c0, packed);
                     }
                 }

@@ -14,7 +14,8 @@
 //   reverse:  exp(a'_t - a'_s) = exp(a'_t - a'_b) * exp(a'_b - a'_s), b = first column of J
 // so a row needs one exp per block and the per-column factors
 //   colf[s] = exp(a_e - a_s) dt_f[s],  colb[s] = exp(a'_b - a'_s) dt_b[s]
-// are shared by all rows. On the diagonal block each entry takes its own exp.
+// are shared by all rows. The diagonal block factorises the same way while its
+// decay span is moderate (mask_diag).
 #pragma once
 
 #include <stdint.h>
@@ -29,73 +30,97 @@ struct MaskVectors {
     const float *colf, *colb;   // per-column factors (see above)
 };
 
-// Columns [32 J + c0, 32 J + c0 + W) of row `row` (W = 16 or 32, c0 = 0 or
-// 16 with W = 16), packed as W/2 bf16 pairs.
+// Largest decay span, within one 32-column block, for which the diagonal
+// block is evaluated in factorised form: the row factor is then at most
+// e^kMaxSpan and the column factor at least e^-kMaxSpan dt, both far inside
+// fp32's range.
+constexpr float kMaxSpan = 60.f;
+
+// Off the diagonal: columns [32 J + c0, 32 J + c0 + W) of row `row` (W = 16 or
+// 32, c0 = 0 or 16 with W = 16) for a column block J other than the row's own,
+// packed as W/2 bf16 pairs. `g` holds the one G these columns need: the
+// forward G_f when J is left of the row (J < row / 32), else the reverse G_b.
+// Both directions share one code path (row factor and column factors picked
+// by direction), so it stays in the instruction cache.
 template <int W>
-__device__ __forceinline__ void mask_cols(int J, int c0, int row, float my_af, float my_ab,
+__device__ __forceinline__ void mask_offdiag(int J, int c0, int row, float my_af, float my_ab,
+                                             const uint32_t (&g)[W], const MaskVectors &v,
+                                             uint32_t (&packed)[W / 2]) {
+    const bool fwd = J < (row >> 5);
+    const int s0 = J * 32;
+    const float r = __expf(fwd ? my_af - v.af[s0 + 31] : my_ab - v.ab[s0]);
+    const float *col = (fwd ? v.colf : v.colb) + s0 + c0;
+    float m[W];
+#pragma unroll
+    for (int q = 0; q < W; q += 4) {
+        const float4 c = *reinterpret_cast<const float4 *>(col + q);
+        m[q + 0] = __uint_as_float(g[q + 0]) * (r * c.x);
+        m[q + 1] = __uint_as_float(g[q + 1]) * (r * c.y);
+        m[q + 2] = __uint_as_float(g[q + 2]) * (r * c.z);
+        m[q + 3] = __uint_as_float(g[q + 3]) * (r * c.w);
+    }
+#pragma unroll
+    for (int q = 0; q < W / 2; ++q) packed[q] = sm100::pack_bf16x2(m[2 * q], m[2 * q + 1]);
+}
+
+// The diagonal block (J = row / 32): columns [32 J + c0, 32 J + c0 + W) of
+// row `row`. Column s is left of the row (forward term only), right of it
+// (reverse term only) or the row's own token (both, decay 1). The decay
+// factorises through the block's edges as off the diagonal, now with a row
+// factor >= 1 and a column factor <= 1:
+//   exp(a_t - a_s)   = exp(a_t - a_e)   * exp(a_e - a_s),     e = last column
+//   exp(a'_t - a'_s) = exp(a'_t - a'_b) * exp(a'_b - a'_s),   b = first column
+// which is exact in fp32 while the block's decay span stays below kMaxSpan;
+// past that (a warp-uniform test) each entry takes its own exponential.
+template <int W>
+__device__ __forceinline__ void mask_diag(int J, int c0, int row, float my_af, float my_ab,
                                           const uint32_t (&gf)[W], const uint32_t (&gb)[W],
                                           const MaskVectors &v, uint32_t (&packed)[W / 2]) {
-    const int wq = row >> 5;
     const int s0 = J * 32;
     const int s1 = s0 + c0;
+    const int rr = row - s1;   // this row's position relative to the first column
     float m[W];
-    if (J < wq) {
-        const float rf = __expf(my_af - v.af[s0 + 31]);
+    const float span_f = v.af[s0] - v.af[s0 + 31], span_b = v.ab[s0 + 31] - v.ab[s0];
+    if (span_f < kMaxSpan && span_b < kMaxSpan) {
+        const float rf = __expf(my_af - v.af[s0 + 31]), rb = __expf(my_ab - v.ab[s0]);
 #pragma unroll
         for (int q = 0; q < W; q += 4) {
-            const float4 c = *reinterpret_cast<const float4 *>(v.colf + s1 + q);
-            m[q + 0] = __uint_as_float(gf[q + 0]) * (rf * c.x);
-            m[q + 1] = __uint_as_float(gf[q + 1]) * (rf * c.y);
-            m[q + 2] = __uint_as_float(gf[q + 2]) * (rf * c.z);
-            m[q + 3] = __uint_as_float(gf[q + 3]) * (rf * c.w);
-        }
-    } else if (J > wq) {
-        const float rb = __expf(my_ab - v.ab[s0]);
-#pragma unroll
-        for (int q = 0; q < W; q += 4) {
-            const float4 c = *reinterpret_cast<const float4 *>(v.colb + s1 + q);
-            m[q + 0] = __uint_as_float(gb[q + 0]) * (rb * c.x);
-            m[q + 1] = __uint_as_float(gb[q + 1]) * (rb * c.y);
-            m[q + 2] = __uint_as_float(gb[q + 2]) * (rb * c.z);
-            m[q + 3] = __uint_as_float(gb[q + 3]) * (rb * c.w);
-        }
-    } else {
-        // diagonal block: column s is either left of the row (forward term
-        // only), right of it (reverse term only) or the row's own token (both,
-        // decay 1), so one exp per entry
-        const int rr = row - s1;   // this row's position relative to the first column
-#pragma unroll
-        for (int q = 0; q < W; q += 4) {
-            const float4 af4 = *reinterpret_cast<const float4 *>(v.af + s1 + q);
-            const float4 ab4 = *reinterpret_cast<const float4 *>(v.ab + s1 + q);
+            const float4 cf4 = *reinterpret_cast<const float4 *>(v.colf + s1 + q);
+            const float4 cb4 = *reinterpret_cast<const float4 *>(v.colb + s1 + q);
             const float4 df4 = *reinterpret_cast<const float4 *>(v.dtf + s1 + q);
             const float4 db4 = *reinterpret_cast<const float4 *>(v.dtb + s1 + q);
-            const float afs[4] = {af4.x, af4.y, af4.z, af4.w};
-            const float abs_[4] = {ab4.x, ab4.y, ab4.z, ab4.w};
-            const float dfs[4] = {df4.x, df4.y, df4.z, df4.w};
-            const float dbs[4] = {db4.x, db4.y, db4.z, db4.w};
+            const float cfs[4] = {cf4.x, cf4.y, cf4.z, cf4.w}, cbs[4] = {cb4.x, cb4.y, cb4.z, cb4.w};
+            const float dfs[4] = {df4.x, df4.y, df4.z, df4.w}, dbs[4] = {db4.x, db4.y, db4.z, db4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int c = q + e;
-                const bool fwd = c < rr, rev = c > rr;
                 const float gfv = __uint_as_float(gf[c]), gbv = __uint_as_float(gb[c]);
-                // the exponent of the selected side is <= 0; the other side is
-                // never used, so its possible overflow is harmless
-                const float x = __expf(fwd ? my_af - afs[e] : my_ab - abs_[e]);
-                const float wv = fwd ? gfv * dfs[e] : gbv * dbs[e];
-                m[c] = (fwd || rev) ? wv * x : gfv * dfs[e] + gbv * dbs[e];
+                m[c] = c < rr ? gfv * (rf * cfs[e]) : c > rr ? gbv * (rb * cbs[e]) : gfv * dfs[e] + gbv * dbs[e];
             }
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < W; ++c) {
+            const int s = s1 + c;
+            const float gfv = __uint_as_float(gf[c]), gbv = __uint_as_float(gb[c]);
+            // the exponent of the selected side is <= 0
+            m[c] = c < rr ? gfv * v.dtf[s] * __expf(my_af - v.af[s])
+                 : c > rr ? gbv * v.dtb[s] * __expf(my_ab - v.ab[s])
+                          : gfv * v.dtf[s] + gbv * v.dtb[s];
         }
     }
 #pragma unroll
     for (int q = 0; q < W / 2; ++q) packed[q] = sm100::pack_bf16x2(m[2 * q], m[2 * q + 1]);
 }
 
-// Columns [32 J, 32 J + 32) of row `row`, packed as 16 bf16 pairs.
+// Columns [32 J, 32 J + 32) of row `row` given both G blocks, packed as 16 bf16 pairs.
 __device__ __forceinline__ void mask_block(int J, int row, float my_af, float my_ab,
                                            const uint32_t (&gf)[32], const uint32_t (&gb)[32],
                                            const MaskVectors &v, uint32_t (&packed)[16]) {
-    mask_cols<32>(J, 0, row, my_af, my_ab, gf, gb, v, packed);
+    const int wq = row >> 5;
+    if (J < wq) mask_offdiag<32>(J, 0, row, my_af, my_ab, gf, v, packed);
+    else if (J > wq) mask_offdiag<32>(J, 0, row, my_af, my_ab, gb, v, packed);
+    else mask_diag<32>(J, 0, row, my_af, my_ab, gf, gb, v, packed);
 }
 
 // Per-column factors of column s (call once per column, before mask_block).

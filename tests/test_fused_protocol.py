@@ -2,7 +2,8 @@
 on the CPU.
 
 A discrete-event model of one CTA: the TMA producer, the MMA issuer, the
-prep/state group (C) and the two mask/output groups (A, B), each taking the
+state-chain group (C) and the two mask/output groups (A, B, which also prepare
+the reverse pass's tiles, alternately), each taking the
 same mbarrier waits and arrivals, named-barrier syncs, TMA loads, MMA commits
 and TMA stores, in the same order, as the kernel. Asynchronous completions
 (TMA loads, MMAs in issue order, the output store's read) land after random,
@@ -176,30 +177,21 @@ def group_c(S, units_list):
     kx = n_s = nvec = n1 = n_xw = 0
     def xw_bar(n):
         return ('XW_READY%d' % (n & 1)) if S.xw2 else 'XW_READY'
-    def chain1(u, i):
-        nonlocal n1
-        yield ('write', ('hbg', u, i), ('hbg', u, i))
-        pb = n1 % 2
-        yield ('wait', 'P1S_READY%d' % pb, n1 >> 1)
-        for b in range(4 * pb, 4 * pb + 4):
-            yield ('read', ('tGf', b), ('S1', u, i))
-        yield ('sync', 'c', 1)
-        yield ('arrive', 'P1S_FREE%d' % pb)
-        n1 += 1
     for u in units_list:
-        pend = None
+        # phase 1: the reverse chain only (groups A and B prepare the tiles)
         for i in range(nt - 1, -1, -1):
-            xs = kx % 2; kx += 1
-            yield ('wait', 'X_FULL%d' % xs, (kx - 1) >> 1)
-            for hh in (0, 1):
-                yield ('read', ('x', xs, hh), ('x', u, 1, i))
-            for hh in (0, 1):
-                yield ('write', ('x', xs, hh), ('xw1', u, i))
-            yield ('arrive', xw_bar(n_xw)); n_xw += 1
-            if pend is not None:
-                yield from chain1(u, pend)
-            pend = i
-        yield from chain1(u, pend)
+            yield ('write', ('hbg', u, i), ('hbg', u, i))
+            pb = n1 % 2
+            yield ('wait', 'G1_READY%d' % (n1 & 3), n1 >> 2)
+            yield ('read', ('gdec', n1 & 3), ('g', u, i))
+            yield ('wait', 'P1S_READY%d' % pb, n1 >> 1)
+            for b in range(4 * pb, 4 * pb + 4):
+                yield ('read', ('tGf', b), ('S1', u, i))
+            yield ('sync', 'c', 1)
+            yield ('arrive', 'P1S_FREE%d' % pb)
+            n1 += 1
+        kx += nt
+        n_xw += nt
         yield ('write', 'hf', ('hf', u, 0))
         yield ('arrive', 'HB_WRITTEN')
         for i in range(nt):
@@ -223,11 +215,27 @@ def group_c(S, units_list):
 
 def group_ab(S, units_list, is_b):
     nt = S.nt
-    kx = n_g = n_y = nvec = 0
+    kx = n_g = n_y = nvec = m1 = 0
     half = 1 if is_b else 0
     blocks = range(half, 8, 2)
+    def xw_bar(n):
+        return ('XW_READY%d' % (n & 1)) if S.xw2 else 'XW_READY'
     for u in units_list:
-        kx += nt
+        # phase 1: every other reverse-pass tile, by the running tile count
+        for i in range(nt - 1, -1, -1):
+            if (m1 & 1) == half:
+                xs = kx % 2
+                yield ('wait', 'X_FULL%d' % xs, kx >> 1)
+                for hh in (0, 1):
+                    yield ('read', ('x', xs, hh), ('x', u, 1, i))
+                for hh in (0, 1):
+                    yield ('write', ('x', xs, hh), ('xw1', u, i))
+                yield ('write', ('gdec', m1 & 3), ('g', u, i))
+                yield ('sync', 'b' if is_b else 'a', 1)
+                yield ('arrive', xw_bar(kx))
+                yield ('arrive', 'G1_READY%d' % (m1 & 3))
+            m1 += 1
+            kx += 1
         for i in range(nt):
             vb = nvec % 2
             yield ('wait', 'VEC_READY%d' % vb, nvec >> 1)

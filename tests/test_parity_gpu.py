@@ -67,6 +67,19 @@ def test_bf16_small(ssd, shape, path):
     check(y, full_oracle(inp), torch.bfloat16, f"{path} {shape}")
 
 
+@pytest.mark.parametrize("path", list(PATHS))
+def test_bf16_decay_range(ssd, path):
+    """Per-head decays from mild to extreme (|A| 1 ... 3000, larger dt): the
+    decay span of a 32-token block runs from below 1 to thousands, so the
+    diagonal mask blocks take both their factorised form and the per-entry
+    exponential beyond it. 160 (batch, head) units: every path runs it."""
+    inp = si.bidir_inputs(40, 256, 4, 64, 128, 4, "bf16", seed=11, device="cuda")
+    inp["A"] = -torch.tensor([[1.0, 50.0, 300.0, 3000.0], [2.0, 80.0, 500.0, 2000.0]], device="cuda")
+    inp["dt"] = (inp["dt"].float() * 3).clamp(max=0.1).to(torch.bfloat16).contiguous()
+    y = run_bidir(ssd, inp, 128, PATHS[path])
+    check(y, full_oracle(inp), torch.bfloat16, f"{path} decay range")
+
+
 @pytest.mark.parametrize("shape", [(2, 300, 4, 128, 2), (1, 64, 3, 64, 3)])
 def test_fp32_small(ssd, shape):
     batch, L, H, N, G = shape

@@ -44,8 +44,9 @@ KERNEL_SOURCE = {
     "chunked": ("ssd_tc.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
     "fused": ("ssd_fused.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
 }
-# name of the kernel each path spends its time in (found in ncu's "Kernel Name")
-KERNEL_NAME = {"simt": "scan_simt_kernel", "chunked": "tc_out_kernel", "fused": "tc_fused_kernel"}
+# kernels one call of each path launches (names as in ncu's "Kernel Name")
+KERNEL_NAMES = {"simt": ("scan_simt_kernel",), "chunked": ("tc_state_kernel", "tc_pass_kernel", "tc_out_kernel"),
+                "fused": ("tc_fused_kernel",)}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -110,29 +111,39 @@ def traffic_record(path: str, workload: str):
     return e.get("dram_bytes_per_launch")
 
 
-def record_traffic(csv_path: str, path: str, workload: str, command: str):
-    """Store dram__bytes_read.sum + dram__bytes_write.sum per launch of the
-    path's dominant kernel, from `ncu -i <report> --page raw --csv` output."""
+def record_traffic(csv_path: str, path: str, workload: str, command: str, scale: float = 1.0,
+                   note: str = ""):
+    """Store dram__bytes_read.sum + dram__bytes_write.sum of one call of the
+    path (summed over one launch of each of its kernels), from
+    `ncu -i <report> --page raw --csv` output of a capture of whole calls.
+    `scale` converts a smaller captured case to the workload (traffic
+    proportional to the tiles processed)."""
     import csv
     with open(csv_path, newline="") as f:
         rows = list(csv.reader(f))
     head, units = rows[0], rows[1]
-    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    unit_scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
     col = {m: head.index(m) for m in ("Kernel Name", "dram__bytes_read.sum", "dram__bytes_write.sum")}
-    per = []
+    names = KERNEL_NAMES[path]
+    per = {n: [] for n in names}
     for r in rows[2:]:
-        if KERNEL_NAME[path] + "<" in r[col["Kernel Name"]] or KERNEL_NAME[path] + "(" in r[col["Kernel Name"]]:
-            per.append(sum(float(r[col[m]].replace(",", "")) * scale[units[col[m]]]
-                           for m in ("dram__bytes_read.sum", "dram__bytes_write.sum")))
-    if not per:
-        raise SystemExit(f"no {KERNEL_NAME[path]} launch in {csv_path}")
+        for n in names:
+            if n + "<" in r[col["Kernel Name"]] or n + "(" in r[col["Kernel Name"]]:
+                per[n].append(sum(float(r[col[m]].replace(",", "")) * unit_scale[units[col[m]]]
+                                  for m in ("dram__bytes_read.sum", "dram__bytes_write.sum")))
+    if any(not v for v in per.values()):
+        raise SystemExit(f"not every kernel of {names} is in {csv_path}")
+    calls = min(len(v) for v in per.values())
     d = {}
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
-    d[f"{workload}:{path}"] = {"dram_bytes_per_launch": round(sum(per) / len(per)),
-                               "launches": len(per), "kernel": KERNEL_NAME[path],
-                               "source_sha": kernel_source_sha(path), "command": command}
+    per_call = sum(sum(v) / len(v) for v in per.values()) * scale
+    e = {"dram_bytes_per_launch": round(per_call), "calls_captured": calls, "kernels": list(names),
+         "source_sha": kernel_source_sha(path), "command": command}
+    if scale != 1.0:
+        e["scaled"] = {"factor": scale, "note": note}
+    d[f"{workload}:{path}"] = e
     with open(TRAFFIC_FILE, "w") as f:
         json.dump(d, f, indent=1, sort_keys=True)
         f.write("\n")
@@ -344,11 +355,14 @@ def main():
                     help="store the dominant kernel's DRAM bytes per launch from an ncu raw CSV "
                          "(with --path and --workload; --capture-command names the capture) and exit")
     ap.add_argument("--capture-command", default="")
+    ap.add_argument("--traffic-scale", type=float, default=1.0)
+    ap.add_argument("--traffic-note", default="")
     args = ap.parse_args()
     if args.record_traffic:
         if args.path == "auto":
             ap.error("--record-traffic needs an explicit --path")
-        record_traffic(args.record_traffic, args.path, args.workload, args.capture_command)
+        record_traffic(args.record_traffic, args.path, args.workload, args.capture_command,
+                       args.traffic_scale, args.traffic_note)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -76,6 +76,10 @@ WORKLOADS = {
         # block-diffusion step: prefix of 262144 tokens, active block of 64, 32 steps
         Workload("blockstep_prefix262144_blk64", 4, 262144, 32, 64, 128, 32, 256, "bf16",
                  block=64, steps=32),
+        # the same step behind a 16384-token prefix (~1 GB on the device: small
+        # enough for a full profiler capture of the block-step kernels)
+        Workload("blockstep_prefix16384_blk64", 4, 16384, 32, 64, 128, 32, 256, "bf16",
+                 block=64, steps=32),
     ]
 }
 

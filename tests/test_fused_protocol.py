@@ -406,7 +406,7 @@ def _schedules(n, xw2, seed0=0):
 
 
 def test_fused_protocol_has_no_overrun_deadlock_or_race():
-    fails = _schedules(1200, xw2=True)
+    fails = _schedules(3000, xw2=True)
     assert not fails, "\n".join(fails[:5])
 
 

@@ -156,10 +156,11 @@ def ssd_bidir_fwd(x, dt, A, B, C, D, out=None, *, chunk: int = 256, path: int = 
     return out
 
 
-def ssd_prefix_state(x, dt, A, B, init=None, out=None, *, chunk: int = 256,
+def ssd_prefix_state(x, dt, A, B, init=None, out=None, *, chunk: int = 256, path: int = SSD_PATH_AUTO,
                      workspace: Workspace | None = None):
-    """Forward-only state after the last token (include/ssd_bidir.h: ssd_prefix_state).
-    dt (batch, L, H), A (H), B (batch, L, G, N): the forward direction's."""
+    """Forward-only state after the last token (include/ssd_bidir.h: ssd_prefix_state,
+    ssd_prefix_state_path). dt (batch, L, H), A (H), B (batch, L, G, N): the forward
+    direction's. `path`: as for ssd_bidir_fwd."""
     _need(x, "x", ndim=4)
     dev, io = x.device, x.dtype
     if io not in _DT:
@@ -187,15 +188,17 @@ def ssd_prefix_state(x, dt, A, B, init=None, out=None, *, chunk: int = 256,
     if nbytes == 0:
         _check(_c.SSD_ERR_UNSUPPORTED, "ssd_prefix_state")
     buf = ws.get(nbytes)
-    rc = lib.ssd_prefix_state(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init), _ptr(out),
-                              batch, L, H, P, N, G, chunk, _DT[io],
-                              _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    rc = lib.ssd_prefix_state_path(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init), _ptr(out),
+                                   batch, L, H, P, N, G, chunk, _DT[io], int(path),
+                                   _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_prefix_state")
     return out
 
 
-def ssd_block_step(x, dt, A, B, C, D, prefix_state, out=None, *, workspace: Workspace | None = None):
-    """One block-diffusion step on the active block (include/ssd_bidir.h: ssd_block_step)."""
+def ssd_block_step(x, dt, A, B, C, D, prefix_state, out=None, *, path: int = SSD_PATH_AUTO,
+                   workspace: Workspace | None = None):
+    """One block-diffusion step on the active block (include/ssd_bidir.h: ssd_block_step,
+    ssd_block_step_path). `path`: as for ssd_bidir_fwd."""
     _need(x, "x", ndim=4)
     dev, io = x.device, x.dtype
     if io not in _DT:
@@ -223,8 +226,8 @@ def ssd_block_step(x, dt, A, B, C, D, prefix_state, out=None, *, workspace: Work
     if nbytes == 0:
         _check(_c.SSD_ERR_UNSUPPORTED, "ssd_block_step")
     buf = ws.get(nbytes)
-    rc = lib.ssd_block_step(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                            _ptr(prefix_state), _ptr(out), batch, T, H, P, N, G, _DT[io],
-                            _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    rc = lib.ssd_block_step_path(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                 _ptr(prefix_state), _ptr(out), batch, T, H, P, N, G, _DT[io],
+                                 int(path), _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_block_step")
     return out

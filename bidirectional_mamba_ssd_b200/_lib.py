@@ -30,6 +30,8 @@ SIGNATURES = {
     "ssd_bidir_fwd_path": (_i, [_vp] * 7 + [_i] * 9 + [_vp, _sz, _vp]),
     "ssd_prefix_state": (_i, [_vp] * 6 + [_i] * 8 + [_vp, _sz, _vp]),
     "ssd_block_step": (_i, [_vp] * 8 + [_i] * 7 + [_vp, _sz, _vp]),
+    "ssd_prefix_state_path": (_i, [_vp] * 6 + [_i] * 9 + [_vp, _sz, _vp]),
+    "ssd_block_step_path": (_i, [_vp] * 8 + [_i] * 8 + [_vp, _sz, _vp]),
     "ssd_bidir_fwd_noalloc": (_i, [_vp] * 7 + [_i] * 8 + [_vp]),
     "ssd_get_device_status": (_i, [_vp, _vp]),
     "ssd_selftest_wait_timeout": (_i, [_vp, _sz, _i, _vp]),

@@ -46,6 +46,11 @@ size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 float *scratch_ptr(void *ws) { return reinterpret_cast<float *>(static_cast<char *>(ws) + ssd::kStatusBytes); }
 
+// Prefix states and block steps take the fused kernel (one (batch, head) per
+// SM at a time, all tiles in one launch) from this many units, else the
+// tile-parallel chunked kernels.
+constexpr long long kFusedMinUnits = 64;
+
 // Kernel choice of SSD_PATH_AUTO: bf16 runs on the tensor cores, in one
 // kernel per (batch, head) when there are enough of those to fill the GPU,
 // else in the tile-parallel chunked kernels; fp32 runs the sequential scan.
@@ -117,7 +122,9 @@ size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdi
             scratch = scratch > c ? scratch : c;
         } else if (op == SSD_OP_BLOCK_STEP) {
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 2);
+            size_t f = ssd::tc_fused_scratch_bytes(batch, seqlen, nheads, dstate);
             scratch = scratch > c ? scratch : c;
+            scratch = scratch > f ? scratch : f;
         }
     }
     return ssd::kStatusBytes + round256(scratch);
@@ -152,12 +159,13 @@ int ssd_bidir_fwd_path(const void *x, const void *dt, const float *A, const void
                       chunk, dtype, path, workspace, ws_bytes, stream);
 }
 
-int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *B,
-                     const float *init_state, float *state_out, int batch, int seqlen, int nheads,
-                     int headdim, int dstate, int ngroups, int chunk, int dtype, void *workspace,
-                     size_t ws_bytes, void *stream) {
+int ssd_prefix_state_path(const void *x, const void *dt, const float *A, const void *B,
+                          const float *init_state, float *state_out, int batch, int seqlen, int nheads,
+                          int headdim, int dstate, int ngroups, int chunk, int dtype, int path,
+                          void *workspace, size_t ws_bytes, void *stream) {
     int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
     if (rc != SSD_OK) return rc;
+    if (path < SSD_PATH_AUTO || path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
     if (!workspace) return SSD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
     if (ws_bytes < ssd_workspace_bytes(SSD_OP_PREFIX_STATE, batch, seqlen, nheads, headdim, dstate,
@@ -171,14 +179,16 @@ int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *
         if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned4(A)) return SSD_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dtype == SSD_BF16 && seqlen > 0) {
+    if (path == SSD_PATH_AUTO && dtype == SSD_BF16 && seqlen > 0)
+        path = (long long)batch * nheads >= kFusedMinUnits ? SSD_PATH_FUSED : SSD_PATH_CHUNKED;
+    if ((path == SSD_PATH_CHUNKED || path == SSD_PATH_FUSED) && dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    // an empty sequence (the state is the initial one) goes to the scan kernel below
+    if ((path == SSD_PATH_CHUNKED || path == SSD_PATH_FUSED) && seqlen > 0) {
         TcArgs t{};
         t.x = x; t.dt = dt; t.A = A; t.B = B; t.init = init_state; t.state_out = state_out;
         t.workspace = workspace; t.ws_bytes = ws_bytes;
         t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 1;
-        cudaError_t e = ssd::launch_tc_chunked(t, s);
-        if (e != cudaErrorNotSupported) return to_status(e);
-        (void)cudaGetLastError();
+        return to_status(path == SSD_PATH_FUSED ? ssd::launch_tc_fused_state(t, s) : ssd::launch_tc_chunked(t, s));
     }
     SimtArgs a{};
     a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = nullptr; a.D = nullptr;
@@ -189,12 +199,21 @@ int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *
     return to_status(ssd::launch_scan_simt(a, dtype == SSD_BF16, dstate, s));
 }
 
-int ssd_block_step(const void *x, const void *dt, const float *A, const void *B, const void *C,
-                   const float *D, const float *prefix_state, void *out, int batch, int blk_len,
-                   int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
-                   size_t ws_bytes, void *stream) {
+int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *B,
+                     const float *init_state, float *state_out, int batch, int seqlen, int nheads,
+                     int headdim, int dstate, int ngroups, int chunk, int dtype, void *workspace,
+                     size_t ws_bytes, void *stream) {
+    return ssd_prefix_state_path(x, dt, A, B, init_state, state_out, batch, seqlen, nheads, headdim,
+                                 dstate, ngroups, chunk, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
+}
+
+int ssd_block_step_path(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                        const float *D, const float *prefix_state, void *out, int batch, int blk_len,
+                        int nheads, int headdim, int dstate, int ngroups, int dtype, int path,
+                        void *workspace, size_t ws_bytes, void *stream) {
     int rc = check_shape(batch, blk_len, nheads, headdim, dstate, ngroups, 64, dtype, false);
     if (rc != SSD_OK) return rc;
+    if (path < SSD_PATH_AUTO || path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
     if (!workspace) return SSD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
     if (ws_bytes < ssd_workspace_bytes(SSD_OP_BLOCK_STEP, batch, blk_len, nheads, headdim, dstate,
@@ -207,17 +226,18 @@ int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
         return SSD_ERR_INVALID_ARG;
     if (prefix_state && !aligned16(prefix_state)) return SSD_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dtype == SSD_BF16) {
-        // the bidirectional chunked tensor-core path over the block, with the
-        // forward scan starting from the cached state and the reverse from zero
+    if (path == SSD_PATH_AUTO && dtype == SSD_BF16)
+        path = (long long)batch * nheads >= kFusedMinUnits ? SSD_PATH_FUSED : SSD_PATH_CHUNKED;
+    if ((path == SSD_PATH_CHUNKED || path == SSD_PATH_FUSED) && dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    if (path == SSD_PATH_CHUNKED || path == SSD_PATH_FUSED) {
+        // both scans over the block, the forward one starting from the cached
+        // state (zero if none) and the reverse one from zero
         TcArgs t{};
         t.x = x; t.dt = dt; t.A = A; t.B = B; t.C = C; t.D = D; t.out = out;
         t.init = prefix_state;
         t.workspace = workspace; t.ws_bytes = ws_bytes;
         t.batch = batch; t.L = blk_len; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
-        cudaError_t e = ssd::launch_tc_chunked(t, s);
-        if (e != cudaErrorNotSupported) return to_status(e);
-        (void)cudaGetLastError();
+        return to_status(path == SSD_PATH_FUSED ? ssd::launch_tc_fused(t, s) : ssd::launch_tc_chunked(t, s));
     }
     SimtArgs a{};
     a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
@@ -229,6 +249,14 @@ int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
     a.batch = batch; a.L = blk_len; a.H = nheads; a.G = ngroups;
     a.ndir = 2; a.has_output = 1;
     return to_status(ssd::launch_scan_simt(a, dtype == SSD_BF16, dstate, s));
+}
+
+int ssd_block_step(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                   const float *D, const float *prefix_state, void *out, int batch, int blk_len,
+                   int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
+                   size_t ws_bytes, void *stream) {
+    return ssd_block_step_path(x, dt, A, B, C, D, prefix_state, out, batch, blk_len, nheads, headdim,
+                               dstate, ngroups, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
 }
 
 int ssd_get_device_status(const void *workspace, void *stream) {

@@ -60,12 +60,32 @@ constexpr int kP = 64;
 constexpr uint32_t kSlab = 16384;       // 128 rows x 128 bytes
 constexpr int kRing = 4;                // B/C ring slots (32 KB each)
 constexpr int kThreads = 448;
+constexpr int kXMax = 2;                // most x slots of any mode
+constexpr int kG1 = 8;                  // state-pass tile decays in flight (>= x slots + 2)
+
+// What one launch computes (a template parameter: each mode is its own kernel)
+enum : int {
+    kModeBidir = 0,      // both scans, summed output
+    kModeBidirInit = 1,  // the same with the forward scan started from a given state
+    kModeState = 2,      // the forward scan's final state only (optionally from a given state)
+};
+
+// x slots: two in every mode. The count must be even: groups A and B take
+// alternate state-pass tiles, and with an even count each group always gets
+// the same slots and waits on every phase of their barriers (with an odd
+// count a group could wait on a slot's next phase before the phase another
+// group used had completed, and the parity wait would pass at once). The
+// state mode pairs each slot with a buffer for the low part of diag(w) X.
+template <int N, int MODE>
+constexpr int x_slots() { return 2; }
 
 struct FusedParams {
-    const __nv_bfloat16 *dt;   // (2, batch, L, H)
-    const float *A;            // (2, H)
+    const __nv_bfloat16 *dt;   // (2, batch, L, H); state mode: (batch, L, H)
+    const float *A;            // (2, H); state mode: (H)
     const float *D;            // (2, H)
     __nv_bfloat16 *hb;         // (units, nt, N, 64) reverse states entering each tile
+    const float *init;         // (batch, H, 64, N) forward start state (init / state modes) or nullptr
+    float *state_out;          // (batch, H, 64, N) final forward state (state mode)
     DeviceStatus *status;
     int batch, L, H, G, nt, units;
 };
@@ -74,9 +94,9 @@ struct FusedParams {
 enum {
     B_RING_FULL = 0,                 // kRing
     B_RING_EMPTY = B_RING_FULL + kRing,
-    B_X_FULL = B_RING_EMPTY + kRing, // 2
-    B_X_EMPTY = B_X_FULL + 2,        // 2
-    B_HB_FULL = B_X_EMPTY + 2,
+    B_X_FULL = B_RING_EMPTY + kRing, // kXMax (x_slots() used)
+    B_X_EMPTY = B_X_FULL + kXMax,    // kXMax
+    B_HB_FULL = B_X_EMPTY + kXMax,
     B_HB_EMPTY,
     B_HB_WRITTEN,                    // group C -> producer: phase-1 states are in global memory
     B_G_READY,                       // MMA -> groups A and B (phase 2)
@@ -84,18 +104,19 @@ enum {
     B_Y_READY,                       // MMA -> groups A and B
     B_P1S_READY,                     // 2: MMA -> group C, phase-1 tile state per TMEM buffer
     B_P1S_FREE = B_P1S_READY + 2,    // 2: group C -> MMA
-    // 2: group C -> MMA, alternating by tile. In phase 1 group C folds tile
-    // states in one tile behind, so it can release diag(w) X of two tiles
-    // before the MMA issuer has taken the first: one barrier would complete
-    // two phases and the issuer's parity wait would miss both.
+    // per x slot (kXMax): diag(w) X of the tile in that slot is ready. One
+    // barrier per slot, not a single one: in the state pass the preparing
+    // groups can release several tiles before the MMA issuer takes the first,
+    // and a single barrier would complete two phases under the issuer's
+    // parity wait; a slot is refilled only after the MMA that read it.
     B_XW_READY = B_P1S_FREE + 2,
-    B_M_READY = B_XW_READY + 2,      // groups A and B -> MMA (count 2)
+    B_M_READY = B_XW_READY + kXMax,  // groups A and B -> MMA (count 2)
     B_S_FREE,                        // group C -> MMA (phase 2)
     B_Y_FREE,                        // group B -> MMA
     B_VEC_READY,                     // 2: group C -> groups A and B, per vector buffer
     B_VEC_FREE = B_VEC_READY + 2,    // 2: groups A and B -> group C (count 2)
-    B_G1_READY = B_VEC_FREE + 2,     // 4: groups A/B -> group C, reverse-pass tile decay per buffer
-    B_MMA_DONE = B_G1_READY + 4,     // MMA issuer, at teardown
+    B_G1_READY = B_VEC_FREE + 2,     // kG1: groups A/B -> group C, state-pass tile decay per buffer
+    B_MMA_DONE = B_G1_READY + kG1,   // MMA issuer, at teardown
     B_COUNT
 };
 
@@ -220,25 +241,33 @@ struct Smem {
     static constexpr uint32_t xw = hf + kH;             // diag(w) x
     static constexpr uint32_t small = xw + kSlab;
     static constexpr uint32_t bytes = small + 7168;     // barriers, scan scratch, 2 tile-vector buffers
+    static __device__ __forceinline__ uint32_t xslot(uint32_t j) { return x0 + j * kSlab; }
+    // state mode: the low part of diag(w) X of x slot j, in the diag(w) X
+    // buffer or the 16 KB from H_b on (H_b alone for N = 128, with H_f for N = 64)
+    static __device__ __forceinline__ uint32_t loslot(uint32_t j) { return j == 0 ? xw : hb; }
+    static_assert(hb + kSlab <= xw, "low-part slot 1");
 };
 
-template <int N>
+template <int N, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
                 const __grid_constant__ CUtensorMap tm_out, const FusedParams p) {
     using S = Smem<N>;
     constexpr int NSLAB = N / 64;
+    constexpr uint32_t kXS = x_slots<N, MODE>();
+    constexpr bool kOut = MODE != kModeState;      // an output pass follows the state pass
+    constexpr bool kFwd1 = MODE == kModeState;     // the state pass runs forward (else reverse)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *g = smem_raw + (base - smem_u32(smem_raw));
     uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
-    static_assert(8 * B_COUNT + 8 <= 320, "barrier area");
-    float *gdec1 = reinterpret_cast<float *>(g + S::small + 320);  // 4 reverse-pass tile decays
-    float *red_ab = reinterpret_cast<float *>(g + S::small + 352); // 2 x 4 floats, groups A and B scans
-    float *red = reinterpret_cast<float *>(g + S::small + 384);    // 8 floats, group C scans
+    static_assert(8 * B_COUNT + 8 <= 416, "barrier area");
+    float *gdec1 = reinterpret_cast<float *>(g + S::small + 416);  // kG1 state-pass tile decays
+    float *red_ab = reinterpret_cast<float *>(g + S::small + 448); // 2 x 4 floats, groups A and B scans
+    float *red = reinterpret_cast<float *>(g + S::small + 480);    // 8 floats, group C scans
     TileVec *vec = reinterpret_cast<TileVec *>(g + S::small + 512);  // 2 buffers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -284,34 +313,39 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                        mbar_wait(bar(B_RING_EMPTY + s), ((kr / kRing) - 1) & 1, abort_flag, p.status, 101);
             };
             auto x_slot = [&](uint32_t &s) -> bool {
-                s = kx & 1;
-                return kx < 2 || mbar_wait(bar(B_X_EMPTY + s), ((kx >> 1) - 1) & 1, abort_flag, p.status, 102);
+                s = kx % kXS;
+                return kx < kXS || mbar_wait(bar(B_X_EMPTY + s), ((kx / kXS) - 1) & 1, abort_flag, p.status, 102);
             };
+            // the state pass's x and B are read once in the state mode; otherwise
+            // the output pass reads them again from L2
+            const uint64_t pol1 = kOut ? keep : stream;
             // after an expired wait anywhere in the CTA, no further loads are issued
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++units_done) {
                 const int b = u / p.H, h = u % p.H, gg = h / hpg;
-                for (int i = nt - 1; ok && i >= 0; --i) {   // phase 1: x, B' right to left
+                for (int k1 = 0; ok && k1 < nt; ++k1) {     // phase 1: x, B of the state pass
+                    const int i = kFwd1 ? k1 : nt - 1 - k1;
                     uint32_t xs, rs;
                     if (!(ok = x_slot(xs))) break;
                     ++kx;
                     mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
-                    tma_load_4d_hint(base + S::x0 + xs * kSlab, &tm_x, bar(B_X_FULL + xs), 0, h, i * kTile, b, keep);
+                    tma_load_4d_hint(base + S::xslot(xs), &tm_x, bar(B_X_FULL + xs), 0, h, i * kTile, b, pol1);
                     if (!(ok = ring_slot(rs))) break;
                     ++kr;
                     mbar_arrive_expect_tx(bar(B_RING_FULL + rs), S::kBC);
                     for (int k = 0; k < NSLAB; ++k)
                         tma_load_5d_hint(base + S::ring + rs * 2 * kSlab + k * kSlab, &tm_b, bar(B_RING_FULL + rs),
-                                         64 * k, gg, i * kTile, b, 1, keep);
+                                         64 * k, gg, i * kTile, b, kFwd1 ? 0 : 1, pol1);
                 }
-                if (!ok || !(ok = mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103))) break;
-                for (int i = 0; ok && i < nt; ++i) {        // phase 2: x, C_f, B_f, C_b, B_b, H_b
+                if (!ok) break;
+                if (kOut && !(ok = mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103))) break;
+                for (int i = 0; kOut && ok && i < nt; ++i) {        // phase 2: x, C_f, B_f, C_b, B_b, H_b
                     const int t0 = i * kTile;
                     uint32_t xs;
                     if (!(ok = x_slot(xs))) break;
                     ++kx;
                     mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
-                    tma_load_4d_hint(base + S::x0 + xs * kSlab, &tm_x, bar(B_X_FULL + xs), 0, h, t0, b, stream);
+                    tma_load_4d_hint(base + S::xslot(xs), &tm_x, bar(B_X_FULL + xs), 0, h, t0, b, stream);
                     const CUtensorMap *maps[4] = {&tm_c, &tm_b, &tm_c, &tm_b};
                     const int dirs[4] = {0, 0, 1, 1};
                     for (int j = 0; ok && j < 4; ++j) {
@@ -334,7 +368,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // after an expired wait, when consumers may have stopped waiting)
             for (uint32_t k = kr > kRing ? kr - kRing : 0; k < kr; ++k)
                 mbar_drain(bar(B_RING_FULL + k % kRing), (k / kRing) & 1);
-            for (uint32_t k = kx > 2 ? kx - 2 : 0; k < kx; ++k) mbar_drain(bar(B_X_FULL + (k & 1)), (k >> 1) & 1);
+            for (uint32_t k = kx > kXS ? kx - kXS : 0; k < kx; ++k) mbar_drain(bar(B_X_FULL + k % kXS), (k / kXS) & 1);
             if (kh >= 1) mbar_drain(bar(B_HB_FULL), (kh - 1) & 1);
         }
     } else if (warp == 1) {
@@ -344,7 +378,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);    // C (K) x B (K)
             constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);      // C (K) x H (MN); M (K) x X (MN)
             uint32_t kr = 0, kx = 0, kh = 0, n1 = 0;
-            uint32_t n_xw = 0, n_m = 0, n_sfree = 0, n_yfree = 0;
+            uint32_t n_m = 0, n_sfree = 0, n_yfree = 0;
             bool first2 = true;
             auto wait_ring = [&](uint32_t k) -> uint32_t {
                 const uint32_t s = k % kRing;
@@ -354,24 +388,29 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             auto slot_addr = [&](uint32_t s) { return base + S::ring + s * 2 * kSlab; };
             // after an expired wait anywhere in the CTA, no further tiles are issued
             for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
-                for (int i = nt - 1; i >= 0 && !*abort_flag; --i, ++n1) {  // phase 1: S' = B'^T (diag(w') X in the x slot)
-                    const uint32_t xs = kx++ & 1;
+                for (int k1 = 0; k1 < nt && !*abort_flag; ++k1, ++n1) {  // phase 1: S = B^T (diag(w) X in the x slot)
+                    const uint32_t n = kx++, xs = n % kXS;
                     const uint32_t rs = wait_ring(kr++);
-                    mbar_wait(bar(B_XW_READY + (n_xw & 1)), (n_xw >> 1) & 1, abort_flag, p.status, 202);
-                    ++n_xw;
+                    mbar_wait(bar(B_XW_READY + xs), (n / kXS) & 1, abort_flag, p.status, 202);
                     const uint32_t pb = n1 & 1;
                     if (n1 >= 2) mbar_wait(bar(B_P1S_FREE + pb), ((n1 >> 1) - 1) & 1, abort_flag, p.status, 203);
                     tc_fence_after();
-                    const uint32_t sB = slot_addr(rs), sX = base + S::x0 + xs * kSlab;
+                    const uint32_t sB = slot_addr(rs), sX = base + S::xslot(xs);
                     for (int k = 0; k < kTile / 16; ++k)
                         mma_bf16_ss(tGf + 64 * pb, sdesc_sw128(sB + k * 2048, kSlab, 1024),
                                     sdesc_sw128(sX + k * 2048, kSlab, 1024), id_state, k > 0);
+                    if constexpr (!kOut) {   // state mode: plus B^T (low part of diag(w) X)
+                        const uint32_t sL = base + S::loslot(xs);
+                        for (int k = 0; k < kTile / 16; ++k)
+                            mma_bf16_ss(tGf + 64 * pb, sdesc_sw128(sB + k * 2048, kSlab, 1024),
+                                        sdesc_sw128(sL + k * 2048, kSlab, 1024), id_state, 1);
+                    }
                     mma_commit(bar(B_P1S_READY + pb));
                     mma_commit(bar(B_RING_EMPTY + rs));
                     mma_commit(bar(B_X_EMPTY + xs));
                 }
-                for (int i = 0; i < nt && !*abort_flag; ++i) {   // phase 2
-                    const uint32_t xs = kx++ & 1;
+                for (int i = 0; kOut && i < nt && !*abort_flag; ++i) {   // phase 2
+                    const uint32_t n = kx++, xs = n % kXS;
                     const uint32_t rCf = wait_ring(kr++), rBf = wait_ring(kr++);
                     const uint32_t rCb = wait_ring(kr++), rBb = wait_ring(kr++);
                     const uint32_t sCf = slot_addr(rCf), sBf = slot_addr(rBf);
@@ -411,8 +450,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     }
                     mma_commit(bar(B_RING_EMPTY + rCb));
                     mma_commit(bar(B_HB_EMPTY));
-                    mbar_wait(bar(B_XW_READY + (n_xw & 1)), (n_xw >> 1) & 1, abort_flag, p.status, 208);
-                    ++n_xw;
+                    mbar_wait(bar(B_XW_READY + xs), (n / kXS) & 1, abort_flag, p.status, 208);
                     tc_fence_after();
                     for (int k = 0; k < kTile / 16; ++k)    // S_f = B_f^T diag(w_f) X
                         mma_bf16_ss(tS, sdesc_sw128(sBf + k * 2048, kSlab, 1024),
@@ -420,9 +458,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     mma_commit(bar(B_S_READY));
                     mma_commit(bar(B_RING_EMPTY + rBf));
                     mbar_wait(bar(B_M_READY), n_m++ & 1, abort_flag, p.status, 209);
-                    mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 204);
+                    mbar_wait(bar(B_X_FULL + xs), (n / kXS) & 1, abort_flag, p.status, 204);
                     tc_fence_after();
-                    const uint32_t sX = base + S::x0 + xs * kSlab;
+                    const uint32_t sX = base + S::xslot(xs);
                     for (int k = 0; k < kTile / 16; ++k)    // Yd = M X, M from TMEM
                         mma_bf16_ts(tYd, tGf + 16 * k, sdesc_sw128(sX + k * 2048, kSlab, 1024), id_o, k > 0);
                     mma_commit(bar(B_Y_READY));
@@ -437,8 +475,20 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const int row = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
         const uint64_t keep = policy_evict_last();
-        uint32_t kx = 0, n_s = 0, nvec = 0, n1 = 0, n_xw = 0;
+        uint32_t kx = 0, n_s = 0, nvec = 0, n1 = 0;
         float hreg[kP];
+        // hreg <- the given forward start state of unit u (row n of the (64, N)
+        // state, transposed: hreg[p] = state[p][n]) or zero
+        auto start_state = [&](int u, bool given) {
+            if (given && p.init && row < N) {
+                const float *ip = p.init + (size_t)u * kP * N + row;
+#pragma unroll
+                for (int j = 0; j < kP; ++j) hreg[j] = ip[(size_t)j * N];
+            } else {
+#pragma unroll
+                for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
+            }
+        };
         // dt of the next output-pass tile is fetched a tile ahead (volatile
         // loads, so the compiler keeps them a tile early)
         uint32_t rawf = 0, rawb = 0;
@@ -458,18 +508,19 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             vb = __uint_as_float(rawb << 16);
         };
         int cu = blockIdx.x, ci = 0;   // the output-pass tile whose dt is in flight
-        load_dt(cu, ci);
+        if constexpr (kOut) load_dt(cu, ci);
         while (cu < p.units) {
             const int u = cu;
             const int h = u % p.H;
-            const float Af = p.A[h], Ab = p.A[p.H + h];
-            // ---------------- phase 1: the reverse chain, right to left. Groups A
-            // and B prepare the tiles (diag(w') X, tile decay); this group stores
-            // the state entering each tile and folds the tile's state in.
-#pragma unroll
-            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
-            for (int i = nt - 1; i >= 0; --i, ++n1) {
-                if (row < N) {
+            const float Af = p.A[h], Ab = kOut ? p.A[p.H + h] : 0.f;
+            // ---------------- phase 1: the state chain (reverse, right to left; in
+            // the state mode forward, from the given state). Groups A and B prepare
+            // the tiles (diag(w) X, tile decay); this group stores the reverse
+            // state entering each tile (output modes) and folds the tile's state in.
+            start_state(u, kFwd1);
+            for (int k1 = 0; k1 < nt; ++k1, ++n1) {
+                const int i = kFwd1 ? k1 : nt - 1 - k1;
+                if (kOut && row < N) {
                     __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -481,8 +532,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     }
                 }
                 const uint32_t pbuf = n1 & 1;
-                mbar_wait(bar(B_G1_READY + (n1 & 3)), (n1 >> 2) & 1, abort_flag, p.status, 303);
-                const float gdec = gdec1[n1 & 3];
+                mbar_wait(bar(B_G1_READY + n1 % kG1), (n1 / kG1) & 1, abort_flag, p.status, 303);
+                const float gdec = gdec1[n1 % kG1];
                 mbar_wait(bar(B_P1S_READY + pbuf), (n1 >> 1) & 1, abort_flag, p.status, 301);
                 tc_fence_after();
 #pragma unroll
@@ -498,21 +549,32 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 sync_c();
                 if (row == 0) mbar_arrive(bar(B_P1S_FREE + pbuf));
             }
-            kx += nt;        // the reverse pass's x loads and diag(w') X releases
-            n_xw += nt;      // belong to groups A and B
-            // phase 2 starts from H_f = 0; the reverse states go to the TMA proxy
-            if (row < N) {
-                uint4 *hf = reinterpret_cast<uint4 *>(g + S::hf + row * 128);
+            if constexpr (!kOut) {
+                // the state mode's result: the forward state after the last tile
+                if (row < N) {
+                    float *op = p.state_out + (size_t)u * kP * N + row;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) hf[c] = make_uint4(0, 0, 0, 0);
+                    for (int j = 0; j < kP; ++j) op[(size_t)j * N] = hreg[j];
+                }
+                cu += gridDim.x;
+                continue;
+            }
+            kx += nt;        // the reverse pass's x loads and diag(w') X releases belong to groups A and B
+            // phase 2 starts from H_f = 0 (the init mode: from the given state); the
+            // reverse states go to the TMA proxy
+            start_state(u, MODE == kModeBidirInit);
+            if (row < N) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(g + S::hf + sw128_offset(row, c)) =
+                        make_uint4(pack_bf16x2(hreg[8 * c], hreg[8 * c + 1]), pack_bf16x2(hreg[8 * c + 2], hreg[8 * c + 3]),
+                                   pack_bf16x2(hreg[8 * c + 4], hreg[8 * c + 5]), pack_bf16x2(hreg[8 * c + 6], hreg[8 * c + 7]));
             }
             fence_proxy_async_smem();
             fence_proxy_async_global();
             sync_c();
             if (row == 0) mbar_arrive(bar(B_HB_WRITTEN));
             // ---------------- phase 2: decay sums, vectors, diag(w_f) X, forward chain
-#pragma unroll
-            for (int j = 0; j < kP; ++j) hreg[j] = 0.f;
             for (int i = 0; i < nt; ++i) {
                 float vf, vb;
                 take_dt(vf, vb);
@@ -541,13 +603,12 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 // diag(w_f) X into the X' buffer (the previous state MMA, which read
                 // it, completed before this group's last state step)
                 const float wf = __expf(Af * (totf - pf)) * vf;   // exp(A sum_{r>s} dt) dt_s
-                const uint32_t xs = kx++ & 1;
-                mbar_wait(bar(B_X_FULL + xs), (kx - 1) >> 1 & 1, abort_flag, p.status, 312);
-                scale_row(g + S::x0 + xs * kSlab, g + S::xw, row, wf);
+                const uint32_t nx = kx++, xs = nx % kXS;
+                mbar_wait(bar(B_X_FULL + xs), (nx / kXS) & 1, abort_flag, p.status, 312);
+                scale_row(g + S::xslot(xs), g + S::xw, row, wf);
                 fence_proxy_async_smem();
                 sync_c();
-                if (row == 0) mbar_arrive(bar(B_XW_READY + (n_xw & 1)));
-                ++n_xw;
+                if (row == 0) mbar_arrive(bar(B_XW_READY + xs));
                 // forward chain: H_f <- exp(A sum dt) H_f + S_f; bf16 copy for C_f.H_f
                 const float gdec = __expf(Af * totf);
                 mbar_wait(bar(B_S_READY), n_s++ & 1, abort_flag, p.status, 313);
@@ -589,49 +650,54 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         float *red_g = red_ab + (is_b ? 4 : 0);
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             const int b = u / p.H, h = u % p.H;
-            const float dsum = p.D[h] + p.D[p.H + h];
-            const float Ab = p.A[p.H + h];
-            // ---------------- phase 1: every other reverse-pass tile (by the CTA's
+            const float dsum = kOut ? p.D[h] + p.D[p.H + h] : 0.f;
+            // the state pass's direction: reverse in the output modes, forward in the state mode
+            const float A1 = kFwd1 ? p.A[h] : p.A[p.H + h];
+            const size_t dt1 = kFwd1 ? 0 : dt_dir;
+            // ---------------- phase 1: every other state-pass tile (by the CTA's
             // running tile count m1: group A the even ones, group B the odd ones):
-            // w'_s = exp(A' sum_{r<s} dt'_r) dt'_s, diag(w') X in place in the x
-            // slot, and the tile decay exp(A' sum dt') for group C's chain.
-            uint32_t rawn = 0;               // dt' of this group's next tile, fetched a tile ahead
+            // w_s = exp(A sum dt_r) dt_s over the rest of the tile in the pass's
+            // direction (reverse: r < s, forward: r > s), diag(w) X in place in
+            // the x slot, and the tile decay exp(A sum dt) for group C's chain.
+            uint32_t rawn = 0;               // dt of this group's next tile, fetched a tile ahead
             bool have = false;
-            for (int i = nt - 1; i >= 0; --i, ++m1, ++kx) {
+            for (int k1 = 0; k1 < nt; ++k1, ++m1, ++kx) {
                 if ((m1 & 1) != (uint32_t)is_b) continue;
+                const int i = kFwd1 ? k1 : nt - 1 - k1;
                 float vb = 0.f;
                 if (have) {
                     vb = bf2f(rawn);
                 } else {
                     const int t = i * kTile + row;
-                    if (t < p.L) vb = __bfloat162float(p.dt[dt_dir + ((size_t)b * p.L + t) * p.H + h]);
+                    if (t < p.L) vb = __bfloat162float(p.dt[dt1 + ((size_t)b * p.L + t) * p.H + h]);
                 }
-                have = i >= 2;
+                have = k1 + 2 < nt;          // this group's next tile, two on in the pass's order
                 rawn = 0;
                 if (have) {
-                    const int t = (i - 2) * kTile + row;
+                    const int t = (kFwd1 ? i + 2 : i - 2) * kTile + row;
                     if (t < p.L) {
-                        const size_t o = dt_dir + ((size_t)b * p.L + t) * p.H + h;
+                        const size_t o = dt1 + ((size_t)b * p.L + t) * p.H + h;
                         asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawn) : "l"(p.dt + o));
                     }
                 }
-                float pb = vb, totb;
-                scan1(pb, totb, row, red_g, sync_g);
-                const float w = __expf(Ab * (pb - vb)) * vb;
-                const uint32_t xs = kx & 1;
-                mbar_wait(bar(B_X_FULL + xs), (kx >> 1) & 1, abort_flag, p.status, 404);
-                uint8_t *xt = g + S::x0 + xs * kSlab;
-                scale_row(xt, xt, row, w);
+                float pb = vb, tot;
+                scan1(pb, tot, row, red_g, sync_g);          // pb: inclusive prefix sum
+                const float w = __expf(A1 * (kFwd1 ? tot - pb : pb - vb)) * vb;
+                const uint32_t xs = kx % kXS;
+                mbar_wait(bar(B_X_FULL + xs), (kx / kXS) & 1, abort_flag, p.status, 404);
+                uint8_t *xt = g + S::xslot(xs);
+                if constexpr (kOut) scale_row(xt, xt, row, w);
+                else scale_row_split(xt, g + S::loslot(xs), row, w);   // the state is a result: 16 bits of w x
                 fence_proxy_async_smem();
-                if (row == 0) gdec1[m1 & 3] = __expf(Ab * totb);
+                if (row == 0) gdec1[m1 % kG1] = __expf(A1 * tot);
                 sync_g();
                 if (row == 0) {
-                    mbar_arrive(bar(B_XW_READY + (kx & 1)));
-                    mbar_arrive(bar(B_G1_READY + (m1 & 3)));
+                    mbar_arrive(bar(B_XW_READY + xs));
+                    mbar_arrive(bar(B_G1_READY + m1 % kG1));
                 }
             }
             // ---------------- phase 2: masked matrix halves and output halves
-            for (int i = 0; i < nt; ++i) {
+            for (int i = 0; kOut && i < nt; ++i) {
                 const int t0 = i * kTile;
                 const uint32_t vb_i = nvec & 1;
                 mbar_wait(bar(B_VEC_READY + vb_i), (nvec >> 1) & 1, abort_flag, p.status, 401);
@@ -668,13 +734,13 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     mbar_arrive(bar(B_VEC_FREE + vb_i));
                 }
                 ++nvec;
-                const uint32_t xs = kx++ & 1;
+                const uint32_t xs = kx++ % kXS;
                 // output columns [2 c0, 2 c0 + 32) of the tile over the x slot
                 // (group A the first half, group B the second), then one TMA store
                 mbar_wait(bar(B_Y_READY), n_y++ & 1, abort_flag, p.status, 403);
                 tc_fence_after();
                 const float ef = __expf(my_af), eb = __expf(my_ab);
-                uint8_t *xt = g + S::x0 + xs * kSlab;
+                uint8_t *xt = g + S::xslot(xs);
                 const int q0 = c0 >> 3;              // 0 or 2: first 16-column quarter
 #pragma unroll 1
                 for (int q = q0; q < q0 + 2; ++q) {
@@ -706,7 +772,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 if (is_b && row == 0) {
                     mbar_arrive(bar(B_Y_FREE));
                     if (!*abort_flag) {
-                        tma_store_4d(&tm_out, base + S::x0 + xs * kSlab, 0, h, t0, b);
+                        tma_store_4d(&tm_out, base + S::xslot(xs), 0, h, t0, b);
                         tma_store_commit();
                     }
                     tma_store_wait_read();      // the store has read the slot
@@ -725,36 +791,57 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-template <int N>
+template <int N, int MODE>
 cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     using S = Smem<N>;
+    constexpr bool kOut = MODE != kModeState;
     const int nt = (a.L + kTile - 1) / kTile;
     const int units = a.batch * a.H;
-    if (a.ws_bytes < kStatusBytes + tc_fused_scratch_bytes(a.batch, a.L, a.H, N)) return cudaErrorInvalidValue;
+    if (a.ws_bytes < kStatusBytes + (kOut ? tc_fused_scratch_bytes(a.batch, a.L, a.H, N) : 0))
+        return cudaErrorInvalidValue;
+    if (MODE == kModeBidirInit && !a.init) return cudaErrorInvalidValue;
+    if (!kOut && !a.state_out) return cudaErrorInvalidValue;
     FusedParams p{};
     p.dt = static_cast<const __nv_bfloat16 *>(a.dt);
     p.A = a.A;
     p.D = a.D;
-    p.hb = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(a.workspace) + kStatusBytes);
+    p.hb = kOut ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(a.workspace) + kStatusBytes) : nullptr;
+    p.init = a.init;
+    p.state_out = a.state_out;
     p.status = static_cast<DeviceStatus *>(a.workspace);
     p.batch = a.batch; p.L = a.L; p.H = a.H; p.G = a.G; p.nt = nt; p.units = units;
 
     CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_out;
-    if (!tmap::map_x(&tm_x, a.x, a.batch, a.L, a.H) || !tmap::map_bc(&tm_b, a.B, 2, a.batch, a.L, a.G, N) ||
-        !tmap::map_bc(&tm_c, a.C, 2, a.batch, a.L, a.G, N) ||
-        !tmap::map_h(&tm_h, p.hb, (long long)units * nt, N) || !tmap::map_x(&tm_out, a.out, a.batch, a.L, a.H))
+    if (!tmap::map_x(&tm_x, a.x, a.batch, a.L, a.H) || !tmap::map_bc(&tm_b, a.B, kOut ? 2 : 1, a.batch, a.L, a.G, N))
         return cudaErrorInvalidValue;
+    if (kOut) {
+        if (!tmap::map_bc(&tm_c, a.C, 2, a.batch, a.L, a.G, N) ||
+            !tmap::map_h(&tm_h, p.hb, (long long)units * nt, N) || !tmap::map_x(&tm_out, a.out, a.batch, a.L, a.H))
+            return cudaErrorInvalidValue;
+    } else {
+        tm_c = tm_h = tm_out = tm_x;   // not read in the state mode
+    }
     int dev = 0, sms = 0;
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    auto k = tc_fused_kernel<N>;
+    auto k = tc_fused_kernel<N, MODE>;
     const size_t smem = S::bytes + 1024;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return e;
     const int grid = units < sms ? units : sms;
     k<<<grid, kThreads, smem, stream>>>(tm_x, tm_b, tm_c, tm_h, tm_out, p);
     return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_mode(const TcArgs &a, cudaStream_t stream) {
+    if (a.L <= 0 || a.batch <= 0) return cudaErrorNotSupported;
+    if (a.N != 64 && a.N != 128) return cudaErrorNotSupported;
+    if (!tmap::encode_fn()) return cudaErrorNotSupported;
+    const long long entries = (long long)a.batch * a.H * ((a.L + kTile - 1) / kTile);
+    if (entries >= (1ll << 31)) return cudaErrorNotSupported;
+    return a.N == 64 ? run_fused<64, MODE>(a, stream) : run_fused<128, MODE>(a, stream);
 }
 
 }  // namespace
@@ -775,11 +862,11 @@ bool tc_fused_supported(int batch, int L, int H, int G, int N) {
 }
 
 cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream) {
-    if (a.L <= 0 || a.batch <= 0) return cudaErrorNotSupported;
-    if (!tmap::encode_fn()) return cudaErrorNotSupported;
-    const long long entries = (long long)a.batch * a.H * ((a.L + kTile - 1) / kTile);
-    if (entries >= (1ll << 31)) return cudaErrorNotSupported;
-    return a.N == 64 ? run_fused<64>(a, stream) : run_fused<128>(a, stream);
+    return a.init ? launch_mode<kModeBidirInit>(a, stream) : launch_mode<kModeBidir>(a, stream);
+}
+
+cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream) {
+    return launch_mode<kModeState>(a, stream);
 }
 
 }  // namespace ssd

@@ -52,6 +52,11 @@ size_t tc_fused_scratch_bytes(int batch, int L, int H, int N);
 bool tc_fused_supported(int batch, int L, int H, int G, int N);
 
 cudaError_t launch_tc_chunked(const TcArgs &a, cudaStream_t stream);
+// Fused kernel, both scans summed; with a.init the forward scan starts from
+// that state (block step).
 cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream);
+// Fused kernel, forward scan only: the final state into a.state_out, from
+// a.init or zero (prefix state); needs no scratch past the status header.
+cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream);
 
 }  // namespace ssd

@@ -153,4 +153,31 @@ __device__ __forceinline__ void scale_row(const uint8_t *src_tile, uint8_t *dst_
     for (int k = 0; k < 8; ++k) d[(k + row) & 7] = v[k];
 }
 
+// Row `row` of diag(w) X kept as two bf16 terms: the rounded product into
+// hi_tile (in place over the x tile is fine) and the remainder into lo_tile,
+// so the pair carries ~16 mantissa bits of w x instead of 8.
+__device__ __forceinline__ void scale_row_split(uint8_t *hi_tile, uint8_t *lo_tile, int row, float w) {
+    uint4 *hi = reinterpret_cast<uint4 *>(hi_tile + row * 128);
+    uint4 *lo = reinterpret_cast<uint4 *>(lo_tile + row * 128);
+    uint4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = hi[(k + row) & 7];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        uint32_t *q = reinterpret_cast<uint32_t *>(&v[k]);
+        uint4 l;
+        uint32_t *ql = reinterpret_cast<uint32_t *>(&l);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a0 = __uint_as_float(q[j] << 16) * w, a1 = __uint_as_float(q[j] & 0xffff0000u) * w;
+            const uint32_t h = sm100::pack_bf16x2(a0, a1);
+            ql[j] = sm100::pack_bf16x2(a0 - __uint_as_float(h << 16), a1 - __uint_as_float(h & 0xffff0000u));
+            q[j] = h;
+        }
+        lo[(k + row) & 7] = l;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) hi[(k + row) & 7] = v[k];
+}
+
 }  // namespace ssd

@@ -140,12 +140,25 @@ int ssd_bidir_fwd_path(const void *x, const void *dt, const float *A, const void
  *   init_state (batch, nheads, headdim, dstate)     fp32, NULL = zero start
  *   state_out  (batch, nheads, headdim, dstate)     fp32; may equal init_state (in-place update,
  *                                                   e.g. committing a finished block)
- * The state is stored as headdim rows of dstate values: state[b][h][p][n] = h[n][p]. */
+ * The state is stored as headdim rows of dstate values: state[b][h][p][n] = h[n][p].
+ * bf16 I/O runs on the tensor cores: with at least 64 (batch, head) units the
+ * fused kernel (one unit per SM at a time, all its tiles in one launch, no
+ * scratch past the status header), else the tile-parallel chunked kernels;
+ * fp32 I/O and seqlen 0 run the sequential fp32 scan. */
 int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *B,
                      const float *init_state, float *state_out,
                      int batch, int seqlen, int nheads, int headdim, int dstate,
                      int ngroups, int chunk, int dtype,
                      void *workspace, size_t ws_bytes, void *stream);
+
+/* ssd_prefix_state with an explicit kernel choice (tests and benchmarks):
+ * SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED or SSD_PATH_FUSED; the last
+ * two take bf16 I/O only (else SSD_ERR_UNSUPPORTED). */
+int ssd_prefix_state_path(const void *x, const void *dt, const float *A, const void *B,
+                          const float *init_state, float *state_out,
+                          int batch, int seqlen, int nheads, int headdim, int dstate,
+                          int ngroups, int chunk, int dtype, int path,
+                          void *workspace, size_t ws_bytes, void *stream);
 
 /* One denoising step on the active block of blk_len tokens: the forward scan
  * starts from the cached prefix state, the reverse scan starts from zero at
@@ -159,13 +172,22 @@ int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *
  *   B, C         (2, batch, blk_len, ngroups, dstate)     io
  *   prefix_state (batch, nheads, headdim, dstate)         fp32, NULL = zero prefix
  *   out          (batch, blk_len, nheads, headdim)        io, overwritten
- * bf16 I/O runs the tensor-core chunked kernels (the prefix state enters the
- * C.H product as a bf16 operand); fp32 I/O runs the sequential fp32 scan. */
+ * bf16 I/O runs on the tensor cores (the prefix state enters the C.H product
+ * as a bf16 operand): with at least 64 (batch, head) units the fused
+ * bidirectional kernel with its forward scan seeded from prefix_state, else
+ * the chunked kernels; fp32 I/O runs the sequential fp32 scan. */
 int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
                    const void *C, const float *D, const float *prefix_state, void *out,
                    int batch, int blk_len, int nheads, int headdim, int dstate,
                    int ngroups, int dtype,
                    void *workspace, size_t ws_bytes, void *stream);
+
+/* ssd_block_step with an explicit kernel choice, as ssd_prefix_state_path. */
+int ssd_block_step_path(const void *x, const void *dt, const float *A, const void *B,
+                        const void *C, const float *D, const float *prefix_state, void *out,
+                        int batch, int blk_len, int nheads, int headdim, int dstate,
+                        int ngroups, int dtype, int path,
+                        void *workspace, size_t ws_bytes, void *stream);
 
 /* ssd_bidir_fwd for callers that cannot allocate device memory when they
  * call the mixer: code running under CUDA graph capture in the global mode,

@@ -25,6 +25,8 @@ import heapq
 import itertools
 import random
 
+import pytest
+
 
 class Bug(Exception):
     pass
@@ -41,9 +43,15 @@ class Bar:
             self.pending = self.count
 
 class Sim:
-    def __init__(self, nt, units, seed, kRing=4, xw2=True, heavy=0.1):
+    """One CTA's schedule. mode: 'bidir' (both scans, output pass; the block
+    step's seeded variant has the same protocol) or 'state' (the forward state
+    pass alone); kxs: x slots; xw_per_slot False plants the earlier single
+    diag(w) X barrier."""
+    def __init__(self, nt, units, seed, kRing=4, mode='bidir', kxs=2, xw_per_slot=True, heavy=0.1):
         self.r = random.Random(seed)
-        self.nt, self.units, self.kRing, self.xw2, self.heavy = nt, units, kRing, xw2, heavy
+        self.nt, self.units, self.kRing, self.heavy = nt, units, kRing, heavy
+        self.mode, self.kxs, self.xw_per_slot = mode, kxs, xw_per_slot
+        self.kG1 = 8
         self.bars = {}
         self.res = {}
         self.t = 0.0
@@ -54,6 +62,11 @@ class Sim:
         if name not in self.bars:
             self.bars[name] = Bar(name, count)
         return self.bars[name]
+    def xw(self, n):
+        """barrier and phase of diag(w) X for the tile with x load index n"""
+        if self.xw_per_slot:
+            return 'XW_READY%d' % (n % self.kxs), n // self.kxs
+        return 'XW_READY', n
     def delay(self):
         d = self.r.expovariate(1.0)
         if self.r.random() < self.heavy:
@@ -80,26 +93,29 @@ class Sim:
 #   ('store', [(res,val)]) then ('store_wait',)
 
 def producer(S, units_list):
-    nt, R = S.nt, S.kRing
+    nt, R, X = S.nt, S.kRing, S.kxs
     kr = kx = kh = 0
     units_done = 0
     for u in units_list:
-        for i in range(nt - 1, -1, -1):
-            xs = kx % 2
-            if kx >= 2:
-                yield ('wait', 'X_EMPTY%d' % xs, (kx >> 1) - 1)
+        for i in range(nt):                      # the state pass's tiles, in its order
+            xs = kx % X
+            if kx >= X:
+                yield ('wait', 'X_EMPTY%d' % xs, kx // X - 1)
             kx += 1
             yield ('tma', 'X_FULL%d' % xs, [(('x', xs, 0), ('x', u, 1, i)), (('x', xs, 1), ('x', u, 1, i))])
             rs = kr % R
             if kr >= R:
                 yield ('wait', 'RING_EMPTY%d' % rs, kr // R - 1)
             kr += 1
-            yield ('tma', 'RING_FULL%d' % rs, [(('ring', rs), ('Bb1', u, i))])
-        yield ('wait', 'HB_WRITTEN', units_done)
+            yield ('tma', 'RING_FULL%d' % rs, [(('ring', rs), ('B1', u, i))])
+        units_done += 1
+        if S.mode == 'state':
+            continue
+        yield ('wait', 'HB_WRITTEN', units_done - 1)
         for i in range(nt):
-            xs = kx % 2
-            if kx >= 2:
-                yield ('wait', 'X_EMPTY%d' % xs, (kx >> 1) - 1)
+            xs = kx % X
+            if kx >= X:
+                yield ('wait', 'X_EMPTY%d' % xs, kx // X - 1)
             kx += 1
             yield ('tma', 'X_FULL%d' % xs, [(('x', xs, 0), ('x', u, 2, i)), (('x', xs, 1), ('x', u, 2, i))])
             for name in ('Cf', 'Bf', 'Cb', 'Bb'):
@@ -112,34 +128,31 @@ def producer(S, units_list):
                 yield ('wait', 'HB_EMPTY', kh - 1)
             kh += 1
             yield ('tma_hb', 'HB_FULL', u, i)
-        units_done += 1
 
 def mma(S, units_list):
-    nt, R = S.nt, S.kRing
+    nt, R, X = S.nt, S.kRing, S.kxs
     kr = kx = kh = n1 = 0
-    n_xw = n_m = n_sfree = n_yfree = 0
+    n_m = n_sfree = n_yfree = 0
     first2 = True
-    def xw_bar(n):
-        return ('XW_READY%d' % (n & 1)) if S.xw2 else 'XW_READY'
-    def xw_phase(n):
-        return (n >> 1) if S.xw2 else n
     for u in units_list:
-        for i in range(nt - 1, -1, -1):
-            xs = kx % 2; kx += 1
+        for i in range(nt):
+            n = kx; xs = n % X; kx += 1
             rs = kr % R
             yield ('wait', 'RING_FULL%d' % rs, kr // R); kr += 1
-            yield ('wait', xw_bar(n_xw), xw_phase(n_xw)); n_xw += 1
+            yield ('wait',) + S.xw(n)
             pb = n1 % 2
             if n1 >= 2:
                 yield ('wait', 'P1S_FREE%d' % pb, (n1 >> 1) - 1)
-            yield ('mma', [(('ring', rs), ('Bb1', u, i)), (('x', xs, 0), ('xw1', u, i)), (('x', xs, 1), ('xw1', u, i))],
+            yield ('mma', [(('ring', rs), ('B1', u, i)), (('x', xs, 0), ('xw1', u, i)), (('x', xs, 1), ('xw1', u, i))],
                    [(('tGf', b), ('S1', u, i)) for b in range(4 * pb, 4 * pb + 4)])
             yield ('commit', 'P1S_READY%d' % pb)
             yield ('commit', 'RING_EMPTY%d' % rs)
             yield ('commit', 'X_EMPTY%d' % xs)
             n1 += 1
+        if S.mode == 'state':
+            continue
         for i in range(nt):
-            xs = kx % 2; kx += 1
+            n = kx; xs = n % X; kx += 1
             slots = []
             for name in ('Cf', 'Bf', 'Cb', 'Bb'):
                 rs = kr % R
@@ -162,36 +175,36 @@ def mma(S, units_list):
             yield ('mma', [(('ring', rCb), ('Cb', u, i)), ('hb', ('hb', u, i))], [(('Yob', 0), ('Yob', u, i)), (('Yob', 1), ('Yob', u, i))])
             yield ('commit', 'RING_EMPTY%d' % rCb)
             yield ('commit', 'HB_EMPTY')
-            yield ('wait', xw_bar(n_xw), xw_phase(n_xw)); n_xw += 1
+            yield ('wait',) + S.xw(n)
             yield ('mma', [(('ring', rBf), ('Bf', u, i)), ('xw', ('xw', u, i))], [('S', ('S', u, i))])
             yield ('commit', 'S_READY')
             yield ('commit', 'RING_EMPTY%d' % rBf)
             yield ('wait', 'M_READY', n_m); n_m += 1
-            yield ('wait', 'X_FULL%d' % xs, (kx - 1) >> 1)
+            yield ('wait', 'X_FULL%d' % xs, n // X)
             yield ('mma', [(('tGf', b), ('M', u, i)) for b in range(8)] + [(('x', xs, 0), ('x', u, 2, i)), (('x', xs, 1), ('x', u, 2, i))],
                    [(('Yd', 0), ('Yd', u, i)), (('Yd', 1), ('Yd', u, i))])
             yield ('commit', 'Y_READY')
 
 def group_c(S, units_list):
-    nt = S.nt
-    kx = n_s = nvec = n1 = n_xw = 0
-    def xw_bar(n):
-        return ('XW_READY%d' % (n & 1)) if S.xw2 else 'XW_READY'
+    nt, X, K = S.nt, S.kxs, S.kG1
+    kx = n_s = nvec = n1 = 0
     for u in units_list:
-        # phase 1: the reverse chain only (groups A and B prepare the tiles)
-        for i in range(nt - 1, -1, -1):
-            yield ('write', ('hbg', u, i), ('hbg', u, i))
+        # phase 1: the state chain only (groups A and B prepare the tiles)
+        for i in range(nt):
+            if S.mode != 'state':
+                yield ('write', ('hbg', u, i), ('hbg', u, i))
             pb = n1 % 2
-            yield ('wait', 'G1_READY%d' % (n1 & 3), n1 >> 2)
-            yield ('read', ('gdec', n1 & 3), ('g', u, i))
+            yield ('wait', 'G1_READY%d' % (n1 % K), n1 // K)
+            yield ('read', ('gdec', n1 % K), ('g', u, i))
             yield ('wait', 'P1S_READY%d' % pb, n1 >> 1)
             for b in range(4 * pb, 4 * pb + 4):
                 yield ('read', ('tGf', b), ('S1', u, i))
             yield ('sync', 'c', 1)
             yield ('arrive', 'P1S_FREE%d' % pb)
             n1 += 1
+        if S.mode == 'state':
+            continue
         kx += nt
-        n_xw += nt
         yield ('write', 'hf', ('hf', u, 0))
         yield ('arrive', 'HB_WRITTEN')
         for i in range(nt):
@@ -201,12 +214,12 @@ def group_c(S, units_list):
             yield ('write', ('vec', vb), ('V', u, i))
             yield ('arrive', 'VEC_READY%d' % vb)
             nvec += 1
-            xs = kx % 2; kx += 1
-            yield ('wait', 'X_FULL%d' % xs, (kx - 1) >> 1)
+            n = kx; xs = n % X; kx += 1
+            yield ('wait', 'X_FULL%d' % xs, n // X)
             for hh in (0, 1):
                 yield ('read', ('x', xs, hh), ('x', u, 2, i))
             yield ('write', 'xw', ('xw', u, i))
-            yield ('arrive', xw_bar(n_xw)); n_xw += 1
+            yield ('arrive', S.xw(n)[0])
             yield ('wait', 'S_READY', n_s); n_s += 1
             yield ('read', 'S', ('S', u, i))
             yield ('write', 'hf', ('hf', u, i + 1))
@@ -214,28 +227,28 @@ def group_c(S, units_list):
             yield ('arrive', 'S_FREE')
 
 def group_ab(S, units_list, is_b):
-    nt = S.nt
+    nt, X, K = S.nt, S.kxs, S.kG1
     kx = n_g = n_y = nvec = m1 = 0
     half = 1 if is_b else 0
     blocks = range(half, 8, 2)
-    def xw_bar(n):
-        return ('XW_READY%d' % (n & 1)) if S.xw2 else 'XW_READY'
     for u in units_list:
-        # phase 1: every other reverse-pass tile, by the running tile count
-        for i in range(nt - 1, -1, -1):
+        # phase 1: every other state-pass tile, by the running tile count
+        for i in range(nt):
             if (m1 & 1) == half:
-                xs = kx % 2
-                yield ('wait', 'X_FULL%d' % xs, kx >> 1)
+                xs = kx % X
+                yield ('wait', 'X_FULL%d' % xs, kx // X)
                 for hh in (0, 1):
                     yield ('read', ('x', xs, hh), ('x', u, 1, i))
                 for hh in (0, 1):
                     yield ('write', ('x', xs, hh), ('xw1', u, i))
-                yield ('write', ('gdec', m1 & 3), ('g', u, i))
+                yield ('write', ('gdec', m1 % K), ('g', u, i))
                 yield ('sync', 'b' if is_b else 'a', 1)
-                yield ('arrive', xw_bar(kx))
-                yield ('arrive', 'G1_READY%d' % (m1 & 3))
+                yield ('arrive', S.xw(kx)[0])
+                yield ('arrive', 'G1_READY%d' % (m1 % K))
             m1 += 1
             kx += 1
+        if S.mode == 'state':
+            continue
         for i in range(nt):
             vb = nvec % 2
             yield ('wait', 'VEC_READY%d' % vb, nvec >> 1)
@@ -251,7 +264,7 @@ def group_ab(S, units_list, is_b):
             yield ('arrive', 'M_READY')
             yield ('arrive', 'VEC_FREE%d' % vb)
             nvec += 1
-            xs = kx % 2; kx += 1
+            xs = kx % X; kx += 1
             yield ('wait', 'Y_READY', n_y); n_y += 1
             for nm in ('Yd', 'Yof', 'Yob'):
                 yield ('read', (nm, half), (nm, u, i))
@@ -391,13 +404,14 @@ def run(S, units_list):
         fn()
 
 
-def _schedules(n, xw2, seed0=0):
+def _schedules(n, mode='bidir', kxs=2, xw_per_slot=True, seed0=0):
     fails = []
     for seed in range(seed0, seed0 + n):
         r = random.Random(seed)
-        nt = r.choice([1, 2, 3, 4, 5])
+        nt = r.choice([1, 2, 3, 4, 5, 9])
         nunits = r.choice([1, 2, 3])
-        S = Sim(nt, nunits, seed, xw2=xw2, heavy=r.choice([0.0, 0.05, 0.2, 0.5]))
+        S = Sim(nt, nunits, seed, mode=mode, kxs=kxs, xw_per_slot=xw_per_slot,
+                heavy=r.choice([0.0, 0.05, 0.2, 0.5]))
         try:
             run(S, list(range(nunits)))
         except Bug as e:
@@ -406,10 +420,25 @@ def _schedules(n, xw2, seed0=0):
 
 
 def test_fused_protocol_has_no_overrun_deadlock_or_race():
-    fails = _schedules(3000, xw2=True)
+    fails = _schedules(2000)
     assert not fails, "\n".join(fails[:5])
 
 
+def test_state_mode_protocol():
+    """The forward state pass alone (its 2 x slots each paired with a low-part
+    buffer that lives and dies with the slot)."""
+    fails = _schedules(1500, mode='state', kxs=2)
+    assert not fails, "\n".join(fails[:5])
+
+
+def test_model_catches_odd_slot_count_in_state_mode():
+    """With an odd number of x slots the alternating preparing groups do not
+    see every phase of a slot: one of them can pass a slot's parity wait
+    before the load another group waited for has landed."""
+    fails = _schedules(200, mode='state', kxs=3)
+    assert fails and any("read ('x'" in f for f in fails)
+
+
 def test_model_catches_single_diag_w_x_barrier():
-    fails = _schedules(100, xw2=False)
+    fails = _schedules(100, xw_per_slot=False)
     assert fails and any("overrun on XW_READY" in f for f in fails)

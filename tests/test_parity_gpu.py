@@ -13,6 +13,7 @@ from ssd_inputs import to_f64
 pytestmark = pytest.mark.gpu
 
 PATHS = {"simt": 1, "chunked": 2, "fused": 3}
+PATHS_ALL = {"auto": 0, **PATHS}
 
 
 @pytest.fixture(scope="module")
@@ -159,29 +160,56 @@ def test_chunk_invariance(ssd, chunk):
 
 # ---------------------------------------------------------------- prefix state
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("L,N,G", [(1000, 128, 4), (256, 64, 1), (1, 128, 4), (0, 128, 4)])
-def test_prefix_state(ssd, dtype, L, N, G):
+def _paths_for(dtype):
+    return ["auto", "simt"] if dtype == "f32" else ["auto", "simt", "chunked", "fused"]
+
+
+@pytest.mark.parametrize("dtype,path", [(d, p) for d in ("f32", "bf16") for p in _paths_for(d)])
+@pytest.mark.parametrize("L,N,G", [(1000, 128, 4), (256, 64, 1), (2000, 64, 2), (1, 128, 4), (0, 128, 4)])
+def test_prefix_state(ssd, dtype, path, L, N, G):
+    """Every path, with and without a start state; 8 and 16 tiles wrap the
+    fused kernel's 5 (N 128) and 3 (N 64) x slots of its state-only mode."""
     inp = si.bidir_inputs(2, L, 4, 64, N, G, dtype, seed=5, device="cuda")
     init = torch.randn(2, 4, 64, N, device="cuda") * 0.5
     for start in (None, init):
-        st = ssd.ssd_prefix_state(inp["x"], inp["dt"][0], inp["A"][0], inp["B"][0], init=start, chunk=128)
+        st = ssd.ssd_prefix_state(inp["x"], inp["dt"][0], inp["A"][0], inp["B"][0], init=start, chunk=128,
+                                  path=PATHS_ALL[path])
         o = oracle.prefix_state(to_f64(inp["x"]), to_f64(inp["dt"][0]), to_f64(inp["A"][0]),
                                 to_f64(inp["B"][0]), init=None if start is None else to_f64(start))
         check(to_f64(st), o, torch.float32 if dtype == "f32" else torch.bfloat16, f"prefix L={L}", state=True)
 
 
-def test_prefix_state_composes_in_place(ssd):
+@pytest.mark.parametrize("path", ["chunked", "fused"])
+def test_prefix_state_composes_in_place(ssd, path):
     inp = si.bidir_inputs(2, 640, 4, 64, 128, 4, "bf16", seed=9, device="cuda")
     k = 384
     x, dt, A, B = inp["x"], inp["dt"][0], inp["A"][0], inp["B"][0]
-    full = ssd.ssd_prefix_state(x, dt, A, B)
-    st = ssd.ssd_prefix_state(x[:, :k].contiguous(), dt[:, :k].contiguous(), A, B[:, :k].contiguous())
+    pid = PATHS[path]
+    full = ssd.ssd_prefix_state(x, dt, A, B, path=pid)
+    st = ssd.ssd_prefix_state(x[:, :k].contiguous(), dt[:, :k].contiguous(), A, B[:, :k].contiguous(), path=pid)
     ssd.ssd_prefix_state(x[:, k:].contiguous(), dt[:, k:].contiguous(), A, B[:, k:].contiguous(),
-                         init=st, out=st)  # committing a block in place
+                         init=st, out=st, path=pid)  # committing a block in place
     o = oracle.prefix_state(to_f64(x), to_f64(dt), to_f64(A), to_f64(B))
     check(to_f64(st), o, torch.bfloat16, "composed", state=True)
     check(to_f64(full), o, torch.bfloat16, "direct", state=True)
+
+
+@pytest.mark.parametrize("path", ["chunked", "fused"])
+def test_prefix_state_and_block_step_many_units(ssd, path):
+    """160 (batch, head) units: more than there are SMs, so the fused kernel's
+    CTAs take two units each and carry their barrier phases across them."""
+    batch, H, N, G = 40, 4, 128, 2
+    data = si.blockstep_inputs(batch, 700, 64, 1, H, 64, N, G, "bf16", seed=13, device="cuda")
+    pid = PATHS[path]
+    st = ssd.ssd_prefix_state(data["x_pre"], data["dt_pre"], data["A"][0], data["B_pre"], path=pid)
+    step = data["steps"][0]
+    y = ssd.ssd_block_step(step["x"], step["dt"], data["A"], step["B"], step["C"], data["D"], st, path=pid)
+    torch.cuda.synchronize()
+    assert ssd.ssd_get_device_status() == 0
+    st_o = oracle.prefix_state(to_f64(data["x_pre"]), to_f64(data["dt_pre"]), to_f64(data["A"][0]),
+                               to_f64(data["B_pre"]))
+    check(to_f64(st), st_o, torch.bfloat16, f"{path} prefix, 160 units", state=True)
+    check(to_f64(y), _block_oracle(step, data["A"], data["D"], st_o), torch.bfloat16, f"{path} block step, 160 units")
 
 
 def test_prefix_state_full_size_sampled(ssd):
@@ -207,16 +235,23 @@ def _block_oracle(step, A, D, state):
                              to_f64(step["C"]), to_f64(D), state)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_block_step_against_oracle(ssd, dtype):
-    data = si.blockstep_inputs(2, 1000, 64, 3, 4, 64, 128, 2, dtype, device="cuda")
+@pytest.mark.parametrize("dtype,path", [(d, p) for d in ("f32", "bf16") for p in _paths_for(d)])
+@pytest.mark.parametrize("blk,N", [(64, 128), (200, 64)])
+def test_block_step_against_oracle(ssd, dtype, path, blk, N):
+    data = si.blockstep_inputs(2, 1000, blk, 3, 4, 64, N, 2, dtype, device="cuda")
     st = ssd.ssd_prefix_state(data["x_pre"], data["dt_pre"], data["A"][0], data["B_pre"])
     st_o = oracle.prefix_state(to_f64(data["x_pre"]), to_f64(data["dt_pre"]), to_f64(data["A"][0]),
                                to_f64(data["B_pre"]))
     io = torch.float32 if dtype == "f32" else torch.bfloat16
     for k, step in enumerate(data["steps"]):
-        y = ssd.ssd_block_step(step["x"], step["dt"], data["A"], step["B"], step["C"], data["D"], st)
-        check(to_f64(y), _block_oracle(step, data["A"], data["D"], st_o), io, f"step {k}")
+        y = ssd.ssd_block_step(step["x"], step["dt"], data["A"], step["B"], step["C"], data["D"], st,
+                               path=PATHS_ALL[path])
+        check(to_f64(y), _block_oracle(step, data["A"], data["D"], st_o), io, f"{path} step {k}")
+    # no prefix state: the forward scan starts from zero
+    step = data["steps"][0]
+    y = ssd.ssd_block_step(step["x"], step["dt"], data["A"], step["B"], step["C"], data["D"], None,
+                           path=PATHS_ALL[path])
+    check(to_f64(y), _block_oracle(step, data["A"], data["D"], None), io, f"{path} step from zero")
 
 
 def test_block_steps_leave_prefix_state_untouched(ssd):

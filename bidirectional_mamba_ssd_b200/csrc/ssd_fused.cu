@@ -296,6 +296,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const uint32_t tGf = tmem, tGb = tmem + 128, tYof = tmem + 256, tYob = tmem + 320,
                    tYd = tmem + 384, tS = tmem + 448;
     const int nt = p.nt;
+    // tiles of the state pass: all of them forward; in reverse all but tile 0,
+    // whose own tile state no tile to its left receives
+    const int n1t = kFwd1 ? nt : nt - 1;
     const int hpg = p.H / p.G;
     const size_t dt_dir = (size_t)p.batch * p.L * p.H;
 
@@ -323,7 +326,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++units_done) {
                 const int b = u / p.H, h = u % p.H, gg = h / hpg;
-                for (int k1 = 0; ok && k1 < nt; ++k1) {     // phase 1: x, B of the state pass
+                for (int k1 = 0; ok && k1 < n1t; ++k1) {    // phase 1: x, B of the state pass
                     const int i = kFwd1 ? k1 : nt - 1 - k1;
                     uint32_t xs, rs;
                     if (!(ok = x_slot(xs))) break;
@@ -388,7 +391,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             auto slot_addr = [&](uint32_t s) { return base + S::ring + s * 2 * kSlab; };
             // after an expired wait anywhere in the CTA, no further tiles are issued
             for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
-                for (int k1 = 0; k1 < nt && !*abort_flag; ++k1, ++n1) {  // phase 1: S = B^T (diag(w) X in the x slot)
+                for (int k1 = 0; k1 < n1t && !*abort_flag; ++k1, ++n1) {  // phase 1: S = B^T (diag(w) X in the x slot)
                     const uint32_t n = kx++, xs = n % kXS;
                     const uint32_t rs = wait_ring(kr++);
                     mbar_wait(bar(B_XW_READY + xs), (n / kXS) & 1, abort_flag, p.status, 202);
@@ -518,7 +521,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // the tiles (diag(w) X, tile decay); this group stores the reverse
             // state entering each tile (output modes) and folds the tile's state in.
             start_state(u, kFwd1);
-            for (int k1 = 0; k1 < nt; ++k1, ++n1) {
+            for (int k1 = 0; k1 < nt; ++k1) {
                 const int i = kFwd1 ? k1 : nt - 1 - k1;
                 if (kOut && row < N) {
                     __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
@@ -531,6 +534,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         st_global_v4_hint(dst + 8 * c, v, keep);
                     }
                 }
+                if (k1 == n1t) break;        // reverse: tile 0's own state is not needed
                 const uint32_t pbuf = n1 & 1;
                 mbar_wait(bar(B_G1_READY + n1 % kG1), (n1 / kG1) & 1, abort_flag, p.status, 303);
                 const float gdec = gdec1[n1 % kG1];
@@ -548,6 +552,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 tc_fence_before();
                 sync_c();
                 if (row == 0) mbar_arrive(bar(B_P1S_FREE + pbuf));
+                ++n1;
             }
             if constexpr (!kOut) {
                 // the state mode's result: the forward state after the last tile
@@ -559,7 +564,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 cu += gridDim.x;
                 continue;
             }
-            kx += nt;        // the reverse pass's x loads and diag(w') X releases belong to groups A and B
+            kx += n1t;       // the reverse pass's x loads and diag(w') X releases belong to groups A and B
             // phase 2 starts from H_f = 0 (the init mode: from the given state); the
             // reverse states go to the TMA proxy
             start_state(u, MODE == kModeBidirInit);
@@ -661,7 +666,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // the x slot, and the tile decay exp(A sum dt) for group C's chain.
             uint32_t rawn = 0;               // dt of this group's next tile, fetched a tile ahead
             bool have = false;
-            for (int k1 = 0; k1 < nt; ++k1, ++m1, ++kx) {
+            for (int k1 = 0; k1 < n1t; ++k1, ++m1, ++kx) {
                 if ((m1 & 1) != (uint32_t)is_b) continue;
                 const int i = kFwd1 ? k1 : nt - 1 - k1;
                 float vb = 0.f;
@@ -671,7 +676,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     const int t = i * kTile + row;
                     if (t < p.L) vb = __bfloat162float(p.dt[dt1 + ((size_t)b * p.L + t) * p.H + h]);
                 }
-                have = k1 + 2 < nt;          // this group's next tile, two on in the pass's order
+                have = k1 + 2 < n1t;         // this group's next tile, two on in the pass's order
                 rawn = 0;
                 if (have) {
                     const int t = (kFwd1 ? i + 2 : i - 2) * kTile + row;

@@ -62,6 +62,9 @@ class Sim:
         if name not in self.bars:
             self.bars[name] = Bar(name, count)
         return self.bars[name]
+    def n1t(self):
+        """tiles of the state pass: all forward; in reverse all but the leftmost"""
+        return self.nt if self.mode == 'state' else self.nt - 1
     def xw(self, n):
         """barrier and phase of diag(w) X for the tile with x load index n"""
         if self.xw_per_slot:
@@ -97,7 +100,7 @@ def producer(S, units_list):
     kr = kx = kh = 0
     units_done = 0
     for u in units_list:
-        for i in range(nt):                      # the state pass's tiles, in its order
+        for i in range(S.n1t()):                 # the state pass's tiles, in its order
             xs = kx % X
             if kx >= X:
                 yield ('wait', 'X_EMPTY%d' % xs, kx // X - 1)
@@ -135,7 +138,7 @@ def mma(S, units_list):
     n_m = n_sfree = n_yfree = 0
     first2 = True
     for u in units_list:
-        for i in range(nt):
+        for i in range(S.n1t()):
             n = kx; xs = n % X; kx += 1
             rs = kr % R
             yield ('wait', 'RING_FULL%d' % rs, kr // R); kr += 1
@@ -189,10 +192,13 @@ def group_c(S, units_list):
     nt, X, K = S.nt, S.kxs, S.kG1
     kx = n_s = nvec = n1 = 0
     for u in units_list:
-        # phase 1: the state chain only (groups A and B prepare the tiles)
+        # phase 1: the state chain only (groups A and B prepare the tiles); the
+        # reverse chain stores nt states and folds all tiles but the last one
         for i in range(nt):
             if S.mode != 'state':
                 yield ('write', ('hbg', u, i), ('hbg', u, i))
+            if i == S.n1t():
+                break
             pb = n1 % 2
             yield ('wait', 'G1_READY%d' % (n1 % K), n1 // K)
             yield ('read', ('gdec', n1 % K), ('g', u, i))
@@ -204,7 +210,7 @@ def group_c(S, units_list):
             n1 += 1
         if S.mode == 'state':
             continue
-        kx += nt
+        kx += S.n1t()
         yield ('write', 'hf', ('hf', u, 0))
         yield ('arrive', 'HB_WRITTEN')
         for i in range(nt):
@@ -233,7 +239,7 @@ def group_ab(S, units_list, is_b):
     blocks = range(half, 8, 2)
     for u in units_list:
         # phase 1: every other state-pass tile, by the running tile count
-        for i in range(nt):
+        for i in range(S.n1t()):
             if (m1 & 1) == half:
                 xs = kx % X
                 yield ('wait', 'X_FULL%d' % xs, kx // X)

@@ -341,7 +341,6 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                          64 * k, gg, i * kTile, b, kFwd1 ? 0 : 1, pol1);
                 }
                 if (!ok) break;
-                if (kOut && !(ok = mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103))) break;
                 for (int i = 0; kOut && ok && i < nt; ++i) {        // phase 2: x, C_f, B_f, C_b, B_b, H_b
                     const int t0 = i * kTile;
                     uint32_t xs;
@@ -361,6 +360,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                              bar(B_RING_FULL + rs), 64 * k, gg, t0, b, dirs[j], stream);
                     }
                     if (!ok) break;
+                    // the unit's reverse states are in global memory once group C is
+                    // past its reverse chain; the x and B/C loads above go out before
+                    if (i == 0 && !(ok = mbar_wait(bar(B_HB_WRITTEN), units_done & 1, abort_flag, p.status, 103)))
+                        break;
                     if (kh >= 1 && !(ok = mbar_wait(bar(B_HB_EMPTY), (kh - 1) & 1, abort_flag, p.status, 104))) break;
                     ++kh;
                     mbar_arrive_expect_tx(bar(B_HB_FULL), S::kH);
@@ -381,7 +384,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);    // C (K) x B (K)
             constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);      // C (K) x H (MN); M (K) x X (MN)
             uint32_t kr = 0, kx = 0, kh = 0, n1 = 0;
-            uint32_t n_m = 0, n_sfree = 0, n_yfree = 0;
+            uint32_t n_m = 0, n_sfree = 0, n_yfree = 0, n_hbw = 0;
             bool first2 = true;
             auto wait_ring = [&](uint32_t k) -> uint32_t {
                 const uint32_t s = k % kRing;
@@ -418,6 +421,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     const uint32_t rCb = wait_ring(kr++), rBb = wait_ring(kr++);
                     const uint32_t sCf = slot_addr(rCf), sBf = slot_addr(rBf);
                     const uint32_t sCb = slot_addr(rCb), sBb = slot_addr(rBb);
+                    // G_f overwrites the reverse pass's TMEM tile states and Y_o,f reads
+                    // H_f: the unit's first output tile waits until group C is done with
+                    // the former and has zeroed (or seeded) the latter
+                    if (i == 0) mbar_wait(bar(B_HB_WRITTEN), n_hbw++ & 1, abort_flag, p.status, 210);
                     tc_fence_after();
                     // G_f = C_f B_f^T, G_b = C_b B_b^T (earlier readers of these TMEM
                     // columns are MMAs issued before, which complete in order)

@@ -114,7 +114,6 @@ def producer(S, units_list):
         units_done += 1
         if S.mode == 'state':
             continue
-        yield ('wait', 'HB_WRITTEN', units_done - 1)
         for i in range(nt):
             xs = kx % X
             if kx >= X:
@@ -127,6 +126,8 @@ def producer(S, units_list):
                     yield ('wait', 'RING_EMPTY%d' % rs, kr // R - 1)
                 kr += 1
                 yield ('tma', 'RING_FULL%d' % rs, [(('ring', rs), (name, u, i))])
+            if i == 0:
+                yield ('wait', 'HB_WRITTEN', units_done - 1)
             if kh >= 1:
                 yield ('wait', 'HB_EMPTY', kh - 1)
             kh += 1
@@ -135,7 +136,7 @@ def producer(S, units_list):
 def mma(S, units_list):
     nt, R, X = S.nt, S.kRing, S.kxs
     kr = kx = kh = n1 = 0
-    n_m = n_sfree = n_yfree = 0
+    n_m = n_sfree = n_yfree = n_hbw = 0
     first2 = True
     for u in units_list:
         for i in range(S.n1t()):
@@ -162,6 +163,8 @@ def mma(S, units_list):
                 yield ('wait', 'RING_FULL%d' % rs, kr // R); kr += 1
                 slots.append(rs)
             rCf, rBf, rCb, rBb = slots
+            if i == 0:
+                yield ('wait', 'HB_WRITTEN', n_hbw); n_hbw += 1
             yield ('mma', [(('ring', rCf), ('Cf', u, i)), (('ring', rBf), ('Bf', u, i))],
                    [(('tGf', b), ('Gf', u, i)) for b in range(8)])
             yield ('mma', [(('ring', rCb), ('Cb', u, i)), (('ring', rBb), ('Bb', u, i))],

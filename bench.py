@@ -34,19 +34,20 @@ sys.path.insert(0, ROOT)
 
 METRIC = "bidir SSD tokens/s at 130M shape L=1024 (1×B200) + % roofline"
 DEFAULT_WORKLOAD = "mixer130m_b32_L1024"
-PATH_IDS = {"auto": 0, "simt": 1, "chunked": 2, "fused": 3}
+PATH_IDS = {"auto": 0, "simt": 1, "chunked": 2, "fused": 3, "segmented": 4}
 # kernels each path launches per ssd_bidir_fwd call (bf16)
-LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1}
+LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1, "segmented": 4}
 # sources each path's kernels compile from (a traffic record is valid only
 # while their hash is unchanged)
 KERNEL_SOURCE = {
     "simt": ("ssd_simt.cu", "ssd_common.cuh"),
     "chunked": ("ssd_tc.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
     "fused": ("ssd_fused.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
+    "segmented": ("ssd_segments.cu", "ssd_fused.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
 }
 # kernels one call of each path launches (names as in ncu's "Kernel Name")
 KERNEL_NAMES = {"simt": ("scan_simt_kernel",), "chunked": ("tc_state_kernel", "tc_pass_kernel", "tc_out_kernel"),
-                "fused": ("tc_fused_kernel",)}
+                "fused": ("tc_fused_kernel",), "segmented": ("tc_fused_kernel", "seg_scan_kernel")}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -138,7 +139,9 @@ def record_traffic(csv_path: str, path: str, workload: str, command: str, scale:
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
-    per_call = sum(sum(v) / len(v) for v in per.values()) * scale
+    # every launch captured, over the calls (the kernel launched fewest times
+    # is launched once per call; the segmented path launches the fused kernel thrice)
+    per_call = sum(sum(v) for v in per.values()) / calls * scale
     e = {"dram_bytes_per_launch": round(per_call), "calls_captured": calls, "kernels": list(names),
          "source_sha": kernel_source_sha(path), "command": command}
     if scale != 1.0:
@@ -473,7 +476,9 @@ def main():
             "peak_source": f"{peaks['source']} STREAM-copy HBM GB/s",
             "algorithmic_bytes_per_launch": abytes,
             "kernel": {"simt": "scan_simt_kernel", "chunked": "tc_state/tc_pass/tc_out kernels (whole step)",
-                       "fused": "tc_fused_kernel"}[path_name]}
+                       "fused": "tc_fused_kernel",
+                       "segmented": "tc_fused_kernel (forward state, reverse state, bidirectional) + seg_scan_kernel "
+                                    "(whole step)"}[path_name]}
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -57,6 +57,11 @@ constexpr long long kFusedMinUnits = 64;
 int auto_path(int batch, int seqlen, int nheads, int ngroups, int dstate, int dtype) {
     if (dtype != SSD_BF16) return SSD_PATH_SIMT;
     if (ssd::tc_fused_supported(batch, seqlen, nheads, ngroups, dstate)) return SSD_PATH_FUSED;
+    // a few long sequences: split them into segments when that leaves at
+    // least 4 tiles per SM to work on
+    const long long units = (long long)batch * nheads, nt = (seqlen + 127) / 128;
+    const int sms = ssd::device_sms();
+    if (units * nt >= 4LL * sms && ssd::seg_count(units, seqlen, sms) > 1) return SSD_PATH_SEGMENTED;
     return SSD_PATH_CHUNKED;
 }
 
@@ -66,7 +71,7 @@ int bidir_impl(const void *x, const void *dt, const float *A, const void *B, con
                size_t ws_bytes, void *stream) {
     int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
     if (rc != SSD_OK) return rc;
-    if (path < SSD_PATH_AUTO || path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
+    if (path < SSD_PATH_AUTO || path > SSD_PATH_SEGMENTED) return SSD_ERR_INVALID_ARG;
     if (!workspace) return SSD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
     if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, seqlen, nheads, headdim, dstate,
@@ -98,6 +103,15 @@ int bidir_impl(const void *x, const void *dt, const float *A, const void *B, con
     t.workspace = workspace; t.ws_bytes = ws_bytes;
     t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
     if (path == SSD_PATH_FUSED) return to_status(ssd::launch_tc_fused(t, s));
+    if (path == SSD_PATH_SEGMENTED) {
+        // at least two segments, even where one would be chosen
+        const int sms = ssd::device_sms();
+        int S = ssd::seg_count((long long)batch * nheads, seqlen, sms > 0 ? sms : 1);
+        for (int k = 2; S < 2 && k <= 64 && seqlen / k >= 128; ++k)
+            if (seqlen % k == 0) S = k;
+        if (S < 2) return SSD_ERR_UNSUPPORTED;
+        return to_status(ssd::launch_tc_segmented(t, S, s));
+    }
     return to_status(ssd::launch_tc_chunked(t, s));
 }
 
@@ -115,8 +129,10 @@ size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdi
         if (op == SSD_OP_BIDIR_FWD) {
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 2);
             size_t f = ssd::tc_fused_scratch_bytes(batch, seqlen, nheads, dstate);
+            size_t g = ssd::tc_segmented_scratch_bytes(batch, seqlen, nheads, dstate);
             scratch = scratch > c ? scratch : c;
             scratch = scratch > f ? scratch : f;
+            scratch = scratch > g ? scratch : g;
         } else if (op == SSD_OP_PREFIX_STATE) {
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 1);
             scratch = scratch > c ? scratch : c;

@@ -68,6 +68,7 @@ enum : int {
     kModeBidir = 0,      // both scans, summed output
     kModeBidirInit = 1,  // the same with the forward scan started from a given state
     kModeState = 2,      // the forward scan's final state only (optionally from a given state)
+    kModeStateRev = 3,   // the reverse scan's final state only (the state at the sequence start)
 };
 
 // x slots: two in every mode. The count must be even: groups A and B take
@@ -85,7 +86,8 @@ struct FusedParams {
     const float *D;            // (2, H)
     __nv_bfloat16 *hb;         // (units, nt, N, 64) reverse states entering each tile
     const float *init;         // (batch, H, 64, N) forward start state (init / state modes) or nullptr
-    float *state_out;          // (batch, H, 64, N) final forward state (state mode)
+    const float *rinit;        // (batch, H, 64, N) reverse start state at the sequence end (init mode) or nullptr
+    float *state_out;          // (batch, H, 64, N) final state of the state modes
     DeviceStatus *status;
     int batch, L, H, G, nt, units;
 };
@@ -256,7 +258,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     using S = Smem<N>;
     constexpr int NSLAB = N / 64;
     constexpr uint32_t kXS = x_slots<N, MODE>();
-    constexpr bool kOut = MODE != kModeState;      // an output pass follows the state pass
+    constexpr bool kOut = MODE == kModeBidir || MODE == kModeBidirInit;   // an output pass follows the state pass
     constexpr bool kFwd1 = MODE == kModeState;     // the state pass runs forward (else reverse)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -296,9 +298,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const uint32_t tGf = tmem, tGb = tmem + 128, tYof = tmem + 256, tYob = tmem + 320,
                    tYd = tmem + 384, tS = tmem + 448;
     const int nt = p.nt;
-    // tiles of the state pass: all of them forward; in reverse all but tile 0,
-    // whose own tile state no tile to its left receives
-    const int n1t = kFwd1 ? nt : nt - 1;
+    // tiles of the state pass: all of them in the state modes; before an output
+    // pass all but tile 0, whose own tile state no tile to its left receives
+    const int n1t = kOut ? nt - 1 : nt;
     const int hpg = p.H / p.G;
     const size_t dt_dir = (size_t)p.batch * p.L * p.H;
 
@@ -487,11 +489,11 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const uint64_t keep = policy_evict_last();
         uint32_t kx = 0, n_s = 0, nvec = 0, n1 = 0;
         float hreg[kP];
-        // hreg <- the given forward start state of unit u (row n of the (64, N)
-        // state, transposed: hreg[p] = state[p][n]) or zero
-        auto start_state = [&](int u, bool given) {
-            if (given && p.init && row < N) {
-                const float *ip = p.init + (size_t)u * kP * N + row;
+        // hreg <- a given start state of unit u (row n of the (64, N) state,
+        // transposed: hreg[p] = state[p][n]) or zero
+        auto start_state = [&](int u, const float *given) {
+            if (given && row < N) {
+                const float *ip = given + (size_t)u * kP * N + row;
 #pragma unroll
                 for (int j = 0; j < kP; ++j) hreg[j] = ip[(size_t)j * N];
             } else {
@@ -527,7 +529,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // the state mode forward, from the given state). Groups A and B prepare
             // the tiles (diag(w) X, tile decay); this group stores the reverse
             // state entering each tile (output modes) and folds the tile's state in.
-            start_state(u, kFwd1);
+            start_state(u, kFwd1 ? p.init : (MODE == kModeBidirInit ? p.rinit : nullptr));
             for (int k1 = 0; k1 < nt; ++k1) {
                 const int i = kFwd1 ? k1 : nt - 1 - k1;
                 if (kOut && row < N) {
@@ -574,7 +576,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             kx += n1t;       // the reverse pass's x loads and diag(w') X releases belong to groups A and B
             // phase 2 starts from H_f = 0 (the init mode: from the given state); the
             // reverse states go to the TMA proxy
-            start_state(u, MODE == kModeBidirInit);
+            start_state(u, MODE == kModeBidirInit ? p.init : nullptr);
             if (row < N) {
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
@@ -806,12 +808,11 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 template <int N, int MODE>
 cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     using S = Smem<N>;
-    constexpr bool kOut = MODE != kModeState;
+    constexpr bool kOut = MODE == kModeBidir || MODE == kModeBidirInit;
     const int nt = (a.L + kTile - 1) / kTile;
     const int units = a.batch * a.H;
     if (a.ws_bytes < kStatusBytes + (kOut ? tc_fused_scratch_bytes(a.batch, a.L, a.H, N) : 0))
         return cudaErrorInvalidValue;
-    if (MODE == kModeBidirInit && !a.init) return cudaErrorInvalidValue;
     if (!kOut && !a.state_out) return cudaErrorInvalidValue;
     FusedParams p{};
     p.dt = static_cast<const __nv_bfloat16 *>(a.dt);
@@ -819,12 +820,15 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     p.D = a.D;
     p.hb = kOut ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(a.workspace) + kStatusBytes) : nullptr;
     p.init = a.init;
+    p.rinit = a.rinit;
     p.state_out = a.state_out;
     p.status = static_cast<DeviceStatus *>(a.workspace);
     p.batch = a.batch; p.L = a.L; p.H = a.H; p.G = a.G; p.nt = nt; p.units = units;
 
     CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_out;
-    if (!tmap::map_x(&tm_x, a.x, a.batch, a.L, a.H) || !tmap::map_bc(&tm_b, a.B, kOut ? 2 : 1, a.batch, a.L, a.G, N))
+    // the forward state mode may be given single-direction B; every other mode reads both directions' layout
+    if (!tmap::map_x(&tm_x, a.x, a.batch, a.L, a.H) ||
+        !tmap::map_bc(&tm_b, a.B, MODE == kModeState ? 1 : 2, a.batch, a.L, a.G, N))
         return cudaErrorInvalidValue;
     if (kOut) {
         if (!tmap::map_bc(&tm_c, a.C, 2, a.batch, a.L, a.G, N) ||
@@ -874,11 +878,15 @@ bool tc_fused_supported(int batch, int L, int H, int G, int N) {
 }
 
 cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream) {
-    return a.init ? launch_mode<kModeBidirInit>(a, stream) : launch_mode<kModeBidir>(a, stream);
+    return a.init || a.rinit ? launch_mode<kModeBidirInit>(a, stream) : launch_mode<kModeBidir>(a, stream);
 }
 
 cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream) {
     return launch_mode<kModeState>(a, stream);
+}
+
+cudaError_t launch_tc_fused_state_rev(const TcArgs &a, cudaStream_t stream) {
+    return launch_mode<kModeStateRev>(a, stream);
 }
 
 }  // namespace ssd

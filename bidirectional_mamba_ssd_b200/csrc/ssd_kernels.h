@@ -38,6 +38,7 @@ struct TcArgs {
     const void *C;            // (2, batch, L, G, N) bf16 or nullptr
     const float *D;           // (2, H)
     const float *init;        // (batch, H, 64, N) forward start state or nullptr
+    const float *rinit = nullptr;  // (batch, H, 64, N) reverse start state (at the sequence end) or nullptr
     float *state_out;         // (batch, H, 64, N) or nullptr
     void *out;                // (batch, L, H, 64) bf16
     void *workspace;          // status header + scratch
@@ -58,5 +59,17 @@ cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream);
 // Fused kernel, forward scan only: the final state into a.state_out, from
 // a.init or zero (prefix state); needs no scratch past the status header.
 cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream);
+// Fused kernel, reverse scan only (direction 1 of the direction-stacked
+// inputs): the state at the sequence start into a.state_out, from zero.
+cudaError_t launch_tc_fused_state_rev(const TcArgs &a, cudaStream_t stream);
+
+// Long sequences with fewer (batch, head) units than SMs: each sequence split
+// into S segments (seg_count: the S, 1 = none, that minimises rounds x tiles
+// per segment on `sms` SMs, S dividing L), states handed across segments,
+// then the fused kernel on the segments.
+int seg_count(long long units, int L, int sms);
+size_t tc_segmented_scratch_bytes(int batch, int L, int H, int N);   // max over the S in use
+cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream);
+int device_sms();   // SM count of the current device, 0 if it cannot be read
 
 }  // namespace ssd

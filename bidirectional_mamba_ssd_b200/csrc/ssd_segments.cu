@@ -1,0 +1,159 @@
+// Bidirectional scan of long sequences split into segments, for batches with
+// fewer (batch, head) units than SMs: the fused kernel takes one unit per SM,
+// so a few long sequences would leave most SMs idle. Each sequence is viewed
+// as S consecutive segments (the row-major tensors reshape for free to
+// batch*S sequences of L/S tokens) and:
+//   1. the fused kernel's forward state mode gives each segment's forward
+//      state at its end, from zero;
+//   2. its reverse state mode gives each segment's reverse state at its
+//      start, from zero;
+//   3. seg_scan_kernel turns those into the state entering each segment from
+//      the left (forward) and from the right (reverse):
+//        Hf_in(s) = sum_{r<s} (prod_{r<q<s} g_f(q)) Sf(r),
+//        Hb_in(s) = sum_{r>s} (prod_{s<q<r} g_b(q)) Sb(r),
+//      with g(q) = exp(A sum of dt over segment q);
+//   4. the fused bidirectional kernel runs on the segments, its forward scan
+//      seeded with Hf_in and its reverse scan with Hb_in.
+// The recurrence is linear in the state, so this equals the scan over the
+// whole sequence up to rounding. The pages describe no such split (they run
+// 65K-token full-sequence denoising: "Training Hybrid Block Diffusion
+// Language Models with Partial Bidirectionality", Key Results); it is the
+// plain consequence of the recurrence, used here to spread a few long
+// sequences over all SMs.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ssd_common.cuh"
+#include "ssd_kernels.h"
+
+namespace ssd {
+namespace {
+
+constexpr int kP = 64;
+constexpr int kMaxSeg = 64;
+constexpr int kScanThreads = 256;
+
+// grid (batch * H, 2 directions), 256 threads.
+__global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(const __nv_bfloat16 *dt, const float *A,
+                                                                const float *Sf, const float *Sb, float *Hf,
+                                                                float *Hb, int batch, int L, int H, int S,
+                                                                int N) {
+    const int u = blockIdx.x, dir = blockIdx.y;
+    const int b = u / H, h = u % H;
+    const int Ls = L / S;
+    __shared__ float lg[kMaxSeg];          // A * (sum of dt over the segment)
+    __shared__ float red[kScanThreads / 32];
+    const __nv_bfloat16 *d = dt + ((size_t)(dir * batch + b) * L) * H + h;
+    const float a = A[dir * H + h];
+    for (int seg = 0; seg < S; ++seg) {
+        float sum = 0.f;
+        for (int t = threadIdx.x; t < Ls; t += kScanThreads)
+            sum += __bfloat162float(d[(size_t)(seg * Ls + t) * H]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float tot = 0.f;
+            for (int w = 0; w < kScanThreads / 32; ++w) tot += red[w];
+            lg[seg] = a * tot;
+        }
+        __syncthreads();
+    }
+    const float *sin = dir ? Sb : Sf;
+    float *hout = dir ? Hb : Hf;
+    const int elems = kP * N;
+    for (int e = threadIdx.x * 4; e < elems; e += kScanThreads * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < S; ++k) {
+            const int seg = dir ? S - 1 - k : k;
+            const size_t su = ((size_t)(b * S + seg) * H + h) * elems + e;   // segment unit of the reshaped batch
+            *reinterpret_cast<float4 *>(hout + su) = acc;
+            const float4 v = *reinterpret_cast<const float4 *>(sin + su);
+            const float g = __expf(lg[seg]);
+            acc = make_float4(fmaf(g, acc.x, v.x), fmaf(g, acc.y, v.y), fmaf(g, acc.z, v.z), fmaf(g, acc.w, v.w));
+        }
+    }
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct SegLayout {
+    size_t fused, states, total;   // fused kernel scratch, then Sf, Sb, Hf, Hb
+};
+
+SegLayout seg_layout(int batch, int L, int H, int N, int S) {
+    SegLayout l;
+    l.fused = align256(tc_fused_scratch_bytes(batch * S, L / S, H, N));
+    l.states = align256((size_t)batch * S * H * kP * N * sizeof(float));
+    l.total = l.fused + 4 * l.states;
+    return l;
+}
+
+}  // namespace
+
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+}
+
+int seg_count(long long units, int L, int sms) {
+    if (sms <= 0 || units >= sms || L < 2 * 128) return 1;
+    const long long nt = (L + 127) / 128;
+    long long best_cost = ((units + sms - 1) / sms) * nt;
+    int best = 1;
+    for (int S = 2; S <= kMaxSeg && L / S >= 128; ++S) {
+        if (L % S) continue;
+        const long long nts = (L / S + 127) / 128;
+        const long long cost = ((units * S + sms - 1) / sms) * nts;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = S;
+        }
+    }
+    return best;
+}
+
+size_t tc_segmented_scratch_bytes(int batch, int L, int H, int N) {
+    size_t m = 0;
+    for (int S = 2; S <= kMaxSeg && L / S >= 128; ++S) {
+        if (L % S) continue;
+        const size_t t = seg_layout(batch, L, H, N, S).total;
+        m = t > m ? t : m;
+    }
+    return m;
+}
+
+cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
+    if (S < 2 || S > kMaxSeg || a.L % S || a.L / S < 1 || a.ndir != 2) return cudaErrorNotSupported;
+    const SegLayout lay = seg_layout(a.batch, a.L, a.H, a.N, S);
+    if (a.ws_bytes < kStatusBytes + lay.total) return cudaErrorInvalidValue;
+    char *scratch = static_cast<char *>(a.workspace) + kStatusBytes;
+    float *Sf = reinterpret_cast<float *>(scratch + lay.fused);
+    float *Sb = reinterpret_cast<float *>(scratch + lay.fused + lay.states);
+    float *Hf = reinterpret_cast<float *>(scratch + lay.fused + 2 * lay.states);
+    float *Hb = reinterpret_cast<float *>(scratch + lay.fused + 3 * lay.states);
+    TcArgs v = a;             // the segments as a batch of batch * S sequences of L / S tokens
+    v.batch = a.batch * S;
+    v.L = a.L / S;
+    v.init = nullptr;
+    v.rinit = nullptr;
+    cudaError_t e;
+    TcArgs f = v;
+    f.state_out = Sf;
+    if ((e = launch_tc_fused_state(f, stream)) != cudaSuccess) return e;
+    TcArgs r = v;
+    r.state_out = Sb;
+    if ((e = launch_tc_fused_state_rev(r, stream)) != cudaSuccess) return e;
+    seg_scan_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(a.dt), a.A, Sf, Sb, Hf, Hb, a.batch, a.L, a.H, S, a.N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    TcArgs o = v;
+    o.init = Hf;
+    o.rinit = Hb;
+    return launch_tc_fused(o, stream);
+}
+
+}  // namespace ssd

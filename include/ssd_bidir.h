@@ -84,7 +84,11 @@ enum {
     SSD_PATH_AUTO = 0,     /* what ssd_bidir_fwd uses */
     SSD_PATH_SIMT = 1,     /* sequential fp32 scan on CUDA cores, any dtype */
     SSD_PATH_CHUNKED = 2,  /* tensor-core chunked path in three kernels (states through the workspace) */
-    SSD_PATH_FUSED = 3     /* tensor-core path, one kernel per (batch, head) */
+    SSD_PATH_FUSED = 3,    /* tensor-core path, one kernel per (batch, head) */
+    SSD_PATH_SEGMENTED = 4 /* long sequences, few (batch, head): each sequence split into S
+                              segments (S divides seqlen); forward and reverse segment states
+                              (fused kernel, state modes), a segment scan, then the fused
+                              kernel on the segments seeded with the handed-over states */
 };
 
 /* The SSD_PATH_* that ssd_bidir_fwd (SSD_PATH_AUTO) runs for these sizes, or

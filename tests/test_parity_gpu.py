@@ -14,6 +14,7 @@ pytestmark = pytest.mark.gpu
 
 PATHS = {"simt": 1, "chunked": 2, "fused": 3}
 PATHS_ALL = {"auto": 0, **PATHS}
+BIDIR_PATHS = {**PATHS, "segmented": 4}
 
 
 @pytest.fixture(scope="module")
@@ -54,13 +55,13 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("path", list(BIDIR_PATHS))
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "b%d_L%d_H%d_N%d_G%d_Q%d" % s)
 def test_bf16_small(ssd, shape, path):
     batch, L, H, N, G, chunk = shape
     inp = si.bidir_inputs(batch, L, H, 64, N, G, "bf16", seed=L + H, device="cuda")
     try:
-        y = run_bidir(ssd, inp, chunk, PATHS[path])
+        y = run_bidir(ssd, inp, chunk, BIDIR_PATHS[path])
     except ssd.SSDError as e:
         if e.status == ssd.SSD_ERR_UNSUPPORTED and path != "simt":
             pytest.skip(f"{path} path not available for this shape")
@@ -68,7 +69,7 @@ def test_bf16_small(ssd, shape, path):
     check(y, full_oracle(inp), torch.bfloat16, f"{path} {shape}")
 
 
-@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("path", list(BIDIR_PATHS))
 def test_bf16_decay_range(ssd, path):
     """Per-head decays from mild to extreme (|A| 1 ... 3000, larger dt): the
     decay span of a 32-token block runs from below 1 to thousands, so the
@@ -77,7 +78,7 @@ def test_bf16_decay_range(ssd, path):
     inp = si.bidir_inputs(40, 256, 4, 64, 128, 4, "bf16", seed=11, device="cuda")
     inp["A"] = -torch.tensor([[1.0, 50.0, 300.0, 3000.0], [2.0, 80.0, 500.0, 2000.0]], device="cuda")
     inp["dt"] = (inp["dt"].float() * 3).clamp(max=0.1).to(torch.bfloat16).contiguous()
-    y = run_bidir(ssd, inp, 128, PATHS[path])
+    y = run_bidir(ssd, inp, 128, BIDIR_PATHS[path])
     check(y, full_oracle(inp), torch.bfloat16, f"{path} decay range")
 
 

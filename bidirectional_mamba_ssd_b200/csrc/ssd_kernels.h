@@ -64,8 +64,8 @@ cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream);
 cudaError_t launch_tc_fused_state_rev(const TcArgs &a, cudaStream_t stream);
 
 // Long sequences with fewer (batch, head) units than SMs: each sequence split
-// into S segments (seg_count: the S, 1 = none, that minimises rounds x tiles
-// per segment on `sms` SMs, S dividing L), states handed across segments,
+// into S segments (seg_count: the fewest, S dividing L, that fill 4/5 of `sms`
+// SMs in one round; 1 = none), states handed across segments,
 // then the fused kernel on the segments.
 int seg_count(long long units, int L, int sms);
 size_t tc_segmented_scratch_bytes(int batch, int L, int H, int N);   // max over the S in use

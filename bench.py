@@ -339,7 +339,9 @@ def bench_blockstep(args, w, dev):
             "prefill": {"ms": round(prefill_ms, 4), "tokens_per_s": round(w.batch * w.seqlen / (prefill_ms / 1e3), 1),
                         "algorithmic_bytes": prefill_bytes,
                         "hbm_frac": round(prefill_bytes / (prefill_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
-            "gpu_launches": args.steps * (3 * w.steps + 2),
+            # the fused kernel (one launch per step or commit) from 64 (batch, head)
+            # units, else the chunked kernels (3 per step, 2 per commit)
+            "gpu_launches": args.steps * ((w.steps + 1) if w.batch * w.nheads >= 64 else (3 * w.steps + 2)),
             "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
 

@@ -88,6 +88,7 @@ struct FusedParams {
     const float *init;         // (batch, H, 64, N) forward start state (init / state modes) or nullptr
     const float *rinit;        // (batch, H, 64, N) reverse start state at the sequence end (init mode) or nullptr
     float *state_out;          // (batch, H, 64, N) final state of the state modes
+    float *decay_out;          // (batch, H) state modes: exp(A * sum of dt) over the sequence, or nullptr
     DeviceStatus *status;
     int batch, L, H, G, nt, units;
 };
@@ -530,6 +531,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // the tiles (diag(w) X, tile decay); this group stores the reverse
             // state entering each tile (output modes) and folds the tile's state in.
             start_state(u, kFwd1 ? p.init : (MODE == kModeBidirInit ? p.rinit : nullptr));
+            float lsum = 0.f;               // state modes: log of the sequence's decay, from the tile decays
             for (int k1 = 0; k1 < nt; ++k1) {
                 const int i = kFwd1 ? k1 : nt - 1 - k1;
                 if (kOut && row < N) {
@@ -547,6 +549,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const uint32_t pbuf = n1 & 1;
                 mbar_wait(bar(B_G1_READY + n1 % kG1), (n1 / kG1) & 1, abort_flag, p.status, 303);
                 const float gdec = gdec1[n1 % kG1];
+                if (!kOut) lsum += __logf(gdec);   // -inf once a tile decays to 0: the product is 0 then
                 mbar_wait(bar(B_P1S_READY + pbuf), (n1 >> 1) & 1, abort_flag, p.status, 301);
                 tc_fence_after();
 #pragma unroll
@@ -570,6 +573,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                     for (int j = 0; j < kP; ++j) op[(size_t)j * N] = hreg[j];
                 }
+                if (row == 0 && p.decay_out) p.decay_out[u] = __expf(lsum);
                 cu += gridDim.x;
                 continue;
             }
@@ -822,6 +826,7 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     p.init = a.init;
     p.rinit = a.rinit;
     p.state_out = a.state_out;
+    p.decay_out = a.decay_out;
     p.status = static_cast<DeviceStatus *>(a.workspace);
     p.batch = a.batch; p.L = a.L; p.H = a.H; p.G = a.G; p.nt = nt; p.units = units;
 

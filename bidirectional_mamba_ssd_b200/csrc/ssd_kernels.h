@@ -39,6 +39,7 @@ struct TcArgs {
     const float *D;           // (2, H)
     const float *init;        // (batch, H, 64, N) forward start state or nullptr
     const float *rinit = nullptr;  // (batch, H, 64, N) reverse start state (at the sequence end) or nullptr
+    float *decay_out = nullptr;    // (batch, H) fused state modes: exp(A * sum of dt) over the sequence
     float *state_out;         // (batch, H, 64, N) or nullptr
     void *out;                // (batch, L, H, 64) bf16
     void *workspace;          // status header + scratch

@@ -11,7 +11,8 @@
 //      the left (forward) and from the right (reverse):
 //        Hf_in(s) = sum_{r<s} (prod_{r<q<s} g_f(q)) Sf(r),
 //        Hb_in(s) = sum_{r>s} (prod_{s<q<r} g_b(q)) Sb(r),
-//      with g(q) = exp(A sum of dt over segment q);
+//      with g(q) = exp(A sum of dt over segment q), which the state passes
+//      also return (the product of their tile decays);
 //   4. the fused bidirectional kernel runs on the segments, its forward scan
 //      seeded with Hf_in and its reverse scan with Hb_in.
 // The recurrence is linear in the state, so this equals the scan over the
@@ -33,44 +34,25 @@ constexpr int kP = 64;
 constexpr int kMaxSeg = 64;
 constexpr int kScanThreads = 256;
 
-// grid (batch * H, 2 directions), 256 threads.
-__global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(const __nv_bfloat16 *dt, const float *A,
-                                                                const float *Sf, const float *Sb, float *Hf,
-                                                                float *Hb, int batch, int L, int H, int S,
-                                                                int N) {
+// grid (batch * H, 2 directions), 256 threads; Gf, Gb: each segment's decay
+// exp(A * sum of dt over the segment), from the state passes.
+__global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(const float *Sf, const float *Sb, const float *Gf,
+                                                                const float *Gb, float *Hf, float *Hb, int H,
+                                                                int S, int N) {
     const int u = blockIdx.x, dir = blockIdx.y;
     const int b = u / H, h = u % H;
-    const int Ls = L / S;
-    __shared__ float lg[kMaxSeg];          // A * (sum of dt over the segment)
-    __shared__ float red[kScanThreads / 32];
-    const __nv_bfloat16 *d = dt + ((size_t)(dir * batch + b) * L) * H + h;
-    const float a = A[dir * H + h];
-    for (int seg = 0; seg < S; ++seg) {
-        float sum = 0.f;
-        for (int t = threadIdx.x; t < Ls; t += kScanThreads)
-            sum += __bfloat162float(d[(size_t)(seg * Ls + t) * H]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float tot = 0.f;
-            for (int w = 0; w < kScanThreads / 32; ++w) tot += red[w];
-            lg[seg] = a * tot;
-        }
-        __syncthreads();
-    }
     const float *sin = dir ? Sb : Sf;
+    const float *gin = dir ? Gb : Gf;
     float *hout = dir ? Hb : Hf;
     const int elems = kP * N;
     for (int e = threadIdx.x * 4; e < elems; e += kScanThreads * 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k = 0; k < S; ++k) {
             const int seg = dir ? S - 1 - k : k;
-            const size_t su = ((size_t)(b * S + seg) * H + h) * elems + e;   // segment unit of the reshaped batch
-            *reinterpret_cast<float4 *>(hout + su) = acc;
-            const float4 v = *reinterpret_cast<const float4 *>(sin + su);
-            const float g = __expf(lg[seg]);
+            const size_t su = (size_t)(b * S + seg) * H + h;   // segment unit of the reshaped batch
+            *reinterpret_cast<float4 *>(hout + su * elems + e) = acc;
+            const float4 v = *reinterpret_cast<const float4 *>(sin + su * elems + e);
+            const float g = gin[su];
             acc = make_float4(fmaf(g, acc.x, v.x), fmaf(g, acc.y, v.y), fmaf(g, acc.z, v.z), fmaf(g, acc.w, v.w));
         }
     }
@@ -79,14 +61,15 @@ __global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(const __nv_bfloa
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct SegLayout {
-    size_t fused, states, total;   // fused kernel scratch, then Sf, Sb, Hf, Hb
+    size_t fused, states, decays, total;   // fused kernel scratch, then Sf, Sb, Hf, Hb, then Gf, Gb
 };
 
 SegLayout seg_layout(int batch, int L, int H, int N, int S) {
     SegLayout l;
     l.fused = align256(tc_fused_scratch_bytes(batch * S, L / S, H, N));
     l.states = align256((size_t)batch * S * H * kP * N * sizeof(float));
-    l.total = l.fused + 4 * l.states;
+    l.decays = align256((size_t)batch * S * H * sizeof(float));
+    l.total = l.fused + 4 * l.states + 2 * l.decays;
     return l;
 }
 
@@ -133,6 +116,8 @@ cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
     float *Sb = reinterpret_cast<float *>(scratch + lay.fused + lay.states);
     float *Hf = reinterpret_cast<float *>(scratch + lay.fused + 2 * lay.states);
     float *Hb = reinterpret_cast<float *>(scratch + lay.fused + 3 * lay.states);
+    float *Gf = reinterpret_cast<float *>(scratch + lay.fused + 4 * lay.states);
+    float *Gb = reinterpret_cast<float *>(scratch + lay.fused + 4 * lay.states + lay.decays);
     TcArgs v = a;             // the segments as a batch of batch * S sequences of L / S tokens
     v.batch = a.batch * S;
     v.L = a.L / S;
@@ -141,12 +126,13 @@ cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
     cudaError_t e;
     TcArgs f = v;
     f.state_out = Sf;
+    f.decay_out = Gf;
     if ((e = launch_tc_fused_state(f, stream)) != cudaSuccess) return e;
     TcArgs r = v;
     r.state_out = Sb;
+    r.decay_out = Gb;
     if ((e = launch_tc_fused_state_rev(r, stream)) != cudaSuccess) return e;
-    seg_scan_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(a.dt), a.A, Sf, Sb, Hf, Hb, a.batch, a.L, a.H, S, a.N);
+    seg_scan_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, Hf, Hb, a.H, S, a.N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     TcArgs o = v;
     o.init = Hf;

@@ -73,6 +73,9 @@ WORKLOADS = {
         Workload("packed128_b512_g1", 512, 128, 24, 64, 128, 1, 64, "bf16"),
         # long-context full-sequence mixer
         Workload("long_L65536", 1, 65536, 32, 64, 128, 32, 256, "bf16"),
+        # the same layout at 16384 tokens (~0.7 GB on the device: small enough
+        # for a full profiler capture of the segmented path's kernels)
+        Workload("long_L16384", 1, 16384, 32, 64, 128, 32, 256, "bf16"),
         # block-diffusion step: prefix of 262144 tokens, active block of 64, 32 steps
         Workload("blockstep_prefix262144_blk64", 4, 262144, 32, 64, 128, 32, 256, "bf16",
                  block=64, steps=32),

@@ -42,8 +42,9 @@ LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1, "segmented": 4}
 KERNEL_SOURCE = {
     "simt": ("ssd_simt.cu", "ssd_common.cuh"),
     "chunked": ("ssd_tc.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
-    "fused": ("ssd_fused.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
-    "segmented": ("ssd_segments.cu", "ssd_fused.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
+    "fused": ("ssd_fused.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
+    "segmented": ("ssd_segments.cu", "ssd_fused.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h",
+                  "ssd_common.cuh"),
 }
 # kernels one call of each path launches (names as in ncu's "Kernel Name")
 KERNEL_NAMES = {"simt": ("scan_simt_kernel",), "chunked": ("tc_state_kernel", "tc_pass_kernel", "tc_out_kernel"),

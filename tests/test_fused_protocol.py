@@ -21,47 +21,21 @@ The model must be kept in step with the kernel when its protocol changes.
 A planted variant with a single diag(w) X barrier (the kernel's earlier
 design, which did overrun on the GPU) must be caught.
 """
-import heapq
-import itertools
 import random
 
-import pytest
+from protocol_sim import Bug, Sched, run_roles
 
 
-class Bug(Exception):
-    pass
-
-class Bar:
-    def __init__(self, name, count):
-        self.name, self.count, self.pending, self.c = name, count, count, 0
-    def arrive(self):
-        self.pending -= 1
-        if self.pending < 0:
-            raise Bug(f"{self.name}: too many arrivals")
-        if self.pending == 0:
-            self.c += 1
-            self.pending = self.count
-
-class Sim:
+class Sim(Sched):
     """One CTA's schedule. mode: 'bidir' (both scans, output pass; the block
     step's seeded variant has the same protocol) or 'state' (the forward state
     pass alone); kxs: x slots; xw_per_slot False plants the earlier single
     diag(w) X barrier."""
     def __init__(self, nt, units, seed, kRing=4, mode='bidir', kxs=2, xw_per_slot=True, heavy=0.1):
-        self.r = random.Random(seed)
-        self.nt, self.units, self.kRing, self.heavy = nt, units, kRing, heavy
+        super().__init__(seed, heavy)
+        self.nt, self.units, self.kRing = nt, units, kRing
         self.mode, self.kxs, self.xw_per_slot = mode, kxs, xw_per_slot
         self.kG1 = 8
-        self.bars = {}
-        self.res = {}
-        self.t = 0.0
-        self.ev = []          # (time, seq, fn)
-        self.seq = itertools.count()
-        self.mma_done_t = 0.0
-    def bar(self, name, count=1):
-        if name not in self.bars:
-            self.bars[name] = Bar(name, count)
-        return self.bars[name]
     def n1t(self):
         """tiles of the state pass: all forward; in reverse all but the leftmost"""
         return self.nt if self.mode == 'state' else self.nt - 1
@@ -70,19 +44,6 @@ class Sim:
         if self.xw_per_slot:
             return 'XW_READY%d' % (n % self.kxs), n // self.kxs
         return 'XW_READY', n
-    def delay(self):
-        d = self.r.expovariate(1.0)
-        if self.r.random() < self.heavy:
-            d *= self.r.choice([10, 50, 200])
-        return d
-    def at(self, t, fn):
-        heapq.heappush(self.ev, (t, next(self.seq), fn))
-    def write(self, k, v):
-        self.res[k] = v
-    def read(self, k, v, who):
-        got = self.res.get(k)
-        if got != v:
-            raise Bug(f"{who}: read {k} expected {v} got {got} at t={self.t:.2f}")
 
 # ---------------------------------------------------------------- roles
 # A role is a generator yielding commands:
@@ -294,123 +255,7 @@ def run(S, units_list):
         'prod': producer(S, units_list), 'mma': mma(S, units_list), 'C': group_c(S, units_list),
         'A': group_ab(S, units_list, False), 'B': group_ab(S, units_list, True),
     }
-    cur = {k: None for k in roles}        # pending command per role
-    ready = {k: 0.0 for k in roles}
-    done = set()
-    syncs = {}                            # name -> set of roles arrived
-    store_pending = {}
-    def bar(n):
-        return S.bar(n, counts.get(n, 1))
-    def step_role(name):
-        """Try to make progress on role `name`; return True if it advanced."""
-        if cur[name] is None:
-            try:
-                cur[name] = next(roles[name])
-            except StopIteration:
-                done.add(name)
-                return True
-        c = cur[name]
-        op = c[0]
-        if op == 'wait':
-            b = bar(c[1]); k = c[2]
-            if b.c >= k + 2:
-                raise Bug(f"{name}: overrun on {c[1]}: waiting for phase {k}, completed {b.c}")
-            if (b.c & 1) != (k & 1):     # the phase with parity k&1 completed (c == k+1)
-                cur[name] = None
-                return True
-            return False
-        if op == 'arrive':
-            bar(c[1]).arrive()
-        elif op == 'tma':
-            bn, writes = c[1], c[2]
-            def land(writes=writes, bn=bn):
-                for k, v in writes:
-                    S.write(k, v)
-                bar(bn).arrive()
-            S.at(S.t + S.delay(), land)
-        elif op == 'tma_hb':
-            bn, u, i = c[1], c[2], c[3]
-            S.read(('hbg', u, i), ('hbg', u, i), name + ' hb load issue')
-            def land(bn=bn, u=u, i=i):
-                S.write('hb', ('hb', u, i))
-                bar(bn).arrive()
-            S.at(S.t + S.delay(), land)
-        elif op == 'mma':
-            reads, writes = c[1], c[2]
-            tdone = max(S.mma_done_t, S.t) + S.delay()
-            S.mma_done_t = tdone
-            def ex(reads=reads, writes=writes):
-                for k, v in reads:
-                    S.read(k, v, 'mma exec')
-                for k, v in writes:
-                    S.write(k, v)
-            S.at(tdone, ex)
-        elif op == 'commit':
-            bn = c[1]
-            S.at(max(S.mma_done_t, S.t) + 1e-6, lambda bn=bn: bar(bn).arrive())
-        elif op == 'read':
-            S.read(c[1], c[2], name)
-        elif op == 'write':
-            S.write(c[1], c[2])
-        elif op == 'sync':
-            nm, n = c[1], c[2]
-            if n == 1:
-                pass
-            else:
-                s = syncs.setdefault(nm, set())
-                s.add(name)
-                if len(s) < n:
-                    return False
-                # all arrived: release the others lazily
-                for other in list(s):
-                    if other != name and cur[other] == c:
-                        cur[other] = None
-                syncs[nm] = set()
-        elif op == 'store':
-            for k, v in c[1]:
-                S.read(k, v, 'store issue')
-            tr = S.t + S.delay()
-            store_pending[name] = (tr, c[1])
-            def rd(items=c[1]):
-                for k, v in items:
-                    S.read(k, v, 'store read')
-            S.at(tr, rd)
-        elif op == 'store_wait':
-            tr, _ = store_pending[name]
-            if S.t < tr:
-                return False
-        cur[name] = None
-        return True
-    while len(done) < len(roles):
-        progressed = True
-        while progressed:
-            progressed = False
-            order = [r for r in roles if r not in done]
-            S.r.shuffle(order)
-            for r in order:
-                if r in done or ready[r] > S.t:
-                    continue
-                # a sync waiter whose partner already released it
-                if step_role(r):
-                    ready[r] = S.t + (S.r.expovariate(4.0) if S.r.random() < 0.5 else 0.0)
-                    progressed = True
-        if len(done) == len(roles):
-            break
-        nxt = [ready[r] for r in roles if r not in done and ready[r] > S.t]
-        tnext = min(nxt) if nxt else None
-        if S.ev and (tnext is None or S.ev[0][0] <= tnext):
-            t, _, fn = heapq.heappop(S.ev)
-            S.t = max(S.t, t)
-            fn()
-        elif tnext is not None:
-            S.t = tnext
-        else:
-            state = {r: cur[r] for r in roles if r not in done}
-            raise Bug(f"deadlock at t={S.t:.2f}: {state}")
-    while S.ev:
-        t, _, fn = heapq.heappop(S.ev)
-        S.t = t
-        fn()
+    run_roles(S, roles, counts)
 
 
 def _schedules(n, mode='bidir', kxs=2, xw_per_slot=True, seed0=0):

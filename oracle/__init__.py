@@ -20,7 +20,11 @@ Parity status: pinned. ``tests/test_oracle_pins.py`` checks this oracle
 against the materialised quadratic form, closed forms (A -> -inf, A = 0, the
 geometric series of a constant input), the flip identity, composability of
 prefix states and a hand-worked golden example; none of those checks calls
-the oracle's own loop to produce its expected value.
+the oracle's own loop to produce its expected value. ``bidir_seeded`` is
+pinned to the other functions: with zero states it is ``block_step`` with no
+prefix; its segments, seeded with the states the rest of the sequence leaves
+(from ``prefix_state`` on either side, the reverse one through the flip
+identity), put together give ``bidir`` over the whole sequence.
 """
 from __future__ import annotations
 
@@ -59,9 +63,10 @@ def configure(lib):
     lib.ssd_oracle_bidir.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, ip, i, i]
     lib.ssd_oracle_prefix_state.argtypes = [dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
     lib.ssd_oracle_block_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
+    lib.ssd_oracle_bidir_seeded.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
     lib.ssd_oracle_threads.argtypes = [i]
     for f in (lib.ssd_oracle_bidir, lib.ssd_oracle_prefix_state,
-              lib.ssd_oracle_block_step, lib.ssd_oracle_threads):
+              lib.ssd_oracle_block_step, lib.ssd_oracle_bidir_seeded, lib.ssd_oracle_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -143,4 +148,30 @@ def block_step(x, dt, A, B, C, D, prefix, nthreads: int = 0) -> np.ndarray:
                                        batch, T, H, P, N, G, int(nthreads))
     if rc != 0:
         raise ValueError("oracle block_step: bad arguments")
+    return out
+
+
+def bidir_seeded(x, dt, A, B, C, D, prefix=None, suffix=None, nthreads: int = 0) -> np.ndarray:
+    """Both scans over a segment with given starting states: the forward scan
+    from `prefix` (the state before the first token), the reverse scan from
+    `suffix` (the reverse state after the last token), plus the D terms.
+    prefix, suffix (batch, H, P, N) or None (zero)."""
+    x = np.asarray(x)
+    batch, L, H, P = x.shape
+    G, N = np.asarray(B).shape[-2:]
+    out = np.zeros((batch, L, H, P))
+    keep = [_f64(a) for a in (x, dt, A, B, C, D)]
+    ptrs = []
+    for s in (prefix, suffix):
+        if s is None:
+            ptrs.append(None)
+        else:
+            a, pa = _f64(s)
+            keep.append((a, pa))
+            ptrs.append(pa)
+    po = out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+    rc = _load().ssd_oracle_bidir_seeded(*(p for _, p in keep[:6]), ptrs[0], ptrs[1], po,
+                                         batch, L, H, P, N, G, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle bidir_seeded: bad arguments")
     return out

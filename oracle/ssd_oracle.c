@@ -223,3 +223,51 @@ int ssd_oracle_block_step(const double *x, const double *dt, const double *A,
     }
     return bad ? -1 : 0;
 }
+
+/* Both scans over a sequence with given starting states: the forward scan
+ * from `prefix` (the forward state before the first token), the reverse scan
+ * from `suffix` (the reverse state after the last token); then the D terms.
+ * This is the mixer over one segment of a longer sequence when prefix and
+ * suffix are the states the tokens outside the segment leave: the recurrence
+ * is the same one as in ssd_oracle_bidir, only its starting states differ.
+ * Layouts as for ssd_oracle_bidir; prefix and suffix (batch, H, P, N), each
+ * may be NULL (zero). */
+int ssd_oracle_bidir_seeded(const double *x, const double *dt, const double *A,
+                            const double *Bm, const double *Cm, const double *D,
+                            const double *prefix, const double *suffix, double *out,
+                            int batch, int L, int H, int P, int N, int G, int nthreads)
+{
+    if (batch < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G) return -1;
+    set_threads(nthreads);
+    const int hpg = H / G;
+    const ptrdiff_t x_ts = (ptrdiff_t)H * P, dt_ts = H, bc_ts = (ptrdiff_t)G * N;
+    const size_t dt_dir = (size_t)batch * L * H;
+    const size_t bc_dir = (size_t)batch * L * G * N;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int u = 0; u < batch * H; ++u) {
+        const int b = u / H, hh = u % H, g = hh / hpg;
+        double *h = (double *)malloc(sizeof(double) * (size_t)N * P);
+        double *y = (double *)calloc((size_t)L * P + 1, sizeof(double));
+        if (!h || !y) { free(h); free(y); bad |= 1; continue; }
+        const double *xu = x + ((size_t)b * L * H + hh) * P;
+        for (int d = 0; d < 2; ++d) {
+            const double *start = d == 0 ? prefix : suffix;
+            for (int n = 0; n < N; ++n)
+                for (int p = 0; p < P; ++p)
+                    h[(size_t)n * P + p] = start ? start[(size_t)u * P * N + (size_t)p * N + n] : 0.0;
+            scan_one_direction(d, L, P, N, xu, x_ts, dt + d * dt_dir + (size_t)b * L * H + hh, dt_ts,
+                               A[d * H + hh], Bm + d * bc_dir + ((size_t)b * L * G + g) * N,
+                               Cm + d * bc_dir + ((size_t)b * L * G + g) * N, bc_ts, h, y);
+        }
+        const double dsum = D[hh] + D[H + hh];
+        for (int t = 0; t < L; ++t) {
+            double *o = out + ((size_t)b * L * H + (size_t)t * H + hh) * P;
+            const double *xt = xu + (size_t)t * x_ts;
+            for (int p = 0; p < P; ++p) o[p] = y[(size_t)t * P + p] + dsum * xt[p];
+        }
+        free(h);
+        free(y);
+    }
+    return bad ? -1 : 0;
+}

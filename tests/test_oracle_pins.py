@@ -263,6 +263,51 @@ def test_block_step_depends_on_prefix_only_through_state():
     assert np.array_equal(oracle.block_step(*args, s1), oracle.block_step(*args, s2))
 
 
+def test_bidir_seeded_with_zero_states_is_the_plain_mixer():
+    rng = np.random.default_rng(21)
+    x, dt, A, B, C, D = rand_problem(rng, batch=2, L=17)
+    y0 = oracle.bidir_seeded(x, dt, A, B, C, D)
+    assert np.array_equal(y0, oracle.block_step(x, dt, A, B, C, D, None))
+    assert rel(y0, oracle.bidir(x, dt, A, B, C, D)) < 1e-14
+
+
+def _reverse_state_after(x, dt, A, B, k):
+    """The reverse state entering token k - 1 from the right: the reverse scan
+    over tokens k..L-1, written as a forward prefix state of the flipped tail
+    (the flip identity), with the reverse direction's parameters."""
+    fl = lambda a: np.flip(a, axis=1).copy()
+    return oracle.prefix_state(fl(x[:, k:]), fl(dt[1][:, k:]), A[1], fl(B[1][:, k:]))
+
+
+def test_bidir_seeded_segments_rebuild_the_whole_sequence():
+    """A sequence cut into segments, each seeded with the forward state the
+    tokens before it leave and the reverse state the tokens after it leave,
+    gives the whole-sequence mixer, segment by segment."""
+    rng = np.random.default_rng(22)
+    x, dt, A, B, C, D = rand_problem(rng, batch=2, L=29)
+    full = oracle.bidir(x, dt, A, B, C, D)
+    cuts = [0, 9, 20, 29]
+    parts = []
+    for k0, k1 in zip(cuts[:-1], cuts[1:]):
+        pre = oracle.prefix_state(x[:, :k0], dt[0][:, :k0], A[0], B[0][:, :k0]) if k0 > 0 else None
+        suf = _reverse_state_after(x, dt, A, B, k1) if k1 < x.shape[1] else None
+        parts.append(oracle.bidir_seeded(x[:, k0:k1], dt[:, :, k0:k1], A, B[:, :, k0:k1], C[:, :, k0:k1], D,
+                                         pre, suf))
+    assert rel(np.concatenate(parts, axis=1), full) < 1e-12
+
+
+def test_bidir_seeded_reverse_start_mirrors_forward_start():
+    """Seeding the reverse scan at the right end is seeding the forward scan of
+    the flipped sequence with the directions swapped."""
+    rng = np.random.default_rng(23)
+    x, dt, A, B, C, D = rand_problem(rng, batch=1, L=11)
+    s = rng.standard_normal((1, 4, 3, 5))
+    y = oracle.bidir_seeded(x, dt, A, B, C, D, None, s)
+    sw = lambda a: np.flip(a[::-1], axis=2).copy()   # swap directions, flip tokens
+    y2 = oracle.bidir_seeded(np.flip(x, 1).copy(), sw(dt), A[::-1].copy(), sw(B), sw(C), D[::-1].copy(), s, None)
+    assert rel(y, np.flip(y2, 1)) < 1e-13
+
+
 def test_units_subset_matches_full():
     rng = np.random.default_rng(12)
     prob = rand_problem(rng, batch=3, L=10, H=4)

@@ -10,6 +10,10 @@ Functions carry the C names:
   ssd_bidir_fwd(x, dt, A, B, C, D, chunk=256)          -> out
   ssd_prefix_state(x, dt, A, B, init=None, chunk=256)  -> state (batch, H, P, N) fp32
   ssd_block_step(x, dt, A, B, C, D, prefix_state)      -> out
+  ssd_segment_states(x, dt, A, B)                      -> (fwd_state, fwd_decay, rev_state, rev_decay)
+  ssd_segment_carry(fwd_states, fwd_decays, rev_states, rev_decays, seg) -> (fwd_in, rev_in)
+  ssd_bidir_fwd_seeded(x, dt, A, B, C, D, fwd_init, rev_init)           -> out
+The sequence-sharded mixer over a process group is in seqshard.py.
 Shapes (row-major, natural token order; [0] forward, [1] reverse):
   x (batch, L, H, P); dt (2, batch, L, H); A, D (2, H) fp32;
   B, C (2, batch, L, G, N); out like x.
@@ -26,7 +30,8 @@ from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSE
                    SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT, SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE,
                    SSD_OP_BLOCK_STEP)
 
-__all__ = ["ssd_bidir_fwd", "ssd_prefix_state", "ssd_block_step", "ssd_workspace_bytes",
+__all__ = ["ssd_bidir_fwd", "ssd_prefix_state", "ssd_block_step", "ssd_segment_states",
+           "ssd_segment_carry", "ssd_bidir_fwd_seeded", "ssd_workspace_bytes",
            "ssd_get_device_status", "SSDError", "Workspace", "lib"]
 
 lib = _c.load()
@@ -230,4 +235,90 @@ def ssd_block_step(x, dt, A, B, C, D, prefix_state, out=None, *, path: int = SSD
                                  _ptr(prefix_state), _ptr(out), batch, T, H, P, N, G, _DT[io],
                                  int(path), _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_block_step")
+    return out
+
+
+def _bidir_args(x, dt, A, B, C, D, what):
+    _need(x, "x", ndim=4)
+    dev, io = x.device, x.dtype
+    if io != torch.bfloat16:
+        raise ValueError(f"{what}: bf16 I/O only (got {io})")
+    _need(dt, "dt", io, dev, 4)
+    _need(B, "B", io, dev, 5)
+    _need(A, "A", torch.float32, dev, 2)
+    batch, L, H, P, G, N = _dims(x, B)
+    if tuple(dt.shape) != (2, batch, L, H) or tuple(B.shape) != (2, batch, L, G, N) or tuple(A.shape) != (2, H):
+        raise ValueError("shape mismatch: want x (b,L,H,P), dt (2,b,L,H), B (2,b,L,G,N), A (2,H)")
+    if C is not None:
+        _need(C, "C", io, dev, 5)
+        _need(D, "D", torch.float32, dev, 2)
+        if tuple(C.shape) != tuple(B.shape) or tuple(D.shape) != (2, H):
+            raise ValueError("shape mismatch: want C like B, D (2,H)")
+    return dev, io, batch, L, H, P, G, N
+
+
+def _state(t, name, dev, shape):
+    if t is not None:
+        _need(t, name, torch.float32, dev, len(shape))
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must be {tuple(shape)}")
+
+
+def ssd_segment_states(x, dt, A, B, *, workspace: Workspace | None = None):
+    """A segment's own states from zero (include/ssd_bidir.h: ssd_segment_states):
+    returns (fwd_state, fwd_decay, rev_state, rev_decay), states (batch, H, P, N)
+    and decays (batch, H), fp32."""
+    dev, io, batch, L, H, P, G, N = _bidir_args(x, dt, A, B, None, None, "ssd_segment_states")
+    fs = torch.empty(batch, H, P, N, dtype=torch.float32, device=dev)
+    rs = torch.empty_like(fs)
+    fd = torch.empty(batch, H, dtype=torch.float32, device=dev)
+    rd = torch.empty_like(fd)
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    buf = ws.get(max(ssd_workspace_bytes(SSD_OP_PREFIX_STATE, batch, L, H, P, N, G, 64, io), 256))
+    rc = lib.ssd_segment_states(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(fs), _ptr(fd), _ptr(rs), _ptr(rd),
+                                batch, L, H, P, N, G, _DT[io], _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_segment_states")
+    return fs, fd, rs, rd
+
+
+def ssd_segment_carry(fwd_states, fwd_decays, rev_states, rev_decays, seg: int):
+    """The states entering segment `seg` from all segments' own states, gathered
+    segment-major (include/ssd_bidir.h: ssd_segment_carry): states (nseg, batch,
+    H, P, N), decays (nseg, batch, H). Returns (fwd_in, rev_in), (batch, H, P, N)."""
+    _need(fwd_states, "fwd_states", torch.float32, None, 5)
+    dev = fwd_states.device
+    nseg, batch, H, P, N = fwd_states.shape
+    _state(rev_states, "rev_states", dev, (nseg, batch, H, P, N))
+    _state(fwd_decays, "fwd_decays", dev, (nseg, batch, H))
+    _state(rev_decays, "rev_decays", dev, (nseg, batch, H))
+    fi = torch.empty(batch, H, P, N, dtype=torch.float32, device=dev)
+    ri = torch.empty_like(fi)
+    rc = lib.ssd_segment_carry(_ptr(fwd_states), _ptr(fwd_decays), _ptr(rev_states), _ptr(rev_decays),
+                               nseg, int(seg), _ptr(fi), _ptr(ri), batch, H, P, N,
+                               ctypes.c_void_p(_stream(dev)))
+    _check(rc, "ssd_segment_carry")
+    return fi, ri
+
+
+def ssd_bidir_fwd_seeded(x, dt, A, B, C, D, fwd_init=None, rev_init=None, out=None, *,
+                         workspace: Workspace | None = None):
+    """Both scans over a segment, the forward one from fwd_init and the reverse
+    one from rev_init at its end (include/ssd_bidir.h: ssd_bidir_fwd_seeded)."""
+    dev, io, batch, L, H, P, G, N = _bidir_args(x, dt, A, B, C, D, "ssd_bidir_fwd_seeded")
+    _state(fwd_init, "fwd_init", dev, (batch, H, P, N))
+    _state(rev_init, "rev_init", dev, (batch, H, P, N))
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _need(out, "out", io, dev, 4)
+        if out.shape != x.shape:
+            raise ValueError("out must have x's shape")
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    buf = ws.get(max(ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, L, H, P, N, G, 64, io), 256))
+    rc = lib.ssd_bidir_fwd_seeded(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(fwd_init),
+                                  _ptr(rev_init), _ptr(out), batch, L, H, P, N, G, _DT[io],
+                                  _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_bidir_fwd_seeded")
     return out

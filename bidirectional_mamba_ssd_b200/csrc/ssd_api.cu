@@ -275,6 +275,83 @@ int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
                                dstate, ngroups, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
 }
 
+int ssd_segment_states(const void *x, const void *dt, const float *A, const void *B, float *fwd_state,
+                       float *fwd_decay, float *rev_state, float *rev_decay, int batch, int seqlen, int nheads,
+                       int headdim, int dstate, int ngroups, int dtype, void *workspace, size_t ws_bytes,
+                       void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype, false);
+    if (rc != SSD_OK) return rc;
+    if (dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_PREFIX_STATE, batch, seqlen, nheads, headdim, dstate, ngroups, 64,
+                                       dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0) return SSD_OK;
+    if (seqlen == 0) return SSD_ERR_UNSUPPORTED;
+    if (!x || !dt || !A || !B || !fwd_state || !fwd_decay || !rev_state || !rev_decay) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned4(A) || !aligned16(fwd_state) ||
+        !aligned16(rev_state) || !aligned4(fwd_decay) || !aligned4(rev_decay))
+        return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the fused kernel's forward and reverse state modes, from zero
+    TcArgs t{};
+    t.x = x; t.dt = dt; t.A = A; t.B = B;
+    t.workspace = workspace; t.ws_bytes = ws_bytes;
+    t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+    TcArgs f = t;
+    f.state_out = fwd_state;
+    f.decay_out = fwd_decay;
+    cudaError_t e = ssd::launch_tc_fused_state(f, s);
+    if (e != cudaSuccess) return to_status(e);
+    TcArgs r = t;
+    r.state_out = rev_state;
+    r.decay_out = rev_decay;
+    return to_status(ssd::launch_tc_fused_state_rev(r, s));
+}
+
+int ssd_segment_carry(const float *fwd_states, const float *fwd_decays, const float *rev_states,
+                      const float *rev_decays, int nseg, int seg, float *fwd_in, float *rev_in, int batch,
+                      int nheads, int headdim, int dstate, void *stream) {
+    if (batch < 0 || nheads <= 0 || nseg <= 0 || seg < 0 || seg >= nseg) return SSD_ERR_INVALID_ARG;
+    if (headdim != 64 || (dstate != 64 && dstate != 128)) return SSD_ERR_UNSUPPORTED;
+    if ((long long)batch * nheads * nseg >= (1ll << 31)) return SSD_ERR_UNSUPPORTED;
+    if (batch == 0) return SSD_OK;
+    if (!fwd_states || !fwd_decays || !rev_states || !rev_decays || !fwd_in || !rev_in) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(fwd_states) || !aligned16(rev_states) || !aligned16(fwd_in) || !aligned16(rev_in) ||
+        !aligned4(fwd_decays) || !aligned4(rev_decays))
+        return SSD_ERR_INVALID_ARG;
+    return to_status(ssd::launch_seg_carry(fwd_states, fwd_decays, rev_states, rev_decays, fwd_in, rev_in, batch,
+                                           nheads, dstate, nseg, seg, static_cast<cudaStream_t>(stream)));
+}
+
+int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                         const float *D, const float *fwd_init, const float *rev_init, void *out, int batch,
+                         int seqlen, int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype, false);
+    if (rc != SSD_OK) return rc;
+    if (dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    if (!x || !dt || !A || !B || !C || !D || !out) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned16(C) || !aligned16(out) || !aligned4(A) ||
+        !aligned4(D))
+        return SSD_ERR_INVALID_ARG;
+    if ((fwd_init && !aligned16(fwd_init)) || (rev_init && !aligned16(rev_init))) return SSD_ERR_INVALID_ARG;
+    // the fused kernel's seeded mode: forward scan from fwd_init, reverse scan
+    // from rev_init at the sequence end (zero where NULL)
+    TcArgs t{};
+    t.x = x; t.dt = dt; t.A = A; t.B = B; t.C = C; t.D = D; t.out = out;
+    t.init = fwd_init; t.rinit = rev_init;
+    t.workspace = workspace; t.ws_bytes = ws_bytes;
+    t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+    return to_status(ssd::launch_tc_fused(t, static_cast<cudaStream_t>(stream)));
+}
+
 int ssd_get_device_status(const void *workspace, void *stream) {
     if (!workspace) return SSD_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

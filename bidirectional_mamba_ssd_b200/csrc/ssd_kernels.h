@@ -72,5 +72,10 @@ int seg_count(long long units, int L, int sms);
 size_t tc_segmented_scratch_bytes(int batch, int L, int H, int N);   // max over the S in use
 cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream);
 int device_sms();   // SM count of the current device, 0 if it cannot be read
+// The forward and reverse states entering segment `seg` of nseg, from every
+// segment's own end states and decays (segment-major arrays; see
+// seg_carry_kernel); Hf, Hb (batch, H, 64, N).
+cudaError_t launch_seg_carry(const float *Sf, const float *Gf, const float *Sb, const float *Gb, float *Hf, float *Hb,
+                             int batch, int H, int N, int nseg, int seg, cudaStream_t stream);
 
 }  // namespace ssd

@@ -193,6 +193,57 @@ int ssd_block_step_path(const void *x, const void *dt, const float *A, const voi
                         int ngroups, int dtype, int path,
                         void *workspace, size_t ws_bytes, void *stream);
 
+/* Sequences split across GPUs (or any other split into segments): each
+ * holder of one segment of every sequence computes its segment's own states,
+ * the holders exchange them (one all-gather of nseg x (2 states + 2 decays)
+ * per (batch, head)), and each then runs its segment seeded with the states
+ * the rest of the sequence leaves. The recurrence is linear in the state, so
+ * this is the whole-sequence mixer up to rounding: the state entering a
+ * segment is the sum of the earlier segments' end states, each decayed over
+ * the segments in between ("Training Hybrid Block Diffusion Language Models
+ * with Partial Bidirectionality", Key Results: full-sequence denoising at
+ * 65K and 262K tokens; the pages describe no split across GPUs, only the
+ * lengths). bf16 I/O only (the fused kernel's state and seeded modes); fp32
+ * returns SSD_ERR_UNSUPPORTED. Workspace: at least
+ * ssd_workspace_bytes(SSD_OP_PREFIX_STATE, ..., chunk 64, SSD_BF16) for
+ * ssd_segment_states, ssd_workspace_bytes(SSD_OP_BIDIR_FWD, ..., chunk 64,
+ * SSD_BF16) for ssd_bidir_fwd_seeded. */
+
+/* A segment's own states, each scan starting from zero at its own end:
+ *   x, dt, A, B  as for ssd_bidir_fwd over the segment (seqlen >= 1)
+ *   fwd_state    (batch, nheads, headdim, dstate) fp32: forward state after the segment's last token
+ *   fwd_decay    (batch, nheads) fp32: exp(A_f[h] * sum of dt_f over the segment)
+ *   rev_state    (batch, nheads, headdim, dstate) fp32: reverse state before its first token
+ *   rev_decay    (batch, nheads) fp32: exp(A_b[h] * sum of dt_b over the segment)
+ * States are stored as headdim rows of dstate values, as ssd_prefix_state's. */
+int ssd_segment_states(const void *x, const void *dt, const float *A, const void *B,
+                       float *fwd_state, float *fwd_decay, float *rev_state, float *rev_decay,
+                       int batch, int seqlen, int nheads, int headdim, int dstate, int ngroups,
+                       int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/* The states entering segment `seg` (0 <= seg < nseg) from the gathered
+ * states of all nseg segments, segment-major: fwd_states / rev_states
+ * (nseg, batch, nheads, headdim, dstate), fwd_decays / rev_decays
+ * (nseg, batch, nheads), all fp32 as ssd_segment_states writes them.
+ *   fwd_in (batch, nheads, headdim, dstate): forward state before the segment
+ *          (zero for seg 0)
+ *   rev_in (batch, nheads, headdim, dstate): reverse state after the segment
+ *          (zero for seg nseg - 1)
+ * No workspace. */
+int ssd_segment_carry(const float *fwd_states, const float *fwd_decays, const float *rev_states,
+                      const float *rev_decays, int nseg, int seg, float *fwd_in, float *rev_in,
+                      int batch, int nheads, int headdim, int dstate, void *stream);
+
+/* Both scans over a segment with given starting states: the forward scan
+ * from fwd_init (state before the first token), the reverse scan from
+ * rev_init (reverse state after the last token); NULL = zero. Other
+ * arguments as ssd_bidir_fwd; out (batch, seqlen, nheads, headdim) io. The
+ * starting states enter the C.H products as bf16 operands. */
+int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const void *B,
+                         const void *C, const float *D, const float *fwd_init, const float *rev_init,
+                         void *out, int batch, int seqlen, int nheads, int headdim, int dstate,
+                         int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream);
+
 /* ssd_bidir_fwd for callers that cannot allocate device memory when they
  * call the mixer: code running under CUDA graph capture in the global mode,
  * where cudaMalloc is not allowed; plug-ins inside a runtime that has already

@@ -132,3 +132,31 @@ def test_prefix_and_block_reject_bad_arguments(lib):
 def test_status_requires_workspace(lib):
     assert lib.ssd_get_device_status(None, None) == -4
     assert lib.ssd_workspace_init(None, 256, None) == -4
+
+
+def test_segment_entry_points_reject_bad_arguments(lib):
+    v = ctypes.c_void_p
+    st = lambda *ints, ws=FAKE, wsb=1 << 40, x=FAKE, so=FAKE: lib.ssd_segment_states(
+        v(x), v(FAKE), v(FAKE), v(FAKE), v(so), v(FAKE), v(FAKE), v(FAKE), *ints, v(ws), wsb, None)
+    assert st(2, 256, 4, 64, 128, 4, 1, ws=0) == -4
+    assert st(2, 256, 4, 64, 128, 3, 1) == -1            # ngroups does not divide nheads
+    assert st(2, 256, 4, 64, 128, 4, 0) == -2            # fp32: not on this path
+    assert st(2, 0, 4, 64, 128, 4, 1) == -2              # an empty segment has no states to compute
+    assert st(2, 256, 4, 64, 128, 4, 1, x=0) == -1
+    assert st(2, 256, 4, 64, 128, 4, 1, so=FAKE + 4) == -1
+    assert st(0, 256, 4, 64, 128, 4, 1, x=0) == 0
+    cy = lambda nseg, seg, *ints, fi=FAKE: lib.ssd_segment_carry(
+        v(FAKE), v(FAKE), v(FAKE), v(FAKE), nseg, seg, v(fi), v(FAKE), *ints, None)
+    assert cy(4, 4, 2, 4, 64, 128) == -1                 # seg out of range
+    assert cy(4, -1, 2, 4, 64, 128) == -1
+    assert cy(0, 0, 2, 4, 64, 128) == -1
+    assert cy(4, 1, 2, 4, 64, 96) == -2
+    assert cy(4, 1, 2, 4, 64, 128, fi=0) == -1
+    assert cy(4, 1, 0, 4, 64, 128, fi=0) == 0
+    sd = lambda *ints, ws=FAKE, wsb=1 << 40, out=FAKE, init=0: lib.ssd_bidir_fwd_seeded(
+        v(FAKE), v(FAKE), v(FAKE), v(FAKE), v(FAKE), v(FAKE), v(init), v(0), v(out), *ints, v(ws), wsb, None)
+    assert sd(2, 256, 4, 64, 128, 4, 1, ws=0) == -4
+    assert sd(2, 256, 4, 64, 128, 4, 0) == -2
+    assert sd(2, 256, 4, 64, 128, 4, 1, out=0) == -1
+    assert sd(2, 256, 4, 64, 128, 4, 1, init=FAKE + 8) == -1
+    assert sd(2, 0, 4, 64, 128, 4, 1, out=0) == 0

@@ -275,7 +275,7 @@ def ssd_segment_states(x, dt, A, B, *, workspace: Workspace | None = None):
     rd = torch.empty_like(fd)
     stream = _stream(dev)
     ws = _workspace(dev, stream, workspace)
-    buf = ws.get(max(ssd_workspace_bytes(SSD_OP_PREFIX_STATE, batch, L, H, P, N, G, 64, io), 256))
+    buf = ws.get(max(ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, L, H, P, N, G, 64, io), 256))
     rc = lib.ssd_segment_states(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(fs), _ptr(fd), _ptr(rs), _ptr(rd),
                                 batch, L, H, P, N, G, _DT[io], _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_segment_states")

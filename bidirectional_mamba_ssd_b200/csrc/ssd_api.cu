@@ -275,6 +275,15 @@ int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
                                dstate, ngroups, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
 }
 
+// Segments to split each sequence into when a call has too few (batch, head)
+// units to fill the GPU (as SSD_PATH_AUTO chooses the segmented path); 1 = none.
+int few_unit_segments(int batch, int seqlen, int nheads) {
+    const long long units = (long long)batch * nheads, nt = (seqlen + 127) / 128;
+    const int sms = ssd::device_sms();
+    if (sms <= 0 || units >= sms || units * nt < 4LL * sms) return 1;
+    return ssd::seg_count(units, seqlen, sms);
+}
+
 int ssd_segment_states(const void *x, const void *dt, const float *A, const void *B, float *fwd_state,
                        float *fwd_decay, float *rev_state, float *rev_decay, int batch, int seqlen, int nheads,
                        int headdim, int dstate, int ngroups, int dtype, void *workspace, size_t ws_bytes,
@@ -284,8 +293,7 @@ int ssd_segment_states(const void *x, const void *dt, const float *A, const void
     if (dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
     if (!workspace) return SSD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
-    if (ws_bytes < ssd_workspace_bytes(SSD_OP_PREFIX_STATE, batch, seqlen, nheads, headdim, dstate, ngroups, 64,
-                                       dtype))
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype))
         return SSD_ERR_WORKSPACE;
     if (batch == 0) return SSD_OK;
     if (seqlen == 0) return SSD_ERR_UNSUPPORTED;
@@ -299,6 +307,9 @@ int ssd_segment_states(const void *x, const void *dt, const float *A, const void
     t.x = x; t.dt = dt; t.A = A; t.B = B;
     t.workspace = workspace; t.ws_bytes = ws_bytes;
     t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+    // few long sequences: state passes over segments of each, then their totals
+    const int S = few_unit_segments(batch, seqlen, nheads);
+    if (S > 1) return to_status(ssd::launch_tc_segment_totals(t, S, fwd_state, fwd_decay, rev_state, rev_decay, s));
     TcArgs f = t;
     f.state_out = fwd_state;
     f.decay_out = fwd_decay;
@@ -349,6 +360,9 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
     t.init = fwd_init; t.rinit = rev_init;
     t.workspace = workspace; t.ws_bytes = ws_bytes;
     t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+    // few long sequences: the segmented path, its scan starting from the seeds
+    const int S = few_unit_segments(batch, seqlen, nheads);
+    if (S > 1) return to_status(ssd::launch_tc_segmented(t, S, static_cast<cudaStream_t>(stream)));
     return to_status(ssd::launch_tc_fused(t, static_cast<cudaStream_t>(stream)));
 }
 

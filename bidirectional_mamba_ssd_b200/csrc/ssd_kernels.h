@@ -71,6 +71,10 @@ cudaError_t launch_tc_fused_state_rev(const TcArgs &a, cudaStream_t stream);
 int seg_count(long long units, int L, int sms);
 size_t tc_segmented_scratch_bytes(int batch, int L, int H, int N);   // max over the S in use
 cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream);
+// The whole sequence's own end states and decays (as the fused state modes
+// give them) from S segments' state passes and one combining kernel.
+cudaError_t launch_tc_segment_totals(const TcArgs &a, int S, float *fwd_state, float *fwd_decay, float *rev_state,
+                                     float *rev_decay, cudaStream_t stream);
 int device_sms();   // SM count of the current device, 0 if it cannot be read
 // The forward and reverse states entering segment `seg` of nseg, from every
 // segment's own end states and decays (segment-major arrays; see

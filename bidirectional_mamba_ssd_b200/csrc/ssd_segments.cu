@@ -12,7 +12,9 @@
 //        Hf_in(s) = sum_{r<s} (prod_{r<q<s} g_f(q)) Sf(r),
 //        Hb_in(s) = sum_{r>s} (prod_{s<q<r} g_b(q)) Sb(r),
 //      with g(q) = exp(A sum of dt over segment q), which the state passes
-//      also return (the product of their tile decays);
+//      also return (the product of their tile decays); given starting states
+//      of the whole sequence (a segment of a longer one) enter as the term
+//      from beyond its ends;
 //   4. the fused bidirectional kernel runs on the segments, its forward scan
 //      seeded with Hf_in and its reverse scan with Hb_in.
 // The recurrence is linear in the state, so this equals the scan over the
@@ -35,18 +37,21 @@ constexpr int kMaxSeg = 64;
 constexpr int kScanThreads = 256;
 
 // grid (batch * H, 2 directions), 256 threads; Gf, Gb: each segment's decay
-// exp(A * sum of dt over the segment), from the state passes.
+// exp(A * sum of dt over the segment), from the state passes. H0f, H0b
+// (batch, H, 64, N) or nullptr: the forward state before the sequence and the
+// reverse state after it.
 __global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(const float *Sf, const float *Sb, const float *Gf,
-                                                                const float *Gb, float *Hf, float *Hb, int H,
-                                                                int S, int N) {
+                                                                const float *Gb, const float *H0f, const float *H0b,
+                                                                float *Hf, float *Hb, int H, int S, int N) {
     const int u = blockIdx.x, dir = blockIdx.y;
     const int b = u / H, h = u % H;
     const float *sin = dir ? Sb : Sf;
     const float *gin = dir ? Gb : Gf;
+    const float *h0 = dir ? H0b : H0f;
     float *hout = dir ? Hb : Hf;
     const int elems = kP * N;
     for (int e = threadIdx.x * 4; e < elems; e += kScanThreads * 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc = h0 ? *reinterpret_cast<const float4 *>(h0 + (size_t)u * elems + e) : make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k = 0; k < S; ++k) {
             const int seg = dir ? S - 1 - k : k;
             const size_t su = (size_t)(b * S + seg) * H + h;   // segment unit of the reshaped batch
@@ -81,6 +86,37 @@ __global__ void __launch_bounds__(kScanThreads) seg_carry_kernel(const float *Sf
             acc = make_float4(fmaf(g, acc.x, v.x), fmaf(g, acc.y, v.y), fmaf(g, acc.z, v.z), fmaf(g, acc.w, v.w));
         }
         *reinterpret_cast<float4 *>(hout + e) = acc;
+    }
+}
+
+// grid (batch * H, 2 directions), 256 threads. From the S segments' own
+// states and decays (reshaped-batch layout, as seg_scan_kernel), the whole
+// sequence's: forward state after its last token, reverse state before its
+// first, and the two decays (the products of the segments').
+__global__ void __launch_bounds__(kScanThreads) seg_total_kernel(const float *Sf, const float *Sb, const float *Gf,
+                                                                 const float *Gb, float *Tf, float *Tb, float *Df,
+                                                                 float *Db, int H, int S, int N) {
+    const int u = blockIdx.x, dir = blockIdx.y;
+    const int b = u / H, h = u % H;
+    const float *sin = dir ? Sb : Sf;
+    const float *gin = dir ? Gb : Gf;
+    float *tout = (dir ? Tb : Tf) + (size_t)u * kP * N;
+    const int elems = kP * N;
+    for (int e = threadIdx.x * 4; e < elems; e += kScanThreads * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < S; ++k) {
+            const int seg = dir ? S - 1 - k : k;
+            const size_t su = (size_t)(b * S + seg) * H + h;
+            const float4 v = *reinterpret_cast<const float4 *>(sin + su * elems + e);
+            const float g = gin[su];
+            acc = make_float4(fmaf(g, acc.x, v.x), fmaf(g, acc.y, v.y), fmaf(g, acc.z, v.z), fmaf(g, acc.w, v.w));
+        }
+        *reinterpret_cast<float4 *>(tout + e) = acc;
+    }
+    if (threadIdx.x == 0) {
+        float g = 1.f;
+        for (int k = 0; k < S; ++k) g *= gin[(size_t)(b * S + k) * H + h];
+        (dir ? Db : Df)[u] = g;
     }
 }
 
@@ -158,7 +194,8 @@ cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
     r.state_out = Sb;
     r.decay_out = Gb;
     if ((e = launch_tc_fused_state_rev(r, stream)) != cudaSuccess) return e;
-    seg_scan_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, Hf, Hb, a.H, S, a.N);
+    seg_scan_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, a.init, a.rinit, Hf, Hb,
+                                                                        a.H, S, a.N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     TcArgs o = v;
     o.init = Hf;
@@ -175,6 +212,35 @@ cudaError_t launch_seg_carry(const float *Sf, const float *Gf, const float *Sb, 
     const int units = batch * H;
     if (units <= 0) return cudaSuccess;
     seg_carry_kernel<<<dim3(units, 2), kScanThreads, 0, stream>>>(Sf, Gf, Sb, Gb, Hf, Hb, units, nseg, seg, kP * N);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_segment_totals(const TcArgs &a, int S, float *fwd_state, float *fwd_decay, float *rev_state,
+                                     float *rev_decay, cudaStream_t stream) {
+    if (S < 2 || S > kMaxSeg || a.L % S || a.ndir != 2) return cudaErrorNotSupported;
+    const SegLayout lay = seg_layout(a.batch, a.L, a.H, a.N, S);
+    if (a.ws_bytes < kStatusBytes + lay.total) return cudaErrorInvalidValue;
+    char *scratch = static_cast<char *>(a.workspace) + kStatusBytes;
+    float *Sf = reinterpret_cast<float *>(scratch + lay.fused);
+    float *Sb = reinterpret_cast<float *>(scratch + lay.fused + lay.states);
+    float *Gf = reinterpret_cast<float *>(scratch + lay.fused + 4 * lay.states);
+    float *Gb = reinterpret_cast<float *>(scratch + lay.fused + 4 * lay.states + lay.decays);
+    TcArgs v = a;             // the segments as a batch of batch * S sequences of L / S tokens
+    v.batch = a.batch * S;
+    v.L = a.L / S;
+    v.init = nullptr;
+    v.rinit = nullptr;
+    cudaError_t e;
+    TcArgs f = v;
+    f.state_out = Sf;
+    f.decay_out = Gf;
+    if ((e = launch_tc_fused_state(f, stream)) != cudaSuccess) return e;
+    TcArgs r = v;
+    r.state_out = Sb;
+    r.decay_out = Gb;
+    if ((e = launch_tc_fused_state_rev(r, stream)) != cudaSuccess) return e;
+    seg_total_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, fwd_state, rev_state,
+                                                                         fwd_decay, rev_decay, a.H, S, a.N);
     return cudaGetLastError();
 }
 

@@ -204,10 +204,11 @@ int ssd_block_step_path(const void *x, const void *dt, const float *A, const voi
  * with Partial Bidirectionality", Key Results: full-sequence denoising at
  * 65K and 262K tokens; the pages describe no split across GPUs, only the
  * lengths). bf16 I/O only (the fused kernel's state and seeded modes); fp32
- * returns SSD_ERR_UNSUPPORTED. Workspace: at least
- * ssd_workspace_bytes(SSD_OP_PREFIX_STATE, ..., chunk 64, SSD_BF16) for
- * ssd_segment_states, ssd_workspace_bytes(SSD_OP_BIDIR_FWD, ..., chunk 64,
- * SSD_BF16) for ssd_bidir_fwd_seeded. */
+ * returns SSD_ERR_UNSUPPORTED. With too few (batch, head) units to fill the
+ * GPU, both calls split each local sequence further into segments, as
+ * SSD_PATH_SEGMENTED does. Workspace: at least
+ * ssd_workspace_bytes(SSD_OP_BIDIR_FWD, ..., chunk 64, SSD_BF16) for
+ * ssd_segment_states and ssd_bidir_fwd_seeded. */
 
 /* A segment's own states, each scan starting from zero at its own end:
  *   x, dt, A, B  as for ssd_bidir_fwd over the segment (seqlen >= 1)

@@ -14,8 +14,11 @@ from ssd_inputs import to_f64
 
 pytestmark = pytest.mark.gpu
 
-# (batch, L, H, N, G): ragged tails, shared and per-head B/C, 8 to 160 units
-SHAPES = [(2, 300, 4, 128, 2), (4, 384, 24, 64, 24), (40, 256, 4, 128, 4), (1, 1, 2, 64, 1)]
+# (batch, L, H, N, G): ragged tails, shared and per-head B/C, 8 to 160 units;
+# the last one has too few units to fill the GPU, so both calls split each
+# sequence into 16 segments of 1024 tokens internally
+SHAPES = [(2, 300, 4, 128, 2), (4, 384, 24, 64, 24), (40, 256, 4, 128, 4), (1, 1, 2, 64, 1),
+          (1, 16384, 8, 128, 8)]
 
 
 @pytest.fixture(scope="module")
@@ -87,8 +90,9 @@ def _sharded_one_gpu(ssd, inp, nseg):
     return torch.cat(outs, dim=1), carried
 
 
-@pytest.mark.parametrize("nseg,shape", [(3, (2, 900, 4, 128, 4)), (4, (3, 1024, 8, 64, 2)), (2, (1, 256, 32, 128, 32))],
-                         ids=["3seg_L900", "4seg_L1024_G2", "2seg_H32"])
+@pytest.mark.parametrize("nseg,shape", [(3, (2, 900, 4, 128, 4)), (4, (3, 1024, 8, 64, 2)), (2, (1, 256, 32, 128, 32)),
+                                        (2, (1, 32768, 8, 128, 8))],
+                         ids=["3seg_L900", "4seg_L1024_G2", "2seg_H32", "2seg_L32768_few_units"])
 def test_sequence_sharded_matches_whole_sequence(ssd, nseg, shape):
     batch, L, H, N, G = shape
     inp = si.bidir_inputs(batch, L, H, 64, N, G, "bf16", seed=L + nseg, device="cuda")

@@ -63,30 +63,31 @@ __global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(const float *Sf,
     }
 }
 
-// grid (batch * H, 2 directions), 256 threads. From the end states S and
-// decays g of all nseg segments of a sequence, laid out segment-major
-// (S (nseg, batch, H, P, N), g (nseg, batch, H)), the state entering segment
-// `seg`: from the left, Hf = sum_{q<seg} (prod_{q<r<seg} g_f(r)) S_f(q); from
-// the right, Hb = sum_{q>seg} (prod_{seg<r<q} g_b(r)) S_b(q). The same
-// recurrence as seg_scan_kernel, for segments that sit on other GPUs.
+// grid (batch * H, 2 directions, elems / 1024), 256 threads, one float4 of
+// the state per thread. From the end states S and decays g of all nseg
+// segments of a sequence, laid out segment-major (S (nseg, batch, H, P, N),
+// g (nseg, batch, H)), the state entering segment `seg`: from the left,
+// Hf = sum_{q<seg} (prod_{q<r<seg} g_f(r)) S_f(q); from the right,
+// Hb = sum_{q>seg} (prod_{seg<r<q} g_b(r)) S_b(q). The same recurrence as
+// seg_scan_kernel, for segments that sit on other GPUs.
 __global__ void __launch_bounds__(kScanThreads) seg_carry_kernel(const float *Sf, const float *Gf, const float *Sb,
                                                                  const float *Gb, float *Hf, float *Hb, int units,
                                                                  int nseg, int seg, int elems) {
     const int u = blockIdx.x, dir = blockIdx.y;
+    const int e = (blockIdx.z * kScanThreads + threadIdx.x) * 4;
+    if (e >= elems) return;
     const float *sin = dir ? Sb : Sf;
     const float *gin = dir ? Gb : Gf;
-    float *hout = (dir ? Hb : Hf) + (size_t)u * elems;
     const int first = dir ? nseg - 1 : 0, last = seg, step = dir ? -1 : 1;
-    for (int e = threadIdx.x * 4; e < elems; e += kScanThreads * 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = first; q != last; q += step) {
-            const size_t su = (size_t)q * units + u;
-            const float4 v = *reinterpret_cast<const float4 *>(sin + su * elems + e);
-            const float g = gin[su];
-            acc = make_float4(fmaf(g, acc.x, v.x), fmaf(g, acc.y, v.y), fmaf(g, acc.z, v.z), fmaf(g, acc.w, v.w));
-        }
-        *reinterpret_cast<float4 *>(hout + e) = acc;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int q = first; q != last; q += step) {
+        const size_t su = (size_t)q * units + u;
+        const float4 v = *reinterpret_cast<const float4 *>(sin + su * elems + e);
+        const float g = gin[su];
+        acc = make_float4(fmaf(g, acc.x, v.x), fmaf(g, acc.y, v.y), fmaf(g, acc.z, v.z), fmaf(g, acc.w, v.w));
     }
+    *reinterpret_cast<float4 *>((dir ? Hb : Hf) + (size_t)u * elems + e) = acc;
 }
 
 // grid (batch * H, 2 directions), 256 threads. From the S segments' own
@@ -211,7 +212,9 @@ cudaError_t launch_seg_carry(const float *Sf, const float *Gf, const float *Sb, 
                              int batch, int H, int N, int nseg, int seg, cudaStream_t stream) {
     const int units = batch * H;
     if (units <= 0) return cudaSuccess;
-    seg_carry_kernel<<<dim3(units, 2), kScanThreads, 0, stream>>>(Sf, Gf, Sb, Gb, Hf, Hb, units, nseg, seg, kP * N);
+    const int elems = kP * N;
+    const int zb = (elems + kScanThreads * 4 - 1) / (kScanThreads * 4);
+    seg_carry_kernel<<<dim3(units, 2, zb), kScanThreads, 0, stream>>>(Sf, Gf, Sb, Gb, Hf, Hb, units, nseg, seg, elems);
     return cudaGetLastError();
 }
 

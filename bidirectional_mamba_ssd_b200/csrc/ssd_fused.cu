@@ -208,6 +208,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
+    // the next kernel in the stream may set itself up while this one runs
+    grid_launch_dependents();
     if (tid == 0) {
         *abort_flag = 0;
         for (int i = 0; i < B_COUNT; ++i)
@@ -218,6 +220,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
+    // the kernel ahead in the stream has finished and its writes are visible
+    // before this one reads or writes global memory
+    grid_dependency_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -783,8 +788,19 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return e;
     const int grid = units < sms ? units : sms;
-    k<<<grid, kThreads, smem, stream>>>(tm_x, tm_b, tm_c, tm_h, tm_out, p);
-    return cudaGetLastError();
+    // programmatic stream serialization: the prologue (barriers, TMEM) overlaps
+    // the end of the kernel ahead; the kernel waits for it before any global access
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, tm_x, tm_b, tm_c, tm_h, tm_out, p);
 }
 
 template <int MODE>

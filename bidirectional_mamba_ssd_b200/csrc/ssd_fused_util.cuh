@@ -56,6 +56,16 @@ __device__ __forceinline__ void st_global_v4_hint(void *p, uint4 v, uint64_t pol
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the kernel ahead of it in the stream has
+// finished; it must wait before touching global memory. Without the launch
+// attribute both are no-ops.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel (if launched that way) start its own prologue.
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // named barriers of the three epilogue groups (128 threads each)
 __device__ __forceinline__ void sync_c() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ void sync_a() { asm volatile("bar.sync 2, 128;" ::: "memory"); }

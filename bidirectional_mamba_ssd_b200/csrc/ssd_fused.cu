@@ -183,7 +183,12 @@ struct Smem {
     static_assert(hb + kSlab <= xw, "low-part slot 1");
 };
 
-template <int N, int MODE>
+// REUSE (one-tile sequences whose B/C are shared by several heads): each CTA
+// takes a contiguous range of units (else every gridDim-th), and an output
+// tile whose C/B tiles are those of the unit before it on the same CTA (same
+// batch element and B/C group) takes them from the ring in place. A template
+// parameter, so that the other shapes' kernels carry none of its code.
+template <int N, int MODE, bool REUSE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
@@ -240,6 +245,18 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     // pass all but tile 0, whose own tile state no tile to its left receives
     const int n1t = kOut ? nt - 1 : nt;
     const int hpg = p.H / p.G;
+    // this CTA's units: [u_begin, u_end) with step u_step (every gridDim-th
+    // unit, or with REUSE a contiguous range)
+    const int per = REUSE ? p.units / (int)gridDim.x : 0, rem = REUSE ? p.units % (int)gridDim.x : 0;
+    const int u_begin = REUSE ? (int)blockIdx.x * per + ((int)blockIdx.x < rem ? (int)blockIdx.x : rem)
+                              : (int)blockIdx.x;
+    const int u_end = REUSE ? u_begin + per + ((int)blockIdx.x < rem ? 1 : 0) : p.units;
+    const int u_step = REUSE ? 1 : (int)gridDim.x;
+    // C/B reuse: unit u's output tile takes the previous unit's C/B tiles
+    auto same_bc = [&](int u) {
+        if constexpr (!REUSE || !kOut) return false;
+        return u > u_begin && u < u_end && (u - 1) / p.H == u / p.H && ((u - 1) % p.H) / hpg == (u % p.H) / hpg;
+    };
     const size_t dt_dir = (size_t)p.batch * p.L * p.H;
 
     if (warp == 0) {
@@ -264,7 +281,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const uint64_t pol1 = kOut ? keep : stream;
             // after an expired wait anywhere in the CTA, no further loads are issued
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++units_done) {
+            for (int u = u_begin; ok && u < u_end; u += u_step, ++units_done) {
                 const int b = u / p.H, h = u % p.H, gg = h / hpg;
                 for (int k1 = 0; ok && k1 < n1t; ++k1) {    // phase 1: x, B of the state pass
                     const int i = kFwd1 ? k1 : nt - 1 - k1;
@@ -290,7 +307,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     tma_load_4d_hint(base + S::xslot(xs), &tm_x, bar(B_X_FULL + xs), 0, h, t0, b, stream);
                     const CUtensorMap *maps[4] = {&tm_c, &tm_b, &tm_c, &tm_b};
                     const int dirs[4] = {0, 0, 1, 1};
-                    for (int j = 0; ok && j < 4; ++j) {
+                    for (int j = 0; ok && !same_bc(u) && j < 4; ++j) {
                         uint32_t rs;
                         if (!(ok = ring_slot(rs))) break;
                         ++kr;
@@ -333,7 +350,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             };
             auto slot_addr = [&](uint32_t s) { return base + S::ring + s * 2 * kSlab; };
             // after an expired wait anywhere in the CTA, no further tiles are issued
-            for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
+            uint32_t rCf = 0, rBf = 0, rCb = 0, rBb = 0;   // the output tile's ring slots
+            for (int u = u_begin; u < u_end && !*abort_flag; u += u_step) {
+                const bool reuse = same_bc(u), keep_bc = same_bc(u + u_step);
                 for (int k1 = 0; k1 < n1t && !*abort_flag; ++k1, ++n1) {  // phase 1: S = B^T (diag(w) X in the x slot)
                     const uint32_t n = kx++, xs = n % kXS;
                     const uint32_t rs = wait_ring(kr++);
@@ -357,8 +376,12 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 for (int i = 0; kOut && i < nt && !*abort_flag; ++i) {   // phase 2
                     const uint32_t n = kx++, xs = n % kXS;
-                    const uint32_t rCf = wait_ring(kr++), rBf = wait_ring(kr++);
-                    const uint32_t rCb = wait_ring(kr++), rBb = wait_ring(kr++);
+                    if (!reuse) {
+                        rCf = wait_ring(kr++);
+                        rBf = wait_ring(kr++);
+                        rCb = wait_ring(kr++);
+                        rBb = wait_ring(kr++);
+                    }
                     const uint32_t sCf = slot_addr(rCf), sBf = slot_addr(rBf);
                     const uint32_t sCb = slot_addr(rCb), sBb = slot_addr(rBb);
                     // G_f overwrites the reverse pass's TMEM tile states and Y_o,f reads
@@ -377,7 +400,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         mma_bf16_ss(tGb, sdesc_sw128(sCb + ko, 0, 1024), sdesc_sw128(sBb + ko, 0, 1024), id_g, k > 0);
                     }
                     mma_commit(bar(B_G_READY));
-                    mma_commit(bar(B_RING_EMPTY + rBb));
+                    if (!keep_bc) mma_commit(bar(B_RING_EMPTY + rBb));
                     // the previous tile's outputs and state are consumed; H_f is this tile's
                     if (!first2) {
                         mbar_wait(bar(B_Y_FREE), n_yfree++ & 1, abort_flag, p.status, 205);
@@ -390,7 +413,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         mma_bf16_ss(tYof, sdesc_sw128(sCf + ko, 0, 1024),
                                     sdesc_sw128(base + S::hf + k * 2048, kSlab, 1024), id_o, k > 0);
                     }
-                    mma_commit(bar(B_RING_EMPTY + rCf));
+                    if (!keep_bc) mma_commit(bar(B_RING_EMPTY + rCf));
                     mbar_wait(bar(B_HB_FULL), kh++ & 1, abort_flag, p.status, 207);
                     tc_fence_after();
                     for (int k = 0; k < N / 16; ++k) {      // Yo_b = C_b H_b
@@ -398,7 +421,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         mma_bf16_ss(tYob, sdesc_sw128(sCb + ko, 0, 1024),
                                     sdesc_sw128(base + S::hb + k * 2048, kSlab, 1024), id_o, k > 0);
                     }
-                    mma_commit(bar(B_RING_EMPTY + rCb));
+                    if (!keep_bc) mma_commit(bar(B_RING_EMPTY + rCb));
                     mma_commit(bar(B_HB_EMPTY));
                     mbar_wait(bar(B_XW_READY + xs), (n / kXS) & 1, abort_flag, p.status, 208);
                     tc_fence_after();
@@ -406,7 +429,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         mma_bf16_ss(tS, sdesc_sw128(sBf + k * 2048, kSlab, 1024),
                                     sdesc_sw128(base + S::xw + k * 2048, kSlab, 1024), id_state, k > 0);
                     mma_commit(bar(B_S_READY));
-                    mma_commit(bar(B_RING_EMPTY + rBf));
+                    if (!keep_bc) mma_commit(bar(B_RING_EMPTY + rBf));
                     mbar_wait(bar(B_M_READY), n_m++ & 1, abort_flag, p.status, 209);
                     mbar_wait(bar(B_X_FULL + xs), (n / kXS) & 1, abort_flag, p.status, 204);
                     tc_fence_after();
@@ -445,7 +468,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         auto load_dt = [&](int u, int i) {
             rawf = 0;
             rawb = 0;
-            if (u >= p.units) return;
+            if (u >= u_end) return;
             const int b = u / p.H, h = u % p.H, t = i * kTile + row;
             if (t < p.L) {
                 const size_t o = ((size_t)b * p.L + t) * p.H + h;
@@ -457,9 +480,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             vf = __uint_as_float(rawf << 16);
             vb = __uint_as_float(rawb << 16);
         };
-        int cu = blockIdx.x, ci = 0;   // the output-pass tile whose dt is in flight
+        int cu = u_begin, ci = 0;   // the output-pass tile whose dt is in flight
         if constexpr (kOut) load_dt(cu, ci);
-        while (cu < p.units) {
+        while (cu < u_end) {
             const int u = cu;
             const int h = u % p.H;
             const float Af = p.A[h], Ab = kOut ? p.A[p.H + h] : 0.f;
@@ -511,7 +534,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     for (int j = 0; j < kP; ++j) op[(size_t)j * N] = hreg[j];
                 }
                 if (row == 0 && p.decay_out) p.decay_out[u] = __expf(lsum);
-                cu += gridDim.x;
+                cu += u_step;
                 continue;
             }
             kx += n1t;       // the reverse pass's x loads and diag(w') X releases belong to groups A and B
@@ -533,7 +556,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             for (int i = 0; i < nt; ++i) {
                 float vf, vb;
                 take_dt(vf, vb);
-                if (++ci == nt) { ci = 0; cu += gridDim.x; }
+                if (++ci == nt) { ci = 0; cu += u_step; }
                 load_dt(cu, ci);
                 float pf = vf, pb = vb, totf, totb;
                 scan2(pf, pb, totf, totb, row, red);
@@ -603,7 +626,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         auto sync_ab = [&]() { asm volatile("bar.sync 4, 256;" ::: "memory"); };
         uint32_t kx = 0, n_g = 0, n_y = 0, nvec = 0, m1 = 0;
         float *red_g = red_ab + (is_b ? 4 : 0);
-        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+        for (int u = u_begin; u < u_end; u += u_step) {
             const int b = u / p.H, h = u % p.H;
             const float dsum = kOut ? p.D[h] + p.D[p.H + h] : 0.f;
             // the state pass's direction: reverse in the output modes, forward in the state mode
@@ -746,7 +769,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-template <int N, int MODE>
+template <int N, int MODE, bool REUSE>
 cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     using S = Smem<N>;
     constexpr bool kOut = MODE == kModeBidir || MODE == kModeBidirInit;
@@ -783,7 +806,7 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    auto k = tc_fused_kernel<N, MODE>;
+    auto k = tc_fused_kernel<N, MODE, REUSE>;
     const size_t smem = S::bytes + 1024;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return e;
@@ -810,7 +833,12 @@ cudaError_t launch_mode(const TcArgs &a, cudaStream_t stream) {
     if (!tmap::encode_fn()) return cudaErrorNotSupported;
     const long long entries = (long long)a.batch * a.H * ((a.L + kTile - 1) / kTile);
     if (entries >= (1ll << 31)) return cudaErrorNotSupported;
-    return a.N == 64 ? run_fused<64, MODE>(a, stream) : run_fused<128, MODE>(a, stream);
+    constexpr bool kOut = MODE == kModeBidir || MODE == kModeBidirInit;
+    // one-tile sequences with B/C shared by several heads: consecutive heads on
+    // one CTA, taking their C/B tiles from the ring in place
+    if (kOut && a.L <= kTile && a.G < a.H)
+        return a.N == 64 ? run_fused<64, MODE, kOut>(a, stream) : run_fused<128, MODE, kOut>(a, stream);
+    return a.N == 64 ? run_fused<64, MODE, false>(a, stream) : run_fused<128, MODE, false>(a, stream);
 }
 
 }  // namespace

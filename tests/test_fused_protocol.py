@@ -31,11 +31,22 @@ class Sim(Sched):
     step's seeded variant has the same protocol) or 'state' (the forward state
     pass alone); kxs: x slots; xw_per_slot False plants the earlier single
     diag(w) X barrier."""
-    def __init__(self, nt, units, seed, kRing=4, mode='bidir', kxs=2, xw_per_slot=True, heavy=0.1):
+    def __init__(self, nt, units, seed, kRing=4, mode='bidir', kxs=2, xw_per_slot=True, heavy=0.1, bc=None,
+                 release_early=False):
         super().__init__(seed, heavy)
         self.nt, self.units, self.kRing = nt, units, kRing
         self.mode, self.kxs, self.xw_per_slot = mode, kxs, xw_per_slot
         self.kG1 = 8
+        # bc[j]: the C/B tiles unit j reads (units of one batch element and B/C
+        # group share them); one-tile units reuse the previous unit's in place
+        self.bc = bc
+        self.release_early = release_early   # planted: release reused slots after each unit
+    def bc_of(self, units_list, j):
+        return self.bc[j] if self.bc is not None else units_list[j]
+    def reuse(self, units_list, j):
+        """unit j takes its C/B tiles from the previous unit's ring slots"""
+        return (self.mode == 'bidir' and self.nt == 1 and self.bc is not None and 0 < j < len(units_list)
+                and self.bc[j] == self.bc[j - 1])
     def n1t(self):
         """tiles of the state pass: all forward; in reverse all but the leftmost"""
         return self.nt if self.mode == 'state' else self.nt - 1
@@ -60,7 +71,7 @@ def producer(S, units_list):
     nt, R, X = S.nt, S.kRing, S.kxs
     kr = kx = kh = 0
     units_done = 0
-    for u in units_list:
+    for j, u in enumerate(units_list):
         for i in range(S.n1t()):                 # the state pass's tiles, in its order
             xs = kx % X
             if kx >= X:
@@ -82,11 +93,13 @@ def producer(S, units_list):
             kx += 1
             yield ('tma', 'X_FULL%d' % xs, [(('x', xs, 0), ('x', u, 2, i)), (('x', xs, 1), ('x', u, 2, i))])
             for name in ('Cf', 'Bf', 'Cb', 'Bb'):
+                if S.reuse(units_list, j):
+                    break
                 rs = kr % R
                 if kr >= R:
                     yield ('wait', 'RING_EMPTY%d' % rs, kr // R - 1)
                 kr += 1
-                yield ('tma', 'RING_FULL%d' % rs, [(('ring', rs), (name, u, i))])
+                yield ('tma', 'RING_FULL%d' % rs, [(('ring', rs), (name, S.bc_of(units_list, j), i))])
             if i == 0:
                 yield ('wait', 'HB_WRITTEN', units_done - 1)
             if kh >= 1:
@@ -99,7 +112,11 @@ def mma(S, units_list):
     kr = kx = kh = n1 = 0
     n_m = n_sfree = n_yfree = n_hbw = 0
     first2 = True
-    for u in units_list:
+    rCf = rBf = rCb = rBb = None
+    for j, u in enumerate(units_list):
+        bcu = S.bc_of(units_list, j)
+        reuse = S.reuse(units_list, j)
+        keep = S.reuse(units_list, j + 1) and not S.release_early
         for i in range(S.n1t()):
             n = kx; xs = n % X; kx += 1
             rs = kr % R
@@ -118,34 +135,39 @@ def mma(S, units_list):
             continue
         for i in range(nt):
             n = kx; xs = n % X; kx += 1
-            slots = []
-            for name in ('Cf', 'Bf', 'Cb', 'Bb'):
-                rs = kr % R
-                yield ('wait', 'RING_FULL%d' % rs, kr // R); kr += 1
-                slots.append(rs)
-            rCf, rBf, rCb, rBb = slots
+            if not reuse:
+                slots = []
+                for name in ('Cf', 'Bf', 'Cb', 'Bb'):
+                    rs = kr % R
+                    yield ('wait', 'RING_FULL%d' % rs, kr // R); kr += 1
+                    slots.append(rs)
+                rCf, rBf, rCb, rBb = slots
             if i == 0:
                 yield ('wait', 'HB_WRITTEN', n_hbw); n_hbw += 1
-            yield ('mma', [(('ring', rCf), ('Cf', u, i)), (('ring', rBf), ('Bf', u, i))],
+            yield ('mma', [(('ring', rCf), ('Cf', bcu, i)), (('ring', rBf), ('Bf', bcu, i))],
                    [(('tGf', b), ('Gf', u, i)) for b in range(8)])
-            yield ('mma', [(('ring', rCb), ('Cb', u, i)), (('ring', rBb), ('Bb', u, i))],
+            yield ('mma', [(('ring', rCb), ('Cb', bcu, i)), (('ring', rBb), ('Bb', bcu, i))],
                    [(('tGb', b), ('Gb', u, i)) for b in range(8)])
             yield ('commit', 'G_READY')
-            yield ('commit', 'RING_EMPTY%d' % rBb)
+            if not keep:
+                yield ('commit', 'RING_EMPTY%d' % rBb)
             if not first2:
                 yield ('wait', 'Y_FREE', n_yfree); n_yfree += 1
                 yield ('wait', 'S_FREE', n_sfree); n_sfree += 1
             first2 = False
-            yield ('mma', [(('ring', rCf), ('Cf', u, i)), ('hf', ('hf', u, i))], [(('Yof', 0), ('Yof', u, i)), (('Yof', 1), ('Yof', u, i))])
-            yield ('commit', 'RING_EMPTY%d' % rCf)
+            yield ('mma', [(('ring', rCf), ('Cf', bcu, i)), ('hf', ('hf', u, i))], [(('Yof', 0), ('Yof', u, i)), (('Yof', 1), ('Yof', u, i))])
+            if not keep:
+                yield ('commit', 'RING_EMPTY%d' % rCf)
             yield ('wait', 'HB_FULL', kh); kh += 1
-            yield ('mma', [(('ring', rCb), ('Cb', u, i)), ('hb', ('hb', u, i))], [(('Yob', 0), ('Yob', u, i)), (('Yob', 1), ('Yob', u, i))])
-            yield ('commit', 'RING_EMPTY%d' % rCb)
+            yield ('mma', [(('ring', rCb), ('Cb', bcu, i)), ('hb', ('hb', u, i))], [(('Yob', 0), ('Yob', u, i)), (('Yob', 1), ('Yob', u, i))])
+            if not keep:
+                yield ('commit', 'RING_EMPTY%d' % rCb)
             yield ('commit', 'HB_EMPTY')
             yield ('wait',) + S.xw(n)
-            yield ('mma', [(('ring', rBf), ('Bf', u, i)), ('xw', ('xw', u, i))], [('S', ('S', u, i))])
+            yield ('mma', [(('ring', rBf), ('Bf', bcu, i)), ('xw', ('xw', u, i))], [('S', ('S', u, i))])
             yield ('commit', 'S_READY')
-            yield ('commit', 'RING_EMPTY%d' % rBf)
+            if not keep:
+                yield ('commit', 'RING_EMPTY%d' % rBf)
             yield ('wait', 'M_READY', n_m); n_m += 1
             yield ('wait', 'X_FULL%d' % xs, n // X)
             yield ('mma', [(('tGf', b), ('M', u, i)) for b in range(8)] + [(('x', xs, 0), ('x', u, 2, i)), (('x', xs, 1), ('x', u, 2, i))],
@@ -258,14 +280,22 @@ def run(S, units_list):
     run_roles(S, roles, counts)
 
 
-def _schedules(n, mode='bidir', kxs=2, xw_per_slot=True, seed0=0):
+def _schedules(n, mode='bidir', kxs=2, xw_per_slot=True, seed0=0, shared_bc=False, release_early=False):
     fails = []
     for seed in range(seed0, seed0 + n):
         r = random.Random(seed)
-        nt = r.choice([1, 2, 3, 4, 5, 9])
-        nunits = r.choice([1, 2, 3])
+        nt = 1 if shared_bc else r.choice([1, 2, 3, 4, 5, 9])
+        nunits = r.choice([3, 5, 8]) if shared_bc else r.choice([1, 2, 3])
+        # runs of units on the same C/B tiles (consecutive heads of one batch element)
+        bc = None
+        if shared_bc:
+            bc, g = [], 0
+            for _ in range(nunits):
+                if bc and r.random() < 0.4:
+                    g += 1
+                bc.append(g)
         S = Sim(nt, nunits, seed, mode=mode, kxs=kxs, xw_per_slot=xw_per_slot,
-                heavy=r.choice([0.0, 0.05, 0.2, 0.5]))
+                heavy=r.choice([0.0, 0.05, 0.2, 0.5]), bc=bc, release_early=release_early)
         try:
             run(S, list(range(nunits)))
         except Bug as e:
@@ -296,3 +326,17 @@ def test_model_catches_odd_slot_count_in_state_mode():
 def test_model_catches_single_diag_w_x_barrier():
     fails = _schedules(100, xw_per_slot=False)
     assert fails and any("overrun on XW_READY" in f for f in fails)
+
+
+def test_one_tile_units_reusing_shared_c_b_tiles():
+    """One-tile sequences whose consecutive units (heads of one batch element
+    and B/C group) take their C/B tiles from the ring in place: the slots are
+    released only after the last unit of a run, and no load is issued for the
+    others."""
+    fails = _schedules(1500, shared_bc=True)
+    assert not fails, "\n".join(fails[:5])
+
+
+def test_model_catches_reused_slots_released_per_unit():
+    fails = _schedules(300, shared_bc=True, release_early=True)
+    assert fails and any("read ('ring'" in f or "overrun" in f for f in fails)

@@ -113,6 +113,19 @@ def test_full_size_sampled(ssd, name, k):
         check(to_f64(out[b, :, h]), o, torch.bfloat16, f"{name} unit {(b, h)}")
 
 
+@pytest.mark.parametrize("shape", [(64, 128, 8, 128, 2), (50, 100, 6, 64, 1), (37, 128, 4, 128, 4)],
+                         ids=["L128_G2", "L100_G1_ragged", "L128_G4_no_sharing"])
+def test_one_tile_sequences_sharing_c_b(ssd, shape):
+    """Hundreds of one-tile sequences: each CTA takes a contiguous range of
+    (batch, head) units and reuses the C/B tiles in its ring for consecutive
+    heads of one batch element and B/C group (G < H); runs break at batch and
+    group boundaries and at the ends of each CTA's range. Every output checked."""
+    batch, L, H, N, G = shape
+    inp = si.bidir_inputs(batch, L, H, 64, N, G, "bf16", seed=batch + G, device="cuda")
+    y = run_bidir(ssd, inp, 64, PATHS["fused"])
+    check(y, full_oracle(inp), torch.bfloat16, f"one-tile {shape}")
+
+
 def _oracle_of(inp):
     return oracle.bidir(*(to_f64(inp[k]) for k in ("x", "dt", "A", "B", "C", "D")))
 

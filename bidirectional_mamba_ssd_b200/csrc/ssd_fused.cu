@@ -252,6 +252,11 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                               : (int)blockIdx.x;
     const int u_end = REUSE ? u_begin + per + ((int)blockIdx.x < rem ? 1 : 0) : p.units;
     const int u_step = REUSE ? 1 : (int)gridDim.x;
+    // the reverse state entering the last tile is zero (no given reverse start
+    // state): it is neither stored nor loaded, C_b H_b is not formed and the
+    // output leaves its term out
+    const bool rzero = MODE == kModeBidir || p.rinit == nullptr;
+    auto hb_zero = [&](int i) { return kOut && rzero && i == nt - 1; };
     // C/B reuse: unit u's output tile takes the previous unit's C/B tiles
     auto same_bc = [&](int u) {
         if constexpr (!REUSE || !kOut) return false;
@@ -323,8 +328,12 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         break;
                     if (kh >= 1 && !(ok = mbar_wait(bar(B_HB_EMPTY), (kh - 1) & 1, abort_flag, p.status, 104))) break;
                     ++kh;
-                    mbar_arrive_expect_tx(bar(B_HB_FULL), S::kH);
-                    tma_load_3d_hint(base + S::hb, &tm_h, bar(B_HB_FULL), 0, 0, u * nt + i, stream);
+                    if (hb_zero(i)) {
+                        mbar_arrive(bar(B_HB_FULL));   // nothing to load: C_b H_b is not formed
+                    } else {
+                        mbar_arrive_expect_tx(bar(B_HB_FULL), S::kH);
+                        tma_load_3d_hint(base + S::hb, &tm_h, bar(B_HB_FULL), 0, 0, u * nt + i, stream);
+                    }
                 }
             }
             // every load issued has landed before the CTA may exit (waited on only
@@ -416,7 +425,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     if (!keep_bc) mma_commit(bar(B_RING_EMPTY + rCf));
                     mbar_wait(bar(B_HB_FULL), kh++ & 1, abort_flag, p.status, 207);
                     tc_fence_after();
-                    for (int k = 0; k < N / 16; ++k) {      // Yo_b = C_b H_b
+                    for (int k = 0; !hb_zero(i) && k < N / 16; ++k) {      // Yo_b = C_b H_b
                         const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
                         mma_bf16_ss(tYob, sdesc_sw128(sCb + ko, 0, 1024),
                                     sdesc_sw128(base + S::hb + k * 2048, kSlab, 1024), id_o, k > 0);
@@ -494,7 +503,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             float lsum = 0.f;               // state modes: log of the sequence's decay, from the tile decays
             for (int k1 = 0; k1 < nt; ++k1) {
                 const int i = kFwd1 ? k1 : nt - 1 - k1;
-                if (kOut && row < N) {
+                if (kOut && row < N && !hb_zero(i)) {
                     __nv_bfloat16 *dst = p.hb + (((size_t)u * nt + i) * N + row) * kP;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -725,7 +734,12 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     uint32_t yd[16], yf[16], yb[16];
                     tmem_ld16(tYd + lane_off + q * 16, yd);
                     tmem_ld16(tYof + lane_off + q * 16, yf);
-                    tmem_ld16(tYob + lane_off + q * 16, yb);
+                    if (hb_zero(i)) {   // warp-uniform: the tile has no C_b H_b term
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) yb[j] = 0u;
+                    } else {
+                        tmem_ld16(tYob + lane_off + q * 16, yb);
+                    }
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {

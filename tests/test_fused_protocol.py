@@ -105,7 +105,11 @@ def producer(S, units_list):
             if kh >= 1:
                 yield ('wait', 'HB_EMPTY', kh - 1)
             kh += 1
-            yield ('tma_hb', 'HB_FULL', u, i)
+            if i == nt - 1:
+                # the reverse state entering the last tile is zero: nothing is loaded
+                yield ('arrive', 'HB_FULL')
+            else:
+                yield ('tma_hb', 'HB_FULL', u, i)
 
 def mma(S, units_list):
     nt, R, X = S.nt, S.kRing, S.kxs
@@ -159,7 +163,8 @@ def mma(S, units_list):
             if not keep:
                 yield ('commit', 'RING_EMPTY%d' % rCf)
             yield ('wait', 'HB_FULL', kh); kh += 1
-            yield ('mma', [(('ring', rCb), ('Cb', bcu, i)), ('hb', ('hb', u, i))], [(('Yob', 0), ('Yob', u, i)), (('Yob', 1), ('Yob', u, i))])
+            if i < nt - 1:   # the last tile has no C_b H_b term
+                yield ('mma', [(('ring', rCb), ('Cb', bcu, i)), ('hb', ('hb', u, i))], [(('Yob', 0), ('Yob', u, i)), (('Yob', 1), ('Yob', u, i))])
             if not keep:
                 yield ('commit', 'RING_EMPTY%d' % rCb)
             yield ('commit', 'HB_EMPTY')
@@ -182,7 +187,8 @@ def group_c(S, units_list):
         # reverse chain stores nt states and folds all tiles but the last one
         for i in range(nt):
             if S.mode != 'state':
-                yield ('write', ('hbg', u, i), ('hbg', u, i))
+                if i < nt - 1:   # the last tile's reverse state is zero and not stored
+                    yield ('write', ('hbg', u, i), ('hbg', u, i))
             if i == S.n1t():
                 break
             pb = n1 % 2
@@ -258,11 +264,12 @@ def group_ab(S, units_list, is_b):
             nvec += 1
             xs = kx % X; kx += 1
             yield ('wait', 'Y_READY', n_y); n_y += 1
-            for nm in ('Yd', 'Yof', 'Yob'):
+            outs = ('Yd', 'Yof', 'Yob') if i < nt - 1 else ('Yd', 'Yof')   # the last tile has no C_b H_b
+            for nm in outs:
                 yield ('read', (nm, half), (nm, u, i))
             yield ('read', ('x', xs, half), ('x', u, 2, i))
             yield ('write', ('x', xs, half), ('y', u, i))
-            for nm in ('Yd', 'Yof', 'Yob'):
+            for nm in outs:
                 yield ('read', (nm, half), (nm, u, i))
             yield ('sync', 'ab', 2)
             if is_b:

@@ -175,3 +175,15 @@ def bidir_seeded(x, dt, A, B, C, D, prefix=None, suffix=None, nthreads: int = 0)
     if rc != 0:
         raise ValueError("oracle bidir_seeded: bad arguments")
     return out
+
+
+def dt_prep(dt_raw, dt_bias, dt_min=0.0, dt_max=np.inf) -> np.ndarray:
+    """The step size a Mamba-2 layer feeds its scan, from the raw projection:
+    dt = clamp(softplus(dt_raw + dt_bias[d, h]), dt_min, dt_max), with
+    softplus(u) = log(1 + exp(u)), in fp64. dt_raw (2, batch, L, H), dt_bias
+    (2, H). The pages name Mamba-2 without printing its parametrisation; this
+    is the standard Mamba-2 one (a positive step from a biased softplus,
+    limited to a range), the input side of the mixer (before the scan)."""
+    u = np.asarray(dt_raw, dtype=np.float64) + np.asarray(dt_bias, dtype=np.float64)[:, None, None, :]
+    sp = np.logaddexp(0.0, u)          # log(1 + exp(u)) without overflow
+    return np.clip(sp, dt_min, dt_max)

@@ -308,6 +308,27 @@ def test_bidir_seeded_reverse_start_mirrors_forward_start():
     assert rel(y, np.flip(y2, 1)) < 1e-13
 
 
+def test_dt_prep_closed_forms():
+    """softplus(0) = ln 2; softplus(u) - softplus(-u) = u; softplus(u) -> u for
+    large u and -> e^u for very negative u; the clamp is applied after."""
+    z = np.zeros((2, 1, 3, 2))
+    assert np.allclose(oracle.dt_prep(z, np.zeros((2, 2))), math.log(2.0), rtol=0, atol=1e-15)
+    u = np.linspace(-30, 30, 61).reshape(1, 1, 61, 1).repeat(2, axis=0)
+    b = np.zeros((2, 1))
+    assert np.allclose(oracle.dt_prep(u, b) - oracle.dt_prep(-u, b), u, rtol=0, atol=1e-12)
+    assert abs(oracle.dt_prep(np.full((2, 1, 1, 1), 40.0), b)[0, 0, 0, 0] - 40.0) < 1e-15
+    assert abs(oracle.dt_prep(np.full((2, 1, 1, 1), -40.0), b)[0, 0, 0, 0] / math.exp(-40.0) - 1) < 1e-15
+    # the bias is per direction and head, added before the softplus
+    bias = np.array([[0.5, -1.0], [2.0, 0.0]])
+    got = oracle.dt_prep(np.zeros((2, 1, 1, 2)), bias)
+    want = np.log1p(np.exp(bias))[:, None, None, :]
+    assert np.allclose(got, want, rtol=1e-15, atol=0)
+    clamped = oracle.dt_prep(np.full((2, 1, 2, 2), -10.0), np.zeros((2, 2)), dt_min=1e-3, dt_max=0.1)
+    assert np.all(clamped == 1e-3)
+    clamped = oracle.dt_prep(np.full((2, 1, 2, 2), 10.0), np.zeros((2, 2)), dt_min=1e-3, dt_max=0.1)
+    assert np.all(clamped == 0.1)
+
+
 def test_units_subset_matches_full():
     rng = np.random.default_rng(12)
     prob = rand_problem(rng, batch=3, L=10, H=4)

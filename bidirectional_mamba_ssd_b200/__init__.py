@@ -13,6 +13,7 @@ Functions carry the C names:
   ssd_segment_states(x, dt, A, B)                      -> (fwd_state, fwd_decay, rev_state, rev_decay)
   ssd_segment_carry(fwd_states, fwd_decays, rev_states, rev_decays, seg) -> (fwd_in, rev_in)
   ssd_bidir_fwd_seeded(x, dt, A, B, C, D, fwd_init, rev_init)           -> out
+  ssd_bidir_fwd_dtraw(x, dt_raw, dt_bias, A, B, C, D, dt_min, dt_max)   -> out
 The sequence-sharded mixer over a process group is in seqshard.py.
 Shapes (row-major, natural token order; [0] forward, [1] reverse):
   x (batch, L, H, P); dt (2, batch, L, H); A, D (2, H) fp32;
@@ -31,7 +32,7 @@ from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSE
                    SSD_OP_BLOCK_STEP)
 
 __all__ = ["ssd_bidir_fwd", "ssd_prefix_state", "ssd_block_step", "ssd_segment_states",
-           "ssd_segment_carry", "ssd_bidir_fwd_seeded", "ssd_workspace_bytes",
+           "ssd_segment_carry", "ssd_bidir_fwd_seeded", "ssd_bidir_fwd_dtraw", "ssd_workspace_bytes",
            "ssd_get_device_status", "SSDError", "Workspace", "lib"]
 
 lib = _c.load()
@@ -321,4 +322,29 @@ def ssd_bidir_fwd_seeded(x, dt, A, B, C, D, fwd_init=None, rev_init=None, out=No
                                   _ptr(rev_init), _ptr(out), batch, L, H, P, N, G, _DT[io],
                                   _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_bidir_fwd_seeded")
+    return out
+
+
+def ssd_bidir_fwd_dtraw(x, dt_raw, dt_bias, A, B, C, D, dt_min: float = 0.0, dt_max: float = float("inf"),
+                        out=None, *, workspace: Workspace | None = None):
+    """The mixer with the step size prepared in the kernel from the raw
+    projection: dt = clamp(softplus(dt_raw + dt_bias), dt_min, dt_max)
+    (include/ssd_bidir.h: ssd_bidir_fwd_dtraw). dt_raw like dt, dt_bias (2, H) fp32."""
+    dev, io, batch, L, H, P, G, N = _bidir_args(x, dt_raw, A, B, C, D, "ssd_bidir_fwd_dtraw")
+    _need(dt_bias, "dt_bias", torch.float32, dev, 2)
+    if tuple(dt_bias.shape) != (2, H):
+        raise ValueError("dt_bias must be (2, H)")
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _need(out, "out", io, dev, 4)
+        if out.shape != x.shape:
+            raise ValueError("out must have x's shape")
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    buf = ws.get(max(ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, L, H, P, N, G, 64, io), 256))
+    rc = lib.ssd_bidir_fwd_dtraw(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), float(dt_min), float(dt_max),
+                                 _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(out), batch, L, H, P, N, G, _DT[io],
+                                 _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_bidir_fwd_dtraw")
     return out

@@ -36,6 +36,7 @@ SIGNATURES = {
     "ssd_segment_states": (_i, [_vp] * 8 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_segment_carry": (_i, [_vp] * 4 + [_i] * 2 + [_vp] * 2 + [_i] * 4 + [_vp]),
     "ssd_bidir_fwd_seeded": (_i, [_vp] * 9 + [_i] * 7 + [_vp, _sz, _vp]),
+    "ssd_bidir_fwd_dtraw": (_i, [_vp] * 3 + [ctypes.c_float] * 2 + [_vp] * 5 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_get_device_status": (_i, [_vp, _vp]),
     "ssd_selftest_wait_timeout": (_i, [_vp, _sz, _i, _vp]),
     "ssd_error_string": (ctypes.c_char_p, [_i]),

@@ -275,6 +275,32 @@ int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
                                dstate, ngroups, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
 }
 
+int ssd_bidir_fwd_dtraw(const void *x, const void *dt_raw, const float *dt_bias, float dt_min, float dt_max,
+                        const float *A, const void *B, const void *C, const float *D, void *out, int batch,
+                        int seqlen, int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
+                        size_t ws_bytes, void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype, false);
+    if (rc != SSD_OK) return rc;
+    if (dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    // NaN bounds fail both comparisons
+    if (!(dt_min >= 0.f) || !(dt_max >= dt_min)) return SSD_ERR_INVALID_ARG;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    if (!x || !dt_raw || !dt_bias || !A || !B || !C || !D || !out) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt_raw) || !aligned16(B) || !aligned16(C) || !aligned16(out) ||
+        !aligned4(dt_bias) || !aligned4(A) || !aligned4(D))
+        return SSD_ERR_INVALID_ARG;
+    TcArgs t{};
+    t.x = x; t.dt = dt_raw; t.A = A; t.B = B; t.C = C; t.D = D; t.out = out;
+    t.dt_bias = dt_bias; t.dt_lo = dt_min; t.dt_hi = dt_max;
+    t.workspace = workspace; t.ws_bytes = ws_bytes;
+    t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+    return to_status(ssd::launch_tc_fused_dtraw(t, static_cast<cudaStream_t>(stream)));
+}
+
 // Segments to split each sequence into when a call has too few (batch, head)
 // units to fill the GPU (as SSD_PATH_AUTO chooses the segmented path); 1 = none.
 int few_unit_segments(int batch, int seqlen, int nheads) {

@@ -93,7 +93,17 @@ struct FusedParams {
     float *decay_out;          // (batch, H) state modes: exp(A * sum of dt) over the sequence, or nullptr
     DeviceStatus *status;
     int batch, L, H, G, nt, units;
+    const float *dt_bias;      // DTRAW: (2, H); dt holds the raw projection
+    float dt_lo, dt_hi;        // DTRAW: the step-size range
 };
+
+// The step size from the raw projection (DTRAW): softplus(raw + bias),
+// clamped to [lo, hi]. softplus(u) = log(1 + e^u), equal to u in fp32 beyond 20.
+__device__ __forceinline__ float dt_from_raw(float raw, float bias, float lo, float hi) {
+    const float u = raw + bias;
+    const float sp = u > 20.f ? u : log1pf(__expf(u));
+    return fminf(fmaxf(sp, lo), hi);
+}
 
 // barrier indices
 enum {
@@ -186,9 +196,11 @@ struct Smem {
 // REUSE (one-tile sequences whose B/C are shared by several heads): each CTA
 // takes a contiguous range of units (else every gridDim-th), and an output
 // tile whose C/B tiles are those of the unit before it on the same CTA (same
-// batch element and B/C group) takes them from the ring in place. A template
-// parameter, so that the other shapes' kernels carry none of its code.
-template <int N, int MODE, bool REUSE>
+// batch element and B/C group) takes them from the ring in place. DTRAW: dt
+// holds the raw projection, and every valid token's step size is
+// dt_from_raw of it (tokens past the end keep 0). Template parameters, so that
+// the other kernels carry none of their code.
+template <int N, int MODE, bool REUSE, bool DTRAW>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_h,
@@ -474,20 +486,27 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // dt of the next output-pass tile is fetched a tile ahead (volatile
         // loads, so the compiler keeps them a tile early)
         uint32_t rawf = 0, rawb = 0;
+        bool dt_valid = false;          // DTRAW: the token of rawf / rawb lies in the sequence
         auto load_dt = [&](int u, int i) {
             rawf = 0;
             rawb = 0;
+            dt_valid = false;
             if (u >= u_end) return;
             const int b = u / p.H, h = u % p.H, t = i * kTile + row;
             if (t < p.L) {
+                dt_valid = true;
                 const size_t o = ((size_t)b * p.L + t) * p.H + h;
                 asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawb) : "l"(p.dt + dt_dir + o));
                 asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawf) : "l"(p.dt + o));
             }
         };
-        auto take_dt = [&](float &vf, float &vb) {
+        auto take_dt = [&](float &vf, float &vb, int h) {
             vf = __uint_as_float(rawf << 16);
             vb = __uint_as_float(rawb << 16);
+            if constexpr (DTRAW) {
+                vf = dt_valid ? dt_from_raw(vf, p.dt_bias[h], p.dt_lo, p.dt_hi) : 0.f;
+                vb = dt_valid ? dt_from_raw(vb, p.dt_bias[p.H + h], p.dt_lo, p.dt_hi) : 0.f;
+            }
         };
         int cu = u_begin, ci = 0;   // the output-pass tile whose dt is in flight
         if constexpr (kOut) load_dt(cu, ci);
@@ -564,7 +583,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // ---------------- phase 2: decay sums, vectors, diag(w_f) X, forward chain
             for (int i = 0; i < nt; ++i) {
                 float vf, vb;
-                take_dt(vf, vb);
+                take_dt(vf, vb, h);
                 if (++ci == nt) { ci = 0; cu += u_step; }
                 load_dt(cu, ci);
                 float pf = vf, pb = vb, totf, totb;
@@ -647,22 +666,28 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // direction (reverse: r < s, forward: r > s), diag(w) X in place in
             // the x slot, and the tile decay exp(A sum dt) for group C's chain.
             uint32_t rawn = 0;               // dt of this group's next tile, fetched a tile ahead
+            bool rawn_valid = false;         // its token lies in the sequence
             bool have = false;
+            // DTRAW: the state pass's step size from the raw projection
+            const float bias1 = DTRAW ? p.dt_bias[kFwd1 ? h : p.H + h] : 0.f;
+            auto dt1_of = [&](float raw) { return DTRAW ? dt_from_raw(raw, bias1, p.dt_lo, p.dt_hi) : raw; };
             for (int k1 = 0; k1 < n1t; ++k1, ++m1, ++kx) {
                 if ((m1 & 1) != (uint32_t)is_b) continue;
                 const int i = kFwd1 ? k1 : nt - 1 - k1;
                 float vb = 0.f;
                 if (have) {
-                    vb = bf2f(rawn);
+                    if (rawn_valid) vb = dt1_of(bf2f(rawn));
                 } else {
                     const int t = i * kTile + row;
-                    if (t < p.L) vb = __bfloat162float(p.dt[dt1 + ((size_t)b * p.L + t) * p.H + h]);
+                    if (t < p.L) vb = dt1_of(__bfloat162float(p.dt[dt1 + ((size_t)b * p.L + t) * p.H + h]));
                 }
                 have = k1 + 2 < n1t;         // this group's next tile, two on in the pass's order
                 rawn = 0;
+                rawn_valid = false;
                 if (have) {
                     const int t = (kFwd1 ? i + 2 : i - 2) * kTile + row;
                     if (t < p.L) {
+                        rawn_valid = true;
                         const size_t o = dt1 + ((size_t)b * p.L + t) * p.H + h;
                         asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(rawn) : "l"(p.dt + o));
                     }
@@ -783,7 +808,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-template <int N, int MODE, bool REUSE>
+template <int N, int MODE, bool REUSE, bool DTRAW>
 cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     using S = Smem<N>;
     constexpr bool kOut = MODE == kModeBidir || MODE == kModeBidirInit;
@@ -803,6 +828,9 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     p.decay_out = a.decay_out;
     p.status = static_cast<DeviceStatus *>(a.workspace);
     p.batch = a.batch; p.L = a.L; p.H = a.H; p.G = a.G; p.nt = nt; p.units = units;
+    p.dt_bias = a.dt_bias;
+    p.dt_lo = a.dt_lo;
+    p.dt_hi = a.dt_hi;
 
     CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_out;
     // the forward state mode may be given single-direction B; every other mode reads both directions' layout
@@ -820,7 +848,7 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    auto k = tc_fused_kernel<N, MODE, REUSE>;
+    auto k = tc_fused_kernel<N, MODE, REUSE, DTRAW>;
     const size_t smem = S::bytes + 1024;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return e;
@@ -840,7 +868,7 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, k, tm_x, tm_b, tm_c, tm_h, tm_out, p);
 }
 
-template <int MODE>
+template <int MODE, bool DTRAW = false>
 cudaError_t launch_mode(const TcArgs &a, cudaStream_t stream) {
     if (a.L <= 0 || a.batch <= 0) return cudaErrorNotSupported;
     if (a.N != 64 && a.N != 128) return cudaErrorNotSupported;
@@ -851,8 +879,8 @@ cudaError_t launch_mode(const TcArgs &a, cudaStream_t stream) {
     // one-tile sequences with B/C shared by several heads: consecutive heads on
     // one CTA, taking their C/B tiles from the ring in place
     if (kOut && a.L <= kTile && a.G < a.H)
-        return a.N == 64 ? run_fused<64, MODE, kOut>(a, stream) : run_fused<128, MODE, kOut>(a, stream);
-    return a.N == 64 ? run_fused<64, MODE, false>(a, stream) : run_fused<128, MODE, false>(a, stream);
+        return a.N == 64 ? run_fused<64, MODE, kOut, DTRAW>(a, stream) : run_fused<128, MODE, kOut, DTRAW>(a, stream);
+    return a.N == 64 ? run_fused<64, MODE, false, DTRAW>(a, stream) : run_fused<128, MODE, false, DTRAW>(a, stream);
 }
 
 }  // namespace
@@ -874,6 +902,11 @@ bool tc_fused_supported(int batch, int L, int H, int G, int N) {
 
 cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream) {
     return a.init || a.rinit ? launch_mode<kModeBidirInit>(a, stream) : launch_mode<kModeBidir>(a, stream);
+}
+
+cudaError_t launch_tc_fused_dtraw(const TcArgs &a, cudaStream_t stream) {
+    if (!a.dt_bias || a.init || a.rinit) return cudaErrorNotSupported;
+    return launch_mode<kModeBidir, true>(a, stream);
 }
 
 cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream) {

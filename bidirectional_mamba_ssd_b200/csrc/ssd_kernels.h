@@ -40,6 +40,8 @@ struct TcArgs {
     const float *init;        // (batch, H, 64, N) forward start state or nullptr
     const float *rinit = nullptr;  // (batch, H, 64, N) reverse start state (at the sequence end) or nullptr
     float *decay_out = nullptr;    // (batch, H) fused state modes: exp(A * sum of dt) over the sequence
+    const float *dt_bias = nullptr;  // (2, H) with launch_tc_fused_dtraw: dt holds the raw projection
+    float dt_lo = 0.f, dt_hi = 0.f;  // with launch_tc_fused_dtraw: the step-size range
     float *state_out;         // (batch, H, 64, N) or nullptr
     void *out;                // (batch, L, H, 64) bf16
     void *workspace;          // status header + scratch
@@ -57,6 +59,10 @@ cudaError_t launch_tc_chunked(const TcArgs &a, cudaStream_t stream);
 // Fused kernel, both scans summed; with a.init the forward scan starts from
 // that state (block step).
 cudaError_t launch_tc_fused(const TcArgs &a, cudaStream_t stream);
+// Fused kernel, both scans, with the step size prepared from the raw
+// projection in the kernel: dt = clamp(softplus(dt_raw + a.dt_bias), a.dt_lo,
+// a.dt_hi) for every token in the sequence (a.dt holds dt_raw).
+cudaError_t launch_tc_fused_dtraw(const TcArgs &a, cudaStream_t stream);
 // Fused kernel, forward scan only: the final state into a.state_out, from
 // a.init or zero (prefix state); needs no scratch past the status header.
 cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream);

@@ -193,6 +193,24 @@ int ssd_block_step_path(const void *x, const void *dt, const float *A, const voi
                         int ngroups, int dtype, int path,
                         void *workspace, size_t ws_bytes, void *stream);
 
+/* ssd_bidir_fwd with the step size prepared inside the kernel from the raw
+ * dt projection of a Mamba-2 layer:
+ *   dt = min(max(softplus(dt_raw + dt_bias[d][h]), dt_min), dt_max),
+ *   softplus(u) = log(1 + exp(u)),
+ * for every token of every sequence (the pages name Mamba-2 without printing
+ * its parametrisation; this is the standard Mamba-2 one, the input side of
+ * the mixer). It saves writing and reading back a prepared dt tensor.
+ *   dt_raw   (2, batch, seqlen, nheads)  io (bf16), the raw projection
+ *   dt_bias  (2, nheads)                 fp32
+ *   dt_min, dt_max                       0 <= dt_min <= dt_max (INFINITY for no upper bound)
+ * Other arguments as ssd_bidir_fwd. bf16 I/O only (the fused kernel, for any
+ * number of (batch, head) units); fp32 returns SSD_ERR_UNSUPPORTED. Workspace:
+ * at least ssd_workspace_bytes(SSD_OP_BIDIR_FWD, ..., chunk 64, SSD_BF16). */
+int ssd_bidir_fwd_dtraw(const void *x, const void *dt_raw, const float *dt_bias, float dt_min, float dt_max,
+                        const float *A, const void *B, const void *C, const float *D, void *out,
+                        int batch, int seqlen, int nheads, int headdim, int dstate, int ngroups,
+                        int dtype, void *workspace, size_t ws_bytes, void *stream);
+
 /* Sequences split across GPUs (or any other split into segments): each
  * holder of one segment of every sequence computes its segment's own states,
  * the holders exchange them (one all-gather of nseg x (2 states + 2 decays)

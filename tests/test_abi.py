@@ -160,3 +160,18 @@ def test_segment_entry_points_reject_bad_arguments(lib):
     assert sd(2, 256, 4, 64, 128, 4, 1, out=0) == -1
     assert sd(2, 256, 4, 64, 128, 4, 1, init=FAKE + 8) == -1
     assert sd(2, 0, 4, 64, 128, 4, 1, out=0) == 0
+
+
+def test_dtraw_rejects_bad_arguments(lib):
+    v = ctypes.c_void_p
+    f = ctypes.c_float
+    call = lambda *ints, lo=0.0, hi=1.0, ws=FAKE, wsb=1 << 40, bias=FAKE, out=FAKE: lib.ssd_bidir_fwd_dtraw(
+        v(FAKE), v(FAKE), v(bias), f(lo), f(hi), v(FAKE), v(FAKE), v(FAKE), v(FAKE), v(out), *ints, v(ws), wsb, None)
+    assert call(2, 256, 4, 64, 128, 4, 1, ws=0) == -4
+    assert call(2, 256, 4, 64, 128, 4, 0) == -2                   # fp32: not on this path
+    assert call(2, 256, 4, 64, 128, 4, 1, lo=-1.0) == -1          # negative lower bound
+    assert call(2, 256, 4, 64, 128, 4, 1, lo=0.2, hi=0.1) == -1   # empty range
+    assert call(2, 256, 4, 64, 128, 4, 1, lo=float("nan")) == -1
+    assert call(2, 256, 4, 64, 128, 4, 1, bias=0) == -1
+    assert call(2, 256, 4, 64, 128, 4, 1, bias=FAKE + 2) == -1
+    assert call(2, 0, 4, 64, 128, 4, 1, out=0) == 0

@@ -39,7 +39,8 @@ int to_status(cudaError_t e) {
 
 size_t simt_scratch(int op, int batch, int seqlen, int nheads) {
     if (op == SSD_OP_PREFIX_STATE) return 0;
-    return sizeof(float) * (size_t)batch * seqlen * nheads * kHeaddim;
+    // one fp32 output buffer per scan direction
+    return 2 * sizeof(float) * (size_t)batch * seqlen * nheads * kHeaddim;
 }
 
 size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }

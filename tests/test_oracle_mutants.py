@@ -24,6 +24,9 @@ PIN_CHECKS = [
     pins.test_prefix_state_closed_form,
     pins.test_prefix_state_composes,
     pins.test_block_step_equals_split_scans,
+    pins.test_bidir_seeded_with_zero_states_is_the_plain_mixer,
+    pins.test_bidir_seeded_segments_rebuild_the_whole_sequence,
+    pins.test_bidir_seeded_reverse_start_mirrors_forward_start,
 ]
 
 # (name, text in ssd_oracle.c, replacement)
@@ -39,6 +42,10 @@ MUTANTS = [
     ("reverse_uses_forward_A", "A[d * H + hh], Bu, Cu", "A[hh], Bu, Cu"),
     ("block_reverse_from_prefix", "(d == 0 && prefix)", "(prefix)"),
     ("output_off_by_one_token", "double *yt = y + (size_t)t * P;", "double *yt = y + (size_t)((t + 1) % L) * P;"),
+    ("seeded_reverse_start_ignored", "const double *start = d == 0 ? prefix : suffix;",
+     "const double *start = d == 0 ? prefix : NULL;"),
+    ("seeded_starts_swapped", "const double *start = d == 0 ? prefix : suffix;",
+     "const double *start = d == 0 ? suffix : prefix;"),
 ]
 
 
@@ -65,3 +72,33 @@ def test_pins_catch_planted_mistake(tmp_path, monkeypatch, name, old, new):
         except (AssertionError, ValueError):
             failed.append(check.__name__)
     assert failed, f"no pin caught mutant {name}"
+
+
+# (name, a mistaken dt_prep): the closed-form pin must reject each
+def _dt_prep_mutants():
+    import numpy as np
+
+    def no_bias(dt_raw, dt_bias, dt_min=0.0, dt_max=np.inf):
+        return np.clip(np.logaddexp(0.0, np.asarray(dt_raw, np.float64)), dt_min, dt_max)
+
+    def exp_not_softplus(dt_raw, dt_bias, dt_min=0.0, dt_max=np.inf):
+        u = np.asarray(dt_raw, np.float64) + np.asarray(dt_bias, np.float64)[:, None, None, :]
+        return np.clip(np.exp(u), dt_min, dt_max)
+
+    def bias_per_direction_swapped(dt_raw, dt_bias, dt_min=0.0, dt_max=np.inf):
+        u = np.asarray(dt_raw, np.float64) + np.asarray(dt_bias, np.float64)[::-1, None, None, :]
+        return np.clip(np.logaddexp(0.0, u), dt_min, dt_max)
+
+    def clamp_before_softplus(dt_raw, dt_bias, dt_min=0.0, dt_max=np.inf):
+        u = np.asarray(dt_raw, np.float64) + np.asarray(dt_bias, np.float64)[:, None, None, :]
+        return np.logaddexp(0.0, np.clip(u, dt_min, dt_max))
+
+    return [("no_bias", no_bias), ("exp_not_softplus", exp_not_softplus),
+            ("bias_directions_swapped", bias_per_direction_swapped), ("clamp_before_softplus", clamp_before_softplus)]
+
+
+@pytest.mark.parametrize("name,fn", _dt_prep_mutants(), ids=[m[0] for m in _dt_prep_mutants()])
+def test_dt_prep_pin_catches_planted_mistake(monkeypatch, name, fn):
+    monkeypatch.setattr(oracle, "dt_prep", fn)
+    with pytest.raises(AssertionError):
+        pins.test_dt_prep_closed_forms()

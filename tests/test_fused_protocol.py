@@ -32,7 +32,7 @@ class Sim(Sched):
     pass alone); kxs: x slots; xw_per_slot False plants the earlier single
     diag(w) X barrier."""
     def __init__(self, nt, units, seed, kRing=4, mode='bidir', kxs=2, xw_per_slot=True, heavy=0.1, bc=None,
-                 release_early=False):
+                 release_early=False, rzero=True):
         super().__init__(seed, heavy)
         self.nt, self.units, self.kRing = nt, units, kRing
         self.mode, self.kxs, self.xw_per_slot = mode, kxs, xw_per_slot
@@ -41,6 +41,11 @@ class Sim(Sched):
         # group share them); one-tile units reuse the previous unit's in place
         self.bc = bc
         self.release_early = release_early   # planted: release reused slots after each unit
+        # the reverse state entering the last tile is zero (no given reverse start
+        # state): not stored, not loaded, no C_b H_b
+        self.rzero = rzero
+    def hb_zero(self, i):
+        return self.rzero and i == self.nt - 1
     def bc_of(self, units_list, j):
         return self.bc[j] if self.bc is not None else units_list[j]
     def reuse(self, units_list, j):
@@ -105,7 +110,7 @@ def producer(S, units_list):
             if kh >= 1:
                 yield ('wait', 'HB_EMPTY', kh - 1)
             kh += 1
-            if i == nt - 1:
+            if S.hb_zero(i):
                 # the reverse state entering the last tile is zero: nothing is loaded
                 yield ('arrive', 'HB_FULL')
             else:
@@ -163,7 +168,7 @@ def mma(S, units_list):
             if not keep:
                 yield ('commit', 'RING_EMPTY%d' % rCf)
             yield ('wait', 'HB_FULL', kh); kh += 1
-            if i < nt - 1:   # the last tile has no C_b H_b term
+            if not S.hb_zero(i):   # a zero reverse state has no C_b H_b term
                 yield ('mma', [(('ring', rCb), ('Cb', bcu, i)), ('hb', ('hb', u, i))], [(('Yob', 0), ('Yob', u, i)), (('Yob', 1), ('Yob', u, i))])
             if not keep:
                 yield ('commit', 'RING_EMPTY%d' % rCb)
@@ -187,7 +192,7 @@ def group_c(S, units_list):
         # reverse chain stores nt states and folds all tiles but the last one
         for i in range(nt):
             if S.mode != 'state':
-                if i < nt - 1:   # the last tile's reverse state is zero and not stored
+                if not S.hb_zero(i):   # a zero reverse state is not stored
                     yield ('write', ('hbg', u, i), ('hbg', u, i))
             if i == S.n1t():
                 break
@@ -264,7 +269,7 @@ def group_ab(S, units_list, is_b):
             nvec += 1
             xs = kx % X; kx += 1
             yield ('wait', 'Y_READY', n_y); n_y += 1
-            outs = ('Yd', 'Yof', 'Yob') if i < nt - 1 else ('Yd', 'Yof')   # the last tile has no C_b H_b
+            outs = ('Yd', 'Yof') if S.hb_zero(i) else ('Yd', 'Yof', 'Yob')   # no C_b H_b for a zero state
             for nm in outs:
                 yield ('read', (nm, half), (nm, u, i))
             yield ('read', ('x', xs, half), ('x', u, 2, i))
@@ -287,7 +292,8 @@ def run(S, units_list):
     run_roles(S, roles, counts)
 
 
-def _schedules(n, mode='bidir', kxs=2, xw_per_slot=True, seed0=0, shared_bc=False, release_early=False):
+def _schedules(n, mode='bidir', kxs=2, xw_per_slot=True, seed0=0, shared_bc=False, release_early=False,
+               rzero=True):
     fails = []
     for seed in range(seed0, seed0 + n):
         r = random.Random(seed)
@@ -302,7 +308,7 @@ def _schedules(n, mode='bidir', kxs=2, xw_per_slot=True, seed0=0, shared_bc=Fals
                     g += 1
                 bc.append(g)
         S = Sim(nt, nunits, seed, mode=mode, kxs=kxs, xw_per_slot=xw_per_slot,
-                heavy=r.choice([0.0, 0.05, 0.2, 0.5]), bc=bc, release_early=release_early)
+                heavy=r.choice([0.0, 0.05, 0.2, 0.5]), bc=bc, release_early=release_early, rzero=rzero)
         try:
             run(S, list(range(nunits)))
         except Bug as e:
@@ -347,3 +353,10 @@ def test_one_tile_units_reusing_shared_c_b_tiles():
 def test_model_catches_reused_slots_released_per_unit():
     fails = _schedules(300, shared_bc=True, release_early=True)
     assert fails and any("read ('ring'" in f or "overrun" in f for f in fails)
+
+
+def test_seeded_reverse_start_loads_the_last_tile_state():
+    """With a given reverse start state the last tile's reverse state is
+    stored, loaded and multiplied like every other tile's."""
+    fails = _schedules(1000, rzero=False)
+    assert not fails, "\n".join(fails[:5])

@@ -1,0 +1,70 @@
+"""Host-side pieces of bench.py: the algorithmic byte count the roofline
+divides by, the parser of ncu's raw CSV that records a path's DRAM traffic,
+and the rule that a record counts only while its kernels' sources are
+unchanged. No GPU."""
+import csv
+import json
+import os
+
+import bench
+import ssd_inputs as si
+
+
+def test_algorithmic_bytes_of_the_130m_shape():
+    # per token: x read once and out written once (24 x 64 bf16 each), dt of
+    # both directions (2 x 24 bf16), B and C of both directions (4 x 24 x 128
+    # bf16): 30 816 bytes; plus A and D (2 x 24 fp32 each)
+    w = si.WORKLOADS["mixer130m_b32_L1024"]
+    assert bench.algorithmic_bytes(w) == 32 * 1024 * 30816 + 4 * 4 * 24 == 1009779072
+
+
+def test_every_path_names_existing_sources_and_kernels():
+    csrc = os.path.join(bench.ROOT, "bidirectional_mamba_ssd_b200", "csrc")
+    for path, files in bench.KERNEL_SOURCE.items():
+        for f in files:
+            assert os.path.exists(os.path.join(csrc, f)), (path, f)
+        assert bench.KERNEL_NAMES[path], path
+        assert len(bench.kernel_source_sha(path)) == 16
+
+
+def _raw_csv(tmp_path, rows):
+    p = tmp_path / "raw.csv"
+    with open(p, "w", newline="") as f:
+        w = csv.writer(f)
+        w.writerow(["ID", "Kernel Name", "dram__bytes_read.sum", "dram__bytes_write.sum"])
+        w.writerow(["", "", "Mbyte", "Gbyte"])
+        for r in rows:
+            w.writerow(r)
+    return str(p)
+
+
+def test_record_traffic_sums_one_call_and_expires_with_the_source(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "traffic.json"))
+    # two calls of the segmented path: each launches the fused kernel three
+    # times and the segment scan once
+    rows = []
+    for _ in range(2):
+        rows += [[0, "void ssd::tc_fused_kernel<128, 2, 0, 0>(CUtensorMap_st, ...)", "1,202.4", "0.003"],
+                 [1, "void ssd::tc_fused_kernel<128, 3, 0, 0>(CUtensorMap_st, ...)", "202.4", "0"],
+                 [2, "ssd::seg_scan_kernel(const float *, ...)", "8.4", "0"],
+                 [3, "void ssd::tc_fused_kernel<128, 1, 0, 0>(CUtensorMap_st, ...)", "806.1", "0.07"]]
+    csv_path = _raw_csv(tmp_path, rows)
+    bench.record_traffic(csv_path, "segmented", "long_L16384", "ncu ...", scale=2.0, note="scaled")
+    d = json.load(open(bench.TRAFFIC_FILE))
+    e = d["long_L16384:segmented"]
+    # reads in Mbyte (with a thousands separator), writes in Gbyte
+    per_call = 1202.4e6 + 0.003e9 + 202.4e6 + 8.4e6 + 806.1e6 + 0.07e9
+    assert e["calls_captured"] == 2
+    assert e["dram_bytes_per_launch"] == round(per_call * 2.0)
+    assert e["scaled"] == {"factor": 2.0, "note": "scaled"}
+    assert bench.traffic_record("segmented", "long_L16384") == e["dram_bytes_per_launch"]
+    # a record taken on other sources no longer counts
+    e["source_sha"] = "0" * 16
+    json.dump(d, open(bench.TRAFFIC_FILE, "w"))
+    assert bench.traffic_record("segmented", "long_L16384") is None
+    assert bench.traffic_record("fused", "no_such_workload") is None
+
+
+def test_whole_job_throughput_and_time_at_one_rank():
+    assert bench.job_time_ms(3.5, 1) == 3.5
+    assert bench.job_throughput(1000, 4, 1, 2.0) == 1000 * 4 / 2e-3

@@ -8,15 +8,20 @@
 // and hands out no allocator, and latency-critical loops where a cudaMalloc or
 // cudaFree would synchronise the device. This entry point needs nothing from
 // them but the inputs and the output: its scratch is a fixed array in the
-// library's own device memory, reserved when the library's module is loaded
-// onto a GPU and kept until the process exits.
+// library's own device memory.
+//
+// When that array is reserved: under CUDA's default lazy module loading, the
+// module holding it is loaded onto a device by the first call on that device
+// (its cudaGetSymbolAddress), so the 32 MiB are reserved then and that first
+// call may allocate and synchronise; with CUDA_MODULE_LOADING=EAGER they are
+// reserved when the context is created. Either way they stay reserved until
+// the process exits. Make the first call on each device before any stream
+// capture begins.
 //
 // It runs the same fused tensor-core kernel as ssd_bidir_fwd (bf16 I/O), with
 // that array as the kernel's workspace: a 256-byte status header, then the
 // reverse scan's per-tile states (batch * nheads * ceil(seqlen/128) * dstate
 // * 64 bf16 values), which is what limits the problem size.
-#include <mutex>
-
 #include "ssd_bidir.h"
 #include "ssd_kernels.h"
 
@@ -29,24 +34,15 @@ constexpr size_t kNoAllocBytes = ssd::kStatusBytes + kNoAllocScratchMax;
 // The scratch itself. Every GPU that loads the library holds it until exit.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-// Device address of g_noalloc_scratch per device. In host code the symbol is
-// only a host-side stand-in, so the address is looked up once per device
-// (with that device current) and passed to the kernel.
-constexpr int kMaxDevices = 128;
-void *g_scratch_addr[kMaxDevices] = {};
-std::mutex g_setup_mutex;
-
+// Device address of g_noalloc_scratch on the current device. In host code the
+// symbol is only a host-side stand-in, so the address is looked up on every
+// call, with the calling device (and its context) current: a cached address
+// could outlive a cudaDeviceReset or belong to another context of the same
+// device. Once the module is loaded the lookup is a cheap host-side query.
 int scratch_address(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SSD_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SSD_ERR_CUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SSD_ERR_CUDA;
+    *out = p;
     return SSD_OK;
 }
 

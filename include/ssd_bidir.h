@@ -272,12 +272,16 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
  *  - bf16 I/O only (the fused tensor-core kernel); fp32 returns
  *    SSD_ERR_UNSUPPORTED.
  *  - Scratch is a fixed 32 MiB array (plus a 256-byte status header) inside
- *    the library, held by every GPU that loads the library until the process
- *    exits. Problems needing more, i.e. batch * nheads * ceil(seqlen / 128) *
- *    dstate * 128 bytes > 32 MiB, return SSD_ERR_WORKSPACE and launch nothing.
- *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
- *  - The first call on each device looks the array's device address up (with
- *    that device current); make that first call before any stream capture.
+ *    the library. Under CUDA's default lazy module loading it is reserved on
+ *    a device by the first call on that device, which may therefore allocate
+ *    and synchronise (with CUDA_MODULE_LOADING=EAGER: when the context is
+ *    created); it stays reserved until the process exits. Make the first call
+ *    on each device before any stream capture. Problems needing more, i.e.
+ *    batch * nheads * ceil(seqlen / 128) * dstate * 128 bytes > 32 MiB,
+ *    return SSD_ERR_WORKSPACE and launch nothing.
+ *  - Allocates nothing after that first call: no cudaMalloc, no cudaFree, no
+ *    allocating library call. Every call looks the array's device address up
+ *    with the calling device current (a cheap host-side query).
  *  - Every call shares the one array: calls that overlap on the GPU (other
  *    streams, other host threads) race and give wrong results. Each call
  *    clears the status header and overwrites the state area before reading it.

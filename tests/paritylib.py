@@ -14,7 +14,13 @@ Why the half ulp is excluded for bf16 outputs: these outputs are heavy
 tailed (max|o| / rms(o) is about 9 at the 130M shape), so rounding the exact
 result to bf16 already moves the largest ones by up to 2^-9 * 9 * rms ~ 0.018
 rms; a bare max-abs bound of 0.02 rms would reject correctly rounded answers.
-The RMS of the error is reported too (rms_err).
+The half-ulp allowance could hide a systematic error of up to 2^-9 relative
+on every element, so bf16 results are also held to an RMS bar:
+  rms(y - o) / rms(o) <= 3e-3.
+Rounding the exact output to bf16 alone gives about 2^-8 / sqrt(12) = 1.1e-3
+(uniform rounding error over the spacing), and the kernels' bf16 MMA operands
+add a little more (1.7e-3 measured at the 130M shape); a bias of 0.3 % on every
+element fails this bar.
 """
 from __future__ import annotations
 
@@ -26,6 +32,7 @@ from ssd_inputs import to_f64
 
 TOL_F32 = 1e-4
 TOL_BF16 = 2e-2
+TOL_BF16_RMS = 3e-3
 
 
 def rms(o):
@@ -68,7 +75,9 @@ def check(y, o, io_dtype, what="", state=False):
         assert e <= TOL_F32, f"{what}: fp32 max rel err {e:.3e} > {TOL_F32}"
     else:
         e = err_bf16(y, o, rounded_output=not state)
-        assert e <= TOL_BF16, f"{what}: bf16 err / rms {e:.3e} > {TOL_BF16} (rms err {rms_err(y, o):.2e})"
+        r = rms_err(y, o)
+        assert e <= TOL_BF16, f"{what}: bf16 err / rms {e:.3e} > {TOL_BF16} (rms err {r:.2e})"
+        assert r <= TOL_BF16_RMS, f"{what}: bf16 rms err {r:.3e} > {TOL_BF16_RMS} (max err / rms {e:.2e})"
     return e
 
 

@@ -83,6 +83,39 @@ def algorithmic_bytes(w) -> int:
     return io * elems + 4 * 4 * w.nheads
 
 
+def intra_chunk_flops(w) -> int:
+    """Algorithmic tensor work of one bidirectional call: per direction, head
+    and chunk of Q tokens, the causal (lower-triangle, Q(Q+1)/2 entries)
+    C.B^T over d_state and the masked matrix times X over headdim, 2 flops per
+    multiply-add. Counted per head (the decay mask differs per head even where
+    B/C are shared)."""
+    q = w.chunk
+    chunks = w.batch * -(-w.seqlen // q)
+    return 2 * w.nheads * chunks * (q * (q + 1) // 2) * 2 * (w.dstate + w.headdim)
+
+
+def roofline_bound(w, seconds: float, peaks: dict) -> dict:
+    """The metric's roofline: the slower of the algorithmic HBM bytes at the
+    measured copy bandwidth and the intra-chunk FLOPs at the measured bf16
+    tensor throughput; the fraction is that bound's time over the measured one."""
+    nbytes, flops = algorithmic_bytes(w), intra_chunk_flops(w)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        achieved = nbytes / seconds / 1e9
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peaks['source']} STREAM-copy HBM GB/s",
+                "algorithmic_bytes_per_launch": nbytes, "intra_chunk_flops_per_launch": flops,
+                "other_bound_us": round(1e6 * t_tc, 2)}
+    achieved = flops / seconds / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peaks['source']} cuBLAS bf16 TFLOP/s (burst)",
+            "algorithmic_bytes_per_launch": nbytes, "intra_chunk_flops_per_launch": flops,
+            "other_bound_us": round(1e6 * t_hbm, 2)}
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -327,7 +360,18 @@ def bench_blockstep(args, w, dev):
                   + 4 * w.batch * w.nheads * w.headdim * w.dstate)
     prefill_bytes = (io * (w.batch * w.seqlen * (w.nheads * w.headdim + w.nheads + w.ngroups * w.dstate))
                      + 4 * w.batch * w.nheads * w.headdim * w.dstate)
+    # the commit: the block's x, forward dt and B read, the state read and written
+    commit_bytes = (io * w.batch * w.block * (w.nheads * w.headdim + w.nheads + w.ngroups * w.dstate)
+                    + 2 * 4 * w.batch * w.nheads * w.headdim * w.dstate)
+    block_bytes = w.steps * step_bytes + commit_bytes
     peaks = measured_peaks()
+    achieved = block_bytes / (ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": f"{peaks['source']} STREAM-copy HBM GB/s",
+            "algorithmic_bytes_per_launch": block_bytes,
+            "kernel": "tc_fused_kernel (32 block steps + the commit, one CUDA graph; bytes of the whole block)",
+            "traffic": None}
     line = {"metric": "block-diffusion denoising tokens/s (block x steps), cached prefix state",
             "value": round(tok / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
@@ -335,6 +379,7 @@ def bench_blockstep(args, w, dev):
             "config": {"workload": w.name, "batch": w.batch, "prefix": w.seqlen, "block": w.block,
                        "denoising_steps": w.steps, "nheads": w.nheads, "headdim": w.headdim,
                        "dstate": w.dstate, "ngroups": w.ngroups, "graph": "one CUDA graph per block"},
+            "roofline": roof,
             "per_denoising_step_us": round(1e3 * ms / (w.steps + 1), 3),
             "algorithmic_bytes_per_denoising_step": step_bytes,
             "prefill": {"ms": round(prefill_ms, 4), "tokens_per_s": round(w.batch * w.seqlen / (prefill_ms / 1e3), 1),
@@ -471,17 +516,13 @@ def main():
         return
 
     peaks = measured_peaks()
-    abytes = algorithmic_bytes(w)
     launches = LAUNCHES_PER_CALL[path_name]
-    achieved = abytes / (ms_step / 1e3) / 1e9
-    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_record(path_name, w.name),
-            "peak_source": f"{peaks['source']} STREAM-copy HBM GB/s",
-            "algorithmic_bytes_per_launch": abytes,
+    roof = roofline_bound(w, ms_step / 1e3, peaks)
+    roof.update({"traffic": traffic_record(path_name, w.name),
             "kernel": {"simt": "scan_simt_kernel", "chunked": "tc_state/tc_pass/tc_out kernels (whole step)",
                        "fused": "tc_fused_kernel",
                        "segmented": "tc_fused_kernel (forward state, reverse state, bidirectional) + seg_scan_kernel "
-                                    "(whole step)"}[path_name]}
+                                    "(whole step)"}[path_name]})
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

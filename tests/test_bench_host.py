@@ -68,3 +68,25 @@ def test_record_traffic_sums_one_call_and_expires_with_the_source(tmp_path, monk
 def test_whole_job_throughput_and_time_at_one_rank():
     assert bench.job_time_ms(3.5, 1) == 3.5
     assert bench.job_throughput(1000, 4, 1, 2.0) == 1000 * 4 / 2e-3
+
+
+def test_intra_chunk_flops_of_the_130m_shape():
+    # per direction, head and 256-token chunk: 256 * 257 / 2 lower-triangle
+    # entries, each a d_state (128) and a headdim (64) multiply-add: 2 flops
+    w = si.WORKLOADS["mixer130m_b32_L1024"]
+    per_chunk = 256 * 257 // 2 * 2 * (128 + 64)
+    assert bench.intra_chunk_flops(w) == 2 * 24 * (32 * 4) * per_chunk == 77611401216
+
+
+def test_roofline_takes_the_slower_bound():
+    peaks = {"hbm_gbs": 6451.5, "bf16_tflops": 1713.8, "source": "measured"}
+    # per-head B/C: 1.01 GB at the copy bandwidth (156 us) outweighs 77.6
+    # GFLOP at the tensor peak (45 us)
+    r = bench.roofline_bound(si.WORKLOADS["mixer130m_b32_L1024"], 260e-6, peaks)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - 1009779072 / 260e-6 / 1e9 / 6451.5) < 1e-4
+    # B/C shared by all heads: 0.238 GB (37 us) is now below the same FLOPs (45 us)
+    r = bench.roofline_bound(si.WORKLOADS["mixer130m_b32_L1024_g1"], 292.5e-6, peaks)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["frac"] - 77611401216 / 292.5e-6 / 1e12 / 1713.8) < 1e-4
+    assert 0.15 < r["frac"] < 0.16

@@ -15,7 +15,7 @@ SSD_F32, SSD_BF16 = 0, 1
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED = 0, -1, -2
 SSD_ERR_CUDA, SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT = -3, -4, -5
 SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE, SSD_OP_BLOCK_STEP = 0, 1, 2
-SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED, SSD_PATH_SEGMENTED = 0, 1, 2, 3, 4
+SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED, SSD_PATH_SEGMENTED, SSD_PATH_PAIR = 0, 1, 2, 3, 4, 5
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int

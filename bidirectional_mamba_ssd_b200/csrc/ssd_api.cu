@@ -52,11 +52,27 @@ float *scratch_ptr(void *ws) { return reinterpret_cast<float *>(static_cast<char
 // tile-parallel chunked kernels.
 constexpr long long kFusedMinUnits = 64;
 
-// Kernel choice of SSD_PATH_AUTO: bf16 runs on the tensor cores, in one
-// kernel per (batch, head) when there are enough of those to fill the GPU,
-// else in the tile-parallel chunked kernels; fp32 runs the sequential scan.
+// Longest sequence, in 128-token tiles, that SSD_PATH_AUTO gives the two-CTA
+// kernel: each cluster keeps up to half a sequence of 32 KB partial tiles live.
+constexpr long long kPairMaxTiles = 16;
+
+// Kernel choice of SSD_PATH_AUTO: bf16 runs on the tensor cores: two CTAs
+// per (batch, head), one per direction, for sequences of 2..16 tiles with a
+// unit for every two SMs; one CTA per (batch, head) when there are enough of
+// those to fill the GPU; else the segmented or tile-parallel chunked kernels;
+// fp32 runs the sequential scan.
 int auto_path(int batch, int seqlen, int nheads, int ngroups, int dstate, int dtype) {
     if (dtype != SSD_BF16) return SSD_PATH_SIMT;
+    // two to 16 tiles and a (batch, head) unit for every two SMs: one cluster of
+    // two CTAs per unit, each running one scan direction (the partial tiles the
+    // directions exchange stay in L2 up to this length)
+    {
+        const long long units = (long long)batch * nheads, nt = (seqlen + 127) / 128;
+        const int sms = ssd::device_sms();
+        if (nt >= 2 && nt <= kPairMaxTiles && sms > 0 && units >= sms / 2 &&
+            ssd::tc_pair_supported(batch, seqlen, nheads, ngroups, dstate))
+            return SSD_PATH_PAIR;
+    }
     if (ssd::tc_fused_supported(batch, seqlen, nheads, ngroups, dstate)) return SSD_PATH_FUSED;
     // a few long sequences: split them into segments when that leaves at
     // least 4 tiles per SM to work on
@@ -72,7 +88,7 @@ int bidir_impl(const void *x, const void *dt, const float *A, const void *B, con
                size_t ws_bytes, void *stream) {
     int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
     if (rc != SSD_OK) return rc;
-    if (path < SSD_PATH_AUTO || path > SSD_PATH_SEGMENTED) return SSD_ERR_INVALID_ARG;
+    if (path < SSD_PATH_AUTO || path > SSD_PATH_PAIR) return SSD_ERR_INVALID_ARG;
     if (!workspace) return SSD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
     if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, seqlen, nheads, headdim, dstate,
@@ -104,6 +120,7 @@ int bidir_impl(const void *x, const void *dt, const float *A, const void *B, con
     t.workspace = workspace; t.ws_bytes = ws_bytes;
     t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
     if (path == SSD_PATH_FUSED) return to_status(ssd::launch_tc_fused(t, s));
+    if (path == SSD_PATH_PAIR) return to_status(ssd::launch_tc_pair(t, s));
     if (path == SSD_PATH_SEGMENTED) {
         // at least two segments, even where one would be chosen
         const int sms = ssd::device_sms();
@@ -131,9 +148,11 @@ size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdi
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 2);
             size_t f = ssd::tc_fused_scratch_bytes(batch, seqlen, nheads, dstate);
             size_t g = ssd::tc_segmented_scratch_bytes(batch, seqlen, nheads, dstate);
+            size_t q = ssd::tc_pair_scratch_bytes(batch, seqlen, nheads, dstate);
             scratch = scratch > c ? scratch : c;
             scratch = scratch > f ? scratch : f;
             scratch = scratch > g ? scratch : g;
+            scratch = scratch > q ? scratch : q;
         } else if (op == SSD_OP_PREFIX_STATE) {
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 1);
             scratch = scratch > c ? scratch : c;

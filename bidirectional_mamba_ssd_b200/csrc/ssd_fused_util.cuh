@@ -66,6 +66,76 @@ __device__ __forceinline__ void grid_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// mbar_wait with its polling loop out of line: the call site holds one
+// try_wait and a call, which keeps kernels with many wait sites small enough
+// for the instruction cache. Same bound and abort rules as mbar_wait.
+static __device__ __noinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                            DeviceStatus *st, uint32_t where) {
+    WaitClock clock;
+    while (true) {
+        if (*abort_flag) return false;
+        if (mbar_try_wait(bar, parity)) return true;
+        if (clock.expired(1000000000ull)) {
+            *abort_flag = 1;
+            report_timeout(st, where);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool mbar_wait_ool(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                              DeviceStatus *st, uint32_t where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_loop(bar, parity, abort_flag, st, where);
+}
+
+// ------------------------------------------------------------ global flags
+// A flag store that publishes the writes before it (of this thread, and of
+// the threads that passed a barrier with it) at GPU scope.
+__device__ __forceinline__ void flag_release(unsigned int *f, unsigned int v) {
+    asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int flag_acquire(const unsigned int *f) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+// Poll a flag until it holds `v`, for at most `limit_ns` of waiting (the same
+// clock rules as mbar_wait). On expiry: timeout in the status header, the
+// CTA's abort flag up, false.
+__device__ __forceinline__ bool flag_wait(const unsigned int *f, unsigned int v, volatile int *abort_flag,
+                                          DeviceStatus *st, uint32_t where, uint64_t limit_ns = 1000000000ull) {
+    if (flag_acquire(f) == v) return true;
+    WaitClock clock;
+    while (true) {
+        if (*abort_flag) return false;
+        if (flag_acquire(f) == v) return true;
+        if (clock.expired(limit_ns)) {
+            *abort_flag = 1;
+            report_timeout(st, where);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+// 16-byte global load that bypasses L1 (data another SM wrote), and store.
+__device__ __forceinline__ float4 ld_cg_f4(const float *p) {
+    float4 v;
+    asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void st_f4(float *p, float a, float b, float c, float d) {
+    asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+// Drop a 128-byte line from L2 without writing it back (its data is dead).
+__device__ __forceinline__ void discard_l2_line(const void *p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+// All threads of both CTAs of a cluster meet; global writes before it are
+// visible to the other CTA after it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // named barriers of the three epilogue groups (128 threads each)
 __device__ __forceinline__ void sync_c() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ void sync_a() { asm volatile("bar.sync 2, 128;" ::: "memory"); }

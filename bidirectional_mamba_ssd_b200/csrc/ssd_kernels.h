@@ -70,6 +70,14 @@ cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream);
 // inputs): the state at the sequence start into a.state_out, from zero.
 cudaError_t launch_tc_fused_state_rev(const TcArgs &a, cudaStream_t stream);
 
+// Two-CTA kernel (ssd_pair.cu): each (batch, head) unit taken by a cluster of
+// two CTAs, one per scan direction, meeting per tile through an fp32 partial
+// in the workspace; both scans summed, a.init / a.rinit as launch_tc_fused.
+// Sequences of at least two 128-token tiles.
+size_t tc_pair_scratch_bytes(int batch, int L, int H, int N);
+bool tc_pair_supported(int batch, int L, int H, int G, int N);
+cudaError_t launch_tc_pair(const TcArgs &a, cudaStream_t stream);
+
 // Long sequences with fewer (batch, head) units than SMs: each sequence split
 // into S segments (seg_count: the fewest, S dividing L, that fill 4/5 of `sms`
 // SMs in one round; 1 = none), states handed across segments,

@@ -113,6 +113,50 @@ __device__ __forceinline__ void mask_diag(int J, int c0, int row, float my_af, f
     for (int q = 0; q < W / 2; ++q) packed[q] = sm100::pack_bf16x2(m[2 * q], m[2 * q + 1]);
 }
 
+// The diagonal block for one direction only (a kernel that runs each scan in
+// its own CTA): forward (FWD) keeps columns s <= t, reverse s >= t, the row's
+// own token with decay 1; `a`, `dt`, `col` are that direction's a_s, dt_s and
+// column factors. Factorised through the block's edge as mask_diag while the
+// block's decay span stays below kMaxSpan, else one exponential per entry;
+// dropped entries are selected as 0, never multiplied.
+template <bool FWD, int W>
+__device__ __forceinline__ void mask_diag1(int J, int c0, int row, float my_a, const uint32_t (&g)[W],
+                                           const float *a, const float *dt, const float *col,
+                                           uint32_t (&packed)[W / 2]) {
+    const int s0 = J * 32;
+    const int s1 = s0 + c0;
+    const int rr = row - s1;
+    float m[W];
+    const float span = FWD ? a[s0] - a[s0 + 31] : a[s0 + 31] - a[s0];
+    if (span < kMaxSpan) {
+        const float r = __expf(my_a - (FWD ? a[s0 + 31] : a[s0]));
+#pragma unroll
+        for (int q = 0; q < W; q += 4) {
+            const float4 c4 = *reinterpret_cast<const float4 *>(col + s1 + q);
+            const float4 d4 = *reinterpret_cast<const float4 *>(dt + s1 + q);
+            const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, ds[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int c = q + e;
+                const float gv = __uint_as_float(g[c]);
+                const bool keep = FWD ? c < rr : c > rr;
+                m[c] = keep ? gv * (r * cs[e]) : c == rr ? gv * ds[e] : 0.f;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < W; ++c) {
+            const int s = s1 + c;
+            const float gv = __uint_as_float(g[c]);
+            const bool keep = FWD ? c < rr : c > rr;
+            // the exponent of a kept entry is <= 0
+            m[c] = keep ? gv * dt[s] * __expf(my_a - a[s]) : c == rr ? gv * dt[s] : 0.f;
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < W / 2; ++q) packed[q] = sm100::pack_bf16x2(m[2 * q], m[2 * q + 1]);
+}
+
 // Columns [32 J, 32 J + 32) of row `row` given both G blocks, packed as 16 bf16 pairs.
 __device__ __forceinline__ void mask_block(int J, int row, float my_af, float my_ab,
                                            const uint32_t (&gf)[32], const uint32_t (&gb)[32],
@@ -151,6 +195,24 @@ __device__ __forceinline__ void scale_row(const uint8_t *src_tile, uint8_t *dst_
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) d[(k + row) & 7] = v[k];
+}
+
+// scale_row for distinct source and destination tiles, one 16-byte chunk at a
+// time in a rolled loop (less code where instruction fetch is the limit).
+__device__ __forceinline__ void scale_row_rolled(const uint8_t *src_tile, uint8_t *dst_tile, int row, float w) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(src_tile + row * 128);
+    uint4 *d = reinterpret_cast<uint4 *>(dst_tile + row * 128);
+#pragma unroll 1
+    for (int k = 0; k < 8; ++k) {
+        uint4 v = src[(k + row) & 7];
+        uint32_t *q = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float lo = __uint_as_float(q[j] << 16) * w, hi = __uint_as_float(q[j] & 0xffff0000u) * w;
+            q[j] = sm100::pack_bf16x2(lo, hi);
+        }
+        d[(k + row) & 7] = v;
+    }
 }
 
 // Row `row` of diag(w) X kept as two bf16 terms: the rounded product into

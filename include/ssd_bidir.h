@@ -85,10 +85,15 @@ enum {
     SSD_PATH_SIMT = 1,     /* sequential fp32 scan on CUDA cores, any dtype */
     SSD_PATH_CHUNKED = 2,  /* tensor-core chunked path in three kernels (states through the workspace) */
     SSD_PATH_FUSED = 3,    /* tensor-core path, one kernel per (batch, head) */
-    SSD_PATH_SEGMENTED = 4 /* long sequences, few (batch, head): each sequence split into S
+    SSD_PATH_SEGMENTED = 4, /* long sequences, few (batch, head): each sequence split into S
                               segments (S divides seqlen); forward and reverse segment states
                               (fused kernel, state modes), a segment scan, then the fused
                               kernel on the segments seeded with the handed-over states */
+    SSD_PATH_PAIR = 5      /* tensor-core path, one cluster of two CTAs per (batch, head):
+                              each CTA runs one scan direction over the tiles in that
+                              direction's order, carrying its state on chip; a tile's two
+                              directions meet through an fp32 partial in the workspace.
+                              seqlen > 128 (at least two 128-token tiles) */
 };
 
 /* The SSD_PATH_* that ssd_bidir_fwd (SSD_PATH_AUTO) runs for these sizes, or

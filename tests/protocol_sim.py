@@ -1,5 +1,5 @@
 """Discrete-event engine for the barrier-protocol models of the persistent
-tensor-core kernels (test_fused_protocol.py, test_bidir2_protocol.py).
+tensor-core kernels (test_fused_protocol.py, test_pair_protocol.py).
 
 Roles are generators that yield the commands below; asynchronous completions
 (TMA loads and stores, MMAs in issue order) land after random, heavy-tailed
@@ -12,13 +12,16 @@ Commands:
   ('wait', bar, k)      wait for completion of phase k (parity k & 1)
   ('arrive', bar)
   ('tma', bar, [(res, val)])          async load: writes then arrives
-  ('mma', [(res,val)] reads, [(res,val)] writes)   in-order async
-  ('commit', bar)                     arrives when all prior MMAs are done
+  ('mma', [(res,val)] reads, [(res,val)] writes[, pipe])   in-order async
+  ('commit', bar[, pipe])             arrives when all prior MMAs (of the pipe) are done
   ('read', res, val) / ('write', res, val)
   ('sync', name, n)                   named barrier over n roles
   ('store', [(res,val)]) then ('store_wait',)      store's shared-memory read
   ('store_g', [(res,val)] smem reads, [(res,val)] global writes)
   ('store_wait_all',)                 all of the role's stores complete
+  ('gset', flag, value)               a release store of a flag in global memory
+  ('gwait', flag, value)              an acquire poll until the flag holds value;
+                                      seeing a later value is an overrun
 """
 import heapq
 import itertools
@@ -49,7 +52,8 @@ class Sched:
         self.t = 0.0
         self.ev = []          # (time, seq, fn)
         self.seq = itertools.count()
-        self.mma_done_t = 0.0
+        self.mma_done = {}    # per tensor pipe: completion time of its last MMA
+        self.flags = {}       # global-memory flags (gset / gwait), start at 0
     def bar(self, name, count=1):
         if name not in self.bars:
             self.bars[name] = Bar(name, count)
@@ -116,8 +120,9 @@ def run_roles(S, roles, counts):
             S.at(S.t + S.delay(), land)
         elif op == 'mma':
             reads, writes = c[1], c[2]
-            tdone = max(S.mma_done_t, S.t) + S.delay()
-            S.mma_done_t = tdone
+            pipe = c[3] if len(c) > 3 else None     # one in-order tensor pipe per CTA
+            tdone = max(S.mma_done.get(pipe, 0.0), S.t) + S.delay()
+            S.mma_done[pipe] = tdone
             def ex(reads=reads, writes=writes):
                 for k, v in reads:
                     S.read(k, v, 'mma exec')
@@ -126,7 +131,8 @@ def run_roles(S, roles, counts):
             S.at(tdone, ex)
         elif op == 'commit':
             bn = c[1]
-            S.at(max(S.mma_done_t, S.t) + 1e-6, lambda bn=bn: bar(bn).arrive())
+            pipe = c[2] if len(c) > 2 else None
+            S.at(max(S.mma_done.get(pipe, 0.0), S.t) + 1e-6, lambda bn=bn: bar(bn).arrive())
         elif op == 'read':
             S.read(c[1], c[2], name)
         elif op == 'write':
@@ -176,6 +182,14 @@ def run_roles(S, roles, counts):
                 return False
         elif op == 'store_wait_all':
             if S.t < store_done.get(name, 0.0):
+                return False
+        elif op == 'gset':
+            S.flags[c[1]] = c[2]
+        elif op == 'gwait':
+            got = S.flags.get(c[1], 0)
+            if got != c[2]:
+                if got > c[2]:
+                    raise Bug(f"{name}: flag {c[1]} overrun: waiting for {c[2]}, holds {got}")
                 return False
         cur[name] = None
         return True

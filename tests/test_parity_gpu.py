@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 PATHS = {"simt": 1, "chunked": 2, "fused": 3}
 PATHS_ALL = {"auto": 0, **PATHS}
-BIDIR_PATHS = {**PATHS, "segmented": 4}
+BIDIR_PATHS = {**PATHS, "segmented": 4, "pair": 5}
 
 
 @pytest.fixture(scope="module")
@@ -111,6 +111,38 @@ def test_full_size_sampled(ssd, name, k):
     ref = oracle_units(inp, units)
     for (b, h), o in ref.items():
         check(to_f64(out[b, :, h]), o, torch.bfloat16, f"{name} unit {(b, h)}")
+
+
+@pytest.mark.parametrize("name,k", [("mixer130m_b32_L1024", 12), ("mixer130m_b32_L1024_g1", 6)])
+def test_full_size_sampled_fused(ssd, name, k):
+    """The one-CTA fused kernel at the 130M shape (the automatic choice there
+    is the two-CTA kernel, tested above), sampled units against the oracle."""
+    w = si.WORKLOADS[name]
+    inp = si.workload_inputs(w, device="cuda")
+    out = ssd.ssd_bidir_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], chunk=w.chunk,
+                            path=BIDIR_PATHS["fused"])
+    torch.cuda.synchronize()
+    assert ssd.ssd_get_device_status() == 0
+    units = sample_units(w.batch, w.nheads, k, seed=5)
+    ref = oracle_units(inp, units)
+    for (b, h), o in ref.items():
+        check(to_f64(out[b, :, h]), o, torch.bfloat16, f"fused {name} unit {(b, h)}")
+
+
+@pytest.mark.parametrize("shape", [(3, 256, 2, 128, 2), (1, 1000, 200, 64, 4), (5, 640, 37, 128, 37)],
+                         ids=["two_tiles", "many_units_ragged", "odd_tiles"])
+def test_pair_every_output(ssd, shape):
+    """The two-CTA kernel over whole problems: two tiles (each direction first
+    on one), more units than clusters with a ragged last tile, and an odd tile
+    count (the middle tile's partial comes from the forward direction); every
+    output against the oracle, twice in a row on the same workspace (the
+    flags of the first call must not satisfy the second)."""
+    batch, L, H, N, G = shape
+    inp = si.bidir_inputs(batch, L, H, 64, N, G, "bf16", seed=L + H, device="cuda")
+    o = full_oracle(inp)
+    for rep in range(2):
+        y = run_bidir(ssd, inp, 128, BIDIR_PATHS["pair"])
+        check(y, o, torch.bfloat16, f"pair {shape} call {rep}")
 
 
 @pytest.mark.parametrize("shape", [(64, 128, 8, 128, 2), (50, 100, 6, 64, 1), (37, 128, 4, 128, 4)],

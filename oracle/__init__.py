@@ -25,6 +25,10 @@ pinned to the other functions: with zero states it is ``block_step`` with no
 prefix; its segments, seeded with the states the rest of the sequence leaves
 (from ``prefix_state`` on either side, the reverse one through the flip
 identity), put together give ``bidir`` over the whole sequence.
+``bidir_bwd`` (gradients) is pinned by central finite differences of
+``bidir``, by the exact adjoint identities of the maps that are linear (y in
+x, in B and in C) and by the closed form of a memoryless scan (A -> -inf);
+``tests/test_oracle_bwd_pins.py``.
 """
 from __future__ import annotations
 
@@ -64,9 +68,10 @@ def configure(lib):
     lib.ssd_oracle_prefix_state.argtypes = [dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
     lib.ssd_oracle_block_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
     lib.ssd_oracle_bidir_seeded.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
+    lib.ssd_oracle_bidir_bwd.argtypes = [dp] * 13 + [i] * 7
     lib.ssd_oracle_threads.argtypes = [i]
-    for f in (lib.ssd_oracle_bidir, lib.ssd_oracle_prefix_state,
-              lib.ssd_oracle_block_step, lib.ssd_oracle_bidir_seeded, lib.ssd_oracle_threads):
+    for f in (lib.ssd_oracle_bidir, lib.ssd_oracle_prefix_state, lib.ssd_oracle_block_step,
+              lib.ssd_oracle_bidir_seeded, lib.ssd_oracle_bidir_bwd, lib.ssd_oracle_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -187,3 +192,21 @@ def dt_prep(dt_raw, dt_bias, dt_min=0.0, dt_max=np.inf) -> np.ndarray:
     u = np.asarray(dt_raw, dtype=np.float64) + np.asarray(dt_bias, dtype=np.float64)[:, None, None, :]
     sp = np.logaddexp(0.0, u)          # log(1 + exp(u)) without overflow
     return np.clip(sp, dt_min, dt_max)
+
+
+def bidir_bwd(x, dt, A, B, C, D, dy, nthreads: int = 0) -> dict:
+    """Gradients of sum(dy * bidir(x, dt, A, B, C, D)) with respect to every
+    input, in fp64, from the adjoint of the recurrence token by token (see
+    ssd_oracle.c). Returns a dict of arrays shaped like the inputs: dx, ddt,
+    dA, dB, dC, dD."""
+    x = np.asarray(x)
+    batch, L, H, P = x.shape
+    G, N = np.asarray(B).shape[-2:]
+    keep = [_f64(a) for a in (x, dt, A, B, C, D, dy)]
+    outs = {"dx": np.zeros((batch, L, H, P)), "ddt": np.zeros((2, batch, L, H)), "dA": np.zeros((2, H)),
+            "dB": np.zeros((2, batch, L, G, N)), "dC": np.zeros((2, batch, L, G, N)), "dD": np.zeros((2, H))}
+    po = [outs[k].ctypes.data_as(ctypes.POINTER(ctypes.c_double)) for k in ("dx", "ddt", "dA", "dB", "dC", "dD")]
+    rc = _load().ssd_oracle_bidir_bwd(*(p for _, p in keep), *po, batch, L, H, P, N, G, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle bidir_bwd: bad arguments")
+    return outs

@@ -271,3 +271,156 @@ int ssd_oracle_bidir_seeded(const double *x, const double *dt, const double *A,
     }
     return bad ? -1 : 0;
 }
+
+/* ------------------------------------------------------------------ gradients
+ * Gradients of the scalar sum_t <dy_t, y_t> over the bidirectional mixer's
+ * inputs (the backward pass a training step of the mixer runs; "Training
+ * Hybrid Block Diffusion Language Models with Partial Bidirectionality", Key
+ * Results and Technical Contribution: the models are trained through the
+ * mixer with a full-block objective).
+ *
+ * Written from the recurrence above by reverse-mode differentiation, one
+ * token after the other in the opposite order of each direction's scan. With
+ * a_t = exp(dt_t A), h_t = a_t h_{t-1} + dt_t B_t x_t^T, y_t = C_t^T h_t, and
+ * g_t the adjoint of h_t (the derivative of the scalar with respect to h_t,
+ * all later tokens included):
+ *   g_t        = C_t dy_t^T + a_{t+1} g_{t+1}            (N x P)
+ *   dC_t[n]   += sum_p h_t[n][p] dy_t[p]
+ *   dx_t[p]   += dt_t sum_n B_t[n] g_t[n][p]
+ *   dB_t[n]   += dt_t sum_p g_t[n][p] x_t[p]
+ *   ddt_t     += sum_{n,p} g_t[n][p] B_t[n] x_t[p] + A a_t <g_t, h_{t-1}>
+ *   dA        += dt_t a_t <g_t, h_{t-1}>
+ * and from the skip term y_t += (D_f + D_b) x_t: dx_t += (D_f + D_b) dy_t,
+ * dD_f = dD_b = sum_t <dy_t, x_t>. "Later" means later in the direction's
+ * own order (t + 1 forward, t - 1 reverse). Every forward state is kept (L + 1
+ * states of N x P doubles per unit), so this is for small problems and
+ * sampled units.
+ *
+ * Layouts as for ssd_oracle_bidir; dy and dx (batch, L, H, P); ddt (2, batch,
+ * L, H); dA, dD (2, H); dB, dC (2, batch, L, G, N). Every output is
+ * overwritten. Heads of a B/C group add into the same dB, dC entries, so the
+ * work is split by (batch, group) with the group's heads in order. */
+int ssd_oracle_bidir_bwd(const double *x, const double *dt, const double *A,
+                         const double *Bm, const double *Cm, const double *D,
+                         const double *dy, double *dx, double *ddt, double *dA,
+                         double *dB, double *dC, double *dD,
+                         int batch, int L, int H, int P, int N, int G, int nthreads)
+{
+    if (batch < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G) return -1;
+    set_threads(nthreads);
+    const int hpg = H / G;
+    const ptrdiff_t x_ts = (ptrdiff_t)H * P, dt_ts = H, bc_ts = (ptrdiff_t)G * N;
+    const size_t dt_dir = (size_t)batch * L * H;
+    const size_t bc_dir = (size_t)batch * L * G * N;
+    memset(dx, 0, sizeof(double) * (size_t)batch * L * H * P);
+    memset(ddt, 0, sizeof(double) * 2 * dt_dir);
+    memset(dB, 0, sizeof(double) * 2 * bc_dir);
+    memset(dC, 0, sizeof(double) * 2 * bc_dir);
+    /* per batch element, summed in order afterwards */
+    double *dA_b = (double *)calloc((size_t)batch * 2 * H + 1, sizeof(double));
+    double *dD_b = (double *)calloc((size_t)batch * H + 1, sizeof(double));
+    if (!dA_b || !dD_b) { free(dA_b); free(dD_b); return -1; }
+    const size_t SN = (size_t)N * P;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int bg = 0; bg < batch * G; ++bg) {
+        const int b = bg / G, g = bg % G;
+        double *hs = (double *)malloc(sizeof(double) * SN * ((size_t)L + 1));
+        double *gadj = (double *)malloc(sizeof(double) * SN);
+        if (!hs || !gadj) { free(hs); free(gadj); bad |= 1; continue; }
+        for (int hh = g * hpg; hh < (g + 1) * hpg; ++hh) {
+            const double *xu = x + ((size_t)b * L * H + hh) * P;
+            const double *dyu = dy + ((size_t)b * L * H + hh) * P;
+            double *dxu = dx + ((size_t)b * L * H + hh) * P;
+            for (int d = 0; d < 2; ++d) {
+                const double Ad = A[d * H + hh];
+                const double *dtu = dt + d * dt_dir + (size_t)b * L * H + hh;
+                double *ddtu = ddt + d * dt_dir + (size_t)b * L * H + hh;
+                const double *Bu = Bm + d * bc_dir + ((size_t)b * L * G + g) * N;
+                const double *Cu = Cm + d * bc_dir + ((size_t)b * L * G + g) * N;
+                double *dBu = dB + d * bc_dir + ((size_t)b * L * G + g) * N;
+                double *dCu = dC + d * bc_dir + ((size_t)b * L * G + g) * N;
+                /* forward through the direction's order: hs[k] is the state after k tokens */
+                memset(hs, 0, sizeof(double) * SN);
+                for (int k = 0; k < L; ++k) {
+                    const int t = d ? (L - 1 - k) : k;
+                    const double dtt = dtu[(ptrdiff_t)t * dt_ts];
+                    const double a = exp(dtt * Ad);
+                    const double *Bt = Bu + (ptrdiff_t)t * bc_ts;
+                    const double *xt = xu + (ptrdiff_t)t * x_ts;
+                    const double *hp = hs + (size_t)k * SN;
+                    double *hn = hs + (size_t)(k + 1) * SN;
+                    for (int n = 0; n < N; ++n)
+                        for (int p = 0; p < P; ++p)
+                            hn[(size_t)n * P + p] = a * hp[(size_t)n * P + p] + dtt * Bt[n] * xt[p];
+                }
+                /* adjoint, in the opposite order */
+                memset(gadj, 0, sizeof(double) * SN);
+                double dA_acc = 0.0;
+                for (int k = L - 1; k >= 0; --k) {
+                    const int t = d ? (L - 1 - k) : k;
+                    const double dtt = dtu[(ptrdiff_t)t * dt_ts];
+                    const double a = exp(dtt * Ad);
+                    const double *Bt = Bu + (ptrdiff_t)t * bc_ts;
+                    const double *Ct = Cu + (ptrdiff_t)t * bc_ts;
+                    const double *xt = xu + (ptrdiff_t)t * x_ts;
+                    const double *dyt = dyu + (ptrdiff_t)t * x_ts;
+                    const double *ht = hs + (size_t)(k + 1) * SN;
+                    const double *hp = hs + (size_t)k * SN;
+                    double *dxt = dxu + (ptrdiff_t)t * x_ts;
+                    /* g_t = C_t dy_t^T + (the decayed adjoint of the later token) */
+                    for (int n = 0; n < N; ++n)
+                        for (int p = 0; p < P; ++p) gadj[(size_t)n * P + p] += Ct[n] * dyt[p];
+                    for (int n = 0; n < N; ++n) {
+                        double s = 0.0;
+                        for (int p = 0; p < P; ++p) s += ht[(size_t)n * P + p] * dyt[p];
+                        dCu[(ptrdiff_t)t * bc_ts + n] += s;
+                    }
+                    for (int p = 0; p < P; ++p) {
+                        double s = 0.0;
+                        for (int n = 0; n < N; ++n) s += Bt[n] * gadj[(size_t)n * P + p];
+                        dxt[p] += dtt * s;
+                    }
+                    double gbx = 0.0, ghp = 0.0;
+                    for (int n = 0; n < N; ++n) {
+                        double s = 0.0;
+                        for (int p = 0; p < P; ++p) {
+                            s += gadj[(size_t)n * P + p] * xt[p];
+                            ghp += gadj[(size_t)n * P + p] * hp[(size_t)n * P + p];
+                        }
+                        dBu[(ptrdiff_t)t * bc_ts + n] += dtt * s;
+                        gbx += Bt[n] * s;
+                    }
+                    ddtu[(ptrdiff_t)t * dt_ts] = gbx + Ad * a * ghp;
+                    dA_acc += dtt * a * ghp;
+                    for (size_t q = 0; q < SN; ++q) gadj[q] *= a;   /* adjoint of h_{t-1}'s share */
+                }
+                dA_b[(size_t)b * 2 * H + d * H + hh] = dA_acc;
+            }
+            /* skip term */
+            const double dsum = D[hh] + D[H + hh];
+            double xdy = 0.0;
+            for (int t = 0; t < L; ++t)
+                for (int p = 0; p < P; ++p) {
+                    dxu[(ptrdiff_t)t * x_ts + p] += dsum * dyu[(ptrdiff_t)t * x_ts + p];
+                    xdy += xu[(ptrdiff_t)t * x_ts + p] * dyu[(ptrdiff_t)t * x_ts + p];
+                }
+            dD_b[(size_t)b * H + hh] = xdy;
+        }
+        free(hs);
+        free(gadj);
+    }
+    for (int d = 0; d < 2; ++d)
+        for (int hh = 0; hh < H; ++hh) {
+            double sa = 0.0, sd = 0.0;
+            for (int b = 0; b < batch; ++b) {
+                sa += dA_b[(size_t)b * 2 * H + d * H + hh];
+                sd += dD_b[(size_t)b * H + hh];
+            }
+            dA[d * H + hh] = sa;
+            dD[d * H + hh] = sd;
+        }
+    free(dA_b);
+    free(dD_b);
+    return bad ? -1 : 0;
+}

@@ -8,6 +8,7 @@ Every step of the computation runs in the library's kernels.
 
 Functions carry the C names:
   ssd_bidir_fwd(x, dt, A, B, C, D, chunk=256)          -> out
+  ssd_bidir_bwd(x, dt, A, B, C, D, dy)                 -> dict of fp32 gradients dx, ddt, dA, dB, dC, dD
   ssd_prefix_state(x, dt, A, B, init=None, chunk=256)  -> state (batch, H, P, N) fp32
   ssd_block_step(x, dt, A, B, C, D, prefix_state)      -> out
   ssd_segment_states(x, dt, A, B)                      -> (fwd_state, fwd_decay, rev_state, rev_decay)
@@ -30,9 +31,9 @@ from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSE
                    SSD_PATH_PAIR,
                    SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA,
                    SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT, SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE,
-                   SSD_OP_BLOCK_STEP)
+                   SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD)
 
-__all__ = ["ssd_bidir_fwd", "ssd_prefix_state", "ssd_block_step", "ssd_segment_states",
+__all__ = ["ssd_bidir_fwd", "ssd_bidir_bwd", "ssd_prefix_state", "ssd_block_step", "ssd_segment_states",
            "ssd_segment_carry", "ssd_bidir_fwd_seeded", "ssd_bidir_fwd_dtraw", "ssd_workspace_bytes",
            "ssd_get_device_status", "SSDError", "Workspace", "lib"]
 
@@ -349,3 +350,38 @@ def ssd_bidir_fwd_dtraw(x, dt_raw, dt_bias, A, B, C, D, dt_min: float = 0.0, dt_
                                  _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_bidir_fwd_dtraw")
     return out
+
+
+def ssd_bidir_bwd(x, dt, A, B, C, D, dy, *, workspace: Workspace | None = None) -> dict:
+    """Gradients of sum(dy * ssd_bidir_fwd(x, dt, A, B, C, D)) with respect to
+    every input (include/ssd_bidir.h: ssd_bidir_bwd), as fp32 tensors shaped
+    like the inputs: dx, ddt, dA, dB, dC, dD."""
+    _need(x, "x", ndim=4)
+    dev, io = x.device, x.dtype
+    if io not in _DT:
+        raise ValueError(f"x dtype {io} not supported (float32 or bfloat16)")
+    _need(dt, "dt", io, dev, 4)
+    _need(B, "B", io, dev, 5)
+    _need(C, "C", io, dev, 5)
+    _need(dy, "dy", io, dev, 4)
+    _need(A, "A", torch.float32, dev, 2)
+    _need(D, "D", torch.float32, dev, 2)
+    batch, L, H, P, G, N = _dims(x, B)
+    if tuple(dt.shape) != (2, batch, L, H) or tuple(B.shape) != (2, batch, L, G, N) \
+            or tuple(C.shape) != tuple(B.shape) or tuple(A.shape) != (2, H) or tuple(D.shape) != (2, H) \
+            or dy.shape != x.shape:
+        raise ValueError("shape mismatch: want x, dy (b,L,H,P), dt (2,b,L,H), B/C (2,b,L,G,N), A/D (2,H)")
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"dx": torch.empty(x.shape, **f32), "ddt": torch.empty(dt.shape, **f32), "dA": torch.empty(A.shape, **f32),
+         "dB": torch.empty(B.shape, **f32), "dC": torch.empty(C.shape, **f32), "dD": torch.empty(D.shape, **f32)}
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    nbytes = ssd_workspace_bytes(SSD_OP_BIDIR_BWD, batch, L, H, P, N, G, 64, io)
+    if nbytes == 0:
+        _check(_c.SSD_ERR_UNSUPPORTED, "ssd_bidir_bwd")
+    buf = ws.get(nbytes)
+    rc = lib.ssd_bidir_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dy),
+                           *(_ptr(g[k]) for k in ("dx", "ddt", "dA", "dB", "dC", "dD")),
+                           batch, L, H, P, N, G, _DT[io], _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_bidir_bwd")
+    return g

@@ -156,6 +156,8 @@ size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdi
         } else if (op == SSD_OP_PREFIX_STATE) {
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 1);
             scratch = scratch > c ? scratch : c;
+        } else if (op == SSD_OP_BIDIR_BWD) {
+            scratch = 0;
         } else if (op == SSD_OP_BLOCK_STEP) {
             size_t c = ssd::tc_chunked_scratch_bytes(batch, seqlen, nheads, dstate, 2);
             size_t f = ssd::tc_fused_scratch_bytes(batch, seqlen, nheads, dstate);
@@ -163,6 +165,7 @@ size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdi
             scratch = scratch > f ? scratch : f;
         }
     }
+    if (op == SSD_OP_BIDIR_BWD) scratch = ssd::bwd_scratch_bytes(batch, seqlen, nheads, dstate);
     return ssd::kStatusBytes + round256(scratch);
 }
 
@@ -410,6 +413,38 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
     const int S = few_unit_segments(batch, seqlen, nheads);
     if (S > 1) return to_status(ssd::launch_tc_segmented(t, S, static_cast<cudaStream_t>(stream)));
     return to_status(ssd::launch_tc_fused(t, static_cast<cudaStream_t>(stream)));
+}
+
+int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, const void *C, const float *D,
+                  const void *dy, float *dx, float *ddt, float *dA, float *dB, float *dC, float *dD, int batch,
+                  int seqlen, int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
+                  size_t ws_bytes, void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype, false);
+    if (rc != SSD_OK) return rc;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_BWD, batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (!dA || !dD || !aligned4(dA) || !aligned4(dD)) return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (batch == 0 || seqlen == 0) {
+        // no tokens: every gradient is zero (dA and dD are the only non-empty ones)
+        if (cudaMemsetAsync(dA, 0, 2 * sizeof(float) * nheads, s) != cudaSuccess ||
+            cudaMemsetAsync(dD, 0, 2 * sizeof(float) * nheads, s) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        return SSD_OK;
+    }
+    if (!x || !dt || !A || !B || !C || !D || !dy || !dx || !ddt || !dB || !dC) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned16(C) || !aligned16(dy) || !aligned16(dx) ||
+        !aligned16(ddt) || !aligned16(dB) || !aligned16(dC) || !aligned4(A) || !aligned4(D))
+        return SSD_ERR_INVALID_ARG;
+    ssd::BwdLaunch l{};
+    l.x = x; l.dt = dt; l.B = B; l.C = C; l.dy = dy; l.A = A; l.D = D;
+    l.dx = dx; l.ddt = ddt; l.dA = dA; l.dB = dB; l.dC = dC; l.dD = dD;
+    l.scratch = scratch_ptr(workspace);
+    l.batch = batch; l.L = seqlen; l.H = nheads; l.G = ngroups; l.N = dstate;
+    l.bf16 = dtype == SSD_BF16;
+    return to_status(ssd::launch_bwd(l, s));
 }
 
 int ssd_get_device_status(const void *workspace, void *stream) {

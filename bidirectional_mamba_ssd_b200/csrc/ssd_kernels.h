@@ -70,6 +70,21 @@ cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream);
 // inputs): the state at the sequence start into a.state_out, from zero.
 cudaError_t launch_tc_fused_state_rev(const TcArgs &a, cudaStream_t stream);
 
+// Backward pass (ssd_bwd.cu): gradients of sum(dy * y) of the bidirectional
+// mixer, fp32 outputs, any I/O dtype; persistent CTAs, each with L states of
+// scratch.
+struct BwdLaunch {
+    const void *x, *dt, *B, *C, *dy;   // io dtype
+    const float *A, *D;
+    float *dx, *ddt, *dA, *dB, *dC, *dD;
+    float *scratch;
+    int batch, L, H, G, N;
+    bool bf16;
+};
+int bwd_grid(int batch, int H);
+size_t bwd_scratch_bytes(int batch, int L, int H, int N);
+cudaError_t launch_bwd(const BwdLaunch &l, cudaStream_t stream);
+
 // Two-CTA kernel (ssd_pair.cu): each (batch, head) unit taken by a cluster of
 // two CTAs, one per scan direction, meeting per tile through an fp32 partial
 // in the workspace; both scans summed, a.init / a.rinit as launch_tc_fused.

@@ -77,7 +77,7 @@ enum {
 };
 
 /* Operation ids for ssd_workspace_bytes. */
-enum { SSD_OP_BIDIR_FWD = 0, SSD_OP_PREFIX_STATE = 1, SSD_OP_BLOCK_STEP = 2 };
+enum { SSD_OP_BIDIR_FWD = 0, SSD_OP_PREFIX_STATE = 1, SSD_OP_BLOCK_STEP = 2, SSD_OP_BIDIR_BWD = 3 };
 
 /* Kernel selection for ssd_bidir_fwd_path (tests and benchmarks). */
 enum {
@@ -267,6 +267,29 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
                          const void *C, const float *D, const float *fwd_init, const float *rev_init,
                          void *out, int batch, int seqlen, int nheads, int headdim, int dstate,
                          int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/* Backward pass of ssd_bidir_fwd: the gradients of the scalar sum(dy * out)
+ * with respect to every input, for training through the mixer.
+ *   dy   (batch, seqlen, nheads, headdim)           io, the gradient of out
+ *   dx   (batch, seqlen, nheads, headdim)           fp32
+ *   ddt  (2, batch, seqlen, nheads)                 fp32
+ *   dA, dD (2, nheads)                              fp32
+ *   dB, dC (2, batch, seqlen, ngroups, dstate)      fp32
+ * Other arguments as for ssd_bidir_fwd (either I/O dtype). Every output is
+ * overwritten. Each (batch, head, direction) runs its scan on CUDA cores in
+ * fp32, keeping every state in the workspace, then the adjoint scan in the
+ * opposite order; the workspace (ssd_workspace_bytes with SSD_OP_BIDIR_BWD)
+ * holds seqlen states of dstate x headdim fp32 per CTA of a persistent grid
+ * (about 4-8 GB at batch 32, seqlen 1024, 24 heads, dstate 128). dx gets
+ * exactly two additions per element and is deterministic; with ngroups <
+ * nheads the heads of a group add into dB and dC atomically, in no fixed
+ * order. Source: "Training Hybrid Block Diffusion Language Models with
+ * Partial Bidirectionality", Key Results and Technical Contribution (the
+ * models are trained through the mixer with a full-block objective). */
+int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                  const float *D, const void *dy, float *dx, float *ddt, float *dA, float *dB,
+                  float *dC, float *dD, int batch, int seqlen, int nheads, int headdim, int dstate,
+                  int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream);
 
 /* ssd_bidir_fwd for callers that cannot allocate device memory when they
  * call the mixer: code running under CUDA graph capture in the global mode,

@@ -10,12 +10,15 @@ Functions carry the C names:
   ssd_bidir_fwd(x, dt, A, B, C, D, chunk=256)          -> out
   ssd_bidir_bwd(x, dt, A, B, C, D, dy)                 -> dict of fp32 gradients dx, ddt, dA, dB, dC, dD
   ssd_prefix_state(x, dt, A, B, init=None, chunk=256)  -> state (batch, H, P, N) fp32
+  ssd_prefix_state_layers(x, dt, A, B, init=None)      -> states (layers, batch, H, P, N) fp32
   ssd_block_step(x, dt, A, B, C, D, prefix_state)      -> out
   ssd_segment_states(x, dt, A, B)                      -> (fwd_state, fwd_decay, rev_state, rev_decay)
   ssd_segment_carry(fwd_states, fwd_decays, rev_states, rev_decays, seg) -> (fwd_in, rev_in)
   ssd_bidir_fwd_seeded(x, dt, A, B, C, D, fwd_init, rev_init)           -> out
   ssd_bidir_fwd_dtraw(x, dt_raw, dt_bias, A, B, C, D, dt_min, dt_max)   -> out
-The sequence-sharded mixer over a process group is in seqshard.py.
+The sequence-sharded mixer over a process group is in seqshard.py; the
+block-diffusion cache of several layers and the CUDA-graph block loop are in
+blockdiff.py.
 Shapes (row-major, natural token order; [0] forward, [1] reverse):
   x (batch, L, H, P); dt (2, batch, L, H); A, D (2, H) fp32;
   B, C (2, batch, L, G, N); out like x.
@@ -33,7 +36,8 @@ from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSE
                    SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT, SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE,
                    SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD)
 
-__all__ = ["ssd_bidir_fwd", "ssd_bidir_bwd", "ssd_prefix_state", "ssd_block_step", "ssd_segment_states",
+__all__ = ["ssd_bidir_fwd", "ssd_bidir_bwd", "ssd_prefix_state", "ssd_prefix_state_layers", "ssd_block_step",
+           "ssd_segment_states",
            "ssd_segment_carry", "ssd_bidir_fwd_seeded", "ssd_bidir_fwd_dtraw", "ssd_workspace_bytes",
            "ssd_get_device_status", "SSDError", "Workspace", "lib"]
 
@@ -200,6 +204,48 @@ def ssd_prefix_state(x, dt, A, B, init=None, out=None, *, chunk: int = 256, path
                                    batch, L, H, P, N, G, chunk, _DT[io], int(path),
                                    _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_prefix_state")
+    return out
+
+
+def ssd_prefix_state_layers(x, dt, A, B, init=None, out=None, *, chunk: int = 256,
+                            workspace: Workspace | None = None):
+    """Forward-only states of several layers at once (include/ssd_bidir.h:
+    ssd_prefix_state_layers): x (layers, batch, L, H, P), dt (layers, batch, L,
+    H), A (layers, H), B (layers, batch, L, G, N), init / out (layers, batch, H,
+    P, N) fp32; out may be init (in-place commit)."""
+    _need(x, "x", ndim=5)
+    dev, io = x.device, x.dtype
+    if io not in _DT:
+        raise ValueError(f"x dtype {io} not supported (float32 or bfloat16)")
+    _need(dt, "dt", io, dev, 4)
+    _need(B, "B", io, dev, 5)
+    _need(A, "A", torch.float32, dev, 2)
+    layers, batch, L, H, P = x.shape
+    G, N = B.shape[-2], B.shape[-1]
+    if tuple(dt.shape) != (layers, batch, L, H) or tuple(B.shape) != (layers, batch, L, G, N) \
+            or tuple(A.shape) != (layers, H):
+        raise ValueError("shape mismatch: want x (l,b,L,H,P), dt (l,b,L,H), B (l,b,L,G,N), A (l,H)")
+    shape = (layers, batch, H, P, N)
+    if init is not None:
+        _need(init, "init", torch.float32, dev, 5)
+        if tuple(init.shape) != shape:
+            raise ValueError("init must be (layers, batch, H, P, N)")
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=dev)
+    else:
+        _need(out, "out", torch.float32, dev, 5)
+        if tuple(out.shape) != shape:
+            raise ValueError("out must be (layers, batch, H, P, N)")
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    nbytes = ssd_workspace_bytes(SSD_OP_PREFIX_STATE, layers * batch, L, H, P, N, G, chunk, io)
+    if nbytes == 0:
+        _check(_c.SSD_ERR_UNSUPPORTED, "ssd_prefix_state_layers")
+    buf = ws.get(nbytes)
+    rc = lib.ssd_prefix_state_layers(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init), _ptr(out),
+                                     layers, batch, L, H, P, N, G, chunk, _DT[io],
+                                     _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_prefix_state_layers")
     return out
 
 

@@ -38,6 +38,7 @@ SIGNATURES = {
     "ssd_bidir_fwd_seeded": (_i, [_vp] * 9 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_bidir_fwd_dtraw": (_i, [_vp] * 3 + [ctypes.c_float] * 2 + [_vp] * 5 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_bidir_bwd": (_i, [_vp] * 13 + [_i] * 7 + [_vp, _sz, _vp]),
+    "ssd_prefix_state_layers": (_i, [_vp] * 6 + [_i] * 9 + [_vp, _sz, _vp]),
     "ssd_get_device_status": (_i, [_vp, _vp]),
     "ssd_selftest_wait_timeout": (_i, [_vp, _sz, _i, _vp]),
     "ssd_error_string": (ctypes.c_char_p, [_i]),

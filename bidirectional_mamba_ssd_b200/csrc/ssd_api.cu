@@ -246,6 +246,48 @@ int ssd_prefix_state(const void *x, const void *dt, const float *A, const void *
                                  dstate, ngroups, chunk, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
 }
 
+int ssd_prefix_state_layers(const void *x, const void *dt, const float *A, const void *B, const float *init_state,
+                            float *state_out, int layers, int batch, int seqlen, int nheads, int headdim, int dstate,
+                            int ngroups, int chunk, int dtype, void *workspace, size_t ws_bytes, void *stream) {
+    if (layers <= 0) return SSD_ERR_INVALID_ARG;
+    if ((long long)layers * batch > (1ll << 31) - 1) return SSD_ERR_UNSUPPORTED;
+    const int lb = layers * batch;
+    int rc = check_shape(lb, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
+    if (rc != SSD_OK) return rc;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_PREFIX_STATE, lb, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (lb == 0) return SSD_OK;
+    if (!state_out || !aligned16(state_out) || (init_state && !aligned16(init_state))) return SSD_ERR_INVALID_ARG;
+    if (seqlen > 0 && (!x || !dt || !A || !B || !aligned16(x) || !aligned16(dt) || !aligned16(B) || !aligned4(A)))
+        return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == SSD_BF16 && seqlen > 0 && (long long)lb * nheads >= kFusedMinUnits) {
+        // one launch: the layers are batch elements that read their own layer's A
+        TcArgs t{};
+        t.x = x; t.dt = dt; t.A = A; t.B = B; t.init = init_state; t.state_out = state_out;
+        t.workspace = workspace; t.ws_bytes = ws_bytes;
+        t.batch = lb; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 1;
+        t.layer_units = batch * nheads;
+        t.A_layer = nheads;
+        return to_status(ssd::launch_tc_fused_state(t, s));
+    }
+    // otherwise one call per layer on that layer's slices
+    const size_t io = dtype == SSD_BF16 ? 2 : 4;
+    const size_t xl = (size_t)batch * seqlen * nheads * headdim, dtl = (size_t)batch * seqlen * nheads;
+    const size_t bl = (size_t)batch * seqlen * ngroups * dstate, sl = (size_t)batch * nheads * headdim * dstate;
+    for (int l = 0; l < layers; ++l) {
+        rc = ssd_prefix_state_path(x ? static_cast<const char *>(x) + l * xl * io : nullptr,
+                                   dt ? static_cast<const char *>(dt) + l * dtl * io : nullptr, A ? A + (size_t)l * nheads : nullptr,
+                                   B ? static_cast<const char *>(B) + l * bl * io : nullptr,
+                                   init_state ? init_state + l * sl : nullptr, state_out + l * sl, batch, seqlen, nheads,
+                                   headdim, dstate, ngroups, chunk, dtype, SSD_PATH_AUTO, workspace, ws_bytes, stream);
+        if (rc != SSD_OK) return rc;
+    }
+    return SSD_OK;
+}
+
 int ssd_block_step_path(const void *x, const void *dt, const float *A, const void *B, const void *C,
                         const float *D, const float *prefix_state, void *out, int batch, int blk_len,
                         int nheads, int headdim, int dstate, int ngroups, int dtype, int path,

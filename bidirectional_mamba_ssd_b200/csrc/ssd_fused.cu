@@ -95,7 +95,13 @@ struct FusedParams {
     int batch, L, H, G, nt, units;
     const float *dt_bias;      // DTRAW: (2, H); dt holds the raw projection
     float dt_lo, dt_hi;        // DTRAW: the step-size range
+    int layer_units, A_layer;  // layers stacked along the batch: A, D of unit u at + (u / layer_units) * A_layer
 };
+
+// A and D of unit u: a layer's own when several layers are stacked along the batch
+__device__ __forceinline__ const float *layer_ptr(const float *base, const FusedParams &p, int u) {
+    return p.layer_units ? base + (size_t)(u / p.layer_units) * p.A_layer : base;
+}
 
 // The step size from the raw projection (DTRAW): softplus(raw + bias),
 // clamped to [lo, hi]. softplus(u) = log(1 + e^u), equal to u in fp32 beyond 20.
@@ -513,7 +519,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         while (cu < u_end) {
             const int u = cu;
             const int h = u % p.H;
-            const float Af = p.A[h], Ab = kOut ? p.A[p.H + h] : 0.f;
+            const float *Au = layer_ptr(p.A, p, u);
+            const float Af = Au[h], Ab = kOut ? Au[p.H + h] : 0.f;
             // ---------------- phase 1: the state chain (reverse, right to left; in
             // the state mode forward, from the given state). Groups A and B prepare
             // the tiles (diag(w) X, tile decay); this group stores the reverse
@@ -656,9 +663,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         float *red_g = red_ab + (is_b ? 4 : 0);
         for (int u = u_begin; u < u_end; u += u_step) {
             const int b = u / p.H, h = u % p.H;
-            const float dsum = kOut ? p.D[h] + p.D[p.H + h] : 0.f;
+            const float *Au = layer_ptr(p.A, p, u), *Du = layer_ptr(p.D, p, u);
+            const float dsum = kOut ? Du[h] + Du[p.H + h] : 0.f;
             // the state pass's direction: reverse in the output modes, forward in the state mode
-            const float A1 = kFwd1 ? p.A[h] : p.A[p.H + h];
+            const float A1 = kFwd1 ? Au[h] : Au[p.H + h];
             const size_t dt1 = kFwd1 ? 0 : dt_dir;
             // ---------------- phase 1: every other state-pass tile (by the CTA's
             // running tile count m1: group A the even ones, group B the odd ones):
@@ -831,6 +839,8 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     p.dt_bias = a.dt_bias;
     p.dt_lo = a.dt_lo;
     p.dt_hi = a.dt_hi;
+    p.layer_units = a.layer_units;
+    p.A_layer = a.A_layer;
 
     CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_out;
     // the forward state mode may be given single-direction B; every other mode reads both directions' layout

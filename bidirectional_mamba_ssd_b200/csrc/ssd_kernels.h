@@ -42,6 +42,10 @@ struct TcArgs {
     float *decay_out = nullptr;    // (batch, H) fused state modes: exp(A * sum of dt) over the sequence
     const float *dt_bias = nullptr;  // (2, H) with launch_tc_fused_dtraw: dt holds the raw projection
     float dt_lo = 0.f, dt_hi = 0.f;  // with launch_tc_fused_dtraw: the step-size range
+    // several layers stacked along the batch: units of layer l are
+    // [l * layer_units, (l + 1) * layer_units) and read A (and D) from
+    // A + l * A_layer (D + l * A_layer); 0 = one layer
+    int layer_units = 0, A_layer = 0;
     float *state_out;         // (batch, H, 64, N) or nullptr
     void *out;                // (batch, L, H, 64) bf16
     void *workspace;          // status header + scratch

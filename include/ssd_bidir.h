@@ -268,6 +268,27 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
                          void *out, int batch, int seqlen, int nheads, int headdim, int dstate,
                          int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream);
 
+/* ssd_prefix_state for several layers at once (block diffusion keeps one
+ * cached forward state per layer; "Training Hybrid Block Diffusion Language
+ * Models with Partial Bidirectionality", Methodology: the states of the
+ * prefix are reused exactly, so committing a finished block updates every
+ * layer's cache). The layers' tensors are stacked along a leading dimension:
+ *   x          (layers, batch, seqlen, nheads, headdim)   io
+ *   dt         (layers, batch, seqlen, nheads)            io (forward direction)
+ *   A          (layers, nheads)                           fp32 (forward direction)
+ *   B          (layers, batch, seqlen, ngroups, dstate)   io (forward direction)
+ *   init_state (layers, batch, nheads, headdim, dstate)   fp32, nullable
+ *   state_out  (layers, batch, nheads, headdim, dstate)   fp32, may alias init_state
+ * With bf16 I/O and at least 64 (layer, batch, head) units this is one
+ * launch of the fused kernel's forward-state mode over all layers (each unit
+ * reads its own layer's A); otherwise one ssd_prefix_state per layer. The
+ * workspace is ssd_workspace_bytes(SSD_OP_PREFIX_STATE, layers * batch, ...).
+ * Returns as ssd_prefix_state. */
+int ssd_prefix_state_layers(const void *x, const void *dt, const float *A, const void *B,
+                            const float *init_state, float *state_out, int layers, int batch,
+                            int seqlen, int nheads, int headdim, int dstate, int ngroups, int chunk,
+                            int dtype, void *workspace, size_t ws_bytes, void *stream);
+
 /* Backward pass of ssd_bidir_fwd: the gradients of the scalar sum(dy * out)
  * with respect to every input, for training through the mixer.
  *   dy   (batch, seqlen, nheads, headdim)           io, the gradient of out

@@ -210,3 +210,94 @@ def bidir_bwd(x, dt, A, B, C, D, dy, nthreads: int = 0) -> dict:
     if rc != 0:
         raise ValueError("oracle bidir_bwd: bad arguments")
     return outs
+
+
+# ------------------------------------------------------------------ mixer block
+# The steps either side of the mixer in a Mamba-2 layer, for the bidirectional
+# model ("DiffMamba - Checkpoints" model card, Model details: forward and
+# flipped-reverse Mamba-2 layers with weight-tied projections, Mamba-2
+# defaults). The pages print none of these steps; they are the standard
+# Mamba-2 ones, read for two directions as follows (listed with the other
+# readings): each direction has its own depthwise conv1d over the projected
+# xBC channels, causal for the forward scan and, for the reverse scan, the
+# flipped sequence's causal conv, i.e. anti-causal in natural order; SiLU
+# after it; the channels split into x (H*P), B (G*N), C (G*N); each direction
+# scans its own x and adds its own D x; the summed output is gated by SiLU(z)
+# and RMS-normalised over its H*P channels with one weight vector.
+
+def silu(v):
+    v = np.asarray(v, dtype=np.float64)
+    return v / (1.0 + np.exp(-v))
+
+
+def conv_silu(xbc, w, bias):
+    """Both directions' depthwise conv1d + SiLU of xbc (batch, L, Cin): w (2,
+    Cin, K), bias (2, Cin). Forward: out[t] = sum_k w[0][c][k] in[t - K + 1 + k];
+    reverse: out[t] = sum_k w[1][c][k] in[t + K - 1 - k]; zero outside the
+    sequence. Returns (2, batch, L, Cin) after SiLU."""
+    xbc = np.asarray(xbc, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    bias = np.asarray(bias, dtype=np.float64)
+    batch, L, cin = xbc.shape
+    K = w.shape[2]
+    out = np.zeros((2, batch, L, cin))
+    for t in range(L):
+        acc_f = np.array(bias[0], dtype=np.float64) * np.ones((batch, cin))
+        acc_b = np.array(bias[1], dtype=np.float64) * np.ones((batch, cin))
+        for k in range(K):
+            s = t - (K - 1) + k            # forward tap k reads token s
+            if 0 <= s < L:
+                acc_f = acc_f + w[0][:, k] * xbc[:, s]
+            r = t + (K - 1) - k            # reverse tap k reads token r
+            if 0 <= r < L:
+                acc_b = acc_b + w[1][:, k] * xbc[:, r]
+        out[0, :, t] = acc_f
+        out[1, :, t] = acc_b
+    return silu(out)
+
+
+def split_xbc(u, H, P, G, N):
+    """(2, batch, L, H*P + 2*G*N) -> x2 (2, batch, L, H, P), B, C (2, batch, L, G, N)."""
+    two, batch, L, _ = u.shape
+    x2 = u[..., :H * P].reshape(two, batch, L, H, P)
+    B = u[..., H * P:H * P + G * N].reshape(two, batch, L, G, N)
+    C = u[..., H * P + G * N:].reshape(two, batch, L, G, N)
+    return x2, B, C
+
+
+def bidir_x2(x2, dt, A, B, C, D, nthreads: int = 0):
+    """The bidirectional mixer with each direction scanning its own x:
+    y = scan_f(x2[0]) + scan_b(x2[1]) + D_f x2[0] + D_b x2[1]. Each direction's
+    part is the pinned bidir() with the other direction's C and D zeroed."""
+    C = np.asarray(C, dtype=np.float64)
+    D = np.asarray(D, dtype=np.float64)
+    parts = []
+    for d in range(2):
+        Cd, Dd = C.copy(), D.copy()
+        Cd[1 - d] = 0.0
+        Dd[1 - d] = 0.0
+        parts.append(bidir(x2[d], dt, A, B, Cd, Dd, nthreads=nthreads))
+    return parts[0] + parts[1]
+
+
+def gated_rmsnorm(y, z, w, eps=1e-5):
+    """Mamba-2's gated RMS norm of the mixer output over its H*P channels:
+    v = y * SiLU(z), out = v / sqrt(mean(v^2) + eps) * w. y, z (batch, L, H,
+    P); w (H*P,)."""
+    y = np.asarray(y, dtype=np.float64)
+    batch, L, H, P = y.shape
+    v = (y * silu(z)).reshape(batch, L, H * P)
+    r = 1.0 / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+    return (v * r * np.asarray(w, dtype=np.float64)).reshape(batch, L, H, P)
+
+
+def mixer_block(xbc, z, dt_raw, conv_w, conv_b, dt_bias, A, D, norm_w, H, P, G, N,
+                dt_min=0.0, dt_max=np.inf, eps=1e-5):
+    """The bidirectional mixer with its input and output steps: conv1d + SiLU
+    per direction, the step size from the raw projection (dt_prep), the mixer
+    with per-direction x, then the gated RMS norm of the sum."""
+    u = conv_silu(xbc, conv_w, conv_b)
+    x2, B, C = split_xbc(u, H, P, G, N)
+    dt = dt_prep(dt_raw, dt_bias, dt_min, dt_max)
+    y = bidir_x2(x2, dt, A, B, C, D)
+    return gated_rmsnorm(y, z, norm_w, eps)

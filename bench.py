@@ -299,59 +299,46 @@ def run_reference(args, w):
 
 
 def bench_blockstep(args, w, dev):
-    """Block diffusion on one GPU: prefill of the cached forward state over the
-    prefix, then per block `steps` denoising steps (each a block step on fresh
-    block inputs, reading the cached state) and the commit of the block into
-    the state. One bench step = one block: all its denoising steps plus the
-    commit, replayed as one CUDA graph. value = block tokens x denoising steps
-    per second."""
+    """Block diffusion on one GPU through the library's block-diffusion helper
+    (bidirectional_mamba_ssd_b200.blockdiff): prefill of the cached forward
+    state over the prefix, then per block `steps` denoising steps (each a block
+    step on fresh block inputs, reading the cached state) and the commit of the
+    block into the state. One bench step = one block: all its denoising steps
+    plus the commit, replayed as one CUDA graph (BlockGraph). value = block
+    tokens x denoising steps per second."""
     import torch
-    import bidirectional_mamba_ssd_b200 as ssd
     import ssd_inputs as si
+    from bidirectional_mamba_ssd_b200.blockdiff import BlockDiffusionCache, BlockGraph
     data = si.blockstep_inputs(w.batch, w.seqlen, w.block, w.steps, w.nheads, w.headdim, w.dstate,
                                w.ngroups, w.dtype, seed=0, device=dev)
-    ws_pre, ws_step, ws_commit = ssd.Workspace(dev), ssd.Workspace(dev), ssd.Workspace(dev)
-    state = torch.empty(w.batch, w.nheads, w.headdim, w.dstate, dtype=torch.float32, device=dev)
+    cache = BlockDiffusionCache(1, w.batch, w.nheads, w.headdim, w.dstate, device=dev)
+    pre = (data["x_pre"][None], data["dt_pre"][None], data["A"][0][None].contiguous(), data["B_pre"][None])
     # prefill timing (outside the graph)
     for _ in range(2):
-        ssd.ssd_prefix_state(data["x_pre"], data["dt_pre"], data["A"][0], data["B_pre"], out=state,
-                             chunk=w.chunk, workspace=ws_pre)
+        cache.prefill(*pre, chunk=w.chunk)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    ssd.ssd_prefix_state(data["x_pre"], data["dt_pre"], data["A"][0], data["B_pre"], out=state,
-                         chunk=w.chunk, workspace=ws_pre)
+    cache.prefill(*pre, chunk=w.chunk)
     e1.record()
     torch.cuda.synchronize()
     prefill_ms = e0.elapsed_time(e1)
-    outs = [torch.empty_like(st["x"]) for st in data["steps"]]
-    commit_state = state.clone()
-
-    def block():
-        for k, st in enumerate(data["steps"]):
-            ssd.ssd_block_step(st["x"], st["dt"], data["A"], st["B"], st["C"], data["D"], state,
-                               out=outs[k], workspace=ws_step)
-        last = data["steps"][-1]
-        ssd.ssd_prefix_state(last["x"], last["dt"][0], data["A"][0], last["B"][0], init=state,
-                             out=commit_state, chunk=w.chunk, workspace=ws_commit)
-
-    stream = torch.cuda.Stream(dev)
-    stream.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(stream):
-        block()   # sizes the workspaces outside the capture
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            block()
+    bg = BlockGraph(cache, w.steps, w.block, w.nheads, w.headdim, w.dstate, w.ngroups)
+    bg.A[0].copy_(data["A"])
+    bg.D[0].copy_(data["D"])
+    for k, st in enumerate(data["steps"]):
+        for n in ("x", "dt", "B", "C"):
+            getattr(bg, n)[k, 0].copy_(st[n])
+    bg.capture()
     torch.cuda.synchronize()
     for _ in range(args.warmup):
-        graph.replay()
+        bg.replay()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
         t0.record()
         for _ in range(args.steps):
-            graph.replay()
+            bg.replay()
         t1.record()
         torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / args.steps
@@ -380,7 +367,8 @@ def bench_blockstep(args, w, dev):
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "prefix": w.seqlen, "block": w.block,
                        "denoising_steps": w.steps, "nheads": w.nheads, "headdim": w.headdim,
-                       "dstate": w.dstate, "ngroups": w.ngroups, "graph": "one CUDA graph per block"},
+                       "dstate": w.dstate, "ngroups": w.ngroups,
+                       "graph": "one CUDA graph per block (blockdiff.BlockGraph: steps + commit)"},
             "roofline": roof,
             "per_denoising_step_us": round(1e3 * ms / (w.steps + 1), 3),
             "algorithmic_bytes_per_denoising_step": step_bytes,

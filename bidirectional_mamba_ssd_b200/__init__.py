@@ -9,6 +9,8 @@ Every step of the computation runs in the library's kernels.
 Functions carry the C names:
   ssd_bidir_fwd(x, dt, A, B, C, D, chunk=256)          -> out
   ssd_bidir_bwd(x, dt, A, B, C, D, dy)                 -> dict of fp32 gradients dx, ddt, dA, dB, dC, dD
+  ssd_bidir_fwd_x2(x2, dt, A, B, C, D)                 -> out (each direction scans its own x, x2 (2,b,L,H,P))
+  ssd_mixer_block_fwd(xbc, z, dt_raw, conv_w, conv_b, dt_bias, A, D, norm_w, H, G, N) -> out
   ssd_prefix_state(x, dt, A, B, init=None, chunk=256)  -> state (batch, H, P, N) fp32
   ssd_prefix_state_layers(x, dt, A, B, init=None)      -> states (layers, batch, H, P, N) fp32
   ssd_block_step(x, dt, A, B, C, D, prefix_state)      -> out
@@ -34,9 +36,10 @@ from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSE
                    SSD_PATH_PAIR,
                    SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA,
                    SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT, SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE,
-                   SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD)
+                   SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD, SSD_OP_BIDIR_FWD_X2, SSD_OP_MIXER_BLOCK)
 
-__all__ = ["ssd_bidir_fwd", "ssd_bidir_bwd", "ssd_prefix_state", "ssd_prefix_state_layers", "ssd_block_step",
+__all__ = ["ssd_bidir_fwd", "ssd_bidir_bwd", "ssd_bidir_fwd_x2", "ssd_mixer_block_fwd", "ssd_prefix_state",
+           "ssd_prefix_state_layers", "ssd_block_step",
            "ssd_segment_states",
            "ssd_segment_carry", "ssd_bidir_fwd_seeded", "ssd_bidir_fwd_dtraw", "ssd_workspace_bytes",
            "ssd_get_device_status", "SSDError", "Workspace", "lib"]
@@ -431,3 +434,76 @@ def ssd_bidir_bwd(x, dt, A, B, C, D, dy, *, workspace: Workspace | None = None) 
                            batch, L, H, P, N, G, _DT[io], _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_bidir_bwd")
     return g
+
+
+def ssd_bidir_fwd_x2(x2, dt, A, B, C, D, out=None, *, workspace: Workspace | None = None):
+    """The bidirectional mixer with each direction scanning its own x
+    (include/ssd_bidir.h: ssd_bidir_fwd_x2): x2 (2, batch, L, H, P)."""
+    _need(x2, "x2", ndim=5)
+    dev, io = x2.device, x2.dtype
+    if io not in _DT:
+        raise ValueError(f"x2 dtype {io} not supported (float32 or bfloat16)")
+    _need(dt, "dt", io, dev, 4)
+    _need(B, "B", io, dev, 5)
+    _need(C, "C", io, dev, 5)
+    _need(A, "A", torch.float32, dev, 2)
+    _need(D, "D", torch.float32, dev, 2)
+    two, batch, L, H, P = x2.shape
+    G, N = B.shape[-2:]
+    if two != 2 or tuple(dt.shape) != (2, batch, L, H) or tuple(B.shape) != (2, batch, L, G, N) \
+            or tuple(C.shape) != tuple(B.shape) or tuple(A.shape) != (2, H) or tuple(D.shape) != (2, H):
+        raise ValueError("shape mismatch: want x2 (2,b,L,H,P), dt (2,b,L,H), B/C (2,b,L,G,N), A/D (2,H)")
+    if out is None:
+        out = torch.empty(x2.shape[1:], dtype=io, device=dev)
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    nbytes = ssd_workspace_bytes(SSD_OP_BIDIR_FWD_X2, batch, L, H, P, N, G, 64, io)
+    if nbytes == 0:
+        _check(_c.SSD_ERR_UNSUPPORTED, "ssd_bidir_fwd_x2")
+    buf = ws.get(nbytes)
+    rc = lib.ssd_bidir_fwd_x2(_ptr(x2), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(out),
+                              batch, L, H, P, N, G, _DT[io], _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    _check(rc, "ssd_bidir_fwd_x2")
+    return out
+
+
+def ssd_mixer_block_fwd(xbc, z, dt_raw, conv_w, conv_b, dt_bias, A, D, norm_w, nheads: int, ngroups: int,
+                        dstate: int, *, dt_min: float = 0.0, dt_max: float = float("inf"), norm_eps: float = 1e-5,
+                        out=None, workspace: Workspace | None = None):
+    """The mixer with its input and output steps (include/ssd_bidir.h:
+    ssd_mixer_block_fwd): xbc (batch, L, H*P + 2*G*N), z (batch, L, H, P),
+    dt_raw (2, batch, L, H), conv_w (2, Cin, K), conv_b (2, Cin), dt_bias, A,
+    D (2, H), norm_w (H*P,). Returns out (batch, L, H, P)."""
+    _need(xbc, "xbc", ndim=3)
+    dev, io = xbc.device, xbc.dtype
+    if io not in _DT:
+        raise ValueError(f"xbc dtype {io} not supported (float32 or bfloat16)")
+    batch, L, cin = xbc.shape
+    P = (cin - 2 * ngroups * dstate) // nheads
+    if nheads * P + 2 * ngroups * dstate != cin:
+        raise ValueError("xbc channels must be nheads*headdim + 2*ngroups*dstate")
+    _need(z, "z", io, dev, 4)
+    _need(dt_raw, "dt_raw", io, dev, 4)
+    for name, t, nd in (("conv_w", conv_w, 3), ("conv_b", conv_b, 2), ("dt_bias", dt_bias, 2), ("A", A, 2),
+                        ("D", D, 2), ("norm_w", norm_w, 1)):
+        _need(t, name, torch.float32, dev, nd)
+    K = conv_w.shape[2]
+    if tuple(z.shape) != (batch, L, nheads, P) or tuple(dt_raw.shape) != (2, batch, L, nheads) \
+            or tuple(conv_w.shape) != (2, cin, K) or tuple(conv_b.shape) != (2, cin) \
+            or tuple(dt_bias.shape) != (2, nheads) or tuple(A.shape) != (2, nheads) or tuple(D.shape) != (2, nheads) \
+            or tuple(norm_w.shape) != (nheads * P,):
+        raise ValueError("shape mismatch in ssd_mixer_block_fwd")
+    if out is None:
+        out = torch.empty(batch, L, nheads, P, dtype=io, device=dev)
+    stream = _stream(dev)
+    ws = _workspace(dev, stream, workspace)
+    nbytes = ssd_workspace_bytes(SSD_OP_MIXER_BLOCK, batch, L, nheads, P, dstate, ngroups, 64, io)
+    if nbytes == 0:
+        _check(_c.SSD_ERR_UNSUPPORTED, "ssd_mixer_block_fwd")
+    buf = ws.get(nbytes)
+    rc = lib.ssd_mixer_block_fwd(_ptr(xbc), _ptr(z), _ptr(dt_raw), _ptr(conv_w), _ptr(conv_b), K, _ptr(dt_bias),
+                                 float(dt_min), float(dt_max), _ptr(A), _ptr(D), _ptr(norm_w), float(norm_eps),
+                                 _ptr(out), batch, L, nheads, P, dstate, ngroups, _DT[io], _ptr(buf), buf.numel(),
+                                 ctypes.c_void_p(stream))
+    _check(rc, "ssd_mixer_block_fwd")
+    return out

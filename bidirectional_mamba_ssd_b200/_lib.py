@@ -15,6 +15,7 @@ SSD_F32, SSD_BF16 = 0, 1
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED = 0, -1, -2
 SSD_ERR_CUDA, SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT = -3, -4, -5
 SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE, SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD = 0, 1, 2, 3
+SSD_OP_BIDIR_FWD_X2, SSD_OP_MIXER_BLOCK = 4, 5
 SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED, SSD_PATH_SEGMENTED, SSD_PATH_PAIR = 0, 1, 2, 3, 4, 5
 
 _vp = ctypes.c_void_p
@@ -39,6 +40,9 @@ SIGNATURES = {
     "ssd_bidir_fwd_dtraw": (_i, [_vp] * 3 + [ctypes.c_float] * 2 + [_vp] * 5 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_bidir_bwd": (_i, [_vp] * 13 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_prefix_state_layers": (_i, [_vp] * 6 + [_i] * 9 + [_vp, _sz, _vp]),
+    "ssd_bidir_fwd_x2": (_i, [_vp] * 7 + [_i] * 7 + [_vp, _sz, _vp]),
+    "ssd_mixer_block_fwd": (_i, [_vp] * 5 + [_i, _vp] + [ctypes.c_float] * 2 + [_vp] * 3 + [ctypes.c_float, _vp]
+                            + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_get_device_status": (_i, [_vp, _vp]),
     "ssd_selftest_wait_timeout": (_i, [_vp, _sz, _i, _vp]),
     "ssd_error_string": (ctypes.c_char_p, [_i]),

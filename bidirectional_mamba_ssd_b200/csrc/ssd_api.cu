@@ -133,6 +133,38 @@ int bidir_impl(const void *x, const void *dt, const float *A, const void *B, con
     return to_status(ssd::launch_tc_chunked(t, s));
 }
 
+// Scratch of ssd_bidir_fwd_x2: the two-CTA kernel's partial tiles (bf16,
+// more than one tile) or the sequential scan's fp32 forward partial.
+size_t x2_scratch(int batch, int seqlen, int nheads, int dstate, int dtype) {
+    size_t s = simt_scratch(SSD_OP_BIDIR_FWD, batch, seqlen, nheads);
+    if (dtype == SSD_BF16 && ssd::tc_pair_supported(batch, seqlen, nheads, 1, dstate)) {
+        const size_t q = ssd::tc_pair_scratch_bytes(batch, seqlen, nheads, dstate);
+        s = s > q ? s : q;
+    }
+    return s;
+}
+
+// Workspace of ssd_mixer_block_fwd after the status header: the mixer's own
+// scratch first (it is passed the workspace as its own), then the
+// intermediates, each 256-byte aligned.
+struct BlockWs {
+    size_t mixer, x2, b2, c2, dt, y, total;
+};
+BlockWs block_ws(int batch, int seqlen, int nheads, int dstate, int ngroups, int dtype) {
+    BlockWs w{};
+    const size_t io = dtype == SSD_BF16 ? 2 : 4;
+    const size_t tok = (size_t)batch * seqlen;
+    w.mixer = round256(x2_scratch(batch, seqlen, nheads, dstate, dtype));
+    size_t o = 0;
+    w.x2 = o; o += round256(2 * tok * nheads * kHeaddim * io);
+    w.b2 = o; o += round256(2 * tok * ngroups * dstate * io);
+    w.c2 = o; o += round256(2 * tok * ngroups * dstate * io);
+    w.dt = o; o += round256(2 * tok * nheads * io);
+    w.y = o; o += round256(tok * nheads * kHeaddim * io);
+    w.total = o;
+    return w;
+}
+
 }  // namespace
 
 extern "C" {
@@ -166,6 +198,11 @@ size_t ssd_workspace_bytes(int op, int batch, int seqlen, int nheads, int headdi
         }
     }
     if (op == SSD_OP_BIDIR_BWD) scratch = ssd::bwd_scratch_bytes(batch, seqlen, nheads, dstate);
+    if (op == SSD_OP_BIDIR_FWD_X2) scratch = x2_scratch(batch, seqlen, nheads, dstate, dtype);
+    if (op == SSD_OP_MIXER_BLOCK) {
+        const BlockWs w = block_ws(batch, seqlen, nheads, dstate, ngroups, dtype);
+        scratch = w.mixer + w.total;
+    }
     return ssd::kStatusBytes + round256(scratch);
 }
 
@@ -487,6 +524,81 @@ int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, 
     l.batch = batch; l.L = seqlen; l.H = nheads; l.G = ngroups; l.N = dstate;
     l.bf16 = dtype == SSD_BF16;
     return to_status(ssd::launch_bwd(l, s));
+}
+
+int ssd_bidir_fwd_x2(const void *x2, const void *dt, const float *A, const void *B, const void *C, const float *D,
+                     void *out, int batch, int seqlen, int nheads, int headdim, int dstate, int ngroups, int dtype,
+                     void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype, false);
+    if (rc != SSD_OK) return rc;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD_X2, batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    if (!x2 || !dt || !A || !B || !C || !D || !out) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x2) || !aligned16(dt) || !aligned16(B) || !aligned16(C) || !aligned16(out) || !aligned4(A) ||
+        !aligned4(D))
+        return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long xdir = (long long)batch * seqlen * nheads * headdim;
+    if (dtype == SSD_BF16 && ssd::tc_pair_supported(batch, seqlen, nheads, ngroups, dstate)) {
+        TcArgs t{};
+        t.x = x2; t.dt = dt; t.A = A; t.B = B; t.C = C; t.D = D; t.out = out;
+        t.workspace = workspace; t.ws_bytes = ws_bytes;
+        t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+        t.x_dir_stride = xdir;
+        return to_status(ssd::launch_tc_pair(t, s));
+    }
+    SimtArgs a{};
+    a.x = x2; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.out = out; a.yacc = scratch_ptr(workspace);
+    a.dt_dir_stride = (long long)batch * seqlen * nheads;
+    a.bc_dir_stride = (long long)batch * seqlen * ngroups * dstate;
+    a.A_dir_stride = nheads;
+    a.x_dir_stride = xdir;
+    a.batch = batch; a.L = seqlen; a.H = nheads; a.G = ngroups;
+    a.ndir = 2; a.has_output = 1;
+    return to_status(ssd::launch_scan_simt(a, dtype == SSD_BF16, dstate, s));
+}
+
+int ssd_mixer_block_fwd(const void *xbc, const void *z, const void *dt_raw, const float *conv_w, const float *conv_b,
+                        int conv_k, const float *dt_bias, float dt_min, float dt_max, const float *A, const float *D,
+                        const float *norm_w, float norm_eps, void *out, int batch, int seqlen, int nheads,
+                        int headdim, int dstate, int ngroups, int dtype, void *workspace, size_t ws_bytes,
+                        void *stream) {
+    int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype, false);
+    if (rc != SSD_OK) return rc;
+    if (conv_k < 1 || conv_k > 4) return SSD_ERR_UNSUPPORTED;
+    if (!(dt_min >= 0.f) || !(dt_max >= dt_min) || !(norm_eps >= 0.f)) return SSD_ERR_INVALID_ARG;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
+    if (ws_bytes < ssd_workspace_bytes(SSD_OP_MIXER_BLOCK, batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype))
+        return SSD_ERR_WORKSPACE;
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    if (!xbc || !z || !dt_raw || !conv_w || !conv_b || !dt_bias || !A || !D || !norm_w || !out)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned16(xbc) || !aligned16(z) || !aligned16(dt_raw) || !aligned16(out) || !aligned4(conv_w) ||
+        !aligned4(conv_b) || !aligned4(dt_bias) || !aligned4(A) || !aligned4(D) || !aligned4(norm_w))
+        return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const BlockWs w = block_ws(batch, seqlen, nheads, dstate, ngroups, dtype);
+    char *inter = static_cast<char *>(workspace) + ssd::kStatusBytes + w.mixer;
+    ssd::BlockLaunch l{};
+    l.xbc = xbc; l.conv_w = conv_w; l.conv_b = conv_b;
+    l.x2 = inter + w.x2; l.B2 = inter + w.b2; l.C2 = inter + w.c2;
+    l.dt_raw = dt_raw; l.dt_bias = dt_bias; l.dt = inter + w.dt;
+    l.y = inter + w.y; l.z = z; l.norm_w = norm_w; l.out = out;
+    l.dt_lo = dt_min; l.dt_hi = dt_max; l.eps = norm_eps;
+    l.batch = batch; l.L = seqlen; l.H = nheads; l.HP = nheads * headdim; l.GN = ngroups * dstate; l.K = conv_k;
+    l.bf16 = dtype == SSD_BF16;
+    if ((rc = to_status(ssd::launch_conv_silu(l, s))) != SSD_OK) return rc;
+    if ((rc = to_status(ssd::launch_dt_prep(l, s))) != SSD_OK) return rc;
+    // the mixer gets the workspace's header and its own scratch
+    rc = ssd_bidir_fwd_x2(l.x2, l.dt, A, l.B2, l.C2, D, const_cast<void *>(l.y), batch, seqlen, nheads, headdim,
+                          dstate, ngroups, dtype, workspace, ssd::kStatusBytes + w.mixer, stream);
+    if (rc != SSD_OK) return rc;
+    return to_status(ssd::launch_gated_rmsnorm(l, s));
 }
 
 int ssd_get_device_status(const void *workspace, void *stream) {

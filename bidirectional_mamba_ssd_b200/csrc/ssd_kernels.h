@@ -22,6 +22,9 @@ struct SimtArgs {
     float *yacc;              // (batch, L, H, 64) fp32 scratch for the forward partial
     long long dt_dir_stride, bc_dir_stride;
     int A_dir_stride;
+    // elements between the two directions' x when each direction scans its own
+    // x (x then holds (2, batch, L, H, 64)); 0 = one x for both directions
+    long long x_dir_stride = 0;
     int batch, L, H, G;
     int ndir;                 // 1: forward only, 2: forward + reverse
     int has_output;
@@ -46,6 +49,9 @@ struct TcArgs {
     // [l * layer_units, (l + 1) * layer_units) and read A (and D) from
     // A + l * A_layer (D + l * A_layer); 0 = one layer
     int layer_units = 0, A_layer = 0;
+    // elements between the two directions' x when each scans its own x
+    // (launch_tc_pair only; x then holds (2, batch, L, H, 64)); 0 = one x
+    long long x_dir_stride = 0;
     float *state_out;         // (batch, H, 64, N) or nullptr
     void *out;                // (batch, L, H, 64) bf16
     void *workspace;          // status header + scratch
@@ -73,6 +79,26 @@ cudaError_t launch_tc_fused_state(const TcArgs &a, cudaStream_t stream);
 // Fused kernel, reverse scan only (direction 1 of the direction-stacked
 // inputs): the state at the sequence start into a.state_out, from zero.
 cudaError_t launch_tc_fused_state_rev(const TcArgs &a, cudaStream_t stream);
+
+// Input and output steps of the mixer block (ssd_block.cu).
+struct BlockLaunch {
+    const void *xbc;            // (batch, L, HP + 2 GN) io
+    const float *conv_w;        // (2, HP + 2 GN, K)
+    const float *conv_b;        // (2, HP + 2 GN)
+    void *x2, *B2, *C2;         // (2, batch, L, HP), (2, batch, L, GN) io
+    const void *dt_raw;         // (2, batch, L, H) io
+    const float *dt_bias;       // (2, H)
+    void *dt;                   // (2, batch, L, H) io
+    const void *y, *z;          // (batch, L, HP) io
+    const float *norm_w;        // (HP)
+    void *out;                  // (batch, L, HP) io
+    float dt_lo, dt_hi, eps;
+    int batch, L, H, HP, GN, K;
+    bool bf16;
+};
+cudaError_t launch_conv_silu(const BlockLaunch &l, cudaStream_t stream);
+cudaError_t launch_dt_prep(const BlockLaunch &l, cudaStream_t stream);
+cudaError_t launch_gated_rmsnorm(const BlockLaunch &l, cudaStream_t stream);
 
 // Backward pass (ssd_bwd.cu): gradients of sum(dy * y) of the bidirectional
 // mixer, fp32 outputs, any I/O dtype; persistent CTAs, each with L states of

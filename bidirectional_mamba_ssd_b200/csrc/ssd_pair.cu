@@ -76,6 +76,7 @@ struct PairParams {
     float *part;               // (clusters, 2, nt) fp32 partial tiles, 16 column chunks x 128 rows x 4
     DeviceStatus *status;
     int batch, L, H, G, nt, units;
+    int x2;                    // each direction scans its own x (tm_xr holds the reverse one's)
 };
 
 enum {
@@ -117,9 +118,9 @@ struct PSmem {
 
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-               const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_out,
-               const PairParams p) {
+tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xr,
+               const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
+               const __grid_constant__ CUtensorMap tm_out, const PairParams p) {
     using S = PSmem<N>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -181,7 +182,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tmap(&tm_x);
+            prefetch_tmap(fwd ? &tm_x : &tm_xr);
             prefetch_tmap(&tm_b);
             prefetch_tmap(&tm_c);
             prefetch_tmap(&tm_out);
@@ -212,7 +213,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     ++kx;
                     // the first reader of an x tile keeps it in L2 for the other direction
                     mbar_arrive_expect_tx(bar(B_X_FULL + xs), kSlab);
-                    tma_load_4d_hint(base + S::xslot(xs), &tm_x, bar(B_X_FULL + xs), 0, h, t0, b,
+                    tma_load_4d_hint(base + S::xslot(xs), fwd ? &tm_x : &tm_xr, bar(B_X_FULL + xs), 0, h, t0, b,
                                      first_at(k) ? keep : stream);
                 }
             }
@@ -432,7 +433,12 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc_fence_after();
             const float e = __expf(my_a);
             const bool yz = hzero(k);
-            const float dsum = p.D[h] + p.D[p.H + h];
+            // D terms: with one x for both directions the second adds (D_f + D_b) x
+            // after the partial; with one x per direction each adds its own D x
+            // before (so the sum is the same whichever comes first)
+            const float d_own = p.x2 ? p.D[dir * p.H + h] : 0.f;
+            const float dsum = p.x2 ? 0.f : p.D[h] + p.D[p.H + h];
+            const bool need_x = second || p.x2;
             uint8_t *xt = g + S::xslot(xs);
             const int q0 = c0 >> 3;              // first 16-column quarter: 0 or 2
 #pragma unroll
@@ -446,10 +452,21 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 } else {
                     tmem_ld16(tYo(m) + lane_off + q * 16, ov);
                 }
+                uint4 xv[2];
+                if (need_x) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) xv[cc] = *reinterpret_cast<const uint4 *>(xt + sw128_offset(row, q * 2 + cc));
+                }
                 tmem_wait_ld();
+                const uint32_t *xu = reinterpret_cast<const uint32_t *>(xv);
+                auto xval = [&](int c) { return bf2f((c & 1) ? (xu[c >> 1] >> 16) : (xu[c >> 1] & 0xffffu)); };
                 float y[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c) y[c] = __uint_as_float(yv[c]) + e * __uint_as_float(ov[c]);
+                if (p.x2) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) y[c] += d_own * xval(c);
+                }
                 if (!second) {
 #pragma unroll
                     for (int e4 = 0; e4 < 4; ++e4)
@@ -463,19 +480,13 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         y[4 * e4 + 2] += pv[4 * qq + e4].z;
                         y[4 * e4 + 3] += pv[4 * qq + e4].w;
                     }
+                    uint4 ov4[2];
+                    uint32_t *ou = reinterpret_cast<uint32_t *>(ov4);
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        uint4 *qp = reinterpret_cast<uint4 *>(xt + sw128_offset(row, q * 2 + cc));
-                        uint4 xv = *qp;
-                        uint32_t *xu = reinterpret_cast<uint32_t *>(&xv);
+                    for (int c2 = 0; c2 < 8; ++c2)
+                        ou[c2] = pack_bf16x2(y[2 * c2] + dsum * xval(2 * c2), y[2 * c2 + 1] + dsum * xval(2 * c2 + 1));
 #pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int i0 = cc * 8 + 2 * e2;
-                            xu[e2] = pack_bf16x2(y[i0] + dsum * bf2f(xu[e2] & 0xffffu),
-                                                 y[i0 + 1] + dsum * bf2f(xu[e2] >> 16));
-                        }
-                        *qp = xv;
-                    }
+                    for (int cc = 0; cc < 2; ++cc) *reinterpret_cast<uint4 *>(xt + sw128_offset(row, q * 2 + cc)) = ov4[cc];
                 }
             }
             fence_proxy_async_smem();
@@ -593,8 +604,11 @@ cudaError_t run_pair(const TcArgs &a, cudaStream_t stream) {
     p.part = reinterpret_cast<float *>((pa + 255) & ~(uintptr_t)255);
     p.batch = a.batch; p.L = a.L; p.H = a.H; p.G = a.G; p.nt = nt; p.units = units;
 
-    CUtensorMap tm_x, tm_b, tm_c, tm_out;
-    if (!tmap::map_x(&tm_x, a.x, a.batch, a.L, a.H) || !tmap::map_bc(&tm_b, a.B, 2, a.batch, a.L, a.G, N) ||
+    p.x2 = a.x_dir_stride != 0;
+    CUtensorMap tm_x, tm_xr, tm_b, tm_c, tm_out;
+    const void *xr = p.x2 ? static_cast<const void *>(static_cast<const __nv_bfloat16 *>(a.x) + a.x_dir_stride) : a.x;
+    if (!tmap::map_x(&tm_x, a.x, a.batch, a.L, a.H) || !tmap::map_x(&tm_xr, xr, a.batch, a.L, a.H) ||
+        !tmap::map_bc(&tm_b, a.B, 2, a.batch, a.L, a.G, N) ||
         !tmap::map_bc(&tm_c, a.C, 2, a.batch, a.L, a.G, N) || !tmap::map_x(&tm_out, a.out, a.batch, a.L, a.H))
         return cudaErrorInvalidValue;
     auto k = tc_pair_kernel<N>;
@@ -625,7 +639,7 @@ cudaError_t run_pair(const TcArgs &a, cudaStream_t stream) {
     const int ncl = active < cmax ? active : cmax;
     cfg.gridDim = dim3(2 * ncl);
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, k, tm_x, tm_b, tm_c, tm_out, p);
+    return cudaLaunchKernelEx(&cfg, k, tm_x, tm_xr, tm_b, tm_c, tm_out, p);
 }
 
 }  // namespace

@@ -58,10 +58,16 @@ scan_simt_seq_kernel(const SimtArgs a) {
     T *out = static_cast<T *>(a.out);
 
     const float dsum = a.has_output ? (a.D[h] + a.D[a.H + h]) : 0.f;
+    // D terms: with one x both go on at the end; with one x per direction each
+    // direction adds its own D x
+    const bool x2 = a.x_dir_stride != 0;
+    const float d_first = (a.has_output && x2) ? a.D[h] : 0.f;
+    const float d_last = (a.has_output && x2) ? a.D[a.H + h] : dsum;
     float hs[NQ];
 
     for (int dir = 0; dir < a.ndir; ++dir) {
         const bool reverse = dir == 1;
+        const T *xd = x + dir * a.x_dir_stride;
         // Starting state: the forward scan may start from a given state.
         if (dir == 0 && a.init) {
             const float *ip = a.init + ((size_t)unit * kP + p) * N + q * NQ;
@@ -89,7 +95,7 @@ scan_simt_seq_kernel(const SimtArgs a) {
             for (int idx = tid; idx < nt * kP; idx += kThreads) {
                 const int i = idx / kP, pp = idx - i * kP;
                 const int t = reverse ? (L - 1 - (t0 + i)) : (t0 + i);
-                xs[idx] = IO<T>::load(x + ((size_t)(b * L + t) * a.H + h) * kP + pp);
+                xs[idx] = IO<T>::load(xd + ((size_t)(b * L + t) * a.H + h) * kP + pp);
             }
             if (tid < nt) {
                 const int t = reverse ? (L - 1 - (t0 + tid)) : (t0 + tid);
@@ -119,10 +125,10 @@ scan_simt_seq_kernel(const SimtArgs a) {
                     const float y = (pi[0] + pi[kP]) + (pi[2 * kP] + pi[3 * kP]);
                     const size_t o = ((size_t)(b * L + t) * a.H + h) * kP + pp;
                     if (dir == 0 && a.ndir == 2) {
-                        a.yacc[o] = y;
+                        a.yacc[o] = x2 ? y + d_first * xs[idx] : y;
                     } else {
                         const float prev = (a.ndir == 2) ? a.yacc[o] : 0.f;
-                        IO<T>::store(out + o, prev + y + dsum * xs[idx]);
+                        IO<T>::store(out + o, prev + y + d_last * xs[idx]);
                     }
                 }
             }
@@ -266,7 +272,7 @@ template <typename T, int N>
 cudaError_t launch_t(const SimtArgs &a, cudaStream_t stream) {
     // both scans side by side while the units take one round of CTAs
     const int sms = device_sms();
-    if (a.ndir == 2 && a.has_output && a.batch * a.H <= (sms > 0 ? sms : 148)) {
+    if (a.ndir == 2 && a.has_output && a.x_dir_stride == 0 && a.batch * a.H <= (sms > 0 ? sms : 148)) {
         const size_t smem = sizeof(float) * 2 * (size_t)stage_floats<N>();
         auto kern = scan_simt_pair_kernel<T, N>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -77,7 +77,10 @@ enum {
 };
 
 /* Operation ids for ssd_workspace_bytes. */
-enum { SSD_OP_BIDIR_FWD = 0, SSD_OP_PREFIX_STATE = 1, SSD_OP_BLOCK_STEP = 2, SSD_OP_BIDIR_BWD = 3 };
+enum {
+    SSD_OP_BIDIR_FWD = 0, SSD_OP_PREFIX_STATE = 1, SSD_OP_BLOCK_STEP = 2, SSD_OP_BIDIR_BWD = 3,
+    SSD_OP_BIDIR_FWD_X2 = 4, SSD_OP_MIXER_BLOCK = 5
+};
 
 /* Kernel selection for ssd_bidir_fwd_path (tests and benchmarks). */
 enum {
@@ -267,6 +270,46 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
                          const void *C, const float *D, const float *fwd_init, const float *rev_init,
                          void *out, int batch, int seqlen, int nheads, int headdim, int dstate,
                          int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/* The bidirectional mixer with each direction scanning its own x (the mixer
+ * of a layer whose two directions have their own input conv, see
+ * ssd_mixer_block_fwd):
+ *   out_t = yf_t(x2[0]) + yb_t(x2[1]) + D_f x2[0]_t + D_b x2[1]_t
+ *   x2   (2, batch, seqlen, nheads, headdim)   io; other arguments as ssd_bidir_fwd
+ * bf16 with seqlen > 128 runs the two-CTA tensor-core kernel, otherwise the
+ * sequential scan. The two directions' fp32 results are added in an order
+ * that does not depend on which direction finishes first. */
+int ssd_bidir_fwd_x2(const void *x2, const void *dt, const float *A, const void *B, const void *C,
+                     const float *D, void *out, int batch, int seqlen, int nheads, int headdim,
+                     int dstate, int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/* A bidirectional Mamba-2 mixer with its input and output steps ("DiffMamba
+ * - Checkpoints" model card, Model details: forward and flipped-reverse
+ * Mamba-2 layers with weight-tied projections, Mamba-2 defaults; the pages
+ * print none of these steps, so they are the standard Mamba-2 ones, read for
+ * two directions):
+ *   1. u_d = SiLU(conv1d_d(xbc) + conv_b_d), depthwise over the channels, causal
+ *      for d = forward, anti-causal (the flipped sequence's causal conv) for
+ *      d = reverse; split into x_d (H*P), B_d (G*N), C_d (G*N);
+ *   2. dt_d = clamp(softplus(dt_raw_d + dt_bias_d), dt_min, dt_max);
+ *   3. y = ssd_bidir_fwd_x2(x_d, dt, A, B, C, D);
+ *   4. out = y SiLU(z) / sqrt(mean_c((y SiLU(z))^2) + norm_eps) * norm_w over
+ *      the H*P channels of each token.
+ *   xbc     (batch, seqlen, nheads*headdim + 2*ngroups*dstate)   io
+ *   z       (batch, seqlen, nheads, headdim)                     io
+ *   dt_raw  (2, batch, seqlen, nheads)                           io
+ *   conv_w  (2, nheads*headdim + 2*ngroups*dstate, conv_k)       fp32, conv_k in 1..4
+ *   conv_b  (2, nheads*headdim + 2*ngroups*dstate)               fp32
+ *   dt_bias, A, D (2, nheads) fp32;  norm_w (nheads*headdim) fp32
+ *   out     (batch, seqlen, nheads, headdim)                     io
+ * The intermediates (u, dt, y) are stored in the I/O dtype in the workspace
+ * (ssd_workspace_bytes with SSD_OP_MIXER_BLOCK). Four launches: conv, dt,
+ * mixer, norm. */
+int ssd_mixer_block_fwd(const void *xbc, const void *z, const void *dt_raw, const float *conv_w,
+                        const float *conv_b, int conv_k, const float *dt_bias, float dt_min, float dt_max,
+                        const float *A, const float *D, const float *norm_w, float norm_eps, void *out,
+                        int batch, int seqlen, int nheads, int headdim, int dstate, int ngroups, int dtype,
+                        void *workspace, size_t ws_bytes, void *stream);
 
 /* ssd_prefix_state for several layers at once (block diffusion keeps one
  * cached forward state per layer; "Training Hybrid Block Diffusion Language

@@ -10,6 +10,11 @@ steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME] [--path auto|simt|chunked|fused|segmented|pair]
+                  [--op bidir|bwd|block]
+
+--op bwd times the backward pass (ssd_bidir_bwd) and --op block the mixer
+with its conv1d + SiLU, dt and gated-norm steps (ssd_mixer_block_fwd) at the
+same workload's sizes; each prints its own metric.
 
 Under torchrun every rank runs the same per-GPU workload (independent
 batches: weak scaling, no collective on the data path); rank 0 prints one
@@ -382,6 +387,78 @@ def bench_blockstep(args, w, dev):
     print(json.dumps(line), flush=True)
 
 
+def bench_op(args, w, dev, world, rank):
+    """The backward pass (--op bwd, one ssd_bidir_bwd call per step) or the
+    mixer block (--op block, one ssd_mixer_block_fwd call per step) at a
+    workload's sizes, on inputs resident in HBM, CUDA events on the launching
+    stream. roofline: algorithmic HBM bytes (inputs read once, outputs written
+    once; intermediates and the backward's saved states are not algorithmic)."""
+    import torch
+    import bidirectional_mamba_ssd_b200 as ssd
+    import ssd_inputs as si
+    io = 2 if w.dtype == "bf16" else 4
+    tok = w.batch * w.seqlen
+    HP, GN, H = w.nheads * w.headdim, w.ngroups * w.dstate, w.nheads
+    if args.op == "bwd":
+        inp = si.workload_inputs(w, seed=rank_seed(rank), device=dev)
+        g = torch.Generator(device=dev).manual_seed(rank_seed(rank) + 1)
+        dy = torch.randn(inp["x"].shape, generator=g, device=dev).to(inp["x"].dtype)
+        names = ("x", "dt", "A", "B", "C", "D")
+        ws = ssd.Workspace(dev)
+
+        def step():
+            ssd.ssd_bidir_bwd(*(inp[n] for n in names), dy, workspace=ws)
+        metric = "bidir SSD backward tokens/s (fp32 gradients of x, dt, A, B, C, D)"
+        nbytes = io * tok * (2 * HP + 2 * H + 4 * GN) + 4 * tok * (HP + 2 * H + 4 * GN) + 4 * 8 * H
+        kernel, launches = "bwd_scan_kernel", 1
+    else:
+        bi = si.block_inputs(w, seed=rank_seed(rank), device=dev)
+        ws = ssd.Workspace(dev)
+
+        def step():
+            ssd.ssd_mixer_block_fwd(bi["xbc"], bi["z"], bi["dt_raw"], bi["conv_w"], bi["conv_b"], bi["dt_bias"],
+                                    bi["A"], bi["D"], bi["norm_w"], w.nheads, w.ngroups, w.dstate,
+                                    dt_min=1e-3, dt_max=0.1, workspace=ws)
+        metric = "bidir Mamba-2 mixer block tokens/s (conv1d + SiLU, dt, mixer, gated RMS norm)"
+        nbytes = io * tok * (HP + 2 * GN + HP + 2 * H + HP) + 4 * (2 * (HP + 2 * GN) * (4 + 1) + 6 * H + HP)
+        kernel, launches = "conv_silu_kernel + dt_prep_kernel + tc_pair_kernel + gated_rmsnorm_kernel", 4
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ws.status() != 0:
+        raise SystemExit("device status after warm-up")
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = job_time_ms(ev0.elapsed_time(ev1), world, dev)
+    if rank != 0:
+        return
+    ms_step = ms / args.steps
+    peaks = measured_peaks()
+    achieved = nbytes / (ms_step / 1e3) / 1e9
+    line = {"metric": metric, "value": round(job_throughput(w.tokens, args.steps, world, ms), 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "op": args.op, **{k: getattr(w, k) for k in
+                       ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups")},
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "peak_source": f"{peaks['source']} STREAM-copy HBM GB/s",
+                         "algorithmic_bytes_per_launch": nbytes, "kernel": kernel, "traffic": None},
+            "gpu_launches": launches * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -390,6 +467,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--path", default="auto", choices=list(PATH_IDS))
+    ap.add_argument("--op", default="bidir", choices=["bidir", "bwd", "block"],
+                    help="bidir: the mixer (default, the headline); bwd: its backward pass (ssd_bidir_bwd); "
+                         "block: the mixer with conv, dt and gated norm (ssd_mixer_block_fwd)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--record-traffic", metavar="CSV",
@@ -411,6 +491,8 @@ def main():
     import ssd_inputs as si
     w = si.WORKLOADS[args.workload]
     if args.impl == "reference":
+        if args.op != "bidir":
+            ap.error("--impl reference times the mixer (--op bidir) only")
         run_reference(args, w)
         return
 
@@ -428,6 +510,9 @@ def main():
     import bidirectional_mamba_ssd_b200 as ssd
     if w.block:
         bench_blockstep(args, w, dev)
+        return
+    if args.op != "bidir":
+        bench_op(args, w, dev, world, rank)
         return
     path = PATH_IDS[args.path]
     if path == 0:

@@ -67,6 +67,10 @@ WORKLOADS = {
         Workload("tiny_fp32_L128", 1, 128, 4, 64, 64, 4, 64, "f32"),
         # DiffMamba ~130M mixer: d_model 768, expand 2 -> 24 heads x 64, per-head B/C
         Workload("mixer130m_b32_L1024", 32, 1024, 24, 64, 128, 24, 256, "bf16"),
+        # the same shape at batch 4 and 8 (profiler captures of the backward
+        # and of the mixer block, a few GB on the device)
+        Workload("mixer130m_b4_L1024", 4, 1024, 24, 64, 128, 24, 256, "bf16"),
+        Workload("mixer130m_b8_L1024", 8, 1024, 24, 64, 128, 24, 256, "bf16"),
         # the same with B/C shared by all heads (ngroups 1)
         Workload("mixer130m_b32_L1024_g1", 32, 1024, 24, 64, 128, 1, 256, "bf16"),
         # LM1B packed-128, batch 512, B/C shared across heads
@@ -169,3 +173,32 @@ def blockstep_inputs(batch, prefix_len, block, steps, nheads, headdim, dstate, n
 def to_f64(t):
     """Exact float64 copy of a (possibly bf16, possibly device) tensor as numpy."""
     return t.detach().to("cpu", torch.float64).numpy()
+
+
+def block_inputs(w: Workload, conv_k: int = 4, seed=0, device="cpu"):
+    """Inputs of the mixer block (ssd_mixer_block_fwd) at a workload's sizes.
+
+    Draw order: xbc (the projected x, B, C channels) ~ N(0, 1), z ~ N(0, 1),
+    dt_raw (2, batch, L, H) ~ N(0, 1); then per direction: conv_w (Cin, K)
+    and conv_b (Cin) ~ U(-1/sqrt(K), 1/sqrt(K)) (the usual depthwise conv
+    initialisation), dt_bias (H) ~ U(-7, -2.3), A = -exp(U(log 1, log 16)),
+    D ~ N(0, 1); norm_w = 1. Activations are rounded to the I/O dtype;
+    parameters are fp32."""
+    io = DTYPES[w.dtype]
+    g = _gen(device, seed)
+    HP, GN = w.nheads * w.headdim, w.ngroups * w.dstate
+    cin = HP + 2 * GN
+    xbc = torch.randn(w.batch, w.seqlen, cin, generator=g, device=device).to(io)
+    z = torch.randn(w.batch, w.seqlen, w.nheads, w.headdim, generator=g, device=device).to(io)
+    dt_raw = torch.randn(2, w.batch, w.seqlen, w.nheads, generator=g, device=device).to(io)
+    bound = 1.0 / (conv_k ** 0.5)
+    cw, cb, db, As, Ds = [], [], [], [], []
+    for _d in range(2):
+        cw.append((torch.rand(cin, conv_k, generator=g, device=device) * 2 - 1) * bound)
+        cb.append((torch.rand(cin, generator=g, device=device) * 2 - 1) * bound)
+        db.append(torch.rand(w.nheads, generator=g, device=device) * 4.7 - 7.0)
+        As.append(_A(g, w.nheads, device))
+        Ds.append(torch.randn(w.nheads, generator=g, device=device))
+    return dict(xbc=xbc, z=z, dt_raw=dt_raw, conv_w=torch.stack(cw).contiguous(), conv_b=torch.stack(cb).contiguous(),
+                dt_bias=torch.stack(db).contiguous(), A=torch.stack(As).float().contiguous(),
+                D=torch.stack(Ds).contiguous(), norm_w=torch.ones(HP, device=device))

@@ -11,7 +11,9 @@
 // tile are added in fp32: the direction that reaches the tile first (the
 // forward one on the left half of the sequence, the reverse one on the right
 // half) stores Y + e Yo as an fp32 partial in global memory, which stays in
-// L2, and publishes it with a flag; the other direction adds it to its own
+// L2, and signals it by arriving on a barrier in the other CTA's shared
+// memory (one barrier per unit parity and tile); the other direction waits on
+// that barrier in its own shared memory, adds the partial to its own
 // Y + e Yo, adds (D_f + D_b) x, rounds once to bf16, stores the tile with TMA,
 // and drops the partial's lines from L2 without a write-back. Addition in
 // fp32 commutes, so the sum does not depend on which direction came first.
@@ -30,19 +32,21 @@
 //   warps 2..5   group C: the step's decay sums and mask vectors, the state
 //                chain H <- exp(A sum dt) H + S (fp32 registers, bf16 copy for
 //                the C.H MMA) and diag(w) X
-//   warps 6..9   group A and warps 10..13 group B: the masked matrix (half of
-//                each 32-column block each, written back into the G buffer as
-//                bf16, the A operand of Y = M X from TMEM), then the previous
-//                step's output (half of the columns each)
+//   warps 6..9   group A and warps 10..13 group B: the masked matrix (A the
+//                32-column blocks 0 and 2, B blocks 1 and 3, written back into
+//                the G buffer as bf16, the A operand of Y = M X from TMEM),
+//                then the previous step's output (half of the columns each)
 // In every group thread r owns tile row r = 32 * (warp % 4) + lane.
 //
-// Partial slots and flags are indexed by (cluster, unit parity, tile): a
-// direction writes a slot for unit j + 2 only after reading the other
-// direction's partials of unit j + 1, which the other direction wrote after
-// it had read every partial of unit j. The barrier and flag protocol is
-// modelled on the CPU (tests/test_pair_protocol.py). Every wait, mbarrier or
-// flag, is bounded in time; an expired wait sets the workspace's timeout flag
-// and the CTA runs to its end without storing.
+// Partial slots and their barriers are indexed by (cluster, unit parity,
+// tile): a direction writes a slot for unit j + 2 only after reading the
+// other direction's partials of unit j + 1, which the other direction wrote
+// after it had read every partial of unit j, so a barrier is never arrived on
+// twice before its waiters saw the first phase. The barrier protocol is modelled on
+// the CPU (tests/test_pair_protocol.py). Every wait is bounded in time; an
+// expired wait sets the workspace's timeout flag and the CTA runs to its end
+// without storing. Both CTAs meet at a cluster barrier before either exits,
+// so no arrival targets the shared memory of a CTA that has left.
 #include <cuda.h>
 #include <stdint.h>
 
@@ -64,6 +68,7 @@ constexpr uint32_t kSlab = 16384;           // 128 rows x 128 bytes
 constexpr int kRing = 4;                    // C/B slots of 32 KB: two tiles
 constexpr int kXS = 3;                      // x slots
 constexpr int kThreads = 448;
+constexpr int kMaxNt = 256;                 // tiles per sequence (one partial barrier per tile and unit parity)
 constexpr size_t kPartFloats = (size_t)kTile * kP;   // one fp32 partial tile (32 KB)
 
 struct PairParams {
@@ -72,7 +77,6 @@ struct PairParams {
     const float *D;            // (2, H)
     const float *init;         // (batch, H, 64, N) forward start state or nullptr
     const float *rinit;        // (batch, H, 64, N) reverse start state (at the sequence end) or nullptr
-    unsigned int *flags;       // (clusters, 2, nt): unit + 1 once the partial of that slot is stored
     float *part;               // (clusters, 2, nt) fp32 partial tiles, 16 column chunks x 128 rows x 4
     DeviceStatus *status;
     int batch, L, H, G, nt, units;
@@ -112,9 +116,57 @@ struct PSmem {
     static constexpr uint32_t h = x0 + kXS * kSlab;        // bf16 (N, 64) state
     static constexpr uint32_t xw = h + N * 128;            // diag(w) X
     static constexpr uint32_t small = xw + kSlab;
-    static constexpr uint32_t bytes = small + 512 + 2 * sizeof(StepVec);
+    static constexpr uint32_t pbar = small + 512 + 2 * sizeof(StepVec);   // (unit parity, tile) barriers
+    static constexpr uint32_t bytes = pbar + 8 * 2 * kMaxNt;
     static __device__ __forceinline__ uint32_t xslot(uint32_t j) { return x0 + j * kSlab; }
 };
+
+
+// ---- partial-ready barriers: a release arrival on the other CTA's barrier
+// (distributed shared memory) after this CTA's partial stores, and an acquire
+// wait at cluster scope on the own barrier before loading the other's partial
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t peer_addr(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+static __device__ __noinline__ bool mbar_wait_cl_loop(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                      DeviceStatus *st, uint32_t where) {
+    WaitClock clock;
+    while (true) {
+        if (*abort_flag) return false;
+        if (mbar_try_wait_cl(bar, parity)) return true;
+        if (clock.expired(1000000000ull)) {
+            *abort_flag = 1;
+            report_timeout(st, where);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                             DeviceStatus *st, uint32_t where) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    return mbar_wait_cl_loop(bar, parity, abort_flag, st, where);
+}
 
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -145,19 +197,18 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const bool two = i == B_M_READY || i == B_M_READY + 1 || i == B_VEC_FREE || i == B_VEC_FREE + 1;
             mbar_init(bar(i), two ? 2 : 1);
         }
-        fence_mbar_init();
     }
+    // the partial-ready barriers: one per (unit parity, tile), completed by the
+    // other CTA's arrival once it has stored its partial of that tile
+    for (int q = tid; q < 2 * p.nt; q += kThreads) mbar_init(base + S::pbar + 8 * q, 1);
+    fence_mbar_init();
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
     // the kernel ahead in the stream has finished before any global access
     grid_dependency_wait();
-    // the cluster's flags start at zero (a previous call left unit numbers in
-    // them); both CTAs pass the cluster barrier before either uses a flag
-    unsigned int *cflags = p.flags + (size_t)cl * 2 * nt;
-    if (dir == 0)
-        for (int q = tid; q < 2 * nt; q += kThreads) cflags[q] = 0u;
+    // both CTAs' barriers are initialised before either arrives on the other's
     tc_fence_before();
     cluster_sync_all();
     tc_fence_after();
@@ -416,12 +467,9 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const bool second = !first_at(k);
             const int j = (u - cl) / ncl;
             const size_t slot = ((size_t)cl * 2 + (j & 1)) * nt + i;
-            unsigned int *flag = p.flags + slot;
+            const uint32_t pb = base + S::pbar + 8 * ((uint32_t)(j & 1) * nt + i);
             float *part = p.part + slot * kPartFloats;
-            if (second) {
-                if (row == 0) flag_wait(flag, (unsigned int)u + 1u, abort_flag, p.status, 801);
-                sync_g();
-            }
+            if (second) mbar_wait_cl(pb, (uint32_t)(j >> 1) & 1u, abort_flag, p.status, 801);
             // the other direction's partial for this thread's 32 columns, loaded
             // before the wait for Y so its L2 latency overlaps it
             float4 pv[8];
@@ -497,7 +545,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             if (is_b && row == 0) {
                 mbar_arrive(bar(B_Y_FREE));
                 if (!second) {
-                    if (!*abort_flag) flag_release(flag, (unsigned int)u + 1u);
+                    if (!*abort_flag) mbar_arrive_peer(peer_addr(pb, cluster_rank() ^ 1u));
                 } else {
                     if (!*abort_flag) {
                         tma_store_4d(&tm_out, base + S::xslot(xs), 0, h, i * kTile, b);
@@ -568,10 +616,10 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     // ------------------------------------------------------------ teardown
     tc_fence_before();
     __syncthreads();
+    // neither CTA leaves while the other may still arrive on its barriers
+    cluster_sync_all();
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
-
-size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 // Clusters a call uses at most: one per two SMs, no more than there are units.
 int pair_clusters_max(int units) {
@@ -580,7 +628,6 @@ int pair_clusters_max(int units) {
     return units < c ? units : c;
 }
 
-size_t flags_bytes(int clusters, int nt) { return align256((size_t)clusters * 2 * nt * sizeof(unsigned int)); }
 
 template <int N>
 cudaError_t run_pair(const TcArgs &a, cudaStream_t stream) {
@@ -597,10 +644,9 @@ cudaError_t run_pair(const TcArgs &a, cudaStream_t stream) {
     p.rinit = a.rinit;
     char *ws = static_cast<char *>(a.workspace);
     p.status = reinterpret_cast<DeviceStatus *>(ws);
-    p.flags = reinterpret_cast<unsigned int *>(ws + kStatusBytes);
     // partial tiles start on a 256-byte boundary whatever the workspace's own
     // alignment (the L2 discard works on whole 128-byte lines)
-    const uintptr_t pa = reinterpret_cast<uintptr_t>(ws + kStatusBytes + flags_bytes(cmax, nt));
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(ws + kStatusBytes);
     p.part = reinterpret_cast<float *>((pa + 255) & ~(uintptr_t)255);
     p.batch = a.batch; p.L = a.L; p.H = a.H; p.G = a.G; p.nt = nt; p.units = units;
 
@@ -649,12 +695,13 @@ size_t tc_pair_scratch_bytes(int batch, int L, int H, int N) {
     const int nt = (L + kTile - 1) / kTile;
     const int cmax = pair_clusters_max(batch * H);
     if (cmax < 1 || nt < 1) return 0;
-    return flags_bytes(cmax, nt) + 256 + (size_t)cmax * 2 * nt * kPartFloats * sizeof(float);
+    return 256 + (size_t)cmax * 2 * nt * kPartFloats * sizeof(float);
 }
 
 bool tc_pair_supported(int batch, int L, int H, int G, int N) {
     (void)G;
     if (L <= kTile || batch <= 0) return false;     // at least two tiles per sequence
+    if ((L + kTile - 1) / kTile > kMaxNt) return false;
     if (N != 64 && N != 128) return false;
     return (long long)batch * H < (1ll << 31);
 }

@@ -96,7 +96,7 @@ enum {
                               each CTA runs one scan direction over the tiles in that
                               direction's order, carrying its state on chip; a tile's two
                               directions meet through an fp32 partial in the workspace.
-                              seqlen > 128 (at least two 128-token tiles) */
+                              128 < seqlen <= 32768 (2 to 256 128-token tiles) */
 };
 
 /* The SSD_PATH_* that ssd_bidir_fwd (SSD_PATH_AUTO) runs for these sizes, or
@@ -276,7 +276,7 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
  * ssd_mixer_block_fwd):
  *   out_t = yf_t(x2[0]) + yb_t(x2[1]) + D_f x2[0]_t + D_b x2[1]_t
  *   x2   (2, batch, seqlen, nheads, headdim)   io; other arguments as ssd_bidir_fwd
- * bf16 with seqlen > 128 runs the two-CTA tensor-core kernel, otherwise the
+ * bf16 with 128 < seqlen <= 32768 runs the two-CTA tensor-core kernel, otherwise the
  * sequential scan. The two directions' fp32 results are added in an order
  * that does not depend on which direction finishes first. */
 int ssd_bidir_fwd_x2(const void *x2, const void *dt, const float *A, const void *B, const void *C,

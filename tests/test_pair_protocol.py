@@ -6,22 +6,24 @@ unit's 128-token tiles left to right, the reverse CTA right to left, each
 with its own producer, MMA issuer, state-chain group (C) and mask/output
 groups (A, B). A tile's two directions meet through global memory: the
 direction that reaches the tile first stores its fp32 partial output and
-then a flag holding unit + 1 (slot by unit parity and tile); the other
-polls the flag, adds the partial and stores the bf16 output. The model
-takes the kernel's mbarrier waits and arrivals, named-barrier syncs, TMA
-loads, MMA commits (one in-order tensor pipe per CTA), flag stores and polls
-and TMA stores, in the kernel's order, with random heavy-tailed delays on
-every asynchronous completion and random stepping order.
+then arrives on a barrier in the other CTA's shared memory (one barrier and
+one partial slot per unit parity and tile); the other waits on that barrier,
+adds the partial and stores the bf16 output. The model takes the kernel's
+mbarrier waits and arrivals (those across the pair included), named-barrier
+syncs, TMA loads, MMA commits (one in-order tensor pipe per CTA) and TMA
+stores, in the kernel's order, with random heavy-tailed delays on every
+asynchronous completion and random stepping order.
 
-Each schedule is checked for phase overrun (a barrier or flag moving two
-steps past a waiter), deadlock (within a CTA or across the pair) and stale
+Each schedule is checked for phase overrun (a barrier moving two phases
+past a waiter), deadlock (within a CTA or across the pair) and stale
 reads of every buffer: the B/C ring, the x slots, H, diag(w) X, the TMEM
 accumulators (G double-buffered, Y, Yo double-buffered, S), the per-tile
 vectors and the partial slots in global memory.
 
 Planted variants that the model must catch: partial slots not split by unit
 parity (the forward CTA overwrites a partial before the reverse CTA has read
-it), a single Yo accumulator (the next tile's C.H overwrites it before the
+it), a partial barrier waited on with the unit's own phase instead of the
+unit pair's, a single Yo accumulator (the next tile's C.H overwrites it before the
 output epilogue has read it) and a single M_READY barrier (two mask phases
 complete under one parity wait).
 """
@@ -35,13 +37,14 @@ class Pair(Sched):
     both CTAs. init[d]: the direction starts from a given state (else zero,
     and the unit's first tile has no C.H term)."""
     def __init__(self, nt, units, seed, heavy=0.1, init=(False, False), par_slots=True, yo_double=True,
-                 m_per_buf=True):
+                 m_per_buf=True, phase_pairs=True):
         super().__init__(seed, heavy)
         self.nt, self.units = nt, units
         self.init = init
         self.par_slots = par_slots      # partial slots split by unit parity
         self.yo_double = yo_double      # two Yo accumulators
         self.m_per_buf = m_per_buf      # one M_READY barrier per G buffer
+        self.phase_pairs = phase_pairs  # a partial barrier completes once per two units
 
     def steps(self, d):
         """(n, j, u, k, i) of every step of direction d (0 forward, 1 reverse)."""
@@ -63,6 +66,12 @@ class Pair(Sched):
 
     def slot(self, j, i):
         return ((j & 1) if self.par_slots else 0, i)
+
+    def part_bar(self, d, j, i):
+        """the partial barrier of tile i, unit j, in CTA d's shared memory, and
+        the phase its waiters wait for (one completion per unit of the slot)"""
+        par, t = self.slot(j, i)
+        return 'fb'[d] + '.PART%d_%d' % (par, t), (j >> 1) if self.par_slots and self.phase_pairs else j
 
     def yo(self, n):
         return n & 1 if self.yo_double else 0
@@ -187,9 +196,8 @@ def group_ab(S, d, is_b):
         second = not S.first(d, k)
         slot = S.slot(j, i)
         if second:
-            # each group's leader polls the flag, then its group syncs
-            yield ('gwait', ('flag',) + slot, u + 1)
-            yield ('sync', g, 1)
+            # every thread waits on the barrier in its own CTA
+            yield ('wait',) + S.part_bar(d, j, i)
         yield ('wait', p + 'Y_READY', n)
         yield ('read', (p + 'Y', half), ('Y', d, u, i))
         if not S.hzero(d, k):
@@ -211,7 +219,8 @@ def group_ab(S, d, is_b):
                        [(('out', u, i), ('y', u, i))])
                 yield ('store_wait',)
             else:
-                yield ('gset', ('flag',) + slot, u + 1)
+                # release arrival on the other CTA's barrier of this slot
+                yield ('arrive', S.part_bar(1 - d, j, i)[0])
             yield ('arrive', p + 'X_EMPTY%d' % xs)
 
     prev = None
@@ -280,3 +289,8 @@ def test_model_catches_single_yo_accumulator():
 def test_model_catches_single_mask_barrier():
     fails = _schedules(300, m_per_buf=False)
     assert fails and any("overrun on" in f and "M_READY" in f for f in fails)
+
+
+def test_model_catches_partial_barrier_phase_per_unit():
+    fails = _schedules(200, phase_pairs=False)
+    assert fails and any("deadlock" in f or "overrun" in f for f in fails)

@@ -364,7 +364,8 @@ def bench_blockstep(args, w, dev):
             "frac": round(achieved / peaks["hbm_gbs"], 4),
             "peak_source": f"{peaks['source']} STREAM-copy HBM GB/s",
             "algorithmic_bytes_per_launch": block_bytes,
-            "kernel": "tc_fused_kernel (32 block steps + the commit, one CUDA graph; bytes of the whole block)",
+            "kernel": "blockstep_kernel (the block steps) + tc_fused_kernel (the commit), one CUDA graph; "
+                      "bytes of the whole block",
             "traffic": None}
     line = {"metric": "block-diffusion denoising tokens/s (block x steps), cached prefix state",
             "value": round(tok / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
@@ -380,9 +381,12 @@ def bench_blockstep(args, w, dev):
             "prefill": {"ms": round(prefill_ms, 4), "tokens_per_s": round(w.batch * w.seqlen / (prefill_ms / 1e3), 1),
                         "algorithmic_bytes": prefill_bytes,
                         "hbm_frac": round(prefill_bytes / (prefill_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
-            # the fused kernel (one launch per step or commit) from 64 (batch, head)
-            # units, else the chunked kernels (3 per step, 2 per commit)
-            "gpu_launches": args.steps * ((w.steps + 1) if w.batch * w.nheads >= 64 else (3 * w.steps + 2)),
+            # one launch per block step (the one-tile kernel for blocks of at most 64
+            # tokens, else the fused kernel from 64 (batch, head) units, else 3
+            # chunked kernels) and one per commit (fused kernel; 2 chunked kernels
+            # under 64 units)
+            "gpu_launches": args.steps * ((w.steps if w.block <= 64 or w.batch * w.nheads >= 64 else 3 * w.steps)
+                                          + (1 if w.batch * w.nheads >= 64 else 2)),
             "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
 

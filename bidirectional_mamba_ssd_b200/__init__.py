@@ -33,7 +33,7 @@ import torch
 
 from . import _lib as _c
 from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED, SSD_PATH_SEGMENTED,  # noqa: F401
-                   SSD_PATH_PAIR,
+                   SSD_PATH_PAIR, SSD_PATH_BLOCK,
                    SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA,
                    SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT, SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE,
                    SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD, SSD_OP_BIDIR_FWD_X2, SSD_OP_MIXER_BLOCK)
@@ -255,7 +255,8 @@ def ssd_prefix_state_layers(x, dt, A, B, init=None, out=None, *, chunk: int = 25
 def ssd_block_step(x, dt, A, B, C, D, prefix_state, out=None, *, path: int = SSD_PATH_AUTO,
                    workspace: Workspace | None = None):
     """One block-diffusion step on the active block (include/ssd_bidir.h: ssd_block_step,
-    ssd_block_step_path). `path`: as for ssd_bidir_fwd."""
+    ssd_block_step_path). `path`: SSD_PATH_AUTO, SIMT, CHUNKED, FUSED or BLOCK (the
+    one-tile kernel, bf16 blocks of at most 64 tokens)."""
     _need(x, "x", ndim=4)
     dev, io = x.device, x.dtype
     if io not in _DT:

@@ -331,7 +331,7 @@ int ssd_block_step_path(const void *x, const void *dt, const float *A, const voi
                         void *workspace, size_t ws_bytes, void *stream) {
     int rc = check_shape(batch, blk_len, nheads, headdim, dstate, ngroups, 64, dtype, false);
     if (rc != SSD_OK) return rc;
-    if (path < SSD_PATH_AUTO || path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
+    if ((path < SSD_PATH_AUTO || path > SSD_PATH_FUSED) && path != SSD_PATH_BLOCK) return SSD_ERR_INVALID_ARG;
     if (!workspace) return SSD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
     if (ws_bytes < ssd_workspace_bytes(SSD_OP_BLOCK_STEP, batch, blk_len, nheads, headdim, dstate,
@@ -344,9 +344,24 @@ int ssd_block_step_path(const void *x, const void *dt, const float *A, const voi
         return SSD_ERR_INVALID_ARG;
     if (prefix_state && !aligned16(prefix_state)) return SSD_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (path == SSD_PATH_AUTO && dtype == SSD_BF16)
-        path = (long long)batch * nheads >= kFusedMinUnits ? SSD_PATH_FUSED : SSD_PATH_CHUNKED;
-    if ((path == SSD_PATH_CHUNKED || path == SSD_PATH_FUSED) && dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    if (path == SSD_PATH_AUTO && dtype == SSD_BF16) {
+        if (ssd::tc_blockstep_supported(batch, blk_len, nheads, ngroups, dstate))
+            path = SSD_PATH_BLOCK;
+        else
+            path = (long long)batch * nheads >= kFusedMinUnits ? SSD_PATH_FUSED : SSD_PATH_CHUNKED;
+    }
+    if ((path == SSD_PATH_CHUNKED || path == SSD_PATH_FUSED || path == SSD_PATH_BLOCK) && dtype != SSD_BF16)
+        return SSD_ERR_UNSUPPORTED;
+    if (path == SSD_PATH_BLOCK) {
+        if (!ssd::tc_blockstep_supported(batch, blk_len, nheads, ngroups, dstate)) return SSD_ERR_UNSUPPORTED;
+        // the two directions stacked as one tile's rows, forward from the cached state
+        TcArgs t{};
+        t.x = x; t.dt = dt; t.A = A; t.B = B; t.C = C; t.D = D; t.out = out;
+        t.init = prefix_state;
+        t.workspace = workspace; t.ws_bytes = ws_bytes;
+        t.batch = batch; t.L = blk_len; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
+        return to_status(ssd::launch_tc_blockstep(t, s));
+    }
     if (path == SSD_PATH_CHUNKED || path == SSD_PATH_FUSED) {
         // both scans over the block, the forward one starting from the cached
         // state (zero if none) and the reverse one from zero

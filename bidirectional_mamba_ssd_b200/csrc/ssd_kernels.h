@@ -123,6 +123,12 @@ size_t tc_pair_scratch_bytes(int batch, int L, int H, int N);
 bool tc_pair_supported(int batch, int L, int H, int G, int N);
 cudaError_t launch_tc_pair(const TcArgs &a, cudaStream_t stream);
 
+// One-tile block step (ssd_blockstep.cu): both scans over a block of at most
+// 64 tokens, forward from a.init (or zero), reverse from zero; bf16, ndir 2,
+// one CTA per (batch, head). Needs only the workspace's status header.
+bool tc_blockstep_supported(int batch, int T, int H, int G, int N);
+cudaError_t launch_tc_blockstep(const TcArgs &a, cudaStream_t stream);
+
 // Long sequences with fewer (batch, head) units than SMs: each sequence split
 // into S segments (seg_count: the fewest, S dividing L, that fill 4/5 of `sms`
 // SMs in one round; 1 = none), states handed across segments,

@@ -92,11 +92,14 @@ enum {
                               segments (S divides seqlen); forward and reverse segment states
                               (fused kernel, state modes), a segment scan, then the fused
                               kernel on the segments seeded with the handed-over states */
-    SSD_PATH_PAIR = 5      /* tensor-core path, one cluster of two CTAs per (batch, head):
+    SSD_PATH_PAIR = 5,     /* tensor-core path, one cluster of two CTAs per (batch, head):
                               each CTA runs one scan direction over the tiles in that
                               direction's order, carrying its state on chip; a tile's two
                               directions meet through an fp32 partial in the workspace.
                               128 < seqlen <= 32768 (2 to 256 128-token tiles) */
+    SSD_PATH_BLOCK = 6     /* ssd_block_step only: one CTA per (batch, head) over a block of at
+                              most 64 tokens, both directions stacked as the rows of one
+                              tensor-core tile */
 };
 
 /* The SSD_PATH_* that ssd_bidir_fwd (SSD_PATH_AUTO) runs for these sizes, or
@@ -185,16 +188,19 @@ int ssd_prefix_state_path(const void *x, const void *dt, const float *A, const v
  *   prefix_state (batch, nheads, headdim, dstate)         fp32, NULL = zero prefix
  *   out          (batch, blk_len, nheads, headdim)        io, overwritten
  * bf16 I/O runs on the tensor cores (the prefix state enters the C.H product
- * as a bf16 operand): with at least 64 (batch, head) units the fused
- * bidirectional kernel with its forward scan seeded from prefix_state, else
- * the chunked kernels; fp32 I/O runs the sequential fp32 scan. */
+ * as a bf16 operand): blocks of at most 64 tokens on the one-tile kernel
+ * (SSD_PATH_BLOCK), longer blocks with at least 64 (batch, head) units on the
+ * fused bidirectional kernel with its forward scan seeded from prefix_state,
+ * else on the chunked kernels; fp32 I/O runs the sequential fp32 scan. */
 int ssd_block_step(const void *x, const void *dt, const float *A, const void *B,
                    const void *C, const float *D, const float *prefix_state, void *out,
                    int batch, int blk_len, int nheads, int headdim, int dstate,
                    int ngroups, int dtype,
                    void *workspace, size_t ws_bytes, void *stream);
 
-/* ssd_block_step with an explicit kernel choice, as ssd_prefix_state_path. */
+/* ssd_block_step with an explicit kernel choice, as ssd_prefix_state_path:
+ * SSD_PATH_AUTO, SIMT, CHUNKED, FUSED or BLOCK (bf16, blk_len <= 64;
+ * SSD_ERR_UNSUPPORTED otherwise). */
 int ssd_block_step_path(const void *x, const void *dt, const float *A, const void *B,
                         const void *C, const float *D, const float *prefix_state, void *out,
                         int batch, int blk_len, int nheads, int headdim, int dstate,

@@ -150,12 +150,22 @@ blockstep_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         tma_load_4d(base + S::x, &tm_x, bar(B_X), 0, h, 0, b);
         tma_load_4d(base + S::x + 8192, &tm_x, bar(B_X), 0, h, 0, b);
     }
-    // decay sums and mask vectors (warps 0..3: forward rows in warps 0, 1,
-    // reverse rows in warps 2, 3); tokens past the block's end have dt = 0
+    // every global load of the threads in flight at once: dt of the row
+    // (warps 0..3: forward rows in warps 0, 1, reverse rows in warps 2, 3;
+    // tokens past the block's end have dt = 0) and this thread's 32 values of
+    // the cached state, row n of H^T (H[p][n] for p in its half of the 64)
     const float A = p.A[(fwd ? 0 : p.H) + h];
+    float v = 0.f;
+    if (ch == 0 && t < p.T) v = __bfloat162float(p.dt[(((size_t)(fwd ? 0 : 1) * p.batch + b) * p.T + t) * p.H + h]);
+    const int n = tid & 127, half = tid >> 7;
+    float hv[32];
+    if (has_h && n < N) {
+        const float *ip = p.prefix + (size_t)u * kP * N + n + (size_t)half * 32 * N;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) hv[j] = __ldg(ip + (size_t)j * N);
+    }
+    // decay sums and mask vectors
     if (ch == 0) {
-        float v = 0.f;
-        if (t < p.T) v = __bfloat162float(p.dt[(((size_t)(fwd ? 0 : 1) * p.batch + b) * p.T + t) * p.H + h]);
         float tot;
         const float pf = scan64(v, lane, q & 1, part + (fwd ? 0 : 2), tot);
         // a_t: decay sum from the block's start (forward) or end (reverse) through t
@@ -168,13 +178,7 @@ blockstep_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         Vcol[row] = __expf(Va[fwd ? (row | 31) : (row & ~31)] - a) * v;
     }
     if (has_h) {
-        // row n of H^T: H[p][n] for p in this thread's 32 of the 64, as bf16
-        const int n = tid & 127, half = tid >> 7;
         if (n < N) {
-            const float *ip = p.prefix + (size_t)u * kP * N + n + (size_t)half * 32 * N;
-            float hv[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) hv[j] = ip[(size_t)j * N];
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 *reinterpret_cast<uint4 *>(g + S::h + sw128_offset(n, half * 4 + c)) =

@@ -8,9 +8,12 @@
 // states h_t = a_t h_{t-1} + dt_t B_t x_t^T (N x P) and their adjoints
 // g_t = C_t dy_t^T + a_{t'} g_{t'} (t' the token after t in the scan's
 // order), one CTA runs
-//   1. the scan in its own order, storing every state h_t (fp32) to its
-//      scratch and forming dC_t = h_t dy_t on the way;
-//   2. the adjoint scan in the opposite order, forming
+//   1. the scan in its own order, storing every kRun-th state h_t (fp32) to
+//      its scratch as a checkpoint and forming dC_t = h_t dy_t on the way;
+//   2. the adjoint scan in the opposite order, one run of kRun tokens at a
+//      time: the run's states are recomputed from its checkpoint into a
+//      kRun-slot buffer (small enough to stay in L2, and each thread reads
+//      back only what it wrote), then the run's tokens form
 //      dx_t += dt_t B_t^T g_t,  dB_t += dt_t g_t x_t,
 //      ddt_t = B_t^T g_t x_t + A a_t <g_t, h_{t-1}>,  dA += dt_t a_t <g_t, h_{t-1}>.
 // The skip term adds (D_f + D_b) dy_t to dx (folded into the forward item's
@@ -24,7 +27,7 @@
 // tokens; reductions over p (dB, dC) use a transposing warp reduction that
 // leaves each lane one finished n, then one add across the quarter's two
 // warps. The grid is persistent (items loop over CTAs), so scratch is
-// L states of N x P fp32 per CTA.
+// ceil(L / kRun) checkpoints plus kRun buffer slots of N x P fp32 per CTA.
 #include "ssd_common.cuh"
 #include "ssd_kernels.h"
 
@@ -34,6 +37,8 @@ namespace {
 constexpr int kP = 64;
 constexpr int kThreads = 256;
 constexpr int kTB = 32;        // tokens staged per round
+constexpr int kRun = 8;        // tokens per checkpoint (divides kTB)
+static_assert(kTB % kRun == 0, "runs tile the staged rounds");
 
 // Sum of v[j] over the 32 lanes of a warp for NQ values j, transposed: on
 // return each lane holds the sum for one index j (transposed_index), and
@@ -79,7 +84,7 @@ struct BwdArgs {
     const void *x, *dt, *B, *C, *dy;
     const float *A, *D;
     float *dx, *ddt, *dA, *dB, *dC, *dD;
-    float *scratch;            // per CTA: L * N * 64 floats
+    float *scratch;            // per CTA: (ceil(L / kRun) + kRun) * N * 64 floats
     int batch, L, H, G;
 };
 
@@ -103,7 +108,9 @@ bwd_scan_kernel(const BwdArgs a) {
     const int items = a.batch * a.H * 2;
     const size_t dt_dir = (size_t)a.batch * L * a.H;
     const size_t bc_dir = (size_t)a.batch * L * a.G * N;
-    float *hsave = a.scratch + (size_t)blockIdx.x * L * N * kP;
+    const int nck = (L + kRun - 1) / kRun;
+    float *ckpt = a.scratch + (size_t)blockIdx.x * (nck + kRun) * N * kP;   // h after tokens kRun j + kRun - 1
+    float *runbuf = ckpt + (size_t)nck * N * kP;                            // h_{s0 - 1 + m}, m < kRun
     const int jt = transposed_index<NQ>(lane);
 
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -157,13 +164,16 @@ bwd_scan_kernel(const BwdArgs a) {
                 const float coef = dtv * xs[i * kP + p];
                 const float dyv = dys[i * kP + p];
                 const float *Bi = Bs + i * N + q * NQ;
-                float *hk = hsave + (size_t)(k0 + i) * N * kP;
                 float w[NQ];
 #pragma unroll
                 for (int j = 0; j < NQ; ++j) {
                     hs[j] = fmaf(decay, hs[j], coef * Bi[j]);
-                    hk[(size_t)(q * NQ + j) * kP + p] = hs[j];
                     w[j] = hs[j] * dyv;
+                }
+                if ((k0 + i) % kRun == kRun - 1) {
+                    float *hk = ckpt + (size_t)((k0 + i) / kRun) * N * kP;
+#pragma unroll
+                    for (int j = 0; j < NQ; ++j) hk[(size_t)(q * NQ + j) * kP + p] = hs[j];
                 }
                 // dC_t[n] = sum_p h_t[n][p] dy_t[p]
                 const float s = warp_transpose_sum<NQ>(w, lane);
@@ -179,33 +189,62 @@ bwd_scan_kernel(const BwdArgs a) {
                 else atomicAdd(a.dC + off, v);
             }
         }
-        __syncthreads();   // the states in scratch are visible to every thread
+        // (each thread reads back only the state elements it wrote: no barrier)
 
         // ---------------- 2. the adjoint scan, in the opposite order
         float gs[NQ];
 #pragma unroll
         for (int j = 0; j < NQ; ++j) gs[j] = 0.f;
         float dA_acc = 0.f, xdy_acc = 0.f;
-        for (int e0 = 0; e0 < L; e0 += kTB) {
-            // chunk of scan-order tokens [k0, k1), walked from k1 - 1 down
-            const int k1 = L - e0, k0 = max(0, k1 - kTB), nt = k1 - k0;
+        for (int c = (L - 1) / kTB; c >= 0; --c) {
+            // staged round of scan-order tokens [k0, k0 + nt), walked from the
+            // top down; rounds start at multiples of kTB, so no run straddles two
+            const int k0 = c * kTB, nt = min(kTB, L - k0);
             stage(k0, nt);
             for (int i = nt - 1; i >= 0; --i) {
                 const int k = k0 + i;
+                const int s0 = k & ~(kRun - 1);   // first token of k's run
+                if (i == nt - 1 || k % kRun == kRun - 1) {
+                    // the run's states h_{s0 - 1} .. h_{k - 1} into slots 0 .. k - s0,
+                    // from the checkpoint before the run (zero before the first token)
+                    float hr[NQ];
+                    if (s0 > 0) {
+                        const float *hc = ckpt + (size_t)(s0 / kRun - 1) * N * kP;
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) hr[j] = hc[(size_t)(q * NQ + j) * kP + p];
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) hr[j] = 0.f;
+                    }
+                    for (int m = 0; m <= k - s0; ++m) {
+                        if (m > 0) {
+                            const int ii = s0 - k0 + m - 1;   // token s0 + m - 1 in the staged round
+                            const float dtm = dts[ii];
+                            const float dec = expf(dtm * Ad);
+                            const float cf = dtm * xs[ii * kP + p];
+                            const float *Bm = Bs + ii * N + q * NQ;
+#pragma unroll
+                            for (int j = 0; j < NQ; ++j) hr[j] = fmaf(dec, hr[j], cf * Bm[j]);
+                        }
+                        float *hb = runbuf + (size_t)m * N * kP;
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) hb[(size_t)(q * NQ + j) * kP + p] = hr[j];
+                    }
+                }
                 const float dtv = dts[i];
                 const float decay = expf(dtv * Ad);
                 const float xv = xs[i * kP + p], dyv = dys[i * kP + p];
                 const float *Bi = Bs + i * N + q * NQ;
                 const float *Ci = Cs + i * N + q * NQ;
-                // h_{t-1}: the state before this token (zero before the scan's first token)
-                const float *hp = hsave + (size_t)(k > 0 ? k - 1 : 0) * N * kP;
+                // h_{t-1}: the state before this token (slot k - s0 of the run's buffer)
+                const float *hp = runbuf + (size_t)(k - s0) * N * kP;
                 float u = 0.f, ghp = 0.f;
                 float w[NQ];
 #pragma unroll
                 for (int j = 0; j < NQ; ++j) {
                     gs[j] = fmaf(Ci[j], dyv, gs[j]);
                     u = fmaf(Bi[j], gs[j], u);
-                    const float hprev = k > 0 ? hp[(size_t)(q * NQ + j) * kP + p] : 0.f;
+                    const float hprev = hp[(size_t)(q * NQ + j) * kP + p];
                     ghp = fmaf(gs[j], hprev, ghp);
                     w[j] = gs[j] * xv;
                 }
@@ -304,7 +343,8 @@ int bwd_grid(int batch, int H) {
 }
 
 size_t bwd_scratch_bytes(int batch, int L, int H, int N) {
-    return (size_t)bwd_grid(batch, H) * L * N * kP * sizeof(float);
+    const size_t nck = ((size_t)L + kRun - 1) / kRun;
+    return (size_t)bwd_grid(batch, H) * (nck + kRun) * N * kP * sizeof(float);
 }
 
 cudaError_t launch_bwd(const BwdLaunch &l, cudaStream_t stream) {

@@ -48,14 +48,17 @@ KERNEL_SOURCE = {
     "simt": ("ssd_simt.cu", "ssd_common.cuh"),
     "chunked": ("ssd_tc.cu", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
     "fused": ("ssd_fused.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
-    "segmented": ("ssd_segments.cu", "ssd_fused.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h",
-                  "ssd_common.cuh"),
+    "segmented": ("ssd_segments.cu", "ssd_fused.cu", "ssd_pair.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh",
+                  "ssd_tmap.h", "ssd_common.cuh"),
     "pair": ("ssd_pair.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
 }
 # kernels one call of each path launches (names as in ncu's "Kernel Name")
 KERNEL_NAMES = {"simt": ("scan_simt_kernel",), "chunked": ("tc_state_kernel", "tc_pass_kernel", "tc_out_kernel"),
                 "fused": ("tc_fused_kernel",), "segmented": ("tc_fused_kernel", "seg_scan_kernel"),
                 "pair": ("tc_pair_kernel",)}
+# kernels a call of the path launches on some shapes only (the segmented
+# path's last step runs the two-CTA kernel where the segments suit it)
+KERNEL_OPTIONAL = {"segmented": ("tc_pair_kernel",)}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -167,14 +170,16 @@ def record_traffic(csv_path: str, path: str, workload: str, command: str, scale:
     unit_scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
     col = {m: head.index(m) for m in ("Kernel Name", "dram__bytes_read.sum", "dram__bytes_write.sum")}
     names = KERNEL_NAMES[path]
-    per = {n: [] for n in names}
+    optional = KERNEL_OPTIONAL.get(path, ())
+    per = {n: [] for n in names + optional}
     for r in rows[2:]:
-        for n in names:
+        for n in names + optional:
             if n + "<" in r[col["Kernel Name"]] or n + "(" in r[col["Kernel Name"]]:
                 per[n].append(sum(float(r[col[m]].replace(",", "")) * unit_scale[units[col[m]]]
                                   for m in ("dram__bytes_read.sum", "dram__bytes_write.sum")))
-    if any(not v for v in per.values()):
+    if any(not per[n] for n in names):
         raise SystemExit(f"not every kernel of {names} is in {csv_path}")
+    per = {n: v for n, v in per.items() if v}
     calls = min(len(v) for v in per.values())
     d = {}
     if os.path.exists(TRAFFIC_FILE):
@@ -183,7 +188,7 @@ def record_traffic(csv_path: str, path: str, workload: str, command: str, scale:
     # every launch captured, over the calls (the kernel launched fewest times
     # is launched once per call; the segmented path launches the fused kernel thrice)
     per_call = sum(sum(v) for v in per.values()) / calls * scale
-    e = {"dram_bytes_per_launch": round(per_call), "calls_captured": calls, "kernels": list(names),
+    e = {"dram_bytes_per_launch": round(per_call), "calls_captured": calls, "kernels": list(per),
          "source_sha": kernel_source_sha(path), "command": command}
     if scale != 1.0:
         e["scaled"] = {"factor": scale, "note": note}
@@ -600,8 +605,8 @@ def main():
     roof.update({"traffic": traffic_record(path_name, w.name),
             "kernel": {"simt": "scan_simt_kernel", "chunked": "tc_state/tc_pass/tc_out kernels (whole step)",
                        "fused": "tc_fused_kernel", "pair": "tc_pair_kernel",
-                       "segmented": "tc_fused_kernel (forward state, reverse state, bidirectional) + seg_scan_kernel "
-                                    "(whole step)"}[path_name]})
+                       "segmented": "tc_fused_kernel (forward state, reverse state) + seg_scan_kernel + the "
+                                    "segments' kernel (tc_pair_kernel, else tc_fused_kernel) (whole step)"}[path_name]})
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -15,8 +15,9 @@
 //      also return (the product of their tile decays); given starting states
 //      of the whole sequence (a segment of a longer one) enter as the term
 //      from beyond its ends;
-//   4. the fused bidirectional kernel runs on the segments, its forward scan
-//      seeded with Hf_in and its reverse scan with Hb_in.
+//   4. the two-CTA kernel (the fused kernel where the segments are too long
+//      or too short for it) runs on the segments, its forward scan seeded
+//      with Hf_in and its reverse scan with Hb_in.
 // The recurrence is linear in the state, so this equals the scan over the
 // whole sequence up to rounding. The pages describe no such split (they run
 // 65K-token full-sequence denoising: "Training Hybrid Block Diffusion
@@ -127,9 +128,17 @@ struct SegLayout {
     size_t fused, states, decays, total;   // fused kernel scratch, then Sf, Sb, Hf, Hb, then Gf, Gb
 };
 
+// the segments' kernel for the last step: the two-CTA kernel when it takes
+// segments of this length
+bool seg_pair(int batch, int L, int H, int G, int N, int S) {
+    return tc_pair_supported(batch * S, L / S, H, G, N);
+}
+
 SegLayout seg_layout(int batch, int L, int H, int N, int S) {
     SegLayout l;
-    l.fused = align256(tc_fused_scratch_bytes(batch * S, L / S, H, N));
+    const size_t f = tc_fused_scratch_bytes(batch * S, L / S, H, N);
+    const size_t q = tc_pair_supported(batch * S, L / S, H, 1, N) ? tc_pair_scratch_bytes(batch * S, L / S, H, N) : 0;
+    l.fused = align256(f > q ? f : q);
     l.states = align256((size_t)batch * S * H * kP * N * sizeof(float));
     l.decays = align256((size_t)batch * S * H * sizeof(float));
     l.total = l.fused + 4 * l.states + 2 * l.decays;
@@ -146,11 +155,36 @@ int device_sms() {
 }
 
 int seg_count(long long units, int L, int sms) {
-    // the fewest segments that give one round over at least 4/5 of the SMs:
-    // every segment adds its own state passes and pass boundaries, and
-    // measured on 32 x 65536 tokens, 4 segments (128 units) beat 8, 16, 32
-    // and 64 (1.12 ms against 1.22 to 1.47 ms)
     if (sms <= 0 || units >= sms || L < 2 * 128) return 1;
+    // segments of 2..256 tiles run on the two-CTA kernel, one cluster of two
+    // SMs each: the S (dividing L) with the lowest estimated time, the fewest
+    // segments on ties. The estimate: rounds of segments over the clusters
+    // times (tiles per segment + 3, the pipeline's fill and drain per
+    // segment), plus the two state passes (one CTA per segment and SM, a tile
+    // there costing about 0.3 of a two-CTA step). Measured on 32 x 65536
+    // tokens: S = 16 1.065 ms, 4 1.137, 8 1.143, 32 1.105, 64 1.266; on
+    // 32 x 16384: S = 4 0.300 ms, 8 0.308, 16 0.315, 32 0.412
+    {
+        const long long ncl = sms / 2 > 0 ? sms / 2 : 1;
+        int best = 0;
+        long long best_cost = 0;
+        for (int S = 2; S <= kMaxSeg; ++S) {
+            if (L % S) continue;
+            const long long nt = (L / S + 127) / 128;
+            if (nt < 2 || nt > 256 || L / S <= 128) continue;
+            const long long rp = (units * S + ncl - 1) / ncl, rf = (units * S + sms - 1) / sms;
+            const long long cost = 5 * rp * (nt + 3) + 3 * rf * nt;
+            if (!best || cost < best_cost) {
+                best = S;
+                best_cost = cost;
+            }
+        }
+        if (best) return best;
+    }
+    // else the fewest segments that give one round of the fused kernel over
+    // at least 4/5 of the SMs: every segment adds its own state passes and
+    // pass boundaries, and measured on 32 x 65536 tokens, 4 segments (128
+    // units) beat 8, 16, 32 and 64 (1.12 ms against 1.22 to 1.47 ms)
     int last = 1;
     for (int S = 2; S <= kMaxSeg && L / S >= 128; ++S) {
         if (L % S) continue;
@@ -201,6 +235,7 @@ cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
     TcArgs o = v;
     o.init = Hf;
     o.rinit = Hb;
+    if (seg_pair(a.batch, a.L, a.H, a.G, a.N, S)) return launch_tc_pair(o, stream);
     return launch_tc_fused(o, stream);
 }
 

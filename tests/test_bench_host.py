@@ -65,6 +65,20 @@ def test_record_traffic_sums_one_call_and_expires_with_the_source(tmp_path, monk
     assert bench.traffic_record("fused", "no_such_workload") is None
 
 
+def test_record_traffic_takes_the_segments_kernel_that_ran(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "traffic.json"))
+    # one call whose last step ran the two-CTA kernel
+    rows = [[0, "void ssd::tc_fused_kernel<128, 2, 0, 0>(CUtensorMap_st, ...)", "200", "0"],
+            [1, "void ssd::tc_fused_kernel<128, 3, 0, 0>(CUtensorMap_st, ...)", "200", "0"],
+            [2, "ssd::seg_scan_kernel(const float *, ...)", "8", "0"],
+            [3, "void ssd::tc_pair_kernel<128>(CUtensorMap_st, ...)", "800", "0.07"]]
+    bench.record_traffic(_raw_csv(tmp_path, rows), "segmented", "long_L65536", "ncu ...")
+    e = json.load(open(bench.TRAFFIC_FILE))["long_L65536:segmented"]
+    assert e["calls_captured"] == 1
+    assert e["kernels"] == ["tc_fused_kernel", "seg_scan_kernel", "tc_pair_kernel"]
+    assert e["dram_bytes_per_launch"] == round(1208e6 + 0.07e9)
+
+
 def test_whole_job_throughput_and_time_at_one_rank():
     assert bench.job_time_ms(3.5, 1) == 3.5
     assert bench.job_throughput(1000, 4, 1, 2.0) == 1000 * 4 / 2e-3

@@ -37,29 +37,47 @@ constexpr int kP = 64;
 constexpr int kMaxSeg = 64;
 constexpr int kScanThreads = 256;
 
-// grid (batch * H, 2 directions), 256 threads; Gf, Gb: each segment's decay
-// exp(A * sum of dt over the segment), from the state passes. H0f, H0b
-// (batch, H, 64, N) or nullptr: the forward state before the sequence and the
-// reverse state after it.
+// grid (batch * H, 2 directions, N * 64 / 1024), 256 threads, one float4 of
+// the state per thread; Gf, Gb: each segment's decay exp(A * sum of dt over
+// the segment), from the state passes. H0f, H0b (batch, H, 64, N) or nullptr:
+// the forward state before the sequence and the reverse state after it. The
+// segments' states are loaded eight at a time before the chain over them, so
+// a thread waits for one round trip per eight segments, not one per segment.
 __global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(const float *Sf, const float *Sb, const float *Gf,
                                                                 const float *Gb, const float *H0f, const float *H0b,
                                                                 float *Hf, float *Hb, int H, int S, int N) {
     const int u = blockIdx.x, dir = blockIdx.y;
     const int b = u / H, h = u % H;
+    const int elems = kP * N;
+    const int e = (blockIdx.z * kScanThreads + threadIdx.x) * 4;
+    if (e >= elems) return;
     const float *sin = dir ? Sb : Sf;
     const float *gin = dir ? Gb : Gf;
     const float *h0 = dir ? H0b : H0f;
     float *hout = dir ? Hb : Hf;
-    const int elems = kP * N;
-    for (int e = threadIdx.x * 4; e < elems; e += kScanThreads * 4) {
-        float4 acc = h0 ? *reinterpret_cast<const float4 *>(h0 + (size_t)u * elems + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < S; ++k) {
-            const int seg = dir ? S - 1 - k : k;
-            const size_t su = (size_t)(b * S + seg) * H + h;   // segment unit of the reshaped batch
-            *reinterpret_cast<float4 *>(hout + su * elems + e) = acc;
-            const float4 v = *reinterpret_cast<const float4 *>(sin + su * elems + e);
-            const float g = gin[su];
-            acc = make_float4(fmaf(g, acc.x, v.x), fmaf(g, acc.y, v.y), fmaf(g, acc.z, v.z), fmaf(g, acc.w, v.w));
+    float4 acc = h0 ? *reinterpret_cast<const float4 *>(h0 + (size_t)u * elems + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    constexpr int kBatch = 8;
+    for (int k0 = 0; k0 < S; k0 += kBatch) {
+        float4 v[kBatch];
+        float g[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            if (k0 + j < S) {
+                const int seg = dir ? S - 1 - (k0 + j) : k0 + j;
+                const size_t su = (size_t)(b * S + seg) * H + h;   // segment unit of the reshaped batch
+                v[j] = *reinterpret_cast<const float4 *>(sin + su * elems + e);
+                g[j] = gin[su];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            if (k0 + j < S) {
+                const int seg = dir ? S - 1 - (k0 + j) : k0 + j;
+                const size_t su = (size_t)(b * S + seg) * H + h;
+                *reinterpret_cast<float4 *>(hout + su * elems + e) = acc;
+                acc = make_float4(fmaf(g[j], acc.x, v[j].x), fmaf(g[j], acc.y, v[j].y), fmaf(g[j], acc.z, v[j].z),
+                                  fmaf(g[j], acc.w, v[j].w));
+            }
         }
     }
 }
@@ -229,8 +247,9 @@ cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
     r.state_out = Sb;
     r.decay_out = Gb;
     if ((e = launch_tc_fused_state_rev(r, stream)) != cudaSuccess) return e;
-    seg_scan_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, a.init, a.rinit, Hf, Hb,
-                                                                        a.H, S, a.N);
+    const int zb = (kP * a.N + kScanThreads * 4 - 1) / (kScanThreads * 4);
+    seg_scan_kernel<<<dim3(a.batch * a.H, 2, zb), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, a.init, a.rinit, Hf, Hb,
+                                                                            a.H, S, a.N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     TcArgs o = v;
     o.init = Hf;

@@ -200,17 +200,60 @@ def record_traffic(csv_path: str, path: str, workload: str, command: str, scale:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled during the timed
+    region: an in-process NVML thread polling every millisecond between
+    __enter__ and __exit__ (read-only queries), else nvidia-smi every 100 ms."""
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.lines = []
+        self.rows = []          # (sm MHz, max sm MHz, reason names) from NVML
+        self.nvml = None
+        self.stop = False
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            props = torch.cuda.get_device_properties(self.index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _sample(self):
+        nv, h = self.nvml
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        self.rows.append((float(sm), float(self.max_mhz), [n for b, n in self.REASONS.items() if bits & b]))
+
+    def _poll(self):
+        while not self.stop:
+            try:
+                self._sample()
+            except Exception:
+                break
+            time.sleep(0.001)
 
     def __enter__(self):
+        try:
+            self.nvml = self._nvml_handle()
+            nv, h = self.nvml
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._sample()            # one sample at the start of the region, whatever its length
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
@@ -228,6 +271,14 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        if self.nvml is not None:
+            self.stop = True
+            self.t.join(timeout=5)
+            try:
+                self._sample()        # and one at its end
+            except Exception:
+                pass
+            return
         if self.proc is not None:
             time.sleep(0.2)
             self.proc.terminate()
@@ -237,21 +288,25 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        rows = []
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != 7:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
-            except ValueError:
-                continue
+        rows = list(self.rows)
+        source = "nvml, 1 ms, during the timed region"
+        if not rows:
+            source = "nvidia-smi, 100 ms"
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for ln in self.lines:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) != 7:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]),
+                                 [names[i] for i, v in enumerate(parts[3:]) if v.lower() == "active"]))
+                except ValueError:
+                    continue
         if not rows:
             return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        reasons = sorted({n for _, _, r in rows for n in r})
         return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": source}
 
 
 def cpu_baseline(w, budget_s: float = 12.0):

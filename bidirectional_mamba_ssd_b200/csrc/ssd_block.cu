@@ -18,113 +18,9 @@
 namespace ssd {
 namespace {
 
-constexpr int kConvThreads = 256;
-constexpr int kConvTokens = 8;       // tokens per thread (its whole input window is loaded at once)
 constexpr int kMaxConv = 4;          // widest conv supported
 
 __device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.f + __expf(-v)); }
-
-// Four consecutive channels of the I/O type as floats (8 bytes of bf16 or 16
-// of fp32; the channel index is a multiple of 4).
-template <typename T> struct Vec4;
-template <> struct Vec4<float> {
-    static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
-        const float4 q = *reinterpret_cast<const float4 *>(p);
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
-        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
-    }
-};
-template <> struct Vec4<__nv_bfloat16> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[4]) {
-        const uint2 q = *reinterpret_cast<const uint2 *>(p);
-        v[0] = __uint_as_float(q.x << 16); v[1] = __uint_as_float(q.x & 0xffff0000u);
-        v[2] = __uint_as_float(q.y << 16); v[3] = __uint_as_float(q.y & 0xffff0000u);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4]) {
-        __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
-        *reinterpret_cast<uint2 *>(p) = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
-    }
-};
-
-// One thread: channels [c, c + 4) of one batch element over kConvTokens
-// tokens. Tap k of the forward conv reads token t - (K - 1) + k, of the
-// reverse conv token t + (K - 1) - k (zero outside the sequence). The inputs
-// its 8 tokens read (t0 - K + 1 .. t0 + 7 + K - 1) are loaded into registers
-// at once, 4 channels per load (coalesced across the channels of a warp), so
-// the thread waits for memory once; the channels' 2 K weights and 2 biases stay
-// in registers. The x, B and C blocks of channels are multiples of 4 wide, so
-// a thread's channels go to one of them.
-template <typename T, int K>
-__global__ void __launch_bounds__(kConvThreads)
-conv_silu_kernel(const T *__restrict__ xbc, const float *__restrict__ w, const float *__restrict__ bias,
-                 T *__restrict__ x2, T *__restrict__ B2, T *__restrict__ C2, int batch, int L, int HP, int GN) {
-    constexpr int R = K - 1;                 // window radius
-    const int cin = HP + 2 * GN;
-    const int c = 4 * (blockIdx.x * kConvThreads + threadIdx.x);
-    const int b = blockIdx.z;
-    const int t0 = blockIdx.y * kConvTokens;
-    if (c >= cin) return;
-    // wf[e][k]: forward tap k of channel c + e (reads token t - R + k); wr[e][k]:
-    // reverse tap k (reads token t + R - k)
-    float wf[4][K], wr[4][K], bf[4], bb[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-            wf[e][k] = w[(size_t)(c + e) * K + k];
-            wr[e][k] = w[(size_t)cin * K + (size_t)(c + e) * K + k];
-        }
-        bf[e] = bias[c + e];
-        bb[e] = bias[cin + c + e];
-    }
-    const T *in = xbc + (size_t)b * L * cin + c;
-    // destination of these channels in each direction
-    T *dst;
-    size_t ld, dir_stride;
-    if (c < HP) {
-        dst = x2 + (size_t)b * L * HP + c; ld = HP; dir_stride = (size_t)batch * L * HP;
-    } else if (c < HP + GN) {
-        dst = B2 + (size_t)b * L * GN + (c - HP); ld = GN; dir_stride = (size_t)batch * L * GN;
-    } else {
-        dst = C2 + (size_t)b * L * GN + (c - HP - GN); ld = GN; dir_stride = (size_t)batch * L * GN;
-    }
-    // every input the thread's tokens read (slot j holds token t0 - R + j),
-    // loaded before any is used
-    float win[kConvTokens + 2 * R][4];
-#pragma unroll
-    for (int j = 0; j < kConvTokens + 2 * R; ++j) {
-        const int t = t0 - R + j;
-        if (t >= 0 && t < L) {
-            Vec4<T>::load(in + (size_t)t * cin, win[j]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) win[j][e] = 0.f;
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < kConvTokens; ++i) {
-        const int t = t0 + i;
-        if (t < L) {
-            float f[4], r[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                f[e] = bf[e];
-                r[e] = bb[e];
-#pragma unroll
-                for (int k = 0; k < K; ++k) {
-                    f[e] = fmaf(wf[e][k], win[i + k][e], f[e]);           // token t - R + k
-                    r[e] = fmaf(wr[e][k], win[i + 2 * R - k][e], r[e]);   // token t + R - k
-                }
-                f[e] = silu(f[e]);
-                r[e] = silu(r[e]);
-            }
-            Vec4<T>::store(dst + (size_t)t * ld, f);
-            Vec4<T>::store(dst + dir_stride + (size_t)t * ld, r);
-        }
-    }
-}
 
 // dt[d][b][t][h] = clamp(softplus(raw + bias[d][h]), lo, hi); softplus(u) =
 // log(1 + e^u), taken as u beyond 20 (where the two agree in fp32).
@@ -173,6 +69,118 @@ template <> struct Vec8<float> {
         reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
     }
 };
+
+// One direction's conv + SiLU for 8 consecutive channels (16 bytes of bf16)
+// of one batch element over a run of kConvRun tokens: the forward conv's tap k
+// reads token t - (K - 1) + k, the reverse conv's tap k token t + (K - 1) - k
+// (zero outside the sequence). The thread keeps its direction's taps for its
+// channels and the last K - 1 input rows in registers and, per group of 8
+// tokens, issues the group's 8 row loads (16 bytes each, 512 contiguous bytes
+// across a warp) before it uses any, so each group waits for memory once. The
+// x, B and C blocks of channels are multiples of 8 wide, so a thread's
+// channels go to one of them.
+// 8 channels of the I/O type kept as loaded (4 registers of bf16 pairs, 8 of
+// fp32) until used.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 q;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { q = *reinterpret_cast<const uint4 *>(p); }
+    __device__ __forceinline__ void zero() { q = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&v)[8]) const {
+        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            v[2 * k] = __uint_as_float(u[k] << 16);
+            v[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+        }
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float *p) {
+        a = reinterpret_cast<const float4 *>(p)[0];
+        b = reinterpret_cast<const float4 *>(p)[1];
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void unpack(float (&v)[8]) const {
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+
+constexpr int kConvRun = 64;     // tokens per thread
+constexpr int kConvGroup = 8;    // rows loaded at once
+constexpr int kConvBlock = 128;  // threads per CTA: 128 chunks of 8 channels
+
+template <typename T, int K>
+__global__ void __launch_bounds__(kConvBlock)
+conv_silu_kernel(const T *__restrict__ xbc, const float *__restrict__ w, const float *__restrict__ bias,
+                 T *__restrict__ x2, T *__restrict__ B2, T *__restrict__ C2, int batch, int L, int HP, int GN) {
+    constexpr int R = K - 1;
+    const int cin = HP + 2 * GN;
+    const int c = 8 * (blockIdx.x * kConvBlock + threadIdx.x);
+    const int dir = blockIdx.y & 1, t0 = (blockIdx.y >> 1) * kConvRun, b = blockIdx.z;
+    if (c >= cin) return;
+    // wk[e][m]: the tap that multiplies window slot m, slot m holding token
+    // t - R + m (forward) or t + m (reverse) for output token t
+    float wk[8][K], bk[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+#pragma unroll
+        for (int m = 0; m < K; ++m)
+            wk[e][m] = w[(size_t)dir * cin * K + (size_t)(c + e) * K + (dir ? R - m : m)];
+        bk[e] = bias[(size_t)dir * cin + c + e];
+    }
+    T *dst;
+    size_t ld;
+    if (c < HP) {
+        dst = x2 + (size_t)b * L * HP + c; ld = HP;
+        if (dir) dst += (size_t)batch * L * HP;
+    } else if (c < HP + GN) {
+        dst = B2 + (size_t)b * L * GN + (c - HP); ld = GN;
+        if (dir) dst += (size_t)batch * L * GN;
+    } else {
+        dst = C2 + (size_t)b * L * GN + (c - HP - GN); ld = GN;
+        if (dir) dst += (size_t)batch * L * GN;
+    }
+    const T *in = xbc + (size_t)b * L * cin + c;
+    // first input row of the window of token t0: t0 - R (forward) or t0 (reverse)
+    const int first = t0 - (dir ? 0 : R);
+    auto load = [&](int t, Raw8<T> &r) {
+        if (t >= 0 && t < L) r.load(in + (size_t)t * cin);
+        else r.zero();
+    };
+    float win[K][8];
+#pragma unroll
+    for (int m = 0; m < R; ++m) {
+        Raw8<T> r;
+        load(first + m, r);
+        r.unpack(win[m]);
+    }
+    const int end = min(t0 + kConvRun, L);
+    for (int g0 = t0; g0 < end; g0 += kConvGroup) {
+        Raw8<T> rows[kConvGroup];
+#pragma unroll
+        for (int i = 0; i < kConvGroup; ++i) load(first + (g0 - t0) + i + R, rows[i]);
+#pragma unroll
+        for (int i = 0; i < kConvGroup; ++i) {
+            rows[i].unpack(win[R]);
+            float o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float a = bk[e];
+#pragma unroll
+                for (int m = 0; m < K; ++m) a = fmaf(wk[e][m], win[m][e], a);
+                o[e] = silu(a);
+            }
+            const int t = g0 + i;
+            if (t < end) Vec8<T>::store(dst + (size_t)t * ld, o);
+#pragma unroll
+            for (int m = 0; m < R; ++m)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) win[m][e] = win[m + 1][e];
+        }
+    }
+}
 
 constexpr int kNormChunks = 8;   // 8-channel chunks per lane held in registers: C <= 32 * 8 * 8
 
@@ -225,10 +233,10 @@ gated_rmsnorm_kernel(const T *__restrict__ y, const T *__restrict__ z, const flo
 template <typename T, int K>
 cudaError_t run_conv_k(const BlockLaunch &l, cudaStream_t s) {
     const int cin = l.HP + 2 * l.GN;
-    dim3 grid((cin / 4 + kConvThreads - 1) / kConvThreads, (l.L + kConvTokens - 1) / kConvTokens, l.batch);
-    conv_silu_kernel<T, K><<<grid, kConvThreads, 0, s>>>(static_cast<const T *>(l.xbc), l.conv_w, l.conv_b,
-                                                         static_cast<T *>(l.x2), static_cast<T *>(l.B2),
-                                                         static_cast<T *>(l.C2), l.batch, l.L, l.HP, l.GN);
+    dim3 grid((cin / 8 + kConvBlock - 1) / kConvBlock, 2 * ((l.L + kConvRun - 1) / kConvRun), l.batch);
+    conv_silu_kernel<T, K><<<grid, kConvBlock, 0, s>>>(static_cast<const T *>(l.xbc), l.conv_w, l.conv_b,
+                                                       static_cast<T *>(l.x2), static_cast<T *>(l.B2),
+                                                       static_cast<T *>(l.C2), l.batch, l.L, l.HP, l.GN);
     return cudaGetLastError();
 }
 
@@ -265,7 +273,7 @@ cudaError_t run_norm(const BlockLaunch &l, cudaStream_t s) {
 
 cudaError_t launch_conv_silu(const BlockLaunch &l, cudaStream_t s) {
     if (l.K < 1 || l.K > kMaxConv) return cudaErrorNotSupported;
-    if (l.HP % 4 || l.GN % 4) return cudaErrorNotSupported;   // 4 channels per thread
+    if (l.HP % 8 || l.GN % 8) return cudaErrorNotSupported;   // 8-channel chunks
     return l.bf16 ? run_conv<__nv_bfloat16>(l, s) : run_conv<float>(l, s);
 }
 

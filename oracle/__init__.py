@@ -69,9 +69,11 @@ def configure(lib):
     lib.ssd_oracle_block_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
     lib.ssd_oracle_bidir_seeded.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i]
     lib.ssd_oracle_bidir_bwd.argtypes = [dp] * 13 + [i] * 7
+    lib.ssd_oracle_bidir_bwd_seeded.argtypes = [dp] * 17 + [i] * 7
     lib.ssd_oracle_threads.argtypes = [i]
     for f in (lib.ssd_oracle_bidir, lib.ssd_oracle_prefix_state, lib.ssd_oracle_block_step,
-              lib.ssd_oracle_bidir_seeded, lib.ssd_oracle_bidir_bwd, lib.ssd_oracle_threads):
+              lib.ssd_oracle_bidir_seeded, lib.ssd_oracle_bidir_bwd, lib.ssd_oracle_bidir_bwd_seeded,
+              lib.ssd_oracle_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -194,19 +196,30 @@ def dt_prep(dt_raw, dt_bias, dt_min=0.0, dt_max=np.inf) -> np.ndarray:
     return np.clip(sp, dt_min, dt_max)
 
 
-def bidir_bwd(x, dt, A, B, C, D, dy, nthreads: int = 0) -> dict:
-    """Gradients of sum(dy * bidir(x, dt, A, B, C, D)) with respect to every
-    input, in fp64, from the adjoint of the recurrence token by token (see
-    ssd_oracle.c). Returns a dict of arrays shaped like the inputs: dx, ddt,
-    dA, dB, dC, dD."""
+def bidir_bwd(x, dt, A, B, C, D, dy, prefix=None, suffix=None, nthreads: int = 0) -> dict:
+    """Gradients of sum(dy * bidir_seeded(x, dt, A, B, C, D, prefix, suffix))
+    (bidir when both states are None) with respect to every input, in fp64,
+    from the adjoint of the recurrence token by token (see ssd_oracle.c).
+    Returns a dict of arrays shaped like the inputs: dx, ddt, dA, dB, dC, dD,
+    and dprefix / dsuffix for the states that are given. With suffix None and
+    a prefix, these are the gradients of the block step."""
     x = np.asarray(x)
     batch, L, H, P = x.shape
     G, N = np.asarray(B).shape[-2:]
-    keep = [_f64(a) for a in (x, dt, A, B, C, D, dy)]
+    keep = [_f64(a) for a in (x, dt, A, B, C, D)]
+    states = [None if s is None else _f64(s) for s in (prefix, suffix)]
+    keep_dy = _f64(dy)
     outs = {"dx": np.zeros((batch, L, H, P)), "ddt": np.zeros((2, batch, L, H)), "dA": np.zeros((2, H)),
             "dB": np.zeros((2, batch, L, G, N)), "dC": np.zeros((2, batch, L, G, N)), "dD": np.zeros((2, H))}
-    po = [outs[k].ctypes.data_as(ctypes.POINTER(ctypes.c_double)) for k in ("dx", "ddt", "dA", "dB", "dC", "dD")]
-    rc = _load().ssd_oracle_bidir_bwd(*(p for _, p in keep), *po, batch, L, H, P, N, G, int(nthreads))
+    if prefix is not None:
+        outs["dprefix"] = np.zeros((batch, H, P, N))
+    if suffix is not None:
+        outs["dsuffix"] = np.zeros((batch, H, P, N))
+    dp = ctypes.POINTER(ctypes.c_double)
+    po = [outs[k].ctypes.data_as(dp) for k in ("dx", "ddt", "dA", "dB", "dC", "dD")]
+    pd = [outs[k].ctypes.data_as(dp) if k in outs else None for k in ("dprefix", "dsuffix")]
+    rc = _load().ssd_oracle_bidir_bwd_seeded(*(p for _, p in keep), *(None if s is None else s[1] for s in states),
+                                             keep_dy[1], *po, *pd, batch, L, H, P, N, G, int(nthreads))
     if rc != 0:
         raise ValueError("oracle bidir_bwd: bad arguments")
     return outs

@@ -299,12 +299,21 @@ int ssd_oracle_bidir_seeded(const double *x, const double *dt, const double *A,
  * Layouts as for ssd_oracle_bidir; dy and dx (batch, L, H, P); ddt (2, batch,
  * L, H); dA, dD (2, H); dB, dC (2, batch, L, G, N). Every output is
  * overwritten. Heads of a B/C group add into the same dB, dC entries, so the
- * work is split by (batch, group) with the group's heads in order. */
-int ssd_oracle_bidir_bwd(const double *x, const double *dt, const double *A,
-                         const double *Bm, const double *Cm, const double *D,
-                         const double *dy, double *dx, double *ddt, double *dA,
-                         double *dB, double *dC, double *dD,
-                         int batch, int L, int H, int P, int N, int G, int nthreads)
+ * work is split by (batch, group) with the group's heads in order.
+ *
+ * ssd_oracle_bidir_bwd_seeded is the same for ssd_oracle_bidir_seeded's
+ * scans: the forward one starts from `prefix`, the reverse one from `suffix`
+ * ((batch, H, P, N) each, NULL for zero), which enter as the state before
+ * each direction's first token; the gradients with respect to them,
+ * dprefix and dsuffix (NULL to skip), are the adjoint of that state:
+ * a_first g_first, the first token's decay times its state's adjoint. With
+ * suffix NULL this is the backward pass of the block step. */
+int ssd_oracle_bidir_bwd_seeded(const double *x, const double *dt, const double *A,
+                                const double *Bm, const double *Cm, const double *D,
+                                const double *prefix, const double *suffix,
+                                const double *dy, double *dx, double *ddt, double *dA,
+                                double *dB, double *dC, double *dD, double *dprefix, double *dsuffix,
+                                int batch, int L, int H, int P, int N, int G, int nthreads)
 {
     if (batch < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G) return -1;
     set_threads(nthreads);
@@ -340,8 +349,16 @@ int ssd_oracle_bidir_bwd(const double *x, const double *dt, const double *A,
                 const double *Cu = Cm + d * bc_dir + ((size_t)b * L * G + g) * N;
                 double *dBu = dB + d * bc_dir + ((size_t)b * L * G + g) * N;
                 double *dCu = dC + d * bc_dir + ((size_t)b * L * G + g) * N;
-                /* forward through the direction's order: hs[k] is the state after k tokens */
-                memset(hs, 0, sizeof(double) * SN);
+                /* forward through the direction's order: hs[k] is the state after k tokens,
+                   hs[0] the given start state (its (P, N) layout transposed) or zero */
+                const double *init = d ? suffix : prefix;
+                if (init) {
+                    const double *iu = init + ((size_t)b * H + hh) * P * N;
+                    for (int n = 0; n < N; ++n)
+                        for (int p = 0; p < P; ++p) hs[(size_t)n * P + p] = iu[(size_t)p * N + n];
+                } else {
+                    memset(hs, 0, sizeof(double) * SN);
+                }
                 for (int k = 0; k < L; ++k) {
                     const int t = d ? (L - 1 - k) : k;
                     const double dtt = dtu[(ptrdiff_t)t * dt_ts];
@@ -396,6 +413,13 @@ int ssd_oracle_bidir_bwd(const double *x, const double *dt, const double *A,
                     for (size_t q = 0; q < SN; ++q) gadj[q] *= a;   /* adjoint of h_{t-1}'s share */
                 }
                 dA_b[(size_t)b * 2 * H + d * H + hh] = dA_acc;
+                /* the start state's adjoint: what is left after the first token */
+                double *dinit = d ? dsuffix : dprefix;
+                if (dinit) {
+                    double *du = dinit + ((size_t)b * H + hh) * P * N;
+                    for (int n = 0; n < N; ++n)
+                        for (int p = 0; p < P; ++p) du[(size_t)p * N + n] = L > 0 ? gadj[(size_t)n * P + p] : 0.0;
+                }
             }
             /* skip term */
             const double dsum = D[hh] + D[H + hh];
@@ -423,4 +447,14 @@ int ssd_oracle_bidir_bwd(const double *x, const double *dt, const double *A,
     free(dA_b);
     free(dD_b);
     return bad ? -1 : 0;
+}
+
+int ssd_oracle_bidir_bwd(const double *x, const double *dt, const double *A,
+                         const double *Bm, const double *Cm, const double *D,
+                         const double *dy, double *dx, double *ddt, double *dA,
+                         double *dB, double *dC, double *dD,
+                         int batch, int L, int H, int P, int N, int G, int nthreads)
+{
+    return ssd_oracle_bidir_bwd_seeded(x, dt, A, Bm, Cm, D, NULL, NULL, dy, dx, ddt, dA, dB, dC, dD, NULL, NULL,
+                                       batch, L, H, P, N, G, nthreads);
 }

@@ -9,7 +9,11 @@ checks:
     <dy, y(v) - y(0)> = <grad, v> up to rounding;
   * the closed form of a memoryless scan (A -> -inf, exp underflows to 0 in
     fp64): y_t = (sum_d dt_d,t C_d,t . B_d,t + D_f + D_b) x_t, whose
-    gradients are written out by hand below.
+    gradients are written out by hand below;
+  * with given start states (the seeded scans, and the block step: forward
+    from a prefix state, reverse from zero): central differences of
+    oracle.bidir_seeded and of oracle.block_step, including along the
+    states, and the adjoint identity of the states (y is affine in them).
 A planted mistake in the backward code must fail at least one of them
 (test_bwd_pins_catch_planted_mistake).
 """
@@ -108,6 +112,67 @@ def test_bwd_memoryless_closed_form():
     assert np.all(g["dA"] == 0.0)
 
 
+def _seeded(seed=3, batch=2, L=6, H=4, P=3, N=5, G=2):
+    inp, dy = _problem(seed, batch, L, H, P, N, G)
+    rng = np.random.default_rng(seed + 100)
+    inp["prefix"] = rng.standard_normal((batch, H, P, N))
+    inp["suffix"] = rng.standard_normal((batch, H, P, N))
+    return inp, dy
+
+
+def _seeded_loss(inp, dy):
+    return float(np.sum(dy * oracle.bidir_seeded(*(inp[k] for k in NAMES), prefix=inp["prefix"],
+                                                  suffix=inp["suffix"])))
+
+
+@pytest.mark.parametrize("name", NAMES + ("prefix", "suffix"))
+def test_seeded_bwd_matches_central_differences(name):
+    inp, dy = _seeded()
+    g = oracle.bidir_bwd(*(inp[k] for k in NAMES), dy, prefix=inp["prefix"], suffix=inp["suffix"])
+    v = np.random.default_rng(4).standard_normal(inp[name].shape)
+    eps = 1e-6 * max(1.0, float(np.max(np.abs(inp[name]))))
+    plus, minus = dict(inp), dict(inp)
+    plus[name] = inp[name] + eps * v
+    minus[name] = inp[name] - eps * v
+    fd = (_seeded_loss(plus, dy) - _seeded_loss(minus, dy)) / (2 * eps)
+    an = float(np.sum(g["d" + name] * v))
+    assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), f"d{name}: finite difference {fd} vs adjoint {an}"
+
+
+def test_state_gradients_adjoint_identity():
+    """y is affine in each start state: <dy, y(s + v) - y(s)> = <ds, v>."""
+    inp, dy = _seeded(seed=5)
+    g = oracle.bidir_bwd(*(inp[k] for k in NAMES), dy, prefix=inp["prefix"], suffix=inp["suffix"])
+    base = oracle.bidir_seeded(*(inp[k] for k in NAMES), prefix=inp["prefix"], suffix=inp["suffix"])
+    rng = np.random.default_rng(6)
+    for name in ("prefix", "suffix"):
+        v = rng.standard_normal(inp[name].shape)
+        moved = dict(inp)
+        moved[name] = inp[name] + v
+        y = oracle.bidir_seeded(*(moved[k] for k in NAMES), prefix=moved["prefix"], suffix=moved["suffix"])
+        lhs, rhs = float(np.sum(dy * (y - base))), float(np.sum(g["d" + name] * v))
+        assert abs(lhs - rhs) <= 1e-10 * max(1.0, abs(lhs)), f"d{name}: {lhs} vs {rhs}"
+
+
+def test_block_step_gradients_match_central_differences():
+    """The block step's gradients (prefix given, no suffix) against central
+    differences of oracle.block_step, its own forward definition."""
+    inp, dy = _seeded(seed=7, L=5)
+    g = oracle.bidir_bwd(*(inp[k] for k in NAMES), dy, prefix=inp["prefix"])
+    assert "dsuffix" not in g
+    rng = np.random.default_rng(8)
+    for name in ("prefix", "dt", "A", "x"):
+        v = rng.standard_normal(inp[name].shape)
+        eps = 1e-6 * max(1.0, float(np.max(np.abs(inp[name]))))
+        f = lambda d: float(np.sum(dy * oracle.block_step(*((inp[k] + d * v) if k == name else inp[k]
+                                                             for k in NAMES),
+                                                           (inp["prefix"] + d * v) if name == "prefix"
+                                                           else inp["prefix"])))
+        fd = (f(eps) - f(-eps)) / (2 * eps)
+        an = float(np.sum(g["d" + name] * v))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), f"block step d{name}: {fd} vs {an}"
+
+
 # (name, text in ssd_oracle.c's backward code, replacement): plausible mistakes
 BWD_MUTANTS = [
     ("ddt_without_decay_term", "ddtu[(ptrdiff_t)t * dt_ts] = gbx + Ad * a * ghp;", "ddtu[(ptrdiff_t)t * dt_ts] = gbx;"),
@@ -119,12 +184,22 @@ BWD_MUTANTS = [
     ("dC_from_previous_state", "s += ht[(size_t)n * P + p] * dyt[p];", "s += hp[(size_t)n * P + p] * dyt[p];"),
     ("reverse_adjoint_walks_forward", "const int t = d ? (L - 1 - k) : k;\n                    const double dtt = dtu[(ptrdiff_t)t * dt_ts];\n                    const double a = exp(dtt * Ad);\n                    const double *Bt = Bu + (ptrdiff_t)t * bc_ts;\n                    const double *Ct",
      "const int t = k;\n                    const double dtt = dtu[(ptrdiff_t)t * dt_ts];\n                    const double a = exp(dtt * Ad);\n                    const double *Bt = Bu + (ptrdiff_t)t * bc_ts;\n                    const double *Ct"),
+    ("start_state_adjoint_without_first_decay",
+     "du[(size_t)p * N + n] = L > 0 ? gadj[(size_t)n * P + p] : 0.0;",
+     "du[(size_t)p * N + n] = L > 0 ? gadj[(size_t)n * P + p] / exp(dtu[(ptrdiff_t)(d ? L - 1 : 0) * dt_ts] * Ad) : 0.0;"),
+    ("start_state_not_transposed", "hs[(size_t)n * P + p] = iu[(size_t)p * N + n];",
+     "hs[(size_t)n * P + p] = iu[(size_t)n * P + p];"),
+    ("start_state_ignored_in_scan", "for (int p = 0; p < P; ++p) hs[(size_t)n * P + p] = iu[(size_t)p * N + n];",
+     "for (int p = 0; p < P; ++p) hs[(size_t)n * P + p] = 0.0 * iu[(size_t)p * N + n];"),
 ]
 
 BWD_PINS = [
     lambda: [test_bwd_matches_central_differences(n) for n in NAMES],
     lambda: [test_bwd_adjoint_identity_of_linear_inputs(n) for n in ("x", "B", "C", "D")],
     test_bwd_memoryless_closed_form,
+    lambda: [test_seeded_bwd_matches_central_differences(n) for n in NAMES + ("prefix", "suffix")],
+    test_state_gradients_adjoint_identity,
+    test_block_step_gradients_match_central_differences,
 ]
 
 

@@ -402,10 +402,14 @@ def ssd_bidir_fwd_dtraw(x, dt_raw, dt_bias, A, B, C, D, dt_min: float = 0.0, dt_
     return out
 
 
-def ssd_bidir_bwd(x, dt, A, B, C, D, dy, *, workspace: Workspace | None = None) -> dict:
+def ssd_bidir_bwd(x, dt, A, B, C, D, dy, *, fwd_init=None, rev_init=None,
+                  workspace: Workspace | None = None) -> dict:
     """Gradients of sum(dy * ssd_bidir_fwd(x, dt, A, B, C, D)) with respect to
     every input (include/ssd_bidir.h: ssd_bidir_bwd), as fp32 tensors shaped
-    like the inputs: dx, ddt, dA, dB, dC, dD."""
+    like the inputs: dx, ddt, dA, dB, dC, dD. With fwd_init / rev_init
+    (batch, H, P, N) fp32, the scans start from those states
+    (ssd_bidir_fwd_seeded; ssd_bidir_bwd_seeded) and the dict also holds
+    d_fwd_init / d_rev_init, their gradients."""
     _need(x, "x", ndim=4)
     dev, io = x.device, x.dtype
     if io not in _DT:
@@ -421,19 +425,43 @@ def ssd_bidir_bwd(x, dt, A, B, C, D, dy, *, workspace: Workspace | None = None) 
             or tuple(C.shape) != tuple(B.shape) or tuple(A.shape) != (2, H) or tuple(D.shape) != (2, H) \
             or dy.shape != x.shape:
         raise ValueError("shape mismatch: want x, dy (b,L,H,P), dt (2,b,L,H), B/C (2,b,L,G,N), A/D (2,H)")
+    for name, st in (("fwd_init", fwd_init), ("rev_init", rev_init)):
+        if st is not None:
+            _need(st, name, torch.float32, dev, 4)
+            if tuple(st.shape) != (batch, H, P, N):
+                raise ValueError(f"{name} must be (batch, H, P, N)")
     f32 = dict(dtype=torch.float32, device=dev)
     g = {"dx": torch.empty(x.shape, **f32), "ddt": torch.empty(dt.shape, **f32), "dA": torch.empty(A.shape, **f32),
          "dB": torch.empty(B.shape, **f32), "dC": torch.empty(C.shape, **f32), "dD": torch.empty(D.shape, **f32)}
+    if fwd_init is not None:
+        g["d_fwd_init"] = torch.empty((batch, H, P, N), **f32)
+    if rev_init is not None:
+        g["d_rev_init"] = torch.empty((batch, H, P, N), **f32)
     stream = _stream(dev)
     ws = _workspace(dev, stream, workspace)
     nbytes = ssd_workspace_bytes(SSD_OP_BIDIR_BWD, batch, L, H, P, N, G, 64, io)
     if nbytes == 0:
         _check(_c.SSD_ERR_UNSUPPORTED, "ssd_bidir_bwd")
     buf = ws.get(nbytes)
-    rc = lib.ssd_bidir_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dy),
-                           *(_ptr(g[k]) for k in ("dx", "ddt", "dA", "dB", "dC", "dD")),
-                           batch, L, H, P, N, G, _DT[io], _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
+    opt = lambda t: _ptr(t) if t is not None else None
+    rc = lib.ssd_bidir_bwd_seeded(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), opt(fwd_init),
+                                  opt(rev_init), _ptr(dy),
+                                  *(_ptr(g[k]) for k in ("dx", "ddt", "dA", "dB", "dC", "dD")),
+                                  opt(g.get("d_fwd_init")), opt(g.get("d_rev_init")),
+                                  batch, L, H, P, N, G, _DT[io], _ptr(buf), buf.numel(), ctypes.c_void_p(stream))
     _check(rc, "ssd_bidir_bwd")
+    return g
+
+
+def ssd_block_step_bwd(x, dt, A, B, C, D, prefix_state, dy, *, workspace: Workspace | None = None) -> dict:
+    """Gradients of sum(dy * ssd_block_step(x, dt, A, B, C, D, prefix_state))
+    with respect to the block's inputs and (as d_prefix_state, when one is
+    given) the cached prefix state: the seeded backward with a forward start
+    state and none for the reverse scan (include/ssd_bidir.h:
+    ssd_bidir_bwd_seeded)."""
+    g = ssd_bidir_bwd(x, dt, A, B, C, D, dy, fwd_init=prefix_state, workspace=workspace)
+    if "d_fwd_init" in g:
+        g["d_prefix_state"] = g.pop("d_fwd_init")
     return g
 
 

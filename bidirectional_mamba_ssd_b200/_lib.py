@@ -40,6 +40,7 @@ SIGNATURES = {
     "ssd_bidir_fwd_seeded": (_i, [_vp] * 9 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_bidir_fwd_dtraw": (_i, [_vp] * 3 + [ctypes.c_float] * 2 + [_vp] * 5 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_bidir_bwd": (_i, [_vp] * 13 + [_i] * 7 + [_vp, _sz, _vp]),
+    "ssd_bidir_bwd_seeded": (_i, [_vp] * 17 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_prefix_state_layers": (_i, [_vp] * 6 + [_i] * 9 + [_vp, _sz, _vp]),
     "ssd_bidir_fwd_x2": (_i, [_vp] * 7 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_mixer_block_fwd": (_i, [_vp] * 5 + [_i, _vp] + [ctypes.c_float] * 2 + [_vp] * 3 + [ctypes.c_float, _vp]

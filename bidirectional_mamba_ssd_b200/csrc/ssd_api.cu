@@ -509,10 +509,11 @@ int ssd_bidir_fwd_seeded(const void *x, const void *dt, const float *A, const vo
     return to_status(ssd::launch_tc_fused(t, static_cast<cudaStream_t>(stream)));
 }
 
-int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, const void *C, const float *D,
-                  const void *dy, float *dx, float *ddt, float *dA, float *dB, float *dC, float *dD, int batch,
-                  int seqlen, int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
-                  size_t ws_bytes, void *stream) {
+int ssd_bidir_bwd_seeded(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                         const float *D, const float *fwd_init, const float *rev_init, const void *dy, float *dx,
+                         float *ddt, float *dA, float *dB, float *dC, float *dD, float *d_fwd_init,
+                         float *d_rev_init, int batch, int seqlen, int nheads, int headdim, int dstate,
+                         int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream) {
     int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype, false);
     if (rc != SSD_OK) return rc;
     if (!workspace) return SSD_ERR_WORKSPACE;
@@ -520,11 +521,17 @@ int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, 
     if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_BWD, batch, seqlen, nheads, headdim, dstate, ngroups, 64, dtype))
         return SSD_ERR_WORKSPACE;
     if (!dA || !dD || !aligned4(dA) || !aligned4(dD)) return SSD_ERR_INVALID_ARG;
+    if ((fwd_init && !aligned4(fwd_init)) || (rev_init && !aligned4(rev_init)) ||
+        (d_fwd_init && !aligned4(d_fwd_init)) || (d_rev_init && !aligned4(d_rev_init)))
+        return SSD_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = sizeof(float) * (size_t)batch * nheads * headdim * dstate;
     if (batch == 0 || seqlen == 0) {
-        // no tokens: every gradient is zero (dA and dD are the only non-empty ones)
+        // no tokens: every gradient is zero (dA, dD and the start states' are the only non-empty ones)
         if (cudaMemsetAsync(dA, 0, 2 * sizeof(float) * nheads, s) != cudaSuccess ||
-            cudaMemsetAsync(dD, 0, 2 * sizeof(float) * nheads, s) != cudaSuccess)
+            cudaMemsetAsync(dD, 0, 2 * sizeof(float) * nheads, s) != cudaSuccess ||
+            (d_fwd_init && state_bytes && cudaMemsetAsync(d_fwd_init, 0, state_bytes, s) != cudaSuccess) ||
+            (d_rev_init && state_bytes && cudaMemsetAsync(d_rev_init, 0, state_bytes, s) != cudaSuccess))
             return SSD_ERR_CUDA;
         return SSD_OK;
     }
@@ -535,10 +542,19 @@ int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, 
     ssd::BwdLaunch l{};
     l.x = x; l.dt = dt; l.B = B; l.C = C; l.dy = dy; l.A = A; l.D = D;
     l.dx = dx; l.ddt = ddt; l.dA = dA; l.dB = dB; l.dC = dC; l.dD = dD;
+    l.init_f = fwd_init; l.init_b = rev_init; l.dinit_f = d_fwd_init; l.dinit_b = d_rev_init;
     l.scratch = scratch_ptr(workspace);
     l.batch = batch; l.L = seqlen; l.H = nheads; l.G = ngroups; l.N = dstate;
     l.bf16 = dtype == SSD_BF16;
     return to_status(ssd::launch_bwd(l, s));
+}
+
+int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, const void *C, const float *D,
+                  const void *dy, float *dx, float *ddt, float *dA, float *dB, float *dC, float *dD, int batch,
+                  int seqlen, int nheads, int headdim, int dstate, int ngroups, int dtype, void *workspace,
+                  size_t ws_bytes, void *stream) {
+    return ssd_bidir_bwd_seeded(x, dt, A, B, C, D, nullptr, nullptr, dy, dx, ddt, dA, dB, dC, dD, nullptr, nullptr,
+                                batch, seqlen, nheads, headdim, dstate, ngroups, dtype, workspace, ws_bytes, stream);
 }
 
 int ssd_bidir_fwd_x2(const void *x2, const void *dt, const float *A, const void *B, const void *C, const float *D,

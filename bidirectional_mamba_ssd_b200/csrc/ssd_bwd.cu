@@ -16,6 +16,11 @@
 //      back only what it wrote), then the run's tokens form
 //      dx_t += dt_t B_t^T g_t,  dB_t += dt_t g_t x_t,
 //      ddt_t = B_t^T g_t x_t + A a_t <g_t, h_{t-1}>,  dA += dt_t a_t <g_t, h_{t-1}>.
+// Each direction's scan may start from a given state (the forward one's
+// prefix, the reverse one's suffix: (batch, H, P, N) fp32), which then also
+// gets its gradient, the adjoint left after the direction's first token
+// (a_first g_first); the block step is the forward scan from a prefix state
+// and the reverse scan from zero.
 // The skip term adds (D_f + D_b) dy_t to dx (folded into the forward item's
 // own contribution, so each dx element receives exactly two fp32 additions,
 // whose sum does not depend on their order) and sum_t <dy_t, x_t> to dD of
@@ -85,6 +90,8 @@ struct BwdArgs {
     const float *A, *D;
     float *dx, *ddt, *dA, *dB, *dC, *dD;
     float *scratch;            // per CTA: (ceil(L / kRun) + kRun) * N * 64 floats
+    const float *init[2];      // start state per direction (batch, H, 64, N), or nullptr (zero)
+    float *dinit[2];           // its gradient per direction, or nullptr
     int batch, L, H, G;
 };
 
@@ -152,9 +159,11 @@ bwd_scan_kernel(const BwdArgs a) {
         auto token_of = [&](int k) { return reverse ? (L - 1 - k) : k; };
 
         // ---------------- 1. the scan: states to scratch, dC on the way
+        // the start state: element (n, p) of unit (b, h) sits at init[((b H + h) 64 + p) N + n]
+        const float *init = a.init[d] ? a.init[d] + ((size_t)(b * a.H + h) * kP + p) * N + q * NQ : nullptr;
         float hs[NQ];
 #pragma unroll
-        for (int j = 0; j < NQ; ++j) hs[j] = 0.f;
+        for (int j = 0; j < NQ; ++j) hs[j] = init ? init[j] : 0.f;
         for (int k0 = 0; k0 < L; k0 += kTB) {
             const int nt = min(kTB, L - k0);
             stage(k0, nt);
@@ -214,7 +223,7 @@ bwd_scan_kernel(const BwdArgs a) {
                         for (int j = 0; j < NQ; ++j) hr[j] = hc[(size_t)(q * NQ + j) * kP + p];
                     } else {
 #pragma unroll
-                        for (int j = 0; j < NQ; ++j) hr[j] = 0.f;
+                        for (int j = 0; j < NQ; ++j) hr[j] = init ? init[j] : 0.f;
                     }
                     for (int m = 0; m <= k - s0; ++m) {
                         if (m > 0) {
@@ -296,6 +305,12 @@ bwd_scan_kernel(const BwdArgs a) {
                 dA_acc += dtv * decay * ghp;
             }
         }
+        // the start state's gradient: the adjoint left after the first token
+        if (a.dinit[d]) {
+            float *di = a.dinit[d] + ((size_t)(b * a.H + h) * kP + p) * N + q * NQ;
+#pragma unroll
+            for (int j = 0; j < NQ; ++j) di[j] = gs[j];
+        }
         // dA over this item's tokens (held by threads 0..kTB-1), dD
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) {
@@ -353,6 +368,8 @@ cudaError_t launch_bwd(const BwdLaunch &l, cudaStream_t stream) {
     a.x = l.x; a.dt = l.dt; a.B = l.B; a.C = l.C; a.dy = l.dy; a.A = l.A; a.D = l.D;
     a.dx = l.dx; a.ddt = l.ddt; a.dA = l.dA; a.dB = l.dB; a.dC = l.dC; a.dD = l.dD;
     a.scratch = l.scratch;
+    a.init[0] = l.init_f; a.init[1] = l.init_b;
+    a.dinit[0] = l.dinit_f; a.dinit[1] = l.dinit_b;
     a.batch = l.batch; a.L = l.L; a.H = l.H; a.G = l.G;
     const int grid = bwd_grid(l.batch, l.H);
     // outputs that receive atomic additions start at zero

@@ -108,6 +108,8 @@ struct BwdLaunch {
     const float *A, *D;
     float *dx, *ddt, *dA, *dB, *dC, *dD;
     float *scratch;
+    const float *init_f = nullptr, *init_b = nullptr;   // start states (batch, H, 64, N) or nullptr
+    float *dinit_f = nullptr, *dinit_b = nullptr;        // their gradients, or nullptr
     int batch, L, H, G, N;
     bool bf16;
 };

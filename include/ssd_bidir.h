@@ -347,10 +347,12 @@ int ssd_prefix_state_layers(const void *x, const void *dt, const float *A, const
  *   dB, dC (2, batch, seqlen, ngroups, dstate)      fp32
  * Other arguments as for ssd_bidir_fwd (either I/O dtype). Every output is
  * overwritten. Each (batch, head, direction) runs its scan on CUDA cores in
- * fp32, keeping every state in the workspace, then the adjoint scan in the
- * opposite order; the workspace (ssd_workspace_bytes with SSD_OP_BIDIR_BWD)
- * holds seqlen states of dstate x headdim fp32 per CTA of a persistent grid
- * (about 4-8 GB at batch 32, seqlen 1024, 24 heads, dstate 128). dx gets
+ * fp32, keeping every 8th state in the workspace, then the adjoint scan in the
+ * opposite order, recomputing each run of 8 states from its checkpoint; the
+ * workspace (ssd_workspace_bytes with SSD_OP_BIDIR_BWD) holds
+ * ceil(seqlen / 8) + 8 states of dstate x headdim fp32 per CTA of a
+ * persistent grid (about 1.3 GB at batch 32, seqlen 1024, 24 heads, dstate
+ * 128). dx gets
  * exactly two additions per element and is deterministic; with ngroups <
  * nheads the heads of a group add into dB and dC atomically, in no fixed
  * order. Source: "Training Hybrid Block Diffusion Language Models with
@@ -360,6 +362,24 @@ int ssd_bidir_bwd(const void *x, const void *dt, const float *A, const void *B, 
                   const float *D, const void *dy, float *dx, float *ddt, float *dA, float *dB,
                   float *dC, float *dD, int batch, int seqlen, int nheads, int headdim, int dstate,
                   int ngroups, int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/* Backward pass of ssd_bidir_fwd_seeded (and so of ssd_block_step: a forward
+ * start state and no reverse one): ssd_bidir_bwd's gradients with each
+ * direction's scan starting from its given state, plus the gradients of the
+ * start states.
+ *   fwd_init, rev_init     (batch, nheads, headdim, dstate)   fp32, read; NULL = zero
+ *   d_fwd_init, d_rev_init (batch, nheads, headdim, dstate)   fp32, overwritten; NULL = not wanted
+ * The start state's gradient is the adjoint of the state before the
+ * direction's first token. Other arguments, workspace and determinism as for
+ * ssd_bidir_bwd. Source: "Training Hybrid Block Diffusion Language Models
+ * with Partial Bidirectionality", Methodology and Technical Contribution
+ * (training through the block-confined scans with the prefix state). */
+int ssd_bidir_bwd_seeded(const void *x, const void *dt, const float *A, const void *B,
+                         const void *C, const float *D, const float *fwd_init,
+                         const float *rev_init, const void *dy, float *dx, float *ddt, float *dA,
+                         float *dB, float *dC, float *dD, float *d_fwd_init, float *d_rev_init,
+                         int batch, int seqlen, int nheads, int headdim, int dstate, int ngroups,
+                         int dtype, void *workspace, size_t ws_bytes, void *stream);
 
 /* ssd_bidir_fwd for callers that cannot allocate device memory when they
  * call the mixer: code running under CUDA graph capture in the global mode,

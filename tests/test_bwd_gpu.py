@@ -98,3 +98,59 @@ def test_bwd_full_size_130m(ssd):
                       ("dC", np.s_[:, b, :, h])):
             e = err_f32(to_f64(g[k])[sl], o[k][sl])
             assert e <= TOL_F32, f"130M {k} unit {(b, h)}: {e:.3e}"
+
+
+# (batch, L, H, N, G, io): the seeded backward, with start states in both
+# directions (ragged length, G < H) and the block step's (a prefix state, no
+# reverse start state)
+SEEDED = [(2, 100, 4, 128, 2, "f32"), (1, 300, 2, 64, 2, "bf16"), (3, 33, 4, 128, 4, "bf16")]
+
+
+def _state(batch, H, N, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    return (torch.randn(batch, H, 64, N, generator=g, device="cuda") * 0.5).contiguous()
+
+
+@pytest.mark.parametrize("shape", SEEDED, ids=lambda s: "b%d_L%d_H%d_N%d_G%d_%s" % s)
+def test_seeded_bwd_against_oracle(ssd, shape):
+    batch, L, H, N, G, io = shape
+    inp = si.bidir_inputs(batch, L, H, 64, N, G, io, seed=L + 2 * H, device="cuda")
+    dy = _dy(inp["x"].shape, inp["x"].dtype, seed=L + 1)
+    pre, suf = _state(batch, H, N, 11), _state(batch, H, N, 12)
+    g = ssd.ssd_bidir_bwd(*(inp[k] for k in NAMES), dy, fwd_init=pre, rev_init=suf)
+    torch.cuda.synchronize()
+    assert ssd.ssd_get_device_status() == 0
+    o = oracle.bidir_bwd(*(to_f64(inp[k]) for k in NAMES), to_f64(dy), prefix=to_f64(pre), suffix=to_f64(suf))
+    _check_all(g, o, f"seeded bwd {shape}")
+    for k, ok in (("d_fwd_init", "dprefix"), ("d_rev_init", "dsuffix")):
+        e = err_f32(to_f64(g[k]), o[ok])
+        assert e <= TOL_F32, f"seeded bwd {shape} {k}: {e:.3e}"
+
+
+@pytest.mark.parametrize("shape", [(2, 64, 4, 128, 4), (3, 50, 6, 64, 3)], ids=["T64_N128", "T50_N64_ragged"])
+def test_block_step_bwd_against_oracle(ssd, shape):
+    """The block step's gradients: forward scan from a cached prefix state,
+    reverse scan from zero at the block end."""
+    batch, T, H, N, G = shape
+    data = si.blockstep_inputs(batch, 96, T, 1, H, 64, N, G, "bf16", seed=T + H, device="cuda")
+    pre_o = oracle.prefix_state(to_f64(data["x_pre"]), to_f64(data["dt_pre"]), to_f64(data["A"][0]),
+                                to_f64(data["B_pre"]))
+    pre = torch.from_numpy(pre_o.astype(np.float32)).to("cuda")
+    step = data["steps"][0]
+    dy = _dy(step["x"].shape, step["x"].dtype, seed=T)
+    g = ssd.ssd_block_step_bwd(step["x"], step["dt"], data["A"], step["B"], step["C"], data["D"], pre, dy)
+    torch.cuda.synchronize()
+    assert ssd.ssd_get_device_status() == 0
+    inp = {"x": step["x"], "dt": step["dt"], "A": data["A"], "B": step["B"], "C": step["C"], "D": data["D"]}
+    o = oracle.bidir_bwd(*(to_f64(inp[k]) for k in NAMES), to_f64(dy), prefix=to_f64(pre))
+    _check_all(g, o, f"block step bwd {shape}")
+    e = err_f32(to_f64(g["d_prefix_state"]), o["dprefix"])
+    assert e <= TOL_F32, f"block step bwd {shape} d_prefix_state: {e:.3e}"
+
+
+def test_seeded_bwd_empty(ssd):
+    inp = si.bidir_inputs(2, 0, 4, 64, 128, 4, "bf16", device="cuda")
+    pre = _state(2, 4, 128, 13)
+    g = ssd.ssd_bidir_bwd(*(inp[k] for k in NAMES), torch.empty_like(inp["x"]), fwd_init=pre)
+    torch.cuda.synchronize()
+    assert float(g["d_fwd_init"].abs().sum()) == 0.0

@@ -35,6 +35,7 @@ SIGNATURES = {
     "ssd_prefix_state_path": (_i, [_vp] * 6 + [_i] * 9 + [_vp, _sz, _vp]),
     "ssd_block_step_path": (_i, [_vp] * 8 + [_i] * 8 + [_vp, _sz, _vp]),
     "ssd_bidir_fwd_noalloc": (_i, [_vp] * 7 + [_i] * 8 + [_vp]),
+    "ssd_noalloc_get_status": (_i, [_vp]),
     "ssd_segment_states": (_i, [_vp] * 8 + [_i] * 7 + [_vp, _sz, _vp]),
     "ssd_segment_carry": (_i, [_vp] * 4 + [_i] * 2 + [_vp] * 2 + [_i] * 4 + [_vp]),
     "ssd_bidir_fwd_seeded": (_i, [_vp] * 9 + [_i] * 7 + [_vp, _sz, _vp]),

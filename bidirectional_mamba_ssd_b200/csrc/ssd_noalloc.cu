@@ -82,3 +82,13 @@ extern "C" int ssd_bidir_fwd_noalloc(const void *x, const void *dt, const float 
     if (e == cudaSuccess) return SSD_OK;
     return e == cudaErrorNotSupported ? SSD_ERR_UNSUPPORTED : SSD_ERR_CUDA;
 }
+
+// The status of the calls made through ssd_bidir_fwd_noalloc: the array's own
+// 256-byte header, read and cleared as ssd_get_device_status does for a
+// workspace (it synchronises the stream; nothing is allocated).
+extern "C" int ssd_noalloc_get_status(void *stream) {
+    void *scratch = nullptr;
+    const int rc = scratch_address(&scratch);
+    if (rc != SSD_OK) return rc;
+    return ssd_get_device_status(scratch, stream);
+}

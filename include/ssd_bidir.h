@@ -404,11 +404,18 @@ int ssd_bidir_bwd_seeded(const void *x, const void *dt, const float *A, const vo
  *    streams, other host threads) race and give wrong results. Each call
  *    clears the status header and overwrites the state area before reading it.
  *  - Device-side wait timeouts are recorded in the array's header and are not
- *    reported by this entry point. */
+ *    reported by this entry point: ssd_noalloc_get_status reads them, before
+ *    the next call clears the header. */
 int ssd_bidir_fwd_noalloc(const void *x, const void *dt, const float *A, const void *B,
                           const void *C, const float *D, void *out,
                           int batch, int seqlen, int nheads, int headdim, int dstate,
                           int ngroups, int chunk, int dtype, void *stream);
+
+/* ssd_get_device_status for ssd_bidir_fwd_noalloc: synchronise `stream`, read
+ * and clear the status header of the no-allocation entry point's own array
+ * (on the current device). Returns as ssd_get_device_status; allocates
+ * nothing. */
+int ssd_noalloc_get_status(void *stream);
 
 /* Synchronise `stream`, read and clear the workspace's status header.
  * Returns SSD_OK, SSD_ERR_TIMEOUT (a bounded device wait expired in a call

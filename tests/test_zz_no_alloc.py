@@ -8,7 +8,8 @@ previous call's contents, so a later call must not see them):
   - against the fp64 oracle, element by element on sampled (batch, head)
     units, at the bf16 parity bar of every other GPU test;
   - against ssd_bidir_fwd forced onto the same fused kernel with a workspace
-    of its own: same kernel, same inputs, so the outputs must be bit-identical.
+    of its own: same kernel, same inputs, so the outputs must be bit-identical;
+  - its status header, read through ssd_noalloc_get_status after each call.
 This file is collected last on purpose.
 """
 import ctypes
@@ -64,6 +65,8 @@ def test_noalloc_matches_oracle_and_fused_path_on_calls_in_a_row():
         exp = oracle_units(inp, units)
         for (b, h), o in exp.items():
             check(y[b, :, h], o, torch.bfloat16, f"call {k} unit ({b},{h})")
+        # the call's own status header: no bounded wait expired
+        assert lib.ssd_noalloc_get_status(ctypes.c_void_p(stream)) == 0, f"call {k}: status"
 
 
 def test_noalloc_rejects_oversized_problem():

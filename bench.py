@@ -39,9 +39,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "bidir SSD tokens/s at 130M shape L=1024 (1×B200) + % roofline"
 DEFAULT_WORKLOAD = "mixer130m_b32_L1024"
-PATH_IDS = {"auto": 0, "simt": 1, "chunked": 2, "fused": 3, "segmented": 4, "pair": 5}
+PATH_IDS = {"auto": 0, "simt": 1, "chunked": 2, "fused": 3, "segmented": 4, "pair": 5, "onetile": 7}
 # kernels each path launches per ssd_bidir_fwd call (bf16)
-LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1, "segmented": 4, "pair": 1}
+LAUNCHES_PER_CALL = {"simt": 1, "chunked": 3, "fused": 1, "segmented": 4, "pair": 1, "onetile": 1}
 # sources each path's kernels compile from (a traffic record is valid only
 # while their hash is unchanged)
 KERNEL_SOURCE = {
@@ -51,11 +51,12 @@ KERNEL_SOURCE = {
     "segmented": ("ssd_segments.cu", "ssd_fused.cu", "ssd_pair.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh",
                   "ssd_tmap.h", "ssd_common.cuh"),
     "pair": ("ssd_pair.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
+    "onetile": ("ssd_onetile.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
 }
 # kernels one call of each path launches (names as in ncu's "Kernel Name")
 KERNEL_NAMES = {"simt": ("scan_simt_kernel",), "chunked": ("tc_state_kernel", "tc_pass_kernel", "tc_out_kernel"),
                 "fused": ("tc_fused_kernel",), "segmented": ("tc_fused_kernel", "seg_scan_kernel"),
-                "pair": ("tc_pair_kernel",)}
+                "pair": ("tc_pair_kernel",), "onetile": ("onetile_kernel",)}
 # kernels a call of the path launches on some shapes only (the segmented
 # path's last step runs the two-CTA kernel where the segments suit it)
 KERNEL_OPTIONAL = {"segmented": ("tc_pair_kernel",)}
@@ -659,7 +660,7 @@ def main():
     roof = roofline_bound(w, ms_step / 1e3, peaks)
     roof.update({"traffic": traffic_record(path_name, w.name),
             "kernel": {"simt": "scan_simt_kernel", "chunked": "tc_state/tc_pass/tc_out kernels (whole step)",
-                       "fused": "tc_fused_kernel", "pair": "tc_pair_kernel",
+                       "fused": "tc_fused_kernel", "pair": "tc_pair_kernel", "onetile": "onetile_kernel",
                        "segmented": "tc_fused_kernel (forward state, reverse state) + seg_scan_kernel + the "
                                     "segments' kernel (tc_pair_kernel, else tc_fused_kernel) (whole step)"}[path_name]})
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

@@ -33,7 +33,7 @@ import torch
 
 from . import _lib as _c
 from ._lib import (SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED, SSD_PATH_SEGMENTED,  # noqa: F401
-                   SSD_PATH_PAIR, SSD_PATH_BLOCK,
+                   SSD_PATH_PAIR, SSD_PATH_BLOCK, SSD_PATH_ONETILE,
                    SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA,
                    SSD_ERR_WORKSPACE, SSD_ERR_TIMEOUT, SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE,
                    SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD, SSD_OP_BIDIR_FWD_X2, SSD_OP_MIXER_BLOCK)

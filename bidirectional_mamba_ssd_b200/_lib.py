@@ -18,6 +18,7 @@ SSD_OP_BIDIR_FWD, SSD_OP_PREFIX_STATE, SSD_OP_BLOCK_STEP, SSD_OP_BIDIR_BWD = 0, 
 SSD_OP_BIDIR_FWD_X2, SSD_OP_MIXER_BLOCK = 4, 5
 SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_CHUNKED, SSD_PATH_FUSED, SSD_PATH_SEGMENTED, SSD_PATH_PAIR = 0, 1, 2, 3, 4, 5
 SSD_PATH_BLOCK = 6
+SSD_PATH_ONETILE = 7
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int

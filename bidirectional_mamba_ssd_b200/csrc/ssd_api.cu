@@ -88,7 +88,7 @@ int bidir_impl(const void *x, const void *dt, const float *A, const void *B, con
                size_t ws_bytes, void *stream) {
     int rc = check_shape(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, dtype, true);
     if (rc != SSD_OK) return rc;
-    if (path < SSD_PATH_AUTO || path > SSD_PATH_PAIR) return SSD_ERR_INVALID_ARG;
+    if ((path < SSD_PATH_AUTO || path > SSD_PATH_PAIR) && path != SSD_PATH_ONETILE) return SSD_ERR_INVALID_ARG;
     if (!workspace) return SSD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return SSD_ERR_INVALID_ARG;
     if (ws_bytes < ssd_workspace_bytes(SSD_OP_BIDIR_FWD, batch, seqlen, nheads, headdim, dstate,
@@ -121,6 +121,7 @@ int bidir_impl(const void *x, const void *dt, const float *A, const void *B, con
     t.batch = batch; t.L = seqlen; t.H = nheads; t.G = ngroups; t.N = dstate; t.ndir = 2;
     if (path == SSD_PATH_FUSED) return to_status(ssd::launch_tc_fused(t, s));
     if (path == SSD_PATH_PAIR) return to_status(ssd::launch_tc_pair(t, s));
+    if (path == SSD_PATH_ONETILE) return to_status(ssd::launch_tc_onetile(t, s));
     if (path == SSD_PATH_SEGMENTED) {
         // at least two segments, even where one would be chosen
         const int sms = ssd::device_sms();

@@ -131,6 +131,13 @@ cudaError_t launch_tc_pair(const TcArgs &a, cudaStream_t stream);
 bool tc_blockstep_supported(int batch, int T, int H, int G, int N);
 cudaError_t launch_tc_blockstep(const TcArgs &a, cudaStream_t stream);
 
+// One-tile sequences (ssd_onetile.cu): seqlen <= 128, both scans summed,
+// bf16, ndir 2, no start states; persistent CTAs over runs of (batch, head)
+// units, G = C B^T of each direction computed once per B/C group. Needs only
+// the workspace's status header.
+bool tc_onetile_supported(int batch, int L, int H, int G, int N);
+cudaError_t launch_tc_onetile(const TcArgs &a, cudaStream_t stream);
+
 // Long sequences with fewer (batch, head) units than SMs: each sequence split
 // into S segments (seg_count: the fewest, S dividing L, that fill 4/5 of `sms`
 // SMs in one round; 1 = none), states handed across segments,

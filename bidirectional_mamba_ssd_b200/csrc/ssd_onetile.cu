@@ -17,14 +17,19 @@
 // packed 128-token shape: "Diffusion Mamba ... (LM1B, packed sequences of
 // 128)" as the pages' second workload.
 //
-// Per CTA: 256 threads, persistent over work units (a batch element, a B/C
-// group and a run of its heads). Thread 0 issues the TMA loads and the MMAs;
-// warp w owns TMEM lanes 32 (w % 4) .. + 31 (tile rows) and the 32-column
-// blocks w / 4 and w / 4 + 2 of the mask, and 32 of the 64 output columns.
-// The next unit's C and B load while the current unit's heads run; each
-// head's x loads while the head before it runs. Every wait is bounded in
-// time; an expired wait sets the workspace's timeout flag and the CTA stores
-// nothing.
+// Per CTA: 384 threads in two roles that hand work over through mbarriers,
+// persistent over a contiguous run of (batch, head) units:
+//  - warps 0..7 build the masked matrix of each head (warp w: TMEM lanes
+//    32 (w % 4) .. + 31, the 16-column half w / 4 of each 32-column block),
+//    into one of two bf16 M buffers in TMEM; thread 0 issues the TMA loads of
+//    C and B, the MMAs (G once per group, Y = M X per head) and their commits;
+//  - warps 8..11 compute each head's decay vectors two heads ahead and run
+//    each head's epilogue (Y from TMEM plus (D_f + D_b) x, written over x in
+//    shared memory, then a TMA store); their first thread issues the x loads,
+//    four heads ahead, and the stores.
+// The next group's C and B load while the current group's heads run. Every
+// wait is bounded in time; an expired wait sets the workspace's timeout flag
+// and the CTA stops storing.
 #include <cuda.h>
 #include <stdint.h>
 
@@ -41,7 +46,7 @@ using namespace sm100;
 using namespace fused;
 
 constexpr int kT = 128;          // tokens of a sequence (at most)
-constexpr int kThreads = 256;
+constexpr int kThreads = 416;    // 8 mask warps, 4 vector and epilogue warps, 1 MMA warp
 constexpr uint32_t kSlab = 16384;   // 128 rows x 128 bytes
 
 struct OneParams {
@@ -53,38 +58,50 @@ struct OneParams {
     int batch, L, H, G, hpg;    // hpg = H / G heads per B/C group
 };
 
+constexpr int kXS = 5;    // x slots (x of a head in, then its y out)
+constexpr int kVS = 3;    // decay-vector buffers
 // mbarriers: C and B of a group loaded; G of a group computed; x of a head
-// loaded (kXS slots); Y of a head computed (two buffers); all MMAs done
-constexpr int kXS = 5;
-enum { B_CB = 0, B_G, B_X, B_Y = B_X + kXS, B_END = B_Y + 2, B_COUNT };
+// loaded; Y of a head computed and read out (two buffers each); a head's
+// vectors written; a head's masked matrix built (two buffers, one arrival per
+// mask warp); all MMAs done
+enum { B_CB = 0, B_G, B_X, B_Y = B_X + kXS, B_YE = B_Y + 2, B_V = B_YE + 2, B_MF = B_V + kVS, B_END = B_MF + 2, B_COUNT };
 
 template <int N>
 struct OSmem {
     static constexpr uint32_t kTile = (N / 64) * kSlab;    // one 128 x N bf16 operand
     static constexpr uint32_t cb = 0;                      // C_f, B_f, C_b, B_b
-    static constexpr uint32_t x = 4 * kTile;               // kXS x slots (x in, then y out)
-    static constexpr uint32_t vec = x + kXS * kSlab;       // two buffers of af, ab, dtf, dtb, colf, colb
-    static constexpr uint32_t small = vec + 2 * 6 * 128 * 4;
-    static constexpr uint32_t bytes = small + 128;
+    static constexpr uint32_t x = 4 * kTile;               // kXS x slots
+    static constexpr uint32_t vec = x + kXS * kSlab;       // kVS buffers of af, ab, dtf, dtb, colf, colb
+    static constexpr uint32_t small = vec + kVS * 6 * 128 * 4;
+    static constexpr uint32_t bytes = small + 256;
 };
 
-// Inclusive prefix sum of v over the 128 threads of one direction (four
-// warps, named barrier `id`, `part` four floats of shared memory); `total`
-// the sum over all of them.
-__device__ __forceinline__ float scan128(float v, int lane, int wq, float *part, int id, float &total) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
+// A (batch, head) unit and the step to the next one in (batch, head) order.
+struct HeadPos {
+    int b, h;
+    __device__ __forceinline__ void next(int H) {
+        if (++h == H) {
+            h = 0;
+            ++b;
+        }
     }
-    if (lane == 31) part[wq] = v;
-    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
-    float before = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-        if (k < wq) before += part[k];
-    total = part[0] + part[1] + part[2] + part[3];
-    return v + before;
+};
+
+// Named barrier over `count` threads that also ORs `pred` across them.
+__device__ __forceinline__ bool bar_or(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void bar_named(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Wait until the shared-memory sources of all but the newest committed bulk
@@ -106,29 +123,24 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
-    float *part = reinterpret_cast<float *>(g + S::small + 96);     // scan partials, four per direction
-    static_assert(8 * B_COUNT + 8 <= 96, "barrier area");
+    float *part = reinterpret_cast<float *>(g + S::small + 192);    // scan partials: 4 forward, 4 reverse
+    static_assert(8 * B_COUNT + 8 <= 192, "barrier area");
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q = warp & 3, k2 = warp >> 2;
+    const int q = warp & 3;                   // TMEM lane quarter of the warp
     const int row = (q << 5) | lane;          // tile row (token t): TMEM lane
-    // the decay vectors: threads 0..127 the forward direction of token tid,
-    // threads 128..255 the reverse direction of token tid - 128
-    const int vdir = tid >> 7, vt = tid & 127;
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     // this CTA's heads: [h0, h0 + n) of the (batch, head) list
     const long long h0 = (long long)blockIdx.x * p.total / gridDim.x;
     const int n = (int)((long long)(blockIdx.x + 1) * p.total / gridDim.x - h0);
-    const long long key_last = (h0 + n - 1) / p.hpg;   // B/C group of the last head
-    auto head_b = [&](int j) { return (int)((h0 + j) / p.H); };
-    auto head_h = [&](int j) { return (int)((h0 + j) % p.H); };
-    auto head_key = [&](int j) { return (h0 + j) / p.hpg; };   // batch * G + group
+    // (batch, head) of the CTA's head j; the loops step these incrementally
+    auto head_at = [&](int j) { return HeadPos{(int)((h0 + j) / p.H), (int)((h0 + j) % p.H)}; };
 
     grid_launch_dependents();
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), i == B_MF || i == B_MF + 1 ? 8 : 1);
         fence_mbar_init();
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_out);
@@ -143,224 +155,297 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM columns: G_f [0,128), G_b [128,256), the masked matrix M [256,384)
-    // (bf16: matrix columns [16 k, 16 k + 16) in TMEM columns [16 k, 16 k + 8)),
-    // Y of even heads [384,448), of odd heads [448,512)
-    const uint32_t tGf = tmem, tGb = tmem + 128, tM = tmem + 256;
+    // TMEM columns: G_f [0,128), G_b [128,256); the masked matrix of even
+    // heads [256,320), of odd heads [320,384) (bf16, two per column: matrix
+    // columns [16 k, 16 k + 16) in TMEM columns [8 k, 8 k + 8)); Y of even
+    // heads [384,448), of odd heads [448,512)
+    const uint32_t tGf = tmem, tGb = tmem + 128;
+    auto tM = [&](int j) { return tmem + 256 + 64 * (j & 1); };
     auto tY = [&](int j) { return tmem + 384 + 64 * (j & 1); };
     const uint32_t lane_off = (uint32_t)(q << 5) << 16;
     auto xslot = [&](int j) { return S::x + (uint32_t)(j % kXS) * kSlab; };
-    auto vbuf = [&](int j) { return reinterpret_cast<float *>(g + S::vec + (j & 1) * 6 * 512); };
+    auto vbuf = [&](int j) { return reinterpret_cast<float *>(g + S::vec + (j % kVS) * 6 * 512); };
     // the kernel ahead in the stream has finished before any global access
     grid_dependency_wait();
 
-    // thread 0's copies in flight: x loads of heads [x_waited, x_issued), C/B
-    // loads of groups [cb_waited, cb_issued)
-    int x_issued = 0, x_waited = 0, cb_issued = 0, cb_waited = 0;
-    auto load_cb = [&](long long key) {
-        const int b = (int)(key / p.G), gg = (int)(key % p.G);
-        mbar_arrive_expect_tx(bar(B_CB), 4 * NSLAB * kSlab);
-        for (int d = 0; d < 2; ++d)
-            for (int sl = 0; sl < NSLAB; ++sl) {
-                tma_load_5d(base + S::cb + (2 * d) * S::kTile + sl * kSlab, &tm_c, bar(B_CB), 64 * sl, gg, 0, b, d);
-                tma_load_5d(base + S::cb + (2 * d + 1) * S::kTile + sl * kSlab, &tm_b, bar(B_CB), 64 * sl, gg, 0, b,
-                            d);
-            }
-        ++cb_issued;
-    };
-    auto load_x = [&](int j) {
-        mbar_arrive_expect_tx(bar(B_X + j % kXS), kSlab);
-        tma_load_4d(base + xslot(j), &tm_x, bar(B_X + j % kXS), 0, head_h(j), 0, head_b(j));
-        ++x_issued;
-    };
-    constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);   // C (K) x B (K)
-    constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);     // M (K) x X (MN)
-    // G_f = C_f B_f^T and G_b = C_b B_b^T of the group in shared memory
-    auto issue_g = [&]() {
-        const bool ok = mbar_wait_ool(bar(B_CB), (uint32_t)cb_waited & 1u, abort_flag, p.status, 1001);
-        ++cb_waited;
-        tc_fence_after();
-        if (ok) {
-            for (int d = 0; d < 2; ++d) {
-                const uint32_t ca = base + S::cb + (2 * d) * S::kTile, ba = ca + S::kTile;
+    if (warp < 8) {
+        // ================= mask builders
+        const int half = warp >> 2, c0 = 16 * half;
+        HeadPos pos = head_at(0);
+        int hg = pos.h % p.hpg;     // head j's place in its B/C group
+        bool ok = true;             // warp-uniform: every wait of this warp so far succeeded
+        int gk = 0;                 // groups begun
 #pragma unroll 1
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
-                    mma_bf16_ss(d ? tGb : tGf, sdesc_sw128(ca + ko, 0, 1024), sdesc_sw128(ba + ko, 0, 1024), id_g,
-                                k > 0);
-                }
-            }
-        }
-        mma_commit(bar(B_G));
-    };
-
-    // the per-head vectors of head j into buffer j & 1: the direction's decay
-    // sums a (forward: A_f times the sum of dt_f over tokens <= t; reverse:
-    // A_b times the sum of dt_b over tokens >= t), dt and the column factors
-    // (exp(a_e - a_s) dt_s with e the last (forward) or first (reverse) token
-    // of the 32-token block of s)
-    auto vectors = [&](int j, float v, float A) {
-        float tot;
-        const float pf = scan128(v, lane, q, part + 4 * vdir, 1 + vdir, tot);
-        const float a = vdir == 0 ? A * pf : A * (tot - pf + v);
-        const float edge = __shfl_sync(0xffffffffu, a, vdir == 0 ? 31 : 0);
-        float *V = vbuf(j);
-        V[vdir * 128 + vt] = a;                          // af, ab
-        V[256 + vdir * 128 + vt] = v;                    // dtf, dtb
-        V[512 + vdir * 128 + vt] = __expf(edge - a) * v; // colf, colb
-    };
-    // dt and A of head j for this thread's direction and token
-    auto load_dt = [&](int j, float &v, float &A) {
-        const int b = head_b(j), h = head_h(j);
-        A = __ldg(p.A + vdir * p.H + h);
-        v = vt < p.L ? __bfloat162float(p.dt[(((size_t)vdir * p.batch + b) * p.L + vt) * p.H + h]) : 0.f;
-    };
-
-    if (tid == 0) {
-        load_cb(head_key(0));
-        load_x(0);
-        if (n > 1) load_x(1);
-    }
-    {
-        float v, A;
-        load_dt(0, v, A);
-        vectors(0, v, A);
-    }
-    if (tid == 0) issue_g();
-    __syncthreads();
-
-    bool ok = true;              // warp-uniform: every wait of this warp so far succeeded
-    int gk = 0;                  // this CTA's group count before the current head
-    float ds_prev = 0.f;         // D_f + D_b of head j - 1
-    bool failed = false;
-#pragma unroll 1
-    for (int j = 0; j <= n; ++j) {
-        float ds_cur = 0.f;
-        if (j < n) {
-            // prefetch the next head's dt and A; D of this head
-            float v_next = 0.f, A_next = 0.f;
-            if (j + 1 < n) load_dt(j + 1, v_next, A_next);
-            const int hj = head_h(j);
-            ds_cur = __ldg(p.D + hj) + __ldg(p.D + p.H + hj);
-            const bool first = j == 0 || head_key(j) != head_key(j - 1);
-            if (first) {
+        for (int j = 0; j < n; ++j) {
+            if (j > 0 && ++hg == p.hpg) hg = 0;
+            if (j == 0 || hg == 0) {
                 ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_G), (uint32_t)gk & 1u, abort_flag, p.status,
                                                                  1002));
                 ++gk;
-                // G of this group is in TMEM: C and B of the next group load
-                if (tid == 0 && ok && head_key(j) < key_last) load_cb(head_key(j) + 1);
             }
-            // ---------------- the masked matrix of head j: row `row`, columns
-            // [32 J + 16 k2, 32 J + 16 k2 + 16) of each 32-column block J
-            // (M is free once head j - 1's MMA has completed)
-            if (j > 0)
-                ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_Y + ((j - 1) & 1)), (uint32_t)((j - 1) >> 1) & 1u,
-                                                                 abort_flag, p.status, 1003));
+            ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_V + j % kVS), (uint32_t)(j / kVS) & 1u,
+                                                             abort_flag, p.status, 1003));
+            // M of head j - 2 has been read by its MMA
+            if (j >= 2)
+                ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_Y + (j & 1)), (uint32_t)((j - 2) >> 1) & 1u,
+                                                                 abort_flag, p.status, 1004));
             tc_fence_after();
             if (ok) {
+                // row `row`, columns [32 J + c0, 32 J + c0 + 16) of every block J:
+                // all G loads first, then the diagonal block and the three others
                 const float *V = vbuf(j);
                 const MaskVectors mv{V, V + 128, V + 256, V + 384, V + 512, V + 640};
                 const float my_af = V[row], my_ab = V[128 + row];
-                const int c0 = 16 * k2;
-#pragma unroll 1
-                for (int J = 0; J < 4; ++J) {
-                    uint32_t packed[8];
-                    if (J == q) {
-                        uint32_t gf[16], gb[16];
-                        tmem_ld16(tGf + lane_off + J * 32 + c0, gf);
-                        tmem_ld16(tGb + lane_off + J * 32 + c0, gb);
-                        tmem_wait_ld();
-                        mask_diag<16>(J, c0, row, my_af, my_ab, gf, gb, mv, packed);
-                    } else {
-                        uint32_t gv[16];
-                        tmem_ld16((J < q ? tGf : tGb) + lane_off + J * 32 + c0, gv);
-                        tmem_wait_ld();
-                        mask_offdiag<16>(J, c0, row, my_af, my_ab, gv, mv, packed);
-                    }
-                    tmem_st8(tM + lane_off + J * 32 + c0, packed);
+                uint32_t gdf[16], gdb[16], go[3][16];
+                tmem_ld16(tGf + lane_off + q * 32 + c0, gdf);
+                tmem_ld16(tGb + lane_off + q * 32 + c0, gdb);
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int J = (q + 1 + k) & 3;
+                    tmem_ld16((J < q ? tGf : tGb) + lane_off + J * 32 + c0, go[k]);
+                }
+                tmem_wait_ld();
+                const uint32_t mrow = tM(j) + lane_off + 8 * half;
+                uint32_t packed[8];
+                mask_diag<16>(q, c0, row, my_af, my_ab, gdf, gdb, mv, packed);
+                tmem_st8(mrow + 16 * q, packed);
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int J = (q + 1 + k) & 3;
+                    mask_offdiag<16>(J, c0, row, my_af, my_ab, go[k], mv, packed);
+                    tmem_st8(mrow + 16 * J, packed);
                 }
                 tmem_wait_st();
             }
-            if (j + 1 < n) vectors(j + 1, v_next, A_next);
+            tc_fence_before();
+            __syncwarp();
+            if (!ok) break;
+            if (lane == 0) mbar_arrive(bar(B_MF + (j & 1)));    // this warp's rows of M_j are built
         }
-        tc_fence_before();
-        failed = __syncthreads_or(!ok);
-        if (failed) break;
-        if (tid == 0) {
-            tc_fence_after();
-            if (j < n) {
-                // Y_j = M X_j
-                const bool xok = mbar_wait_ool(bar(B_X + j % kXS), (uint32_t)(j / kXS) & 1u, abort_flag, p.status, 1004);
-                ++x_waited;
-                if (xok && !*abort_flag) {
-                    const uint32_t xa = base + xslot(j);
-#pragma unroll 1
-                    for (int k = 0; k < 128 / 16; ++k)
-                        mma_bf16_ts(tY(j), tM + 16 * k, sdesc_sw128(xa + k * 2048, kSlab, 1024), id_o, k > 0);
-                }
-                mma_commit(bar(B_Y + (j & 1)));
-                // the next head starts a new group: its G, once all rows of M_j are built
-                if (j + 1 < n && head_key(j + 1) != head_key(j)) issue_g();
-            }
-            // y of head j - 2 (written over its x in the epilogue of the last iteration)
-            if (j >= 2) {
-                tma_store_4d(&tm_out, base + xslot(j - 2), 0, head_h(j - 2), 0, head_b(j - 2));
-                tma_store_commit();
-            }
-            // x of head j + 2 into the slot of head j - 3, once its y has left
-            if (j + 2 < n) {
-                tma_store_wait_read1();
-                load_x(j + 2);
-            }
-        }
-        // ---------------- epilogue of head j - 1: y = Y + (D_f + D_b) x, in
-        // place of x (row `row`, columns [32 k2, 32 k2 + 32))
-        if (j > 0) {
-            const int e = j - 1;
-            ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_Y + (e & 1)), (uint32_t)(e >> 1) & 1u, abort_flag,
-                                                             p.status, 1005) &&
-                                             mbar_wait_ool(bar(B_X + e % kXS), (uint32_t)(e / kXS) & 1u, abort_flag,
-                                                           p.status, 1006));
-            tc_fence_after();
-            if (ok) {
-                uint32_t yv[32];
-                tmem_ld32(tY(e) + lane_off + k2 * 32, yv);
-                tmem_wait_ld();
-                uint8_t *xs = g + xslot(e);
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint4 *ptr = reinterpret_cast<uint4 *>(xs + sw128_offset(row, k2 * 4 + cc));
-                    const uint4 xv = *ptr;
-                    const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int j2 = 0; j2 < 4; ++j2) {
-                        const int c = cc * 8 + 2 * j2;
-                        o[j2] = pack_bf16x2(__uint_as_float(yv[c]) + ds_prev * bf2f(xu[j2] & 0xffffu),
-                                            __uint_as_float(yv[c + 1]) + ds_prev * bf2f(xu[j2] >> 16));
+    } else if (warp == 12) {
+        // ================= C/B loads and the MMAs (one thread)
+        if (lane == 0) {
+            constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);   // C (K) x B (K)
+            constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);     // M (K) x X (MN)
+            // C/B loads in flight: groups [cb_waited, cb_issued)
+            int cb_issued = 0, cb_waited = 0;
+            auto load_cb = [&](long long key) {
+                const int b = (int)(key / p.G), gg = (int)(key % p.G);
+                mbar_arrive_expect_tx(bar(B_CB), 4 * NSLAB * kSlab);
+                for (int d = 0; d < 2; ++d)
+                    for (int sl = 0; sl < NSLAB; ++sl) {
+                        tma_load_5d(base + S::cb + (2 * d) * S::kTile + sl * kSlab, &tm_c, bar(B_CB), 64 * sl, gg,
+                                    0, b, d);
+                        tma_load_5d(base + S::cb + (2 * d + 1) * S::kTile + sl * kSlab, &tm_b, bar(B_CB), 64 * sl,
+                                    gg, 0, b, d);
                     }
-                    *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+                ++cb_issued;
+            };
+            // G_f = C_f B_f^T and G_b = C_b B_b^T of the group in shared memory
+            auto issue_g = [&]() {
+                const bool okc = mbar_wait_ool(bar(B_CB), (uint32_t)cb_waited & 1u, abort_flag, p.status, 1001);
+                ++cb_waited;
+                tc_fence_after();
+                if (okc) {
+                    for (int d = 0; d < 2; ++d) {
+                        const uint32_t ca = base + S::cb + (2 * d) * S::kTile, ba = ca + S::kTile;
+#pragma unroll 1
+                        for (int k = 0; k < N / 16; ++k) {
+                            const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
+                            mma_bf16_ss(d ? tGb : tGf, sdesc_sw128(ca + ko, 0, 1024), sdesc_sw128(ba + ko, 0, 1024),
+                                        id_g, k > 0);
+                        }
+                    }
                 }
-                fence_proxy_async_smem();
+                mma_commit(bar(B_G));
+            };
+            // head j: its batch element, its group `gg` and its place `hg` in the group
+            HeadPos pos = head_at(0);
+            int gg = pos.h / p.hpg, hg = pos.h - gg * p.hpg;
+            load_cb((long long)pos.b * p.G + gg);
+            issue_g();
+            int gk = 0;
+#pragma unroll 1
+            for (int j = 0; j < n; ++j) {
+                if (j > 0) {
+                    pos.next(p.H);
+                    if (++hg == p.hpg) {
+                        hg = 0;
+                        gg = pos.h == 0 ? 0 : gg + 1;
+                    }
+                }
+                bool okm = true;
+                if (j == 0 || hg == 0) {
+                    // G of this group is in TMEM: C and B of the next group, if this
+                    // CTA has one, may load
+                    okm = mbar_wait_ool(bar(B_G), (uint32_t)gk & 1u, abort_flag, p.status, 1009);
+                    ++gk;
+                    if (okm && j + (p.hpg - hg) < n) load_cb((long long)pos.b * p.G + gg + 1);
+                }
+                // Y_j = M_j X_j, once M_j is built, x_j is in and Y of head j - 2 has been read out
+                okm = okm && mbar_wait_ool(bar(B_MF + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_flag, p.status, 1010);
+                okm = okm && mbar_wait_ool(bar(B_X + j % kXS), (uint32_t)(j / kXS) & 1u, abort_flag, p.status, 1005);
+                if (j >= 2)
+                    okm = okm && mbar_wait_ool(bar(B_YE + (j & 1)), (uint32_t)((j - 2) >> 1) & 1u, abort_flag,
+                                               p.status, 1006);
+                tc_fence_after();
+                if (!okm) break;
+                const uint32_t xa = base + xslot(j);
+#pragma unroll 1
+                for (int k = 0; k < 128 / 16; ++k)
+                    mma_bf16_ts(tY(j), tM(j) + 8 * k, sdesc_sw128(xa + k * 2048, kSlab, 1024), id_o, k > 0);
+                mma_commit(bar(B_Y + (j & 1)));
+                // the next head starts a new group: its G, now that every row of M_j is built
+                if (j + 1 < n && hg + 1 == p.hpg) issue_g();
+            }
+            // teardown: every MMA and C/B load of this thread has finished
+            mma_commit(bar(B_END));
+            mbar_drain(bar(B_END), 0);
+            for (int k = cb_waited; k < cb_issued; ++k) mbar_drain(bar(B_CB), (uint32_t)k & 1u);
+        }
+        __syncwarp();
+    } else {
+        // ================= decay vectors, epilogue, x loads and y stores (warps 8..11)
+        const int r = tid - 256;                  // token of the vectors; tile row of the epilogue
+        const bool leader = r == 0;
+        int x_issued = 0, x_seen = 0;             // the leader's x loads: heads [x_seen, x_issued) in flight
+        HeadPos pos_x = head_at(0);               // the leader's next x load
+        auto load_x = [&](int j) {
+            mbar_arrive_expect_tx(bar(B_X + j % kXS), kSlab);
+            tma_load_4d(base + xslot(j), &tm_x, bar(B_X + j % kXS), 0, pos_x.h, 0, pos_x.b);
+            pos_x.next(p.H);
+            ++x_issued;
+        };
+        if (leader)
+            for (int j = 0; j < kXS - 1 && j < n; ++j) load_x(j);
+        // dt of a head at token r, both directions, and its A
+        struct DtA { float vf, vb, af, ab; };
+        HeadPos pos_dt = head_at(0);              // the next dt load
+        auto load_dt = [&](int j) {
+            DtA d{0.f, 0.f, 0.f, 0.f};
+            if (j < n) {
+                const int b = pos_dt.b, h = pos_dt.h;
+                pos_dt.next(p.H);
+                d.af = __ldg(p.A + h);
+                d.ab = __ldg(p.A + p.H + h);
+                if (r < p.L) {
+                    d.vf = __bfloat162float(p.dt[((size_t)b * p.L + r) * p.H + h]);
+                    d.vb = __bfloat162float(p.dt[(((size_t)p.batch + b) * p.L + r) * p.H + h]);
+                }
+            }
+            return d;
+        };
+        // the vectors of head j into buffer j % kVS: the decay sums (forward:
+        // A_f times the sum of dt_f over tokens <= t; reverse: A_b times the
+        // sum of dt_b over tokens >= t), dt and the column factors (exp(a_e -
+        // a_s) dt_s, e the last (forward) or first (reverse) token of the
+        // 32-token block of s); then the mask builders may take head j
+        auto vectors = [&](int j, const DtA &d) {
+            float pf = d.vf, pb = d.vb;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float nf = __shfl_up_sync(0xffffffffu, pf, o), nb = __shfl_up_sync(0xffffffffu, pb, o);
+                if (lane >= o) {
+                    pf += nf;
+                    pb += nb;
+                }
+            }
+            if (lane == 31) {
+                part[q] = pf;
+                part[4 + q] = pb;
+            }
+            bar_named(2, 128);
+            float bf = 0.f, bb = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (k < q) {
+                    bf += part[k];
+                    bb += part[4 + k];
+                }
+            const float totb = part[4] + part[5] + part[6] + part[7];
+            const float af = d.af * (pf + bf);
+            const float ab = d.ab * (totb - (pb + bb) + d.vb);
+            const float ef = __shfl_sync(0xffffffffu, af, 31), eb = __shfl_sync(0xffffffffu, ab, 0);
+            float *V = vbuf(j);
+            V[r] = af;
+            V[128 + r] = ab;
+            V[256 + r] = d.vf;
+            V[384 + r] = d.vb;
+            V[512 + r] = __expf(ef - af) * d.vf;
+            V[640 + r] = __expf(eb - ab) * d.vb;
+            bar_named(2, 128);
+            if (leader) mbar_arrive(bar(B_V + j % kVS));
+        };
+        // vectors of heads 0 and 1; dt of head 2 in flight
+        DtA dn = load_dt(0);
+        vectors(0, dn);
+        dn = load_dt(1);
+        DtA dn2 = load_dt(2);
+        if (n > 1) vectors(1, dn);
+        dn = dn2;
+        bool ok = true;
+        HeadPos pos_e = head_at(0);               // head i of the epilogue
+#pragma unroll 1
+        for (int i = 0; i < n; ++i) {
+            if (i > 0) pos_e.next(p.H);
+            // vectors of head i + 2 (their buffer was last read by the mask of head
+            // i - 1, whose MMA the epilogue of head i - 1 has seen complete)
+            if (i + 2 < n) {
+                dn2 = load_dt(i + 3);
+                vectors(i + 2, dn);
+                dn = dn2;
+            }
+            const int hi = pos_e.h;
+            const float ds = __ldg(p.D + hi) + __ldg(p.D + p.H + hi);
+            // ---------------- epilogue of head i: y = Y + (D_f + D_b) x, written over x
+            ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_Y + (i & 1)), (uint32_t)(i >> 1) & 1u, abort_flag,
+                                                             p.status, 1007) &&
+                                             mbar_wait_ool(bar(B_X + i % kXS), (uint32_t)(i / kXS) & 1u, abort_flag,
+                                                           p.status, 1008));
+            if (leader) x_seen = i + 1;
+            tc_fence_after();
+            uint32_t ya[32], yb[32];
+            if (ok) {
+                tmem_ld32(tY(i) + lane_off, ya);
+                tmem_ld32(tY(i) + lane_off + 32, yb);
+                tmem_wait_ld();
+            }
+            tc_fence_before();
+            if (bar_or(2, 128, !ok)) break;
+            if (leader) mbar_arrive(bar(B_YE + (i & 1)));    // Y_i read out: the MMA of head i + 2 may write it
+            uint8_t *xs = g + xslot(i);
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                uint4 *ptr = reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc));
+                const uint4 xv = *ptr;
+                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int j2 = 0; j2 < 4; ++j2) {
+                    const int c = (cc & 3) * 8 + 2 * j2;
+                    const uint32_t y0 = cc < 4 ? ya[c] : yb[c], y1 = cc < 4 ? ya[c + 1] : yb[c + 1];
+                    o[j2] = pack_bf16x2(__uint_as_float(y0) + ds * bf2f(xu[j2] & 0xffffu),
+                                        __uint_as_float(y1) + ds * bf2f(xu[j2] >> 16));
+                }
+                *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            fence_proxy_async_smem();
+            bar_named(2, 128);
+            if (leader) {
+                tma_store_4d(&tm_out, base + xslot(i), 0, hi, 0, pos_e.b);
+                tma_store_commit();
+                // x of head i + 4 into the slot of head i - 1, once its y has left
+                if (i + kXS - 1 < n) {
+                    tma_store_wait_read1();
+                    load_x(i + kXS - 1);
+                }
             }
         }
-        ds_prev = ds_cur;
-    }
-    // y of the last head
-    tc_fence_before();
-    failed = __syncthreads_or(failed || !ok);
-    if (tid == 0) {
-        if (!failed && n >= 1) {
-            tma_store_4d(&tm_out, base + xslot(n - 1), 0, head_h(n - 1), 0, head_b(n - 1));
-            tma_store_commit();
+        if (leader) {
+            // teardown: this thread's x loads and y stores have finished
+            for (int k = x_seen; k < x_issued; ++k) mbar_drain(bar(B_X + k % kXS), (uint32_t)(k / kXS) & 1u);
+            tma_store_wait_all();
         }
-        // teardown: every MMA, load and store of this CTA has finished before
-        // its shared memory and TMEM are released
-        mma_commit(bar(B_END));
-        mbar_drain(bar(B_END), 0);
-        for (int k = x_waited; k < x_issued; ++k) mbar_drain(bar(B_X + k % kXS), (uint32_t)(k / kXS) & 1u);
-        for (int k = cb_waited; k < cb_issued; ++k) mbar_drain(bar(B_CB), (uint32_t)k & 1u);
-        tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();

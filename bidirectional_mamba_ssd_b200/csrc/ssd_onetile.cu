@@ -87,6 +87,86 @@ struct HeadPos {
     }
 };
 
+// ---- packed fp32 pairs (sm_100a f32x2 arithmetic): two IEEE products per
+// instruction, bit-identical to two scalar multiplies
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2u(uint32_t lo, uint32_t hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float lo_of(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_of(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+// a pair of fp32 values rounded to a bf16 pair (low element in the low half)
+__device__ __forceinline__ uint32_t bf16x2_of(uint64_t v) {
+    uint32_t d;
+    asm("{\n\t.reg .f32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}" : "=r"(d) : "l"(v));
+    return d;
+}
+
+// Off the diagonal: 16 columns [s1, s1 + 16) of one row of the masked matrix,
+// g * (r * col[s]) with r the row's factor for the column block (forward or
+// reverse, as in mask_offdiag) and col the direction's column factors.
+__device__ __forceinline__ void offdiag16(const uint32_t (&g)[16], float r, const float *col,
+                                          uint32_t (&packed)[8]) {
+    const uint64_t rr = f2(r, r);
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+        const float4 c = *reinterpret_cast<const float4 *>(col + k);
+        packed[k / 2] = bf16x2_of(mul2(f2u(g[k], g[k + 1]), mul2(rr, f2(c.x, c.y))));
+        packed[k / 2 + 1] = bf16x2_of(mul2(f2u(g[k + 2], g[k + 3]), mul2(rr, f2(c.z, c.w))));
+    }
+}
+
+// The diagonal block: columns [s1, s1 + 16) of row `row` (s1 = 32 J + c0, J =
+// row / 32). The forward term g_f (r_f colf) is kept for s <= t and the reverse
+// term g_b (r_b colb) for s >= t; on the row's own token both are kept, each
+// equal to G dt there (the two factors of exp(a_t - a_e) exp(a_e - a_t)).
+// Factorised while the block's decay span is below kMaxSpan, else one
+// exponential per entry (as mask_diag).
+__device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, float my_ab, const uint32_t (&gf)[16],
+                                       const uint32_t (&gb)[16], const MaskVectors &v, uint32_t (&packed)[8]) {
+    const int s0 = J * 32, s1 = s0 + c0;
+    const int rr = row - s1;   // the row's token relative to the first column
+    const float span_f = v.af[s0] - v.af[s0 + 31], span_b = v.ab[s0 + 31] - v.ab[s0];
+    if (span_f < kMaxSpan && span_b < kMaxSpan) {
+        const uint64_t rf = f2(__expf(my_af - v.af[s0 + 31]), __expf(my_af - v.af[s0 + 31]));
+        const uint64_t rb = f2(__expf(my_ab - v.ab[s0]), __expf(my_ab - v.ab[s0]));
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+            const float2 cf = *reinterpret_cast<const float2 *>(v.colf + s1 + k);
+            const float2 cb = *reinterpret_cast<const float2 *>(v.colb + s1 + k);
+            const uint64_t pf = mul2(f2u(gf[k], gf[k + 1]), mul2(rf, f2(cf.x, cf.y)));
+            const uint64_t pb = mul2(f2u(gb[k], gb[k + 1]), mul2(rb, f2(cb.x, cb.y)));
+            const float m0 = (k <= rr ? lo_of(pf) : 0.f) + (k >= rr ? lo_of(pb) : 0.f);
+            const float m1 = (k + 1 <= rr ? hi_of(pf) : 0.f) + (k + 1 >= rr ? hi_of(pb) : 0.f);
+            packed[k / 2] = pack_bf16x2(m0, m1);
+        }
+    } else {
+        float m[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const int s = s1 + c;
+            const float gfv = __uint_as_float(gf[c]), gbv = __uint_as_float(gb[c]);
+            // the exponent of the selected side is <= 0
+            m[c] = c < rr ? gfv * v.dtf[s] * __expf(my_af - v.af[s])
+                 : c > rr ? gbv * v.dtb[s] * __expf(my_ab - v.ab[s])
+                          : gfv * v.dtf[s] + gbv * v.dtb[s];
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) packed[k] = pack_bf16x2(m[2 * k], m[2 * k + 1]);
+    }
+}
+
 // Named barrier over `count` threads that also ORs `pred` across them.
 __device__ __forceinline__ bool bar_or(int id, int count, bool pred) {
     uint32_t r;
@@ -207,12 +287,15 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tmem_wait_ld();
                 const uint32_t mrow = tM(j) + lane_off + 8 * half;
                 uint32_t packed[8];
-                mask_diag<16>(q, c0, row, my_af, my_ab, gdf, gdb, mv, packed);
+                diag16(q, c0, row, my_af, my_ab, gdf, gdb, mv, packed);
                 tmem_st8(mrow + 16 * q, packed);
 #pragma unroll
                 for (int k = 0; k < 3; ++k) {
                     const int J = (q + 1 + k) & 3;
-                    mask_offdiag<16>(J, c0, row, my_af, my_ab, go[k], mv, packed);
+                    // forward blocks (left of the row's own) scale by exp(a_t - a_e), e
+                    // the block's last token; reverse ones by exp(a'_t - a'_b), b its first
+                    const float r = J < q ? __expf(my_af - V[J * 32 + 31]) : __expf(my_ab - V[128 + J * 32]);
+                    offdiag16(go[k], r, (J < q ? V + 512 : V + 640) + J * 32 + c0, packed);
                     tmem_st8(mrow + 16 * J, packed);
                 }
                 tmem_wait_st();

@@ -46,7 +46,7 @@ using namespace sm100;
 using namespace fused;
 
 constexpr int kT = 128;          // tokens of a sequence (at most)
-constexpr int kThreads = 416;    // 8 mask warps, 4 vector and epilogue warps, 1 MMA warp
+constexpr int kThreads = 512;    // 8 mask warps, 4 epilogue warps, 1 MMA warp, 3 vector warps
 constexpr uint32_t kSlab = 16384;   // 128 rows x 128 bytes
 
 struct OneParams {
@@ -63,8 +63,11 @@ constexpr int kVS = 3;    // decay-vector buffers
 // mbarriers: C and B of a group loaded; G of a group computed; x of a head
 // loaded; Y of a head computed and read out (two buffers each); a head's
 // vectors written; a head's masked matrix built (two buffers, one arrival per
-// mask warp); all MMAs done
-enum { B_CB = 0, B_G, B_X, B_Y = B_X + kXS, B_YE = B_Y + 2, B_V = B_YE + 2, B_MF = B_V + kVS, B_END = B_MF + 2, B_COUNT };
+// mask warp); a vector buffer read by every mask warp; all MMAs done
+enum {
+    B_CB = 0, B_G, B_X, B_Y = B_X + kXS, B_YE = B_Y + 2, B_V = B_YE + 2, B_MF = B_V + kVS, B_VE = B_MF + 2,
+    B_END = B_VE + kVS, B_COUNT
+};
 
 template <int N>
 struct OSmem {
@@ -203,7 +206,6 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     uint64_t *bars = reinterpret_cast<uint64_t *>(g + S::small);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g + S::small + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(g + S::small + 8 * B_COUNT + 4);
-    float *part = reinterpret_cast<float *>(g + S::small + 192);    // scan partials: 4 forward, 4 reverse
     static_assert(8 * B_COUNT + 8 <= 192, "barrier area");
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -220,7 +222,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     grid_launch_dependents();
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), i == B_MF || i == B_MF + 1 ? 8 : 1);
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), (i >= B_MF && i < B_VE + kVS) ? 8 : 1);
         fence_mbar_init();
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_out);
@@ -303,7 +305,95 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc_fence_before();
             __syncwarp();
             if (!ok) break;
-            if (lane == 0) mbar_arrive(bar(B_MF + (j & 1)));    // this warp's rows of M_j are built
+            if (lane == 0) {
+                mbar_arrive(bar(B_MF + (j & 1)));    // this warp's rows of M_j are built
+                mbar_arrive(bar(B_VE + j % kVS));    // and it is done with head j's vectors
+            }
+        }
+    } else if (warp >= 13) {
+        // ================= decay vectors: warp 13 + k takes heads j = k (mod 3),
+        // the whole head in one warp (lane l: tokens 4 l .. 4 l + 3, both
+        // directions), into buffer j % 3 once the mask warps are done with head
+        // j - 3. Per head: the decay sums (forward: A_f times the sum of dt_f
+        // over tokens <= t; reverse: A_b times the sum of dt_b over tokens >=
+        // t), dt, and the column factors exp(a_e - a_s) dt_s (e the last
+        // (forward) or first (reverse) token of the 32-token block of s)
+        const int vw = warp - 13;
+        const int t0 = 4 * lane;
+        bool ok = true;
+        HeadPos pos = head_at(vw);
+        float vf[4], vb[4], Af = 0.f, Ab = 0.f;
+        auto load = [&](int j) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) vf[k] = vb[k] = 0.f;
+            if (j < n) {
+                Af = __ldg(p.A + pos.h);
+                Ab = __ldg(p.A + p.H + pos.h);
+                const __nv_bfloat16 *df = p.dt + (size_t)pos.b * p.L * p.H + pos.h;
+                const __nv_bfloat16 *db = df + (size_t)p.batch * p.L * p.H;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (t0 + k < p.L) {
+                        vf[k] = __bfloat162float(df[(size_t)(t0 + k) * p.H]);
+                        vb[k] = __bfloat162float(db[(size_t)(t0 + k) * p.H]);
+                    }
+                pos.next(p.H);
+                pos.next(p.H);
+                pos.next(p.H);
+            }
+        };
+        load(vw);
+#pragma unroll 1
+        for (int j = vw; j < n; j += kVS) {
+            const float cf[4] = {vf[0], vf[1], vf[2], vf[3]}, cb[4] = {vb[0], vb[1], vb[2], vb[3]};
+            const float A_f = Af, A_b = Ab;
+            load(j + kVS);     // this warp's next head, in flight while this one is computed
+            // inclusive sums over the lane's four tokens, then across the warp
+            float sf[4], sb[4];
+            sf[0] = cf[0];
+            sb[0] = cb[0];
+#pragma unroll
+            for (int k = 1; k < 4; ++k) {
+                sf[k] = sf[k - 1] + cf[k];
+                sb[k] = sb[k - 1] + cb[k];
+            }
+            float xf = sf[3], xb = sb[3];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float nf = __shfl_up_sync(0xffffffffu, xf, o), nb = __shfl_up_sync(0xffffffffu, xb, o);
+                if (lane >= o) {
+                    xf += nf;
+                    xb += nb;
+                }
+            }
+            const float tot_b = __shfl_sync(0xffffffffu, xb, 31);
+            const float pre_f = xf - sf[3], pre_b = xb - sb[3];     // sums over the lanes before this one
+            float af[4], ab[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                af[k] = A_f * (pre_f + sf[k]);
+                ab[k] = A_b * (tot_b - (pre_b + sb[k]) + cb[k]);
+            }
+            // block edges: the last token of the lane's 32-token block (forward),
+            // its first (reverse)
+            const float ef = __shfl_sync(0xffffffffu, af[3], lane | 7), eb = __shfl_sync(0xffffffffu, ab[0], lane & ~7);
+            if (j >= kVS)
+                ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_VE + j % kVS), (uint32_t)(j / kVS - 1) & 1u,
+                                                                 abort_flag, p.status, 1011));
+            if (!ok) break;
+            float *V = vbuf(j);
+            *reinterpret_cast<float4 *>(V + t0) = make_float4(af[0], af[1], af[2], af[3]);
+            *reinterpret_cast<float4 *>(V + 128 + t0) = make_float4(ab[0], ab[1], ab[2], ab[3]);
+            *reinterpret_cast<float4 *>(V + 256 + t0) = make_float4(cf[0], cf[1], cf[2], cf[3]);
+            *reinterpret_cast<float4 *>(V + 384 + t0) = make_float4(cb[0], cb[1], cb[2], cb[3]);
+            *reinterpret_cast<float4 *>(V + 512 + t0) =
+                make_float4(__expf(ef - af[0]) * cf[0], __expf(ef - af[1]) * cf[1], __expf(ef - af[2]) * cf[2],
+                            __expf(ef - af[3]) * cf[3]);
+            *reinterpret_cast<float4 *>(V + 640 + t0) =
+                make_float4(__expf(eb - ab[0]) * cb[0], __expf(eb - ab[1]) * cb[1], __expf(eb - ab[2]) * cb[2],
+                            __expf(eb - ab[3]) * cb[3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_V + j % kVS));
         }
     } else if (warp == 12) {
         // ================= C/B loads and the MMAs (one thread)
@@ -388,8 +478,8 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         }
         __syncwarp();
     } else {
-        // ================= decay vectors, epilogue, x loads and y stores (warps 8..11)
-        const int r = tid - 256;                  // token of the vectors; tile row of the epilogue
+        // ================= epilogue, x loads and y stores (warps 8..11)
+        const int r = tid - 256;                  // tile row of the epilogue
         const bool leader = r == 0;
         int x_issued = 0, x_seen = 0;             // the leader's x loads: heads [x_seen, x_issued) in flight
         HeadPos pos_x = head_at(0);               // the leader's next x load
@@ -401,83 +491,11 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         };
         if (leader)
             for (int j = 0; j < kXS - 1 && j < n; ++j) load_x(j);
-        // dt of a head at token r, both directions, and its A
-        struct DtA { float vf, vb, af, ab; };
-        HeadPos pos_dt = head_at(0);              // the next dt load
-        auto load_dt = [&](int j) {
-            DtA d{0.f, 0.f, 0.f, 0.f};
-            if (j < n) {
-                const int b = pos_dt.b, h = pos_dt.h;
-                pos_dt.next(p.H);
-                d.af = __ldg(p.A + h);
-                d.ab = __ldg(p.A + p.H + h);
-                if (r < p.L) {
-                    d.vf = __bfloat162float(p.dt[((size_t)b * p.L + r) * p.H + h]);
-                    d.vb = __bfloat162float(p.dt[(((size_t)p.batch + b) * p.L + r) * p.H + h]);
-                }
-            }
-            return d;
-        };
-        // the vectors of head j into buffer j % kVS: the decay sums (forward:
-        // A_f times the sum of dt_f over tokens <= t; reverse: A_b times the
-        // sum of dt_b over tokens >= t), dt and the column factors (exp(a_e -
-        // a_s) dt_s, e the last (forward) or first (reverse) token of the
-        // 32-token block of s); then the mask builders may take head j
-        auto vectors = [&](int j, const DtA &d) {
-            float pf = d.vf, pb = d.vb;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float nf = __shfl_up_sync(0xffffffffu, pf, o), nb = __shfl_up_sync(0xffffffffu, pb, o);
-                if (lane >= o) {
-                    pf += nf;
-                    pb += nb;
-                }
-            }
-            if (lane == 31) {
-                part[q] = pf;
-                part[4 + q] = pb;
-            }
-            bar_named(2, 128);
-            float bf = 0.f, bb = 0.f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                if (k < q) {
-                    bf += part[k];
-                    bb += part[4 + k];
-                }
-            const float totb = part[4] + part[5] + part[6] + part[7];
-            const float af = d.af * (pf + bf);
-            const float ab = d.ab * (totb - (pb + bb) + d.vb);
-            const float ef = __shfl_sync(0xffffffffu, af, 31), eb = __shfl_sync(0xffffffffu, ab, 0);
-            float *V = vbuf(j);
-            V[r] = af;
-            V[128 + r] = ab;
-            V[256 + r] = d.vf;
-            V[384 + r] = d.vb;
-            V[512 + r] = __expf(ef - af) * d.vf;
-            V[640 + r] = __expf(eb - ab) * d.vb;
-            bar_named(2, 128);
-            if (leader) mbar_arrive(bar(B_V + j % kVS));
-        };
-        // vectors of heads 0 and 1; dt of head 2 in flight
-        DtA dn = load_dt(0);
-        vectors(0, dn);
-        dn = load_dt(1);
-        DtA dn2 = load_dt(2);
-        if (n > 1) vectors(1, dn);
-        dn = dn2;
         bool ok = true;
         HeadPos pos_e = head_at(0);               // head i of the epilogue
 #pragma unroll 1
         for (int i = 0; i < n; ++i) {
             if (i > 0) pos_e.next(p.H);
-            // vectors of head i + 2 (their buffer was last read by the mask of head
-            // i - 1, whose MMA the epilogue of head i - 1 has seen complete)
-            if (i + 2 < n) {
-                dn2 = load_dt(i + 3);
-                vectors(i + 2, dn);
-                dn = dn2;
-            }
             const int hi = pos_e.h;
             const float ds = __ldg(p.D + hi) + __ldg(p.D + p.H + hi);
             // ---------------- epilogue of head i: y = Y + (D_f + D_b) x, written over x

@@ -74,8 +74,11 @@ struct OSmem {
     static constexpr uint32_t kTile = (N / 64) * kSlab;    // one 128 x N bf16 operand
     static constexpr uint32_t cb = 0;                      // C_f, B_f, C_b, B_b
     static constexpr uint32_t x = 4 * kTile;               // kXS x slots
-    static constexpr uint32_t vec = x + kXS * kSlab;       // kVS buffers of af, ab, dtf, dtb, colf, colb
-    static constexpr uint32_t small = vec + kVS * 6 * 128 * 4;
+    // kVS buffers of af, ab, dtf, dtb, colf, colb (128 floats each) and the
+    // head's D_f + D_b
+    static constexpr uint32_t kVecBytes = 6 * 512 + 128;
+    static constexpr uint32_t vec = x + kXS * kSlab;
+    static constexpr uint32_t small = vec + kVS * kVecBytes;
     static constexpr uint32_t bytes = small + 256;
 };
 
@@ -133,11 +136,14 @@ __device__ __forceinline__ void offdiag16(const uint32_t (&g)[16], float r, cons
 // The diagonal block: columns [s1, s1 + 16) of row `row` (s1 = 32 J + c0, J =
 // row / 32). The forward term g_f (r_f colf) is kept for s <= t and the reverse
 // term g_b (r_b colb) for s >= t; on the row's own token both are kept, each
-// equal to G dt there (the two factors of exp(a_t - a_e) exp(a_e - a_t)).
+// equal to G dt there (the two factors of exp(a_t - a_e) exp(a_e - a_t)), and
+// the skip coefficient dsum = D_f + D_b is added, so that the product with X
+// carries the skip term (D_f + D_b) x_t as well.
 // Factorised while the block's decay span is below kMaxSpan, else one
 // exponential per entry (as mask_diag).
-__device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, float my_ab, const uint32_t (&gf)[16],
-                                       const uint32_t (&gb)[16], const MaskVectors &v, uint32_t (&packed)[8]) {
+__device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, float my_ab, float dsum,
+                                       const uint32_t (&gf)[16], const uint32_t (&gb)[16], const MaskVectors &v,
+                                       uint32_t (&packed)[8]) {
     const int s0 = J * 32, s1 = s0 + c0;
     const int rr = row - s1;   // the row's token relative to the first column
     const float span_f = v.af[s0] - v.af[s0 + 31], span_b = v.ab[s0 + 31] - v.ab[s0];
@@ -150,8 +156,9 @@ __device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, floa
             const float2 cb = *reinterpret_cast<const float2 *>(v.colb + s1 + k);
             const uint64_t pf = mul2(f2u(gf[k], gf[k + 1]), mul2(rf, f2(cf.x, cf.y)));
             const uint64_t pb = mul2(f2u(gb[k], gb[k + 1]), mul2(rb, f2(cb.x, cb.y)));
-            const float m0 = (k <= rr ? lo_of(pf) : 0.f) + (k >= rr ? lo_of(pb) : 0.f);
-            const float m1 = (k + 1 <= rr ? hi_of(pf) : 0.f) + (k + 1 >= rr ? hi_of(pb) : 0.f);
+            const float m0 = (k <= rr ? lo_of(pf) : 0.f) + (k >= rr ? lo_of(pb) : 0.f) + (k == rr ? dsum : 0.f);
+            const float m1 =
+                (k + 1 <= rr ? hi_of(pf) : 0.f) + (k + 1 >= rr ? hi_of(pb) : 0.f) + (k + 1 == rr ? dsum : 0.f);
             packed[k / 2] = pack_bf16x2(m0, m1);
         }
     } else {
@@ -163,7 +170,7 @@ __device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, floa
             // the exponent of the selected side is <= 0
             m[c] = c < rr ? gfv * v.dtf[s] * __expf(my_af - v.af[s])
                  : c > rr ? gbv * v.dtb[s] * __expf(my_ab - v.ab[s])
-                          : gfv * v.dtf[s] + gbv * v.dtb[s];
+                          : gfv * v.dtf[s] + gbv * v.dtb[s] + dsum;
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) packed[k] = pack_bf16x2(m[2 * k], m[2 * k + 1]);
@@ -246,7 +253,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     auto tY = [&](int j) { return tmem + 384 + 64 * (j & 1); };
     const uint32_t lane_off = (uint32_t)(q << 5) << 16;
     auto xslot = [&](int j) { return S::x + (uint32_t)(j % kXS) * kSlab; };
-    auto vbuf = [&](int j) { return reinterpret_cast<float *>(g + S::vec + (j % kVS) * 6 * 512); };
+    auto vbuf = [&](int j) { return reinterpret_cast<float *>(g + S::vec + (j % kVS) * S::kVecBytes); };
     // the kernel ahead in the stream has finished before any global access
     grid_dependency_wait();
 
@@ -289,7 +296,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tmem_wait_ld();
                 const uint32_t mrow = tM(j) + lane_off + 8 * half;
                 uint32_t packed[8];
-                diag16(q, c0, row, my_af, my_ab, gdf, gdb, mv, packed);
+                diag16(q, c0, row, my_af, my_ab, V[768], gdf, gdb, mv, packed);
                 tmem_st8(mrow + 16 * q, packed);
 #pragma unroll
                 for (int k = 0; k < 3; ++k) {
@@ -322,13 +329,14 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int t0 = 4 * lane;
         bool ok = true;
         HeadPos pos = head_at(vw);
-        float vf[4], vb[4], Af = 0.f, Ab = 0.f;
+        float vf[4], vb[4], Af = 0.f, Ab = 0.f, Dn = 0.f;
         auto load = [&](int j) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) vf[k] = vb[k] = 0.f;
             if (j < n) {
                 Af = __ldg(p.A + pos.h);
                 Ab = __ldg(p.A + p.H + pos.h);
+                Dn = __ldg(p.D + pos.h) + __ldg(p.D + p.H + pos.h);
                 const __nv_bfloat16 *df = p.dt + (size_t)pos.b * p.L * p.H + pos.h;
                 const __nv_bfloat16 *db = df + (size_t)p.batch * p.L * p.H;
 #pragma unroll
@@ -346,7 +354,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll 1
         for (int j = vw; j < n; j += kVS) {
             const float cf[4] = {vf[0], vf[1], vf[2], vf[3]}, cb[4] = {vb[0], vb[1], vb[2], vb[3]};
-            const float A_f = Af, A_b = Ab;
+            const float A_f = Af, A_b = Ab, Ds = Dn;
             load(j + kVS);     // this warp's next head, in flight while this one is computed
             // inclusive sums over the lane's four tokens, then across the warp
             float sf[4], sb[4];
@@ -382,6 +390,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                                                  abort_flag, p.status, 1011));
             if (!ok) break;
             float *V = vbuf(j);
+            if (lane == 0) V[768] = Ds;
             *reinterpret_cast<float4 *>(V + t0) = make_float4(af[0], af[1], af[2], af[3]);
             *reinterpret_cast<float4 *>(V + 128 + t0) = make_float4(ab[0], ab[1], ab[2], ab[3]);
             *reinterpret_cast<float4 *>(V + 256 + t0) = make_float4(cf[0], cf[1], cf[2], cf[3]);
@@ -464,7 +473,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tc_fence_after();
                 if (!okm) break;
                 const uint32_t xa = base + xslot(j);
-#pragma unroll 1
+#pragma unroll
                 for (int k = 0; k < 128 / 16; ++k)
                     mma_bf16_ts(tY(j), tM(j) + 8 * k, sdesc_sw128(xa + k * 2048, kSlab, 1024), id_o, k > 0);
                 mma_commit(bar(B_Y + (j & 1)));
@@ -497,8 +506,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int i = 0; i < n; ++i) {
             if (i > 0) pos_e.next(p.H);
             const int hi = pos_e.h;
-            const float ds = __ldg(p.D + hi) + __ldg(p.D + p.H + hi);
-            // ---------------- epilogue of head i: y = Y + (D_f + D_b) x, written over x
+            // ---------------- epilogue of head i: y = Y (the skip term rides on M's diagonal), written over x
             ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_Y + (i & 1)), (uint32_t)(i >> 1) & 1u, abort_flag,
                                                              p.status, 1007) &&
                                              mbar_wait_ool(bar(B_X + i % kXS), (uint32_t)(i / kXS) & 1u, abort_flag,
@@ -514,21 +522,18 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc_fence_before();
             if (bar_or(2, 128, !ok)) break;
             if (leader) mbar_arrive(bar(B_YE + (i & 1)));    // Y_i read out: the MMA of head i + 2 may write it
+            // y as bf16 over x (whose MMA has completed), for the TMA store
             uint8_t *xs = g + xslot(i);
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) {
-                uint4 *ptr = reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc));
-                const uint4 xv = *ptr;
-                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
                 uint32_t o[4];
 #pragma unroll
                 for (int j2 = 0; j2 < 4; ++j2) {
                     const int c = (cc & 3) * 8 + 2 * j2;
                     const uint32_t y0 = cc < 4 ? ya[c] : yb[c], y1 = cc < 4 ? ya[c + 1] : yb[c + 1];
-                    o[j2] = pack_bf16x2(__uint_as_float(y0) + ds * bf2f(xu[j2] & 0xffffu),
-                                        __uint_as_float(y1) + ds * bf2f(xu[j2] >> 16));
+                    o[j2] = pack_bf16x2(__uint_as_float(y0), __uint_as_float(y1));
                 }
-                *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async_smem();
             bar_named(2, 128);

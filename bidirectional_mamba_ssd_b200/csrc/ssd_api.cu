@@ -56,13 +56,15 @@ constexpr long long kFusedMinUnits = 64;
 // kernel: each cluster keeps up to half a sequence of 32 KB partial tiles live.
 constexpr long long kPairMaxTiles = 16;
 
-// Kernel choice of SSD_PATH_AUTO: bf16 runs on the tensor cores: two CTAs
-// per (batch, head), one per direction, for sequences of 2..16 tiles with a
-// unit for every two SMs; one CTA per (batch, head) when there are enough of
-// those to fill the GPU; else the segmented or tile-parallel chunked kernels;
-// fp32 runs the sequential scan.
+// Kernel choice of SSD_PATH_AUTO: bf16 runs on the tensor cores: the one-tile
+// kernel for sequences of at most one 128-token tile; two CTAs per (batch,
+// head), one per direction, for sequences of 2..16 tiles with a unit for
+// every two SMs; one CTA per (batch, head) when there are enough of those to
+// fill the GPU; else the segmented or tile-parallel chunked kernels; fp32
+// runs the sequential scan.
 int auto_path(int batch, int seqlen, int nheads, int ngroups, int dstate, int dtype) {
     if (dtype != SSD_BF16) return SSD_PATH_SIMT;
+    if (ssd::tc_onetile_supported(batch, seqlen, nheads, ngroups, dstate)) return SSD_PATH_ONETILE;
     // two to 16 tiles and a (batch, head) unit for every two SMs: one cluster of
     // two CTAs per unit, each running one scan direction (the partial tiles the
     // directions exchange stay in L2 up to this length)

@@ -100,10 +100,11 @@ enum {
     SSD_PATH_BLOCK = 6,    /* ssd_block_step only: one CTA per (batch, head) over a block of at
                               most 64 tokens, both directions stacked as the rows of one
                               tensor-core tile */
-    SSD_PATH_ONETILE = 7   /* ssd_bidir_fwd_path, seqlen <= 128 (one tensor-core tile): each
-                              CTA takes a run of (batch, head) units, computes both
+    SSD_PATH_ONETILE = 7   /* bf16, seqlen <= 128 (one tensor-core tile), dstate 64 or 128:
+                              each CTA takes a run of (batch, head) units, computes both
                               directions' C B^T once per B/C group and reuses it for every
-                              head of the group (mask and one MMA per head) */
+                              head of the group (mask and one MMA per head); what
+                              SSD_PATH_AUTO runs for these sizes */
 };
 
 /* The SSD_PATH_* that ssd_bidir_fwd (SSD_PATH_AUTO) runs for these sizes, or

@@ -17,16 +17,18 @@
 // packed 128-token shape: "Diffusion Mamba ... (LM1B, packed sequences of
 // 128)" as the pages' second workload.
 //
-// Per CTA: 384 threads in two roles that hand work over through mbarriers,
+// Per CTA: 512 threads in four roles that hand work over through mbarriers,
 // persistent over a contiguous run of (batch, head) units:
 //  - warps 0..7 build the masked matrix of each head (warp w: TMEM lanes
-//    32 (w % 4) .. + 31, the 16-column half w / 4 of each 32-column block),
-//    into one of two bf16 M buffers in TMEM; thread 0 issues the TMA loads of
-//    C and B, the MMAs (G once per group, Y = M X per head) and their commits;
-//  - warps 8..11 compute each head's decay vectors two heads ahead and run
-//    each head's epilogue (Y from TMEM plus (D_f + D_b) x, written over x in
-//    shared memory, then a TMA store); their first thread issues the x loads,
-//    four heads ahead, and the stores.
+//    32 (w % 4) .. + 31, the 16-column half w / 4 of each 32-column block)
+//    into one of two bf16 M buffers in TMEM, (D_f + D_b) on its diagonal;
+//  - warps 8..11 run each head's epilogue: Y (= y) from TMEM to bf16 over the
+//    head's x in shared memory, then a TMA store; their first thread issues
+//    the x loads, four heads ahead, and the stores;
+//  - warp 12 (one thread) issues the C/B loads and the MMAs: G once per
+//    group, Y = M X per head;
+//  - warps 13..15 compute the decay vectors, each a whole head at a time,
+//    heads j = 0, 1, 2 (mod 3) respectively, up to three heads ahead.
 // The next group's C and B load while the current group's heads run. Every
 // wait is bounded in time; an expired wait sets the workspace's timeout flag
 // and the CTA stops storing.

@@ -96,6 +96,11 @@ struct FusedParams {
     const float *dt_bias;      // DTRAW: (2, H); dt holds the raw projection
     float dt_lo, dt_hi;        // DTRAW: the step-size range
     int layer_units, A_layer;  // layers stacked along the batch: A, D of unit u at + (u / layer_units) * A_layer
+    // 0: the next kernel may start its prologue at once, and this one waits for
+    // the kernel ahead before touching global memory; 1: the next kernel may
+    // start only after this one's wait (so it need not wait itself); 2: no wait
+    // (launched right after an order-1 kernel, whose wait covers its inputs)
+    int launch_order;
 };
 
 // A and D of unit u: a layer's own when several layers are stacked along the batch
@@ -232,7 +237,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     // the next kernel in the stream may set itself up while this one runs
-    grid_launch_dependents();
+    if (p.launch_order != 1) grid_launch_dependents();
     if (tid == 0) {
         *abort_flag = 0;
         for (int i = 0; i < B_COUNT; ++i)
@@ -245,7 +250,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
     // the kernel ahead in the stream has finished and its writes are visible
     // before this one reads or writes global memory
-    grid_dependency_wait();
+    if (p.launch_order != 2) grid_dependency_wait();
+    if (p.launch_order == 1) grid_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -841,6 +847,7 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     p.dt_hi = a.dt_hi;
     p.layer_units = a.layer_units;
     p.A_layer = a.A_layer;
+    p.launch_order = a.launch_order;
 
     CUtensorMap tm_x, tm_b, tm_c, tm_h, tm_out;
     // the forward state mode may be given single-direction B; every other mode reads both directions' layout
@@ -862,7 +869,8 @@ cudaError_t run_fused(const TcArgs &a, cudaStream_t stream) {
     const size_t smem = S::bytes + 1024;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return e;
-    const int grid = units < sms ? units : sms;
+    int grid = units < sms ? units : sms;
+    if (a.grid_cap > 0 && grid > a.grid_cap) grid = a.grid_cap;
     // programmatic stream serialization: the prologue (barriers, TMEM) overlaps
     // the end of the kernel ahead; the kernel waits for it before any global access
     cudaLaunchConfig_t cfg = {};

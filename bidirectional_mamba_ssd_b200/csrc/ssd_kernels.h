@@ -52,6 +52,9 @@ struct TcArgs {
     // elements between the two directions' x when each scans its own x
     // (launch_tc_pair only; x then holds (2, batch, L, H, 64)); 0 = one x
     long long x_dir_stride = 0;
+    // fused kernel only: at most this many CTAs (0 = one per SM), and the
+    // launch order of its kernel (FusedParams::launch_order)
+    int grid_cap = 0, launch_order = 0;
     float *state_out;         // (batch, H, 64, N) or nullptr
     void *out;                // (batch, L, H, 64) bf16
     void *workspace;          // status header + scratch

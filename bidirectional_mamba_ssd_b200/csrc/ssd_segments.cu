@@ -222,6 +222,20 @@ size_t tc_segmented_scratch_bytes(int batch, int L, int H, int N) {
     return m;
 }
 
+// The forward and reverse state passes read the same x. With units enough
+// for both halves of the GPU they run side by side, each on half the SMs: the
+// reverse pass is released only once the forward pass's wait for the kernel
+// ahead is over and does not wait itself, so the two CTAs on a unit run at the
+// same time and the second read of each x tile comes from L2.
+static void share_state_passes(TcArgs &f, TcArgs &r) {
+    const int sms = device_sms();
+    if (sms < 2 || (long long)f.batch * f.H < sms) return;
+    f.grid_cap = sms / 2;
+    f.launch_order = 1;
+    r.grid_cap = sms - sms / 2;
+    r.launch_order = 2;
+}
+
 cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
     if (S < 2 || S > kMaxSeg || a.L % S || a.L / S < 1 || a.ndir != 2) return cudaErrorNotSupported;
     const SegLayout lay = seg_layout(a.batch, a.L, a.H, a.N, S);
@@ -242,11 +256,13 @@ cudaError_t launch_tc_segmented(const TcArgs &a, int S, cudaStream_t stream) {
     TcArgs f = v;
     f.state_out = Sf;
     f.decay_out = Gf;
-    if ((e = launch_tc_fused_state(f, stream)) != cudaSuccess) return e;
     TcArgs r = v;
     r.state_out = Sb;
     r.decay_out = Gb;
+    share_state_passes(f, r);
+    if ((e = launch_tc_fused_state(f, stream)) != cudaSuccess) return e;
     if ((e = launch_tc_fused_state_rev(r, stream)) != cudaSuccess) return e;
+    // launched without programmatic serialization: waits for both passes
     const int zb = (kP * a.N + kScanThreads * 4 - 1) / (kScanThreads * 4);
     seg_scan_kernel<<<dim3(a.batch * a.H, 2, zb), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, a.init, a.rinit, Hf, Hb,
                                                                             a.H, S, a.N);
@@ -291,11 +307,13 @@ cudaError_t launch_tc_segment_totals(const TcArgs &a, int S, float *fwd_state, f
     TcArgs f = v;
     f.state_out = Sf;
     f.decay_out = Gf;
-    if ((e = launch_tc_fused_state(f, stream)) != cudaSuccess) return e;
     TcArgs r = v;
     r.state_out = Sb;
     r.decay_out = Gb;
+    share_state_passes(f, r);
+    if ((e = launch_tc_fused_state(f, stream)) != cudaSuccess) return e;
     if ((e = launch_tc_fused_state_rev(r, stream)) != cudaSuccess) return e;
+    // launched without programmatic serialization: waits for both passes
     seg_total_kernel<<<dim3(a.batch * a.H, 2), kScanThreads, 0, stream>>>(Sf, Sb, Gf, Gb, fwd_state, rev_state,
                                                                          fwd_decay, rev_decay, a.H, S, a.N);
     return cudaGetLastError();

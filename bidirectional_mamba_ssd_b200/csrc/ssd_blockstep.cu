@@ -25,10 +25,13 @@
 // "DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone", Technical
 // Summary, 2. Methodology, Core Architecture.
 //
-// Per CTA: 256 threads. Thread 0 issues the TMA loads and the MMAs; warp w
-// owns TMEM lanes 32 (w % 4) .. + 31 (tile rows) and column half w / 4 of
-// every per-row step (the mask's 64-column halves, the output's 32-column
-// halves). Every wait is bounded in time; an expired wait sets the
+// Per CTA: 288 threads. Warp 8 (its lane 0) issues the TMA loads and the
+// MMAs, each as soon as its operands are ready: G = C B^T while warps 0..3
+// compute the decay vectors and every mask warp converts its part of the
+// cached state; C H once the state is in shared memory; Y once the mask is
+// built. Warps 0..7 own TMEM lanes 32 (w % 4) .. + 31 (tile rows) and column
+// half w / 4 of every per-row step (the mask's 64-column halves, the output's
+// 32-column halves). Every wait is bounded in time; an expired wait sets the
 // workspace's timeout flag and the CTA stores nothing.
 #include <cuda.h>
 #include <stdint.h>
@@ -47,7 +50,8 @@ using namespace fused;
 
 constexpr int kT = 64;          // tokens of a block (at most)
 constexpr int kP = 64;          // headdim
-constexpr int kThreads = 256;
+constexpr int kThreads = 288;       // 8 mask and epilogue warps, 1 issuing warp
+constexpr int kIssueWarp = 8;       // lane 0: the TMA loads and the MMAs
 constexpr uint32_t kSlab = 16384;   // 128 rows x 128 bytes
 
 struct BlockParams {
@@ -61,7 +65,10 @@ struct BlockParams {
     int batch, T, H, G;
 };
 
-enum { B_LOAD = 0, B_X, B_G, B_Y, B_COUNT };
+// mbarriers: C and B loaded; x loaded; G computed; the cached state in shared
+// memory (one arrival per mask warp); the masked matrix built (one arrival per
+// mask warp); Y and C H computed
+enum { B_LOAD = 0, B_X, B_G, B_H, B_M, B_Y, B_COUNT };
 
 template <int N>
 struct BSmem {
@@ -117,7 +124,7 @@ blockstep_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     grid_launch_dependents();
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), i == B_H || i == B_M ? 8 : 1);
         fence_mbar_init();
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_b);
@@ -137,88 +144,112 @@ blockstep_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     // the kernel ahead in the stream has finished before any global access
     grid_dependency_wait();
 
-    if (tid == 0) {
-        // [C_f; C_b] and [B_f; B_b]: a 64-row box per direction and 64-column slab
-        mbar_arrive_expect_tx(bar(B_LOAD), 4 * NSLAB * 8192);
-        for (int d = 0; d < 2; ++d)
-            for (int sl = 0; sl < NSLAB; ++sl) {
-                tma_load_5d(base + S::c + sl * kSlab + d * 8192, &tm_c, bar(B_LOAD), 64 * sl, gg, 0, b, d);
-                tma_load_5d(base + S::b + sl * kSlab + d * 8192, &tm_b, bar(B_LOAD), 64 * sl, gg, 0, b, d);
-            }
-        // x twice: the K rows of both halves of M
-        mbar_arrive_expect_tx(bar(B_X), 2 * 8192);
-        tma_load_4d(base + S::x, &tm_x, bar(B_X), 0, h, 0, b);
-        tma_load_4d(base + S::x + 8192, &tm_x, bar(B_X), 0, h, 0, b);
-    }
-    // every global load of the threads in flight at once: dt of the row
-    // (warps 0..3: forward rows in warps 0, 1, reverse rows in warps 2, 3;
-    // tokens past the block's end have dt = 0) and this thread's 32 values of
-    // the cached state, row n of H^T (H[p][n] for p in its half of the 64)
-    const float A = p.A[(fwd ? 0 : p.H) + h];
-    float v = 0.f;
-    if (ch == 0 && t < p.T) v = __bfloat162float(p.dt[(((size_t)(fwd ? 0 : 1) * p.batch + b) * p.T + t) * p.H + h]);
-    const int n = tid & 127, half = tid >> 7;
-    float hv[32];
-    if (has_h && n < N) {
-        const float *ip = p.prefix + (size_t)u * kP * N + n + (size_t)half * 32 * N;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) hv[j] = __ldg(ip + (size_t)j * N);
-    }
-    // decay sums and mask vectors
-    if (ch == 0) {
-        float tot;
-        const float pf = scan64(v, lane, q & 1, part + (fwd ? 0 : 2), tot);
-        // a_t: decay sum from the block's start (forward) or end (reverse) through t
-        const float a = fwd ? A * pf : A * (tot - pf + v);
-        Va[row] = a;
-        Vdt[row] = v;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // column factor exp(a_e - a_s) dt_s, e the 32-column block's last
-        // (forward) or first (reverse) column
-        Vcol[row] = __expf(Va[fwd ? (row | 31) : (row & ~31)] - a) * v;
-    }
-    if (has_h) {
-        if (n < N) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<uint4 *>(g + S::h + sw128_offset(n, half * 4 + c)) =
-                    make_uint4(pack_bf16x2(hv[8 * c], hv[8 * c + 1]), pack_bf16x2(hv[8 * c + 2], hv[8 * c + 3]),
-                               pack_bf16x2(hv[8 * c + 4], hv[8 * c + 5]), pack_bf16x2(hv[8 * c + 6], hv[8 * c + 7]));
-        }
-        fence_proxy_async_smem();
-    }
-    __syncthreads();
-
     constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, false);   // [C_f; C_b] (K) x [B_f; B_b] (K)
     constexpr uint32_t id_o = idesc_bf16_f32(128, 64, false, true);     // C (K) x H (MN); M (K) x [X; X] (MN)
-    if (tid == 0) {
-        if (mbar_wait_ool(bar(B_LOAD), 0, abort_flag, p.status, 901)) {
+    if (warp == kIssueWarp) {
+        // ================= the issuing thread: loads, then each MMA as soon as
+        // its operands are ready (G while the vectors and the state are prepared)
+        if (lane == 0) {
+            // [C_f; C_b] and [B_f; B_b]: a 64-row box per direction and 64-column slab
+            mbar_arrive_expect_tx(bar(B_LOAD), 4 * NSLAB * 8192);
+            for (int d = 0; d < 2; ++d)
+                for (int sl = 0; sl < NSLAB; ++sl) {
+                    tma_load_5d(base + S::c + sl * kSlab + d * 8192, &tm_c, bar(B_LOAD), 64 * sl, gg, 0, b, d);
+                    tma_load_5d(base + S::b + sl * kSlab + d * 8192, &tm_b, bar(B_LOAD), 64 * sl, gg, 0, b, d);
+                }
+            // x twice: the K rows of both halves of M
+            mbar_arrive_expect_tx(bar(B_X), 2 * 8192);
+            tma_load_4d(base + S::x, &tm_x, bar(B_X), 0, h, 0, b);
+            tma_load_4d(base + S::x + 8192, &tm_x, bar(B_X), 0, h, 0, b);
+            bool ok = mbar_wait_ool(bar(B_LOAD), 0, abort_flag, p.status, 901);
             tc_fence_after();
-#pragma unroll 1
-            for (int k = 0; k < N / 16; ++k) {
-                const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
-                mma_bf16_ss(tG, sdesc_sw128(base + S::c + ko, 0, 1024), sdesc_sw128(base + S::b + ko, 0, 1024),
-                            id_g, k > 0);
-            }
-            mma_commit(bar(B_G));
-            if (has_h) {
+            if (ok) {
 #pragma unroll 1
                 for (int k = 0; k < N / 16; ++k) {
                     const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
-                    mma_bf16_ss(tYo, sdesc_sw128(base + S::c + ko, 0, 1024),
-                                sdesc_sw128(base + S::h + k * 2048, kSlab, 1024), id_o, k > 0);
+                    mma_bf16_ss(tG, sdesc_sw128(base + S::c + ko, 0, 1024), sdesc_sw128(base + S::b + ko, 0, 1024),
+                                id_g, k > 0);
+                }
+                mma_commit(bar(B_G));
+            }
+            // C H once the cached state is in shared memory
+            if (ok && has_h) {
+                ok = mbar_wait_ool(bar(B_H), 0, abort_flag, p.status, 906);
+                tc_fence_after();
+                if (ok) {
+#pragma unroll 1
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * kSlab + (k & 3) * 32;
+                        mma_bf16_ss(tYo, sdesc_sw128(base + S::c + ko, 0, 1024),
+                                    sdesc_sw128(base + S::h + k * 2048, kSlab, 1024), id_o, k > 0);
+                    }
                 }
             }
+            // Y = M [X; X] once every row of M is built and x is in: rows 0..63
+            // the forward output, rows 64..127 the reverse one
+            ok = ok && mbar_wait_ool(bar(B_M), 0, abort_flag, p.status, 907) &&
+                 mbar_wait_ool(bar(B_X), 0, abort_flag, p.status, 903);
+            tc_fence_after();
+            if (ok && !*abort_flag) {
+#pragma unroll 1
+                for (int k = 0; k < 128 / 16; ++k)
+                    mma_bf16_ts(tY, tG + 16 * k, sdesc_sw128(base + S::x + k * 2048, kSlab, 1024), id_o, k > 0);
+            }
+            mma_commit(bar(B_Y));
         }
-    }
+        __syncwarp();
+    } else {
+        // ================= warps 0..7: the decay vectors (warps 0..3), the
+        // cached state's bf16 copy, then the mask. Every global load in flight
+        // at once: dt of the row (warps 0..3: forward rows in warps 0, 1,
+        // reverse rows in warps 2, 3; tokens past the block's end have dt = 0)
+        // and this thread's 32 values of the cached state, row n of H^T (H[p][n]
+        // for p in its half of the 64)
+        const float A = p.A[(fwd ? 0 : p.H) + h];
+        float v = 0.f;
+        if (ch == 0 && t < p.T) v = __bfloat162float(p.dt[(((size_t)(fwd ? 0 : 1) * p.batch + b) * p.T + t) * p.H + h]);
+        const int n = tid & 127, half = tid >> 7;
+        float hv[32];
+        if (has_h && n < N) {
+            const float *ip = p.prefix + (size_t)u * kP * N + n + (size_t)half * 32 * N;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) hv[j] = __ldg(ip + (size_t)j * N);
+        }
+        // decay sums and mask vectors
+        if (ch == 0) {
+            float tot;
+            const float pf = scan64(v, lane, q & 1, part + (fwd ? 0 : 2), tot);
+            // a_t: decay sum from the block's start (forward) or end (reverse) through t
+            const float a = fwd ? A * pf : A * (tot - pf + v);
+            Va[row] = a;
+            Vdt[row] = v;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            // column factor exp(a_e - a_s) dt_s, e the 32-column block's last
+            // (forward) or first (reverse) column
+            Vcol[row] = __expf(Va[fwd ? (row | 31) : (row & ~31)] - a) * v;
+        }
+        // the cached state as the bf16 N x 64 operand of C H
+        if (has_h) {
+            if (n < N) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4 *>(g + S::h + sw128_offset(n, half * 4 + c)) =
+                        make_uint4(pack_bf16x2(hv[8 * c], hv[8 * c + 1]), pack_bf16x2(hv[8 * c + 2], hv[8 * c + 3]),
+                                   pack_bf16x2(hv[8 * c + 4], hv[8 * c + 5]), pack_bf16x2(hv[8 * c + 6], hv[8 * c + 7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_H));
+        }
+        __syncwarp();
+        asm volatile("bar.sync 3, 256;" ::: "memory");    // the vectors, to every mask warp
 
-    // ---------------- the masked matrix, in place of G: this thread's row, the
-    // direction's 32-column block `ch` of its 64 columns, and zero over the
-    // other direction's block `ch`
-    const int lq = q & 1;                       // the row's 32-row block within its direction
-    const int vo = fwd ? 0 : 64;                // the direction's vectors
-    const float my_a = Va[row];
-    {
+        // ---------------- the masked matrix, in place of G: this thread's row, the
+        // direction's 32-column block `ch` of its 64 columns, and zero over the
+        // other direction's block `ch`
+        const int lq = q & 1;                       // the row's 32-row block within its direction
+        const int vo = fwd ? 0 : 64;                // the direction's vectors
+        const float my_a = Va[row];
         const int Jm = fwd ? ch : ch + 2, Jz = fwd ? ch + 2 : ch;
         uint32_t packed[16];
         const bool zero = fwd ? ch > lq : ch < lq;
@@ -245,39 +276,36 @@ blockstep_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             tmem_st8(tG + lane_off + Jz * 32 + 16, zz);
             tmem_wait_st();
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_M));      // this warp's part of M is built
     }
-    tc_fence_before();
-    __syncthreads();
-    // ---------------- Y = M [X; X], on top of nothing: rows 0..63 the forward
-    // output, rows 64..127 the reverse one
-    if (tid == 0) {
-        tc_fence_after();
-        if (!*abort_flag && mbar_wait_ool(bar(B_X), 0, abort_flag, p.status, 903)) {
-#pragma unroll 1
-            for (int k = 0; k < 128 / 16; ++k)
-                mma_bf16_ts(tY, tG + 16 * k, sdesc_sw128(base + S::x + k * 2048, kSlab, 1024), id_o, k > 0);
-        }
-        mma_commit(bar(B_Y));
-    }
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_ool(bar(B_Y), 0, abort_flag, p.status, 904) &&
-                                                mbar_wait_ool(bar(B_X), 0, abort_flag, p.status, 905));
-    tc_fence_after();
-    // the reverse rows' y into shared memory over B (fp32, 64 floats a row,
-    // 16-byte chunks permuted by the row so a warp's stores spread over banks)
+
+    // ---------------- the epilogue (warps 0..7)
+    const bool mine = warp < kIssueWarp;
+    bool ok = true;
     uint8_t *yb = g + S::b;
-    if (ok && !fwd) {
-        uint32_t v[32];
-        tmem_ld32(tY + lane_off + ch * 32, v);
-        tmem_wait_ld();
+    if (mine) {
+        ok = __all_sync(0xffffffffu, mbar_wait_ool(bar(B_Y), 0, abort_flag, p.status, 904) &&
+                                         mbar_wait_ool(bar(B_X), 0, abort_flag, p.status, 905));
+        tc_fence_after();
+        // the reverse rows' y into shared memory over B (fp32, 64 floats a row,
+        // 16-byte chunks permuted by the row so a warp's stores spread over banks)
+        if (ok && !fwd) {
+            uint32_t v[32];
+            tmem_ld32(tY + lane_off + ch * 32, v);
+            tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4)
-            *reinterpret_cast<uint4 *>(yb + t * 256 + (((ch * 8 + c4) ^ (t & 15)) << 4)) =
-                make_uint4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+            for (int c4 = 0; c4 < 8; ++c4)
+                *reinterpret_cast<uint4 *>(yb + t * 256 + (((ch * 8 + c4) ^ (t & 15)) << 4)) =
+                    make_uint4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+        }
     }
     __syncthreads();
     // ---------------- out = y_f + exp(a_t) Yo + y_b + (D_f + D_b) x: the forward
     // rows, 32 columns a thread (rows past the block's end load but do not store)
-    if (fwd && __all_sync(0xffffffffu, ok && !*abort_flag)) {
+    if (mine && fwd && __all_sync(0xffffffffu, ok && !*abort_flag)) {
+        const float my_a = Va[row];
         uint32_t yv[32], ov[32];
         tmem_ld32(tY + lane_off + ch * 32, yv);
         if (has_h) tmem_ld32(tYo + lane_off + ch * 32, ov);
@@ -309,7 +337,7 @@ blockstep_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         }
     }
     // ---------------- teardown: the MMAs are complete (B_Y) before TMEM is released
-    if (tid == 0) mbar_drain(bar(B_Y), 0);
+    if (warp == kIssueWarp && lane == 0) mbar_drain(bar(B_Y), 0);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);

@@ -522,6 +522,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tmem_wait_ld();
             }
             tc_fence_before();
+            __syncwarp();    // the named barriers are warp-collective: reconverge after the leader's steps
             if (bar_or(2, 128, !ok)) break;
             if (leader) mbar_arrive(bar(B_YE + (i & 1)));    // Y_i read out: the MMA of head i + 2 may write it
             // y as bf16 over x (whose MMA has completed), for the TMA store
@@ -538,6 +539,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 *reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async_smem();
+            __syncwarp();
             bar_named(2, 128);
             if (leader) {
                 tma_store_4d(&tm_out, base + xslot(i), 0, hi, 0, pos_e.b);

@@ -9,7 +9,7 @@ total ~1 GB per GPU, well above the 126 MB L2, so no flush is needed between
 steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--path auto|simt|chunked|fused|segmented|pair]
+                  [--workload NAME] [--path auto|simt|chunked|fused|segmented|pair|onetile]
                   [--op bidir|bwd|block]
 
 --op bwd times the backward pass (ssd_bidir_bwd) and --op block the mixer

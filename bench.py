@@ -54,12 +54,13 @@ KERNEL_SOURCE = {
     "onetile": ("ssd_onetile.cu", "ssd_fused_util.cuh", "ssd_mask.cuh", "sm100.cuh", "ssd_tmap.h", "ssd_common.cuh"),
 }
 # kernels one call of each path launches (names as in ncu's "Kernel Name")
-KERNEL_NAMES = {"simt": ("scan_simt_kernel",), "chunked": ("tc_state_kernel", "tc_pass_kernel", "tc_out_kernel"),
+KERNEL_NAMES = {"simt": ("scan_simt_pair_kernel",), "chunked": ("tc_state_kernel", "tc_pass_kernel", "tc_out_kernel"),
                 "fused": ("tc_fused_kernel",), "segmented": ("tc_fused_kernel", "seg_scan_kernel"),
                 "pair": ("tc_pair_kernel",), "onetile": ("onetile_kernel",)}
 # kernels a call of the path launches on some shapes only (the segmented
-# path's last step runs the two-CTA kernel where the segments suit it)
-KERNEL_OPTIONAL = {"segmented": ("tc_pair_kernel",)}
+# path's last step runs the two-CTA kernel where the segments suit it; the
+# fp32 scan runs one kernel per direction beyond one unit per SM)
+KERNEL_OPTIONAL = {"segmented": ("tc_pair_kernel",), "simt": ("scan_simt_seq_kernel",)}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -659,7 +660,7 @@ def main():
     launches = LAUNCHES_PER_CALL[path_name]
     roof = roofline_bound(w, ms_step / 1e3, peaks)
     roof.update({"traffic": traffic_record(path_name, w.name),
-            "kernel": {"simt": "scan_simt_kernel", "chunked": "tc_state/tc_pass/tc_out kernels (whole step)",
+            "kernel": {"simt": "scan_simt_pair_kernel (both scans side by side; scan_simt_seq_kernel beyond one unit per SM)", "chunked": "tc_state/tc_pass/tc_out kernels (whole step)",
                        "fused": "tc_fused_kernel", "pair": "tc_pair_kernel", "onetile": "onetile_kernel",
                        "segmented": "tc_fused_kernel (forward state, reverse state) + seg_scan_kernel + the "
                                     "segments' kernel (tc_pair_kernel, else tc_fused_kernel) (whole step)"}[path_name]})

@@ -21,10 +21,10 @@
 // persistent over a contiguous run of (batch, head) units:
 //  - warps 0..7 build the masked matrix of each head (warp w: TMEM lanes
 //    32 (w % 4) .. + 31, the 16-column half w / 4 of each 32-column block)
-//    into one of two bf16 M buffers in TMEM, (D_f + D_b) on its diagonal;
-//  - warps 8..11 run each head's epilogue: Y (= y) from TMEM to bf16 over the
-//    head's x in shared memory, then a TMA store; their first thread issues
-//    the x loads, four heads ahead, and the stores;
+//    into one of two bf16 M buffers in TMEM;
+//  - warps 8..11 run each head's epilogue: y = Y + (D_f + D_b) x in fp32,
+//    rounded to bf16 over the head's x in shared memory, then a TMA store;
+//    their first thread issues the x loads, four heads ahead, and the stores;
 //  - warp 12 (one thread) issues the C/B loads and the MMAs: G once per
 //    group, Y = M X per head;
 //  - warps 13..15 compute the decay vectors, each a whole head at a time,
@@ -76,9 +76,8 @@ struct OSmem {
     static constexpr uint32_t kTile = (N / 64) * kSlab;    // one 128 x N bf16 operand
     static constexpr uint32_t cb = 0;                      // C_f, B_f, C_b, B_b
     static constexpr uint32_t x = 4 * kTile;               // kXS x slots
-    // kVS buffers of af, ab, dtf, dtb, colf, colb (128 floats each) and the
-    // head's D_f + D_b
-    static constexpr uint32_t kVecBytes = 6 * 512 + 128;
+    // kVS buffers of af, ab, dtf, dtb, colf, colb (128 floats each)
+    static constexpr uint32_t kVecBytes = 6 * 512;
     static constexpr uint32_t vec = x + kXS * kSlab;
     static constexpr uint32_t small = vec + kVS * kVecBytes;
     static constexpr uint32_t bytes = small + 256;
@@ -112,6 +111,12 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+// a * b + c on each element of the pairs, one rounding each (as fmaf)
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 __device__ __forceinline__ float lo_of(uint64_t v) { return __uint_as_float((uint32_t)v); }
 __device__ __forceinline__ float hi_of(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
 // a pair of fp32 values rounded to a bf16 pair (low element in the low half)
@@ -138,12 +143,10 @@ __device__ __forceinline__ void offdiag16(const uint32_t (&g)[16], float r, cons
 // The diagonal block: columns [s1, s1 + 16) of row `row` (s1 = 32 J + c0, J =
 // row / 32). The forward term g_f (r_f colf) is kept for s <= t and the reverse
 // term g_b (r_b colb) for s >= t; on the row's own token both are kept, each
-// equal to G dt there (the two factors of exp(a_t - a_e) exp(a_e - a_t)), and
-// the skip coefficient dsum = D_f + D_b is added, so that the product with X
-// carries the skip term (D_f + D_b) x_t as well.
+// equal to G dt there (the two factors of exp(a_t - a_e) exp(a_e - a_t)).
 // Factorised while the block's decay span is below kMaxSpan, else one
 // exponential per entry (as mask_diag).
-__device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, float my_ab, float dsum,
+__device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, float my_ab,
                                        const uint32_t (&gf)[16], const uint32_t (&gb)[16], const MaskVectors &v,
                                        uint32_t (&packed)[8]) {
     const int s0 = J * 32, s1 = s0 + c0;
@@ -158,9 +161,8 @@ __device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, floa
             const float2 cb = *reinterpret_cast<const float2 *>(v.colb + s1 + k);
             const uint64_t pf = mul2(f2u(gf[k], gf[k + 1]), mul2(rf, f2(cf.x, cf.y)));
             const uint64_t pb = mul2(f2u(gb[k], gb[k + 1]), mul2(rb, f2(cb.x, cb.y)));
-            const float m0 = (k <= rr ? lo_of(pf) : 0.f) + (k >= rr ? lo_of(pb) : 0.f) + (k == rr ? dsum : 0.f);
-            const float m1 =
-                (k + 1 <= rr ? hi_of(pf) : 0.f) + (k + 1 >= rr ? hi_of(pb) : 0.f) + (k + 1 == rr ? dsum : 0.f);
+            const float m0 = (k <= rr ? lo_of(pf) : 0.f) + (k >= rr ? lo_of(pb) : 0.f);
+            const float m1 = (k + 1 <= rr ? hi_of(pf) : 0.f) + (k + 1 >= rr ? hi_of(pb) : 0.f);
             packed[k / 2] = pack_bf16x2(m0, m1);
         }
     } else {
@@ -172,7 +174,7 @@ __device__ __forceinline__ void diag16(int J, int c0, int row, float my_af, floa
             // the exponent of the selected side is <= 0
             m[c] = c < rr ? gfv * v.dtf[s] * __expf(my_af - v.af[s])
                  : c > rr ? gbv * v.dtb[s] * __expf(my_ab - v.ab[s])
-                          : gfv * v.dtf[s] + gbv * v.dtb[s] + dsum;
+                          : gfv * v.dtf[s] + gbv * v.dtb[s];
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) packed[k] = pack_bf16x2(m[2 * k], m[2 * k + 1]);
@@ -298,7 +300,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tmem_wait_ld();
                 const uint32_t mrow = tM(j) + lane_off + 8 * half;
                 uint32_t packed[8];
-                diag16(q, c0, row, my_af, my_ab, V[768], gdf, gdb, mv, packed);
+                diag16(q, c0, row, my_af, my_ab, gdf, gdb, mv, packed);
                 tmem_st8(mrow + 16 * q, packed);
 #pragma unroll
                 for (int k = 0; k < 3; ++k) {
@@ -331,14 +333,13 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int t0 = 4 * lane;
         bool ok = true;
         HeadPos pos = head_at(vw);
-        float vf[4], vb[4], Af = 0.f, Ab = 0.f, Dn = 0.f;
+        float vf[4], vb[4], Af = 0.f, Ab = 0.f;
         auto load = [&](int j) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) vf[k] = vb[k] = 0.f;
             if (j < n) {
                 Af = __ldg(p.A + pos.h);
                 Ab = __ldg(p.A + p.H + pos.h);
-                Dn = __ldg(p.D + pos.h) + __ldg(p.D + p.H + pos.h);
                 const __nv_bfloat16 *df = p.dt + (size_t)pos.b * p.L * p.H + pos.h;
                 const __nv_bfloat16 *db = df + (size_t)p.batch * p.L * p.H;
 #pragma unroll
@@ -356,7 +357,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll 1
         for (int j = vw; j < n; j += kVS) {
             const float cf[4] = {vf[0], vf[1], vf[2], vf[3]}, cb[4] = {vb[0], vb[1], vb[2], vb[3]};
-            const float A_f = Af, A_b = Ab, Ds = Dn;
+            const float A_f = Af, A_b = Ab;
             load(j + kVS);     // this warp's next head, in flight while this one is computed
             // inclusive sums over the lane's four tokens, then across the warp
             float sf[4], sb[4];
@@ -392,7 +393,6 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                                                  abort_flag, p.status, 1011));
             if (!ok) break;
             float *V = vbuf(j);
-            if (lane == 0) V[768] = Ds;
             *reinterpret_cast<float4 *>(V + t0) = make_float4(af[0], af[1], af[2], af[3]);
             *reinterpret_cast<float4 *>(V + 128 + t0) = make_float4(ab[0], ab[1], ab[2], ab[3]);
             *reinterpret_cast<float4 *>(V + 256 + t0) = make_float4(cf[0], cf[1], cf[2], cf[3]);
@@ -508,7 +508,8 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int i = 0; i < n; ++i) {
             if (i > 0) pos_e.next(p.H);
             const int hi = pos_e.h;
-            // ---------------- epilogue of head i: y = Y (the skip term rides on M's diagonal), written over x
+            const float ds = __ldg(p.D + hi) + __ldg(p.D + p.H + hi);
+            // ---------------- epilogue of head i: y = Y + (D_f + D_b) x, written over x
             ok = __all_sync(0xffffffffu, ok && mbar_wait_ool(bar(B_Y + (i & 1)), (uint32_t)(i >> 1) & 1u, abort_flag,
                                                              p.status, 1007) &&
                                              mbar_wait_ool(bar(B_X + i % kXS), (uint32_t)(i / kXS) & 1u, abort_flag,
@@ -525,18 +526,23 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             __syncwarp();    // the named barriers are warp-collective: reconverge after the leader's steps
             if (bar_or(2, 128, !ok)) break;
             if (leader) mbar_arrive(bar(B_YE + (i & 1)));    // Y_i read out: the MMA of head i + 2 may write it
-            // y as bf16 over x (whose MMA has completed), for the TMA store
+            // y = Y + (D_f + D_b) x in fp32 (fused, two at a time), rounded once to
+            // bf16 over x (whose MMA has completed) for the TMA store
             uint8_t *xs = g + xslot(i);
+            const uint64_t dd = f2(ds, ds);
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) {
+                uint4 *ptr = reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc));
+                const uint4 xv = *ptr;
+                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
                 uint32_t o[4];
 #pragma unroll
                 for (int j2 = 0; j2 < 4; ++j2) {
                     const int c = (cc & 3) * 8 + 2 * j2;
                     const uint32_t y0 = cc < 4 ? ya[c] : yb[c], y1 = cc < 4 ? ya[c + 1] : yb[c + 1];
-                    o[j2] = pack_bf16x2(__uint_as_float(y0), __uint_as_float(y1));
+                    o[j2] = bf16x2_of(fma2(dd, f2u(xu[j2] << 16, xu[j2] & 0xffff0000u), f2u(y0, y1)));
                 }
-                *reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *ptr = make_uint4(o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async_smem();
             __syncwarp();

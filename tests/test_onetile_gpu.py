@@ -41,7 +41,7 @@ def full_oracle(inp):
 # (batch, L, H, N, G)
 SHAPES = [(3, 128, 4, 128, 1), (2, 100, 6, 64, 2), (5, 1, 2, 128, 1), (4, 77, 8, 128, 8),
           (40, 128, 24, 128, 1), (64, 128, 8, 128, 2), (50, 100, 6, 64, 1), (37, 128, 4, 128, 4),
-          (7, 128, 6, 64, 3), (200, 128, 3, 128, 3)]
+          (7, 128, 6, 64, 3), (200, 128, 3, 128, 3), (6, 100, 8, 128, 2)]
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "b%d_L%d_H%d_N%d_G%d" % s)

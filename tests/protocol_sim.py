@@ -1,5 +1,6 @@
 """Discrete-event engine for the barrier-protocol models of the persistent
-tensor-core kernels (test_fused_protocol.py, test_pair_protocol.py).
+tensor-core kernels (test_fused_protocol.py, test_pair_protocol.py,
+test_onetile_protocol.py).
 
 Roles are generators that yield the commands below; asynchronous completions
 (TMA loads and stores, MMAs in issue order) land after random, heavy-tailed
@@ -17,6 +18,8 @@ Commands:
   ('read', res, val) / ('write', res, val)
   ('sync', name, n)                   named barrier over n roles
   ('store', [(res,val)]) then ('store_wait',)      store's shared-memory read
+  ('store_wait1',)                    the shared-memory reads of all but the
+                                      role's newest store (bulk wait_group.read 1)
   ('store_g', [(res,val)] smem reads, [(res,val)] global writes)
   ('store_wait_all',)                 all of the role's stores complete
   ('gset', flag, value)               a release store of a flag in global memory
@@ -81,6 +84,7 @@ def run_roles(S, roles, counts):
     done = set()
     syncs = {}                            # name -> set of roles arrived
     store_pending = {}
+    store_reads = {}                      # role -> shared-memory read times of its stores, in order
     store_done = {}                       # role -> completion time of its last global store
     def bar(n):
         return S.bar(n, counts.get(n, 1))
@@ -167,6 +171,7 @@ def run_roles(S, roles, counts):
             tr = S.t + S.delay()
             tc = tr + S.delay()
             store_pending[name] = (tr, c[1])
+            store_reads.setdefault(name, []).append(tr)
             store_done[name] = max(store_done.get(name, 0.0), tc)
             def rd(items=c[1]):
                 for k, v in items:
@@ -179,6 +184,9 @@ def run_roles(S, roles, counts):
         elif op == 'store_wait':
             tr, _ = store_pending[name]
             if S.t < tr:
+                return False
+        elif op == 'store_wait1':
+            if S.t < max(store_reads.get(name, [0.0])[:-1], default=0.0):
                 return False
         elif op == 'store_wait_all':
             if S.t < store_done.get(name, 0.0):

@@ -530,11 +530,14 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             // bf16 over x (whose MMA has completed) for the TMA store
             uint8_t *xs = g + xslot(i);
             const uint64_t dd = f2(ds, ds);
+            // every x chunk of the row first (the stores below would otherwise
+            // hold each load back: the swizzled addresses are not known apart)
+            uint4 xv[8];
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) xv[cc] = *reinterpret_cast<const uint4 *>(xs + sw128_offset(r, cc));
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) {
-                uint4 *ptr = reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc));
-                const uint4 xv = *ptr;
-                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+                const uint32_t xu[4] = {xv[cc].x, xv[cc].y, xv[cc].z, xv[cc].w};
                 uint32_t o[4];
 #pragma unroll
                 for (int j2 = 0; j2 < 4; ++j2) {
@@ -542,7 +545,7 @@ onetile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const uint32_t y0 = cc < 4 ? ya[c] : yb[c], y1 = cc < 4 ? ya[c + 1] : yb[c + 1];
                     o[j2] = bf16x2_of(fma2(dd, f2u(xu[j2] << 16, xu[j2] & 0xffff0000u), f2u(y0, y1)));
                 }
-                *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(xs + sw128_offset(r, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async_smem();
             __syncwarp();

@@ -6,16 +6,17 @@
 //   y = (M_f + M_b) X + (D_f + D_b) x,
 //   M_f[t][s] = G_f[t][s] exp(a_t - a_s) dt_f[s] (s <= t),
 //   M_b[t][s] = G_b[t][s] exp(a'_t - a'_s) dt_b[s] (s >= t),
-// with G = C B^T of each direction. G depends only on the B/C group, not on
-// the head, so the kernel takes one (batch, B/C group) at a time, forms G_f
-// and G_b once on the tensor cores (TMEM, fp32), and then, for each head of
-// the group, builds the head's mask from G and its own decays (bf16, in
-// TMEM), runs Y = M X and writes y. With B/C shared by all heads (Mamba-2's
-// ngroups = 1) the 24 heads of a batch element share two G tiles.
+// with G = C B^T of each direction. G depends only on the batch element and
+// the B/C group, not on the head. Each CTA takes a contiguous run of (batch,
+// head) units; for each B/C group in its run it forms G_f and G_b once on the
+// tensor cores (TMEM, fp32), and then, for each head of the group, builds the
+// head's mask from G and its own decays (bf16, in TMEM), runs Y = M X and
+// writes y. With B/C shared by all heads (Mamba-2's ngroups = 1) the 24
+// heads of a batch element share two G tiles.
 // The two scans, added: "DiffuMamba: High-Throughput Diffusion LMs with Mamba
-// Backbone", Technical Summary, 2. Methodology, Core Architecture; the
-// packed 128-token shape: "Diffusion Mamba ... (LM1B, packed sequences of
-// 128)" as the pages' second workload.
+// Backbone", Technical Summary, 2. Methodology, Core Architecture. The
+// packed 128-token, batch-512 shape: the "Waspr/mdlm-lm1b-gpt2-packed"
+// model page (LM1B packed to 128 tokens, batch 512).
 //
 // Per CTA: 512 threads in four roles that hand work over through mbarriers,
 // persistent over a contiguous run of (batch, head) units:

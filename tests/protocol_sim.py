@@ -1,6 +1,6 @@
 """Discrete-event engine for the barrier-protocol models of the persistent
 tensor-core kernels (test_fused_protocol.py, test_pair_protocol.py,
-test_onetile_protocol.py).
+test_onetile_protocol.py, test_blockstep_protocol.py).
 
 Roles are generators that yield the commands below; asynchronous completions
 (TMA loads and stores, MMAs in issue order) land after random, heavy-tailed

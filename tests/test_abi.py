@@ -129,6 +129,18 @@ def test_prefix_and_block_reject_bad_arguments(lib):
     assert bs(0, 64, 32, 64, 128, 32, 1, ptr=0) == 0
 
 
+def test_auto_path_takes_the_one_tile_kernel_for_short_bf16_sequences(lib):
+    """ssd_select_path (host only): bf16 sequences of at most 128 tokens with
+    d_state 64 or 128 run the one-tile kernel (SSD_PATH_ONETILE = 7) whatever
+    the batch and grouping; longer ones, fp32 and other d_state do not."""
+    sp = lambda *a: lib.ssd_select_path(*a)
+    for batch, L, H, N, G in [(512, 128, 24, 128, 1), (1, 1, 2, 64, 1), (6, 100, 8, 128, 2), (3, 77, 8, 64, 8)]:
+        assert sp(batch, L, H, 64, N, G, 64, 1) == 7, (batch, L, H, N, G)
+    assert sp(512, 129, 24, 64, 128, 1, 64, 1) != 7
+    assert sp(512, 128, 24, 64, 128, 1, 64, 0) == 1          # fp32: the sequential scan
+    assert sp(4, 128, 24, 64, 32, 1, 64, 1) != 7             # d_state 32 is not a one-tile shape
+
+
 def test_status_requires_workspace(lib):
     assert lib.ssd_get_device_status(None, None) == -4
     assert lib.ssd_workspace_init(None, 256, None) == -4
